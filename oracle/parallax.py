@@ -1,0 +1,118 @@
+"""Float64 CPU oracle for Parallax attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code
+with the CUDA path (the seeded input generator is the only module both sides
+use), and it is deliberately plain and slow.
+
+What it computes ("Parallax: Parameterized Local Linear Attention for Language
+Modeling", arXiv 2605.29157):
+
+* The layer output is softmax attention minus a covariance correction,
+  ``o_i = o^SA_i - Sigma_KV^(i) rho_i`` (gist.science summary, "Mecanismo
+  central", the one printed formula), where ``rho_i`` is the per-query probe
+  (agihunt.info summary: rho = W_R x, with its own RMSNorm and RoPE; the
+  kernels receive it as the tensor R).
+* ``Sigma_KV^(i)`` is the softmax-weighted covariance of the visible values
+  and keys, ``sum_j p_ij (v_j - vbar_i)(k_j - kbar_i)^T``, with
+  ``p_ij = softmax_j(q_i . k_j / sqrt(d))`` (rainbus.top summary, "Softmax
+  Attention" and the six-step forward in "方法步骤详情": softmax weights, key
+  differences, probe inner products, corrected weights, two outputs, combine).
+* The boundary amplification factor eta is zero (gist.science, "Eliminación
+  de la Amplificación de Frontera"), so nothing multiplies the correction.
+
+The function below writes that definition out in two passes per query row:
+first the softmax weights and the weighted means kbar and vbar, then the
+centred second moment applied to rho.  It never uses the streamed
+(O1, O2, tbar) rearrangement that the kernels use; the tests pin the two
+against each other.
+
+Readings of the pages adopted here (the pages print no layout or mask rule):
+scores are scaled by 1/sqrt(d) and the probe term is not scaled; the causal
+mask lets query i see keys j <= i; a decode query at KV length n sees keys
+0..n-1; Q, K, V, R are [B, H, N, d] and all heads have their own K and V.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def parallax_row(q: np.ndarray, rho: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """Parallax output for one query over its visible keys.
+
+    q, rho: [d]; K, V: [n, d] (only the keys the query may see, n >= 1).
+    Returns float64 [d] = vbar - sum_j p_j (v_j - vbar) ((k_j - kbar) . rho).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    rho = np.asarray(rho, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    d = q.shape[0]
+    # Softmax weights over the visible keys.
+    s = (K @ q) / math.sqrt(d)
+    w = np.exp(s - s.max())
+    p = w / w.sum()
+    # First pass: weighted means.
+    kbar = p @ K
+    vbar = p @ V
+    # Second pass: centred covariance applied to the probe.
+    kc = K - kbar
+    vc = V - vbar
+    probe = kc @ rho                     # (k_j - kbar) . rho   for every j
+    correction = vc.T @ (p * probe)      # Sigma_KV rho
+    return vbar - correction
+
+
+def prefill_ref(Q, K, V, R, causal: bool = True, rows=None) -> np.ndarray:
+    """Oracle for a prefill.
+
+    Q, K, V, R: float64 arrays [B, H, N, d].  ``rows`` is None (every output
+    row) or an iterable of (b, h, i) triples; the result is then [len(rows), d]
+    in the same order.
+    """
+    B, H, N, d = Q.shape
+    if rows is None:
+        out = np.empty((B, H, N, d), dtype=np.float64)
+        for b in range(B):
+            for h in range(H):
+                for i in range(N):
+                    n = i + 1 if causal else N
+                    out[b, h, i] = parallax_row(Q[b, h, i], R[b, h, i], K[b, h, :n], V[b, h, :n])
+        return out
+    res = []
+    for (b, h, i) in rows:
+        n = i + 1 if causal else N
+        res.append(parallax_row(Q[b, h, i], R[b, h, i], K[b, h, :n], V[b, h, :n]))
+    return np.stack(res) if res else np.zeros((0, d))
+
+
+def decode_ref(q, r, Kc, Vc, seqlens, units=None) -> np.ndarray:
+    """Oracle for one decode step.
+
+    q, r: [B, H, d]; Kc, Vc: [B, H, L, d]; seqlens: [B] ints in 1..L.  The
+    query of sequence b sits at position seqlens[b]-1 and sees keys
+    0..seqlens[b]-1.  ``units`` is None (all (b, h)) or a list of (b, h).
+    """
+    B, H, d = q.shape
+    if units is None:
+        units = [(b, h) for b in range(B) for h in range(H)]
+        full = True
+    else:
+        full = False
+    res = []
+    for (b, h) in units:
+        n = int(seqlens[b])
+        res.append(parallax_row(q[b, h], r[b, h], Kc[b, h, :n], Vc[b, h, :n]))
+    out = np.stack(res)
+    return out.reshape(B, H, d) if full else out
+
+
+def softmax_weights_row(q, K) -> np.ndarray:
+    """p_j for one query (exposed for the invariant tests on s_ij)."""
+    q = np.asarray(q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    s = (K @ q) / math.sqrt(q.shape[0])
+    w = np.exp(s - s.max())
+    return w / w.sum()

@@ -1,0 +1,50 @@
+"""Host side of the seeded input generator (CPU only)."""
+import numpy as np
+import torch
+
+from local_linear_attention_streamed_b200 import synth
+
+
+def test_splitmix64_published_sequence():
+    # SplitMix64 seeded with 0: first outputs as published with the reference
+    # implementation (Vigna's splitmix64.c) — 0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4.
+    h = synth.raw_hash(0, np.arange(2, dtype=np.uint64))
+    assert int(h[0]) == 0xE220A8397B1DCDAF
+    assert int(h[1]) == 0x6E789E6AA1B965F4
+
+
+def test_deterministic_and_sliceable():
+    a = synth.draw(7, synth.TID_K, 0, 4096, synth.RMS_ROWS, synth.BF16, row=128)
+    b = synth.draw(7, synth.TID_K, 0, 4096, synth.RMS_ROWS, synth.BF16, row=128)
+    assert np.array_equal(a, b)
+    c = synth.draw(7, synth.TID_K, 1024, 2048, synth.RMS_ROWS, synth.BF16, row=128)
+    assert np.array_equal(a[1024:3072], c)
+    d = synth.draw(8, synth.TID_K, 0, 4096, synth.RMS_ROWS, synth.BF16, row=128)
+    assert not np.array_equal(a, d)
+
+
+def test_distribution_moments():
+    x = synth.draw_f64(3, synth.TID_V, 0, 1 << 20, synth.NORMAL, sigma=0.25)
+    assert abs(x.mean()) < 2e-3
+    assert abs(x.std() - 0.25) < 2e-3
+    assert np.abs(x).max() <= 0.25 * np.sqrt(3.0) * 2.0 + 1e-12
+    r = synth.draw_f64(3, synth.TID_Q, 0, 128 * 512, synth.RMS_ROWS, row=128).reshape(-1, 128)
+    np.testing.assert_allclose(np.sqrt((r * r).mean(axis=1)), 1.0, rtol=0, atol=1e-14)
+
+
+def test_bf16_rounding_matches_torch():
+    x = synth.draw_f64(5, synth.TID_Q, 0, 1 << 16, synth.NORMAL, sigma=3.0).astype(np.float32)
+    ours = synth.f32_to_bf16_bits(x)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    np.testing.assert_array_equal(synth.bf16_bits_to_f64(ours),
+                                  torch.from_numpy(x).to(torch.bfloat16).double().numpy())
+
+
+def test_seqlens_range():
+    s = synth.seqlens(11, 4096, 1000, ragged=True)
+    assert s.min() >= 500 and s.max() <= 1000
+    assert len(np.unique(s)) > 400
+    assert (synth.seqlens(11, 8, 64, ragged=False) == 64).all()
+    s1 = synth.seqlens(11, 64, 1, ragged=True)
+    assert (s1 == 1).all()
