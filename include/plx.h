@@ -1,0 +1,154 @@
+/*
+ * plx.h — C ABI of libplx.so: Parallax attention forward on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Parallax: Parameterized Local Linear Attention for Language Modeling"
+ * (arXiv 2605.29157).  Per query i over its visible keys J_i:
+ *
+ *   p_ij  = softmax_j(q_i . k_j / sqrt(d))                (rainbus.top summary, "Softmax Attention")
+ *   out_i = o^SA_i - Sigma_KV^(i) rho_i                    (gist.science summary, "Mecanismo central")
+ *         = sum_j p_ij (1 - t_ij + tbar_i) v_j,  t_ij = rho_i . k_j,  tbar_i = sum_j p_ij t_ij
+ *
+ * computed in the streamed form with one running max and one rescale factor
+ * shared by the softmax branch and the covariance branch (rainbus.top summary,
+ * "方法步骤详情": per KV block S1 = QK^T and S2 = RK^T, then O1 = sum w v and
+ * O2 = sum w t v accumulated together; agihunt.info summary, hardware paragraph).
+ * The boundary amplification factor eta is zero (gist.science, "Eliminación de la
+ * Amplificación de Frontera").  rho_i (R) is an input: the probe W_R x after its
+ * RMSNorm and RoPE.
+ *
+ * Conventions (the pages give no layout):
+ *   - Prefill tensors Q, K, V, R, out are [B, H, N, d], row-major, d fastest.
+ *   - Decode: q, r, out are [B, H, d]; Kcache, Vcache are [B, H, L, d] with each
+ *     sequence padded to stride L; seqlens is int32 [B] with 1 <= seqlens[b] <= L.
+ *     The query of sequence b sits at position seqlens[b]-1 and sees keys
+ *     0 .. seqlens[b]-1.
+ *   - Scores are scaled by 1/sqrt(d); the probe term t = rho . k is not scaled.
+ *   - causal != 0: query row i sees keys 0..i (diagonal included).  causal == 0:
+ *     every row sees all N keys.
+ *   - Every head has its own K and V (no grouping).
+ *   - out has the dtype of the inputs; arithmetic is fp32.
+ *
+ * Memory and ownership: every tensor pointer is a DEVICE pointer owned by the
+ * caller; the library keeps no reference after the call returns.  Calls are
+ * asynchronous on the given CUDA stream (void* stands for cudaStream_t; NULL is
+ * the legacy default stream).  All tensor pointers must be 16-byte aligned.
+ *
+ * Errors: every entry point returns PLX_OK (0) or a negative code.  Argument
+ * errors are detected on the host before anything is launched.  Errors found by
+ * a kernel (a seqlen outside 1..L, a bounded wait that ran out) are recorded in a
+ * per-device status word that plx_get_device_status() reads and clears; such a
+ * kernel writes zeros for the affected outputs and never traps.
+ */
+#ifndef PLX_H
+#define PLX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PLX_ABI_VERSION 1
+
+/* Element type of all tensors of one call. */
+typedef enum { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
+
+/* Status codes. */
+#define PLX_OK 0
+#define PLX_ERR_INVALID_ARG (-1)  /* null pointer, non-positive size, bad enum      */
+#define PLX_ERR_UNSUPPORTED (-2)  /* head dim or dtype combination not implemented */
+#define PLX_ERR_MISALIGNED (-3)   /* a tensor pointer is not 16-byte aligned       */
+#define PLX_ERR_CUDA (-4)         /* a CUDA runtime/driver call or launch failed   */
+#define PLX_ERR_WORKSPACE (-5)    /* caller workspace smaller than required        */
+#define PLX_ERR_BAD_SEQLEN (-6)   /* device-reported: a seqlens[b] outside 1..L    */
+#define PLX_ERR_TIMEOUT (-7)      /* device-reported: a bounded wait gave up       */
+
+/* Supported shapes: bf16 with d in {64, 128}; f32 with d a multiple of 32 and
+ * d <= 128.  B, H, N, L >= 1. */
+
+/*
+ * Causal (or full) prefill forward.  bf16 on the legacy default stream.
+ * Q, K, V, R, out: [B, H, N, d].
+ */
+int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void* out,
+                int B, int H, int N, int d, int causal);
+
+/* As plx_prefill with an explicit element type and stream. */
+int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, void* out,
+                   int B, int H, int N, int d, int causal, int dtype, void* stream);
+
+/*
+ * One decode step with split-KV: every (b, h) streams its cache rows
+ * 0..seqlens[b]-1; partial results (running max m, omega = sum w, T = sum w t,
+ * O1, O2) of the key chunks are merged inside the kernel by the last chunk to
+ * finish.  bf16 on the legacy default stream with a library-owned workspace.
+ */
+int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vcache,
+               const int32_t* seqlens, void* out, int B, int H, int L, int d);
+
+/*
+ * As plx_decode with an explicit element type, workspace and stream.
+ * workspace: device memory of at least plx_decode_workspace_bytes(B, H, L, d)
+ * bytes, 256-byte aligned, ZEROED by the caller before its first use (the kernel
+ * leaves its counters at zero again when it finishes).  NULL selects a
+ * library-owned workspace, grown on demand, one per device.  Two calls that
+ * share a workspace must not run concurrently.
+ */
+int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                  const int32_t* seqlens, void* out, int B, int H, int L, int d, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace plx_decode_ex needs for these sizes (0 if none is needed). */
+size_t plx_decode_workspace_bytes(int B, int H, int L, int d);
+
+/*
+ * Number of key chunks each (b, h) is split into for these sizes (the partial
+ * records per (b, h) the workspace holds).  For tests and diagnostics.
+ */
+int plx_decode_num_splits(int B, int H, int L, int d);
+
+/*
+ * Per-head RMSNorm (unit weight, eps) followed by rotate-half RoPE (frequencies
+ * base^(-2k/d), position = token index) of a projected activation, with the
+ * head split folded in: x is bf16 [B, N, H*d] (token-major, as a GEMM writes it),
+ * y is bf16 [B, H, N, d].  The agihunt.info summary states that rho gets its own
+ * RMSNorm and RoPE; q and k take the same treatment (Qwen-3 style).
+ */
+int plx_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,
+                      float rope_base, void* stream);
+
+/* The library-owned scratch a full layer forward needs, in bytes. */
+size_t plx_layer_workspace_bytes(int B, int N, int H, int d);
+
+/*
+ * Full Parallax attention layer, bf16 (projections with fp32 accumulation):
+ *   q,k,v,rho = x W_Q, x W_K, x W_V, x W_R     (W stored [in, out] = [H*d, H*d])
+ *   q,k,rho  <- RoPE(RMSNorm(.)) per head     (plx_qkr_norm_rope, eps 1e-6, base 10000)
+ *   o         = causal Parallax prefill over [B, H, N, d]
+ *   y         = o W_O                          (o merged back to [B, N, H*d])
+ * x, y: bf16 [B, N, H*d].  workspace: device memory of plx_layer_workspace_bytes()
+ * bytes, or NULL for a library-owned one.
+ */
+int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void* WV,
+                      const void* WR, const void* WO, void* y, int B, int N, int H, int d,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Waits for `stream`, then reads and clears this device's kernel status word.
+ * Returns PLX_OK, or the first device-reported error since the last read
+ * (PLX_ERR_BAD_SEQLEN, PLX_ERR_TIMEOUT), or PLX_ERR_CUDA if the wait failed.
+ */
+int plx_get_device_status(void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* plx_status_string(int code);
+
+/* PLX_ABI_VERSION of the loaded library. */
+int plx_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PLX_H */

@@ -1,0 +1,318 @@
+// C ABI of libplx.so (declared in include/plx.h): host-side validation,
+// kernel selection, library-owned workspaces and the per-device status word.
+#include "plx_internal.cuh"
+
+#include <cublas_v2.h>
+
+#include <mutex>
+
+#include "../../include/plx.h"
+
+namespace plx {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+// Per-device kernel status word (bits of kStatus*); kernels atomicOr into it.
+__device__ int g_status;
+
+struct DeviceCache {
+  bool init = false;
+  int num_sms = 0;
+  int* status = nullptr;  // device address of g_status on this device
+  void* decode_ws = nullptr;
+  size_t decode_ws_bytes = 0;
+  void* layer_ws = nullptr;
+  size_t layer_ws_bytes = 0;
+  cublasHandle_t cublas = nullptr;
+};
+
+std::mutex g_mu;
+DeviceCache g_dev[kMaxDevices];
+
+int current_device(DeviceCache** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
+  DeviceCache& c = g_dev[dev];
+  if (!c.init) {
+    if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return PLX_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&c.status), g_status) != cudaSuccess)
+      return PLX_ERR_CUDA;
+    c.init = true;
+  }
+  *out = &c;
+  return PLX_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+
+// Shapes each kernel family supports.
+int check_head_dim(int d, int dtype) {
+  if (dtype == PLX_BF16) return (d == 64 || d == 128) ? PLX_OK : PLX_ERR_UNSUPPORTED;
+  if (dtype == PLX_F32) return (d >= 32 && d <= 128 && d % 32 == 0) ? PLX_OK : PLX_ERR_UNSUPPORTED;
+  return PLX_ERR_INVALID_ARG;
+}
+
+// Grows a library-owned buffer; new memory is zeroed (decode counters start at 0).
+int grow(void** ptr, size_t* bytes, size_t need, cudaStream_t st) {
+  if (*bytes >= need) return PLX_OK;
+  if (*ptr) {
+    if (cudaFree(*ptr) != cudaSuccess) return PLX_ERR_CUDA;
+    *ptr = nullptr;
+    *bytes = 0;
+  }
+  if (cudaMalloc(ptr, need) != cudaSuccess) {
+    *ptr = nullptr;
+    return PLX_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(*ptr, 0, need, st) != cudaSuccess) return PLX_ERR_CUDA;
+  *bytes = need;
+  return PLX_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk,
+                        size_t* partial_off) {
+  decode_split_plan(B, H, L, num_sms, splits, chunk);
+  if (*splits <= 1) {
+    *partial_off = 0;
+    return 0;
+  }
+  size_t counters = round_up(sizeof(int) * (size_t)B * H, 256);
+  *partial_off = counters;
+  return counters + sizeof(float) * (size_t)B * H * (size_t)(*splits) * (size_t)(2 * d + 4);
+}
+
+int num_sms_or_default() {
+  DeviceCache* c = nullptr;
+  if (current_device(&c) == PLX_OK) return c->num_sms;
+  return 148;
+}
+
+}  // namespace
+}  // namespace plx
+
+using namespace plx;
+
+extern "C" {
+
+int plx_abi_version(void) { return PLX_ABI_VERSION; }
+
+const char* plx_status_string(int code) {
+  switch (code) {
+    case PLX_OK: return "ok";
+    case PLX_ERR_INVALID_ARG: return "invalid argument (null pointer, non-positive size or bad enum)";
+    case PLX_ERR_UNSUPPORTED: return "unsupported head dimension / dtype combination";
+    case PLX_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case PLX_ERR_CUDA: return "CUDA runtime or launch failure";
+    case PLX_ERR_WORKSPACE: return "workspace too small";
+    case PLX_ERR_BAD_SEQLEN: return "device reported a seqlens entry outside 1..L";
+    case PLX_ERR_TIMEOUT: return "device reported a bounded wait that ran out";
+    default: return "unknown status code";
+  }
+}
+
+int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
+                   int H, int N, int d, int causal, int dtype, void* stream) {
+  if (!Q || !K || !V || !R || !out) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  int rc = check_head_dim(d, dtype);
+  if (rc != PLX_OK) return rc;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(R) || !aligned16(out))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  PrefillArgs a{Q, K, V, R, out, B, H, N, d, causal ? 1 : 0, dc->status};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == PLX_BF16 && prefill_tc_supported(d)) {
+    e = launch_prefill_tc(a, st, dc->num_sms);
+  } else {
+    e = launch_prefill_simt(a, dtype == PLX_BF16, st);
+  }
+  return e == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
+                int H, int N, int d, int causal) {
+  return plx_prefill_ex(Q, K, V, R, out, B, H, N, d, causal, PLX_BF16, nullptr);
+}
+
+int plx_decode_num_splits(int B, int H, int L, int d) {
+  (void)d;
+  if (B < 1 || H < 1 || L < 1) return 0;
+  int splits = 1, chunk = 0;
+  decode_split_plan(B, H, L, num_sms_or_default(), &splits, &chunk);
+  return splits;
+}
+
+size_t plx_decode_workspace_bytes(int B, int H, int L, int d) {
+  if (B < 1 || H < 1 || L < 1 || d < 1) return 0;
+  int splits = 1, chunk = 0;
+  size_t off = 0;
+  return decode_ws_layout(B, H, L, d, num_sms_or_default(), &splits, &chunk, &off);
+}
+
+int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                  const int32_t* seqlens, void* out, int B, int H, int L, int d, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !r || !Kcache || !Vcache || !seqlens || !out) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || L < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  int rc = check_head_dim(d, dtype);
+  if (rc != PLX_OK) return rc;
+  if (!aligned16(q) || !aligned16(r) || !aligned16(Kcache) || !aligned16(Vcache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.q = q;
+  a.r = r;
+  a.K = Kcache;
+  a.V = Vcache;
+  a.seqlens = seqlens;
+  a.out = out;
+  a.B = B;
+  a.H = H;
+  a.L = L;
+  a.d = d;
+  a.status = dc->status;
+  if (dtype == PLX_F32) {
+    return launch_decode_simt(a, false, st) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  }
+  size_t off = 0;
+  size_t need = decode_ws_layout(B, H, L, d, dc->num_sms, &a.splits, &a.chunk, &off);
+  if (need > 0) {
+    char* ws = nullptr;
+    if (workspace) {
+      if (workspace_bytes < need) return PLX_ERR_WORKSPACE;
+      if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PLX_ERR_MISALIGNED;
+      ws = static_cast<char*>(workspace);
+    } else {
+      std::lock_guard<std::mutex> lk(g_mu);
+      if ((rc = grow(&dc->decode_ws, &dc->decode_ws_bytes, need, st)) != PLX_OK) return rc;
+      ws = static_cast<char*>(dc->decode_ws);
+    }
+    a.counters = reinterpret_cast<int*>(ws);
+    a.partials = reinterpret_cast<float*>(ws + off);
+  }
+  return launch_decode_bf16(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vcache,
+               const int32_t* seqlens, void* out, int B, int H, int L, int d) {
+  return plx_decode_ex(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, PLX_BF16, nullptr, 0,
+                       nullptr);
+}
+
+int plx_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,
+                      float rope_base, void* stream) {
+  if (!x || !y) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || !(eps >= 0.f) || !(rope_base > 0.f)) return PLX_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(y)) return PLX_ERR_MISALIGNED;
+  return launch_qkr_norm_rope(x, y, B, N, H, d, eps, rope_base,
+                              reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PLX_OK
+             : PLX_ERR_CUDA;
+}
+
+size_t plx_layer_workspace_bytes(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  size_t t = round_up((size_t)B * N * H * d * 2, 256);
+  return 9 * t;  // 4 projections, 4 head-split tensors, attention output
+}
+
+int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void* WV, const void* WR,
+                      const void* WO, void* y, int B, int N, int H, int d, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  if (!x || !WQ || !WK || !WV || !WR || !WO || !y) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1) return PLX_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(WQ) || !aligned16(WK) || !aligned16(WV) || !aligned16(WR) ||
+      !aligned16(WO) || !aligned16(y))
+    return PLX_ERR_MISALIGNED;
+  DeviceCache* dc = nullptr;
+  int rc = current_device(&dc);
+  if (rc != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  size_t need = plx_layer_workspace_bytes(B, N, H, d);
+  char* ws = nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (workspace) {
+    if (workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PLX_ERR_MISALIGNED;
+    ws = static_cast<char*>(workspace);
+  } else {
+    if ((rc = grow(&dc->layer_ws, &dc->layer_ws_bytes, need, st)) != PLX_OK) return rc;
+    ws = static_cast<char*>(dc->layer_ws);
+  }
+  if (!dc->cublas) {
+    if (cublasCreate(&dc->cublas) != CUBLAS_STATUS_SUCCESS) {
+      dc->cublas = nullptr;
+      return PLX_ERR_CUDA;
+    }
+  }
+  if (cublasSetStream(dc->cublas, st) != CUBLAS_STATUS_SUCCESS) return PLX_ERR_CUDA;
+  const size_t t = round_up((size_t)B * N * H * d * 2, 256);
+  void* proj[4] = {ws, ws + t, ws + 2 * t, ws + 3 * t};          // q, k, v, rho: [B, N, H*d]
+  void* head[4] = {ws + 4 * t, ws + 5 * t, ws + 6 * t, ws + 7 * t};  // [B, H, N, d]
+  void* attn = ws + 8 * t;                                       // [B, H, N, d]
+  const void* W[4] = {WQ, WK, WV, WR};
+  const int D = H * d;
+  const long long M = (long long)B * N;
+  const float one = 1.f, zero = 0.f;
+  // Row-major Y[M, D] = X[M, D] W[D, D] is column-major Y^T = W^T X^T.
+  for (int i = 0; i < 4; ++i) {
+    if (cublasGemmEx(dc->cublas, CUBLAS_OP_N, CUBLAS_OP_N, D, (int)M, D, &one, W[i], CUDA_R_16BF, D,
+                     x, CUDA_R_16BF, D, &zero, proj[i], CUDA_R_16BF, D, CUBLAS_COMPUTE_32F,
+                     CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+      return PLX_ERR_CUDA;
+  }
+  const float eps = 1e-6f, base = 10000.f;
+  if (launch_qkr_norm_rope(proj[0], head[0], B, N, H, d, eps, base, st) != cudaSuccess ||
+      launch_qkr_norm_rope(proj[1], head[1], B, N, H, d, eps, base, st) != cudaSuccess ||
+      launch_swap_axes(proj[2], head[2], B, N, H, d, st) != cudaSuccess ||
+      launch_qkr_norm_rope(proj[3], head[3], B, N, H, d, eps, base, st) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  PrefillArgs a{head[0], head[1], head[2], head[3], attn, B, H, N, d, 1, dc->status};
+  cudaError_t e = prefill_tc_supported(d) ? launch_prefill_tc(a, st, dc->num_sms)
+                                          : launch_prefill_simt(a, true, st);
+  if (e != cudaSuccess) return PLX_ERR_CUDA;
+  // Merge heads back to [B, N, H*d] (reusing the q projection buffer), then W_O.
+  if (launch_swap_axes(attn, proj[0], B, H, N, d, st) != cudaSuccess) return PLX_ERR_CUDA;
+  if (cublasGemmEx(dc->cublas, CUBLAS_OP_N, CUBLAS_OP_N, D, (int)M, D, &one, WO, CUDA_R_16BF, D,
+                   proj[0], CUDA_R_16BF, D, &zero, y, CUDA_R_16BF, D, CUBLAS_COMPUTE_32F,
+                   CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+    return PLX_ERR_CUDA;
+  return PLX_OK;
+}
+
+int plx_get_device_status(void* stream) {
+  DeviceCache* dc = nullptr;
+  int rc = current_device(&dc);
+  if (rc != PLX_OK) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, dc->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  if (word != 0) {
+    int zero = 0;
+    if (cudaMemcpy(dc->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return PLX_ERR_CUDA;
+  }
+  if (word & kStatusBadSeqlen) return PLX_ERR_BAD_SEQLEN;
+  if (word & kStatusTimeout) return PLX_ERR_TIMEOUT;
+  return PLX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// Internal declarations shared by the translation units of libplx.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace plx {
+
+// Bits of the per-device status word that kernels set (atomicOr); the host
+// maps the lowest set bit to a status code.
+enum : int {
+  kStatusBadSeqlen = 1,
+  kStatusTimeout = 2,
+};
+
+// Iteration cap of every bounded wait in the kernels (mbarrier try_wait loops).
+// A wait that reaches it sets kStatusTimeout and abandons the tile.
+constexpr long long kWaitCap = 1ll << 26;
+
+struct PrefillArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const void* R;
+  void* out;
+  int B, H, N, d;
+  int causal;
+  int* status;
+};
+
+struct DecodeArgs {
+  const void* q;
+  const void* r;
+  const void* K;
+  const void* V;
+  const int32_t* seqlens;
+  void* out;
+  int B, H, L, d;
+  int splits;       // key chunks per (b, h)
+  int chunk;        // keys per chunk (multiple of 64)
+  float* partials;  // [B*H, splits, 2*d + 4] fp32: (m, omega, T, pad, O1[d], O2[d])
+  int* counters;    // [B*H] arrival counters, zero between calls
+  int* status;
+};
+
+// SIMT kernels: any d that is a multiple of 32 up to 128, f32 or bf16 storage.
+cudaError_t launch_prefill_simt(const PrefillArgs& a, bool bf16, cudaStream_t st);
+cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
+
+// bf16 split-KV decode on tensor-core MMAs, d in {64, 128}.
+cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms);
+// Split heuristic shared by the launcher and the workspace-size query.
+void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk);
+
+// bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
+bool prefill_tc_supported(int d);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms);
+
+// Per-head RMSNorm + RoPE with the head split folded in.
+cudaError_t launch_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,
+                                 float base, cudaStream_t st);
+// bf16 [B, A1, A2, d] -> [B, A2, A1, d] (head split and merge of a layer).
+cudaError_t launch_swap_axes(const void* src, void* dst, int B, int A1, int A2, int d,
+                             cudaStream_t st);
+
+}  // namespace plx

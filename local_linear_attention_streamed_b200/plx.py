@@ -1,0 +1,158 @@
+"""Thin ctypes binding over libplx.so (include/plx.h).
+
+Argument marshalling only: torch tensors are passed as raw device pointers and
+the current torch stream; every step of the computation runs in the library's
+CUDA kernels.  Loading fails loudly when the library is missing; there is no
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+PLX_F32 = 0
+PLX_BF16 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libplx.so")
+
+# Exported symbols and their C signatures (mirrors include/plx.h).
+_vp, _i, _sz, _f = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = {
+    "plx_prefill": (_i, [_vp] * 5 + [_i] * 5),
+    "plx_prefill_ex": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
+    "plx_decode": (_i, [_vp] * 6 + [_i] * 4),
+    "plx_decode_ex": (_i, [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]),
+    "plx_decode_workspace_bytes": (_sz, [_i] * 4),
+    "plx_decode_num_splits": (_i, [_i] * 4),
+    "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
+    "plx_layer_workspace_bytes": (_sz, [_i] * 4),
+    "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
+    "plx_get_device_status": (_i, [_vp]),
+    "plx_status_string": (ctypes.c_char_p, [_i]),
+    "plx_abi_version": (_i, []),
+}
+
+
+class PlxError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with __graft_entry__.build() "
+                           "(python -m local_linear_attention_streamed_b200._build)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_string(code: int) -> str:
+    return lib.plx_status_string(int(code)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise PlxError(rc, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return PLX_BF16
+    if t.dtype == torch.float32:
+        return PLX_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def prefill(Q, K, V, R, causal: bool = True, out=None, stream=None):
+    """Parallax prefill over [B, H, N, d] tensors (bf16 or fp32); returns out."""
+    B, H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("R", R)):
+        if t.shape != Q.shape or t.dtype != Q.dtype:
+            raise ValueError(f"{n} must match Q in shape and dtype")
+    if out is None:
+        out = torch.empty_like(Q)
+    rc = lib.plx_prefill_ex(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                            B, H, N, d, int(bool(causal)), _dtype_code(Q), _stream_ptr(stream))
+    _check(rc, "plx_prefill_ex")
+    return out
+
+
+def decode_workspace_bytes(B: int, H: int, L: int, d: int) -> int:
+    return int(lib.plx_decode_workspace_bytes(B, H, L, d))
+
+
+def decode(q, r, Kcache, Vcache, seqlens, out=None, workspace=None, stream=None):
+    """One decode step: q, r [B, H, d]; caches [B, H, L, d]; seqlens int32 [B]."""
+    B, H, L, d = Kcache.shape
+    if q.shape != (B, H, d) or r.shape != (B, H, d) or Vcache.shape != Kcache.shape:
+        raise ValueError("shape mismatch")
+    if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
+        raise ValueError("seqlens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.plx_decode_ex(_dev(q, "q"), _dev(r, "r"), _dev(Kcache, "Kcache"), _dev(Vcache, "Vcache"),
+                           _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, L, d, _dtype_code(q),
+                           ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(rc, "plx_decode_ex")
+    return out
+
+
+def qkr_norm_rope(x, H: int, eps: float = 1e-6, base: float = 10000.0, out=None, stream=None):
+    """x bf16 [B, N, H*d] -> RoPE(RMSNorm(.)) per head as [B, H, N, d]."""
+    B, N, D = x.shape
+    d = D // H
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=x.dtype, device=x.device)
+    rc = lib.plx_qkr_norm_rope(_dev(x, "x"), _dev(out, "out"), B, N, H, d, eps, base,
+                               _stream_ptr(stream))
+    _check(rc, "plx_qkr_norm_rope")
+    return out
+
+
+def layer_forward(x, WQ, WK, WV, WR, WO, H: int, out=None, workspace=None, stream=None):
+    """Full Parallax attention layer: x bf16 [B, N, H*d], W* bf16 [H*d, H*d] stored [in, out]."""
+    B, N, D = x.shape
+    d = D // H
+    if out is None:
+        out = torch.empty_like(x)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.plx_layer_forward(_dev(x, "x"), _dev(WQ, "WQ"), _dev(WK, "WK"), _dev(WV, "WV"),
+                               _dev(WR, "WR"), _dev(WO, "WO"), _dev(out, "out"), B, N, H, d,
+                               ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(rc, "plx_layer_forward")
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronises the stream, returns and clears the device status code."""
+    return int(lib.plx_get_device_status(_stream_ptr(stream)))

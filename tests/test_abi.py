@@ -1,0 +1,92 @@
+"""C ABI of libplx.so on the CPU: it loads, exports what include/*.h declares,
+and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+PKG = os.path.join(ROOT, "local_linear_attention_streamed_b200")
+
+
+def _declared(header):
+    text = open(os.path.join(ROOT, "include", header)).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(plx_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from local_linear_attention_streamed_b200 import plx
+    return plx.lib
+
+
+@pytest.mark.parametrize("header,so", [("plx.h", "libplx.so"), ("plx_synth.h", "libplx_synth.so")])
+def test_exports_every_declared_symbol(header, so):
+    names = _declared(header)
+    assert names, header
+    dll = ctypes.CDLL(os.path.join(PKG, so))
+    missing = [n for n in names if not hasattr(dll, n)]
+    assert not missing, f"{so} lacks {missing}"
+
+
+def test_binding_covers_header(lib):
+    from local_linear_attention_streamed_b200 import plx
+    assert set(_declared("plx.h")) == set(plx.SIGNATURES)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.plx_abi_version() == 1
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
+        s = lib.plx_status_string(code).decode()
+        assert s and s != "unknown status code"
+    assert lib.plx_status_string(-99).decode() == "unknown status code"
+
+
+A = 0x10000  # aligned fake device addresses: validation fails before they are used
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    ok = [A, A, A, A, A]
+    assert lib.plx_prefill_ex(None, A, A, A, A, 1, 1, 8, 64, 1, 1, None) == -1
+    assert lib.plx_prefill_ex(*ok, 0, 1, 8, 64, 1, 1, None) == -1
+    assert lib.plx_prefill_ex(*ok, 1, 1, 0, 64, 1, 1, None) == -1
+    assert lib.plx_prefill_ex(*ok, 1, 1, 8, 64, 1, 7, None) == -1
+    assert lib.plx_prefill_ex(*ok, 1, 1, 8, 96, 1, 1, None) == -2   # bf16 needs d in {64, 128}
+    assert lib.plx_prefill_ex(*ok, 1, 1, 8, 160, 1, 0, None) == -2  # f32 needs d <= 128
+    assert lib.plx_prefill_ex(*ok, 1, 1, 8, 48, 1, 0, None) == -2   # f32 needs d % 32 == 0
+    assert lib.plx_prefill_ex(A, A + 2, A, A, A, 1, 1, 8, 64, 1, 1, None) == -3
+
+
+def test_decode_rejects_bad_arguments(lib):
+    ok = [A] * 6
+    assert lib.plx_decode_ex(A, A, A, A, None, A, 1, 1, 8, 128, 1, None, 0, None) == -1
+    assert lib.plx_decode_ex(*ok, 1, 0, 8, 128, 1, None, 0, None) == -1
+    assert lib.plx_decode_ex(*ok, 1, 1, 8, 32, 1, None, 0, None) == -2
+    assert lib.plx_decode_ex(A, A, A, A + 8, A, A, 1, 1, 8, 128, 1, None, 0, None) == -3
+    assert lib.plx_decode_ex(A, A, A, A, A + 2, A, 1, 1, 8, 128, 1, None, 0, None) == -3
+
+
+def test_layer_and_norm_rope_reject_bad_arguments(lib):
+    assert lib.plx_qkr_norm_rope(None, A, 1, 8, 2, 128, 1e-6, 1e4, None) == -1
+    assert lib.plx_qkr_norm_rope(A, A, 1, 8, 2, 96, 1e-6, 1e4, None) == -2
+    assert lib.plx_qkr_norm_rope(A, A, 1, 8, 2, 128, -1.0, 1e4, None) == -1
+    assert lib.plx_layer_forward(*([A] * 6), None, 1, 8, 2, 128, None, 0, None) == -1
+    assert lib.plx_layer_forward(*([A] * 7), 1, 8, 2, 32, None, 0, None) == -2
+    assert lib.plx_layer_forward(*([A] * 6), A + 4, 1, 8, 2, 128, None, 0, None) == -3
+
+
+def test_decode_split_plan(lib):
+    for (B, H, L) in [(64, 16, 4096), (1, 16, 32768), (2048, 16, 4096), (1, 1, 1), (3, 5, 1000),
+                      (1, 16, 128), (8, 16, 16384)]:
+        S = lib.plx_decode_num_splits(B, H, L, 128)
+        assert 1 <= S <= max(1, L // 256) + 1
+        ws = lib.plx_decode_workspace_bytes(B, H, L, 128)
+        if S == 1:
+            assert ws == 0
+        else:
+            assert ws >= B * H * S * (2 * 128 + 4) * 4 + B * H * 4
+    # Small batches split the context; large ones do not need to.
+    assert lib.plx_decode_num_splits(1, 16, 32768, 128) > 8
+    assert lib.plx_decode_num_splits(2048, 16, 4096, 128) == 1
