@@ -90,10 +90,13 @@ int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vca
 /*
  * As plx_decode with an explicit element type, workspace and stream.
  * workspace: device memory of at least plx_decode_workspace_bytes(B, H, L, d)
- * bytes, 256-byte aligned, ZEROED by the caller before its first use (the kernel
- * leaves its counters at zero again when it finishes).  NULL selects a
- * library-owned workspace, grown on demand, one per device.  Two calls that
- * share a workspace must not run concurrently.
+ * bytes, 256-byte aligned, for the fp32 partial records of the key chunks (no
+ * initial contents needed), or NULL for a library-owned workspace, grown on
+ * demand, one per device.  The last chunk of each (b, h) to finish is found
+ * with an arrival counter; the counters live in a small library-owned array per
+ * device (allocated and zeroed on first use, left at zero by every call).
+ * Because of that array and of the library-owned workspace, decode calls on one
+ * device must be ordered (one stream, or synchronised), not run concurrently.
  */
 int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
                   const int32_t* seqlens, void* out, int B, int H, int L, int d, int dtype,

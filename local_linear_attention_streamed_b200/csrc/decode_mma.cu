@@ -13,7 +13,8 @@
 //   whose A tile carries q in row 0 and rho in row 1 (the pages' packing of the
 //   QK and RK products into one MMA; agihunt.info summary, decode paragraph).
 //   O1 and O2 come out of one MMA as well: V^T times [w ; w t] gives O1 and O2
-//   as the two columns of one accumulator.  The contraction dims and the key
+//   as columns of one accumulator (each weight split into a bf16 hi + lo pair
+//   that fills two of the MMA's otherwise idle columns).  The contraction dims and the key
 //   order inside a block are permuted consistently on both operands, so the
 //   16-byte vectors as loaded ARE the MMA fragments (V needs one byte-permute
 //   per two elements to pair keys); no shared-memory transpose is needed.
@@ -105,7 +106,7 @@ __device__ __forceinline__ void load_block(Frag<D>& f, const __nv_bfloat16* Kbh,
 template <int D>
 struct WarpState {
   static constexpr int MT = D / 16;
-  float O[MT][4];  // value-MMA accumulators: rows = dims, columns 0/1 = O1/O2
+  float O[MT][4];  // value-MMA accumulators: rows = dims, columns (0+1) = O1, (2+3) = O2
   float m;         // running max (log2 domain), warp-uniform
   float omega, T;  // partial sums held by lanes 0..3
 };
@@ -129,24 +130,21 @@ __device__ __forceinline__ void compute_block(WarpState<D>& s, const Frag<D>& f,
       mma_bf16(S[nt], aq[ks][0], 0u, aq[ks][1], 0u, b0, b1);
     }
   }
-  // Lanes 0..3 hold s1 (row 0) and lanes 4..7 s2 (row 1) of keys 4t..4t+3.
-  float own[4] = {S[0][0], S[0][1], S[1][0], S[1][1]};
-  float oth[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) oth[e] = __shfl_xor_sync(0xffffffffu, own[e], 4);
+  // Lane t holds s1 (row 0) and lane 4+t holds s2 (row 1) of keys 4t..4t+3;
+  // every lane fetches both for its own t.
   float s1[4], s2[4];
   float mloc = -CUDART_INF_F;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
+    float own = (e < 2) ? S[0][e] : S[1][e - 2];
+    float a = __shfl_sync(0xffffffffu, own, t);
+    s2[e] = __shfl_sync(0xffffffffu, own, 4 + t);
     bool valid = j0 + 4 * t + e < kend;
-    float a = (g == 0) ? own[e] : oth[e];
-    s2[e] = (g == 0) ? oth[e] : own[e];
     s1[e] = valid ? a * c_log2 : -CUDART_INF_F;
     mloc = fmaxf(mloc, s1[e]);
   }
   mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-  mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-  const float mblk = __shfl_sync(0xffffffffu, mloc, 0);
+  const float mblk = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));  // same in every lane
   if (mblk > s.m + kLazyTau) {  // warp-uniform; also taken on the first block (m = -inf)
     const float alpha = exp2f(s.m - mblk);
 #pragma unroll
@@ -165,14 +163,22 @@ __device__ __forceinline__ void compute_block(WarpState<D>& s, const Frag<D>& f,
     s.omega += (w[0] + w[1]) + (w[2] + w[3]);
     s.T += (w[0] * s2[0] + w[1] * s2[1]) + (w[2] * s2[2] + w[3] * s2[3]);
   }
-  // ---- [O1 O2] += V^T x [w ; w t]: B columns 0/1 come from lanes with g = 0/1.
+  // ---- [O1 O2] += V^T x [w_hi, w_lo, wt_hi, wt_lo]: column n comes from lanes
+  // with g = n.  Each weight travels as a bf16 pair hi + lo (lo = the bf16 of
+  // the remainder), so the products carry ~16 mantissa bits: the combine
+  // (1 + tbar) O1 - O2 cancels by up to |t| on queries with few keys, and a
+  // single bf16 rounding of w t would show through it.
   uint32_t b0 = 0u, b1 = 0u;
-  if (g == 0) {
-    b0 = pack_bf16(w[0], w[1]);
-    b1 = pack_bf16(w[2], w[3]);
-  } else if (g == 1) {
-    b0 = pack_bf16(w[0] * s2[0], w[1] * s2[1]);
-    b1 = pack_bf16(w[2] * s2[2], w[3] * s2[3]);
+  if (g < 4) {
+    float x[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float v = (g < 2) ? w[e] : w[e] * s2[e];
+      if (g & 1) v -= __bfloat162float(__float2bfloat16_rn(v));
+      x[e] = v;
+    }
+    b0 = pack_bf16(x[0], x[1]);
+    b1 = pack_bf16(x[2], x[3]);
   }
 #pragma unroll
   for (int mt = 0; mt < WarpState<D>::MT; ++mt) {
@@ -290,13 +296,12 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
       sm.omega[warp] = s.omega;
       sm.T[warp] = s.T;
     }
-    if (t == 0) {
+    if (t < 2) {  // lane t = 0 holds columns 0, 1 (O1 hi + lo); t = 1 holds 2, 3 (O2)
+      float* dst = (t == 0) ? sm.O1[warp] : sm.O2[warp];
 #pragma unroll
       for (int mt = 0; mt < WarpState<D>::MT; ++mt) {
-        sm.O1[warp][dim_row<D>(g, mt, 0)] = s.O[mt][0];
-        sm.O2[warp][dim_row<D>(g, mt, 0)] = s.O[mt][1];
-        sm.O1[warp][dim_row<D>(g, mt, 1)] = s.O[mt][2];
-        sm.O2[warp][dim_row<D>(g, mt, 1)] = s.O[mt][3];
+        dst[dim_row<D>(g, mt, 0)] = s.O[mt][0] + s.O[mt][1];
+        dst[dim_row<D>(g, mt, 1)] = s.O[mt][2] + s.O[mt][3];
       }
     }
     __syncthreads();

@@ -20,8 +20,10 @@ struct DeviceCache {
   bool init = false;
   int num_sms = 0;
   int* status = nullptr;  // device address of g_status on this device
-  void* decode_ws = nullptr;
+  void* decode_ws = nullptr;  // partial records (library-owned workspace)
   size_t decode_ws_bytes = 0;
+  void* counters = nullptr;   // arrival counters, one per (b, h); zero between calls
+  size_t counters_bytes = 0;
   void* layer_ws = nullptr;
   size_t layer_ws_bytes = 0;
   cublasHandle_t cublas = nullptr;
@@ -74,16 +76,11 @@ int grow(void** ptr, size_t* bytes, size_t need, cudaStream_t st) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk,
-                        size_t* partial_off) {
+// Bytes of partial records a split decode needs (0 when keys are not split).
+size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk) {
   decode_split_plan(B, H, L, num_sms, splits, chunk);
-  if (*splits <= 1) {
-    *partial_off = 0;
-    return 0;
-  }
-  size_t counters = round_up(sizeof(int) * (size_t)B * H, 256);
-  *partial_off = counters;
-  return counters + sizeof(float) * (size_t)B * H * (size_t)(*splits) * (size_t)(2 * d + 4);
+  if (*splits <= 1) return 0;
+  return sizeof(float) * (size_t)B * H * (size_t)(*splits) * (size_t)(2 * d + 4);
 }
 
 int num_sms_or_default() {
@@ -154,8 +151,7 @@ int plx_decode_num_splits(int B, int H, int L, int d) {
 size_t plx_decode_workspace_bytes(int B, int H, int L, int d) {
   if (B < 1 || H < 1 || L < 1 || d < 1) return 0;
   int splits = 1, chunk = 0;
-  size_t off = 0;
-  return decode_ws_layout(B, H, L, d, num_sms_or_default(), &splits, &chunk, &off);
+  return decode_ws_layout(B, H, L, d, num_sms_or_default(), &splits, &chunk);
 }
 
 int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
@@ -188,21 +184,22 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
   if (dtype == PLX_F32) {
     return launch_decode_simt(a, false, st) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
   }
-  size_t off = 0;
-  size_t need = decode_ws_layout(B, H, L, d, dc->num_sms, &a.splits, &a.chunk, &off);
+  size_t need = decode_ws_layout(B, H, L, d, dc->num_sms, &a.splits, &a.chunk);
   if (need > 0) {
-    char* ws = nullptr;
+    if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLX_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    // The counters live apart from the partial records so that no call's
+    // records can ever land where a later call (other B*H) keeps counters.
+    if ((rc = grow(&dc->counters, &dc->counters_bytes, sizeof(int) * (size_t)B * H, st)) != PLX_OK)
+      return rc;
+    a.counters = static_cast<int*>(dc->counters);
     if (workspace) {
-      if (workspace_bytes < need) return PLX_ERR_WORKSPACE;
-      if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PLX_ERR_MISALIGNED;
-      ws = static_cast<char*>(workspace);
+      a.partials = static_cast<float*>(workspace);
     } else {
-      std::lock_guard<std::mutex> lk(g_mu);
       if ((rc = grow(&dc->decode_ws, &dc->decode_ws_bytes, need, st)) != PLX_OK) return rc;
-      ws = static_cast<char*>(dc->decode_ws);
+      a.partials = static_cast<float*>(dc->decode_ws);
     }
-    a.counters = reinterpret_cast<int*>(ws);
-    a.partials = reinterpret_cast<float*>(ws + off);
   }
   return launch_decode_bf16(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
