@@ -191,7 +191,7 @@ def run_gpu(args, rank, world, dist):
     seed = 1002 + 1000 * rank
 
     # ---- Decode (headline).
-    B, H, L, d = DECODE["B"], DECODE["H"], DECODE["L"], DECODE["d"]
+    B, H, L, d = args.decode_batch, DECODE["H"], DECODE["L"], DECODE["d"]
     specs = synth.decode_specs(B, H, L, d)
     t = {}
     for name, spec in specs.items():
@@ -257,7 +257,7 @@ def run_gpu(args, rank, world, dist):
     # ---- Prefill.
     prefill = None
     if not args.no_prefill:
-        pB, pH, pN, pd = PREFILL["B"], PREFILL["H"], PREFILL["N"], PREFILL["d"]
+        pB, pH, pN, pd = args.prefill_batch, PREFILL["H"], PREFILL["N"], PREFILL["d"]
         pspecs = synth.prefill_specs(pB, pH, pN, pd)
         pt = {}
         for name, spec in pspecs.items():
@@ -280,7 +280,7 @@ def run_gpu(args, rank, world, dist):
             "metric": "causal prefill TFLOP/s", "unit": "TFLOP/s",
             "value": round(sum_over_ranks(flops * psteps, dist) / (p_total * 1e-3) / 1e12, 2),
             "ms_per_step": round(p_total / psteps, 3), "steps": psteps,
-            "config": {"workload": "causal prefill B=8 H=16 N=4096 d=128 bf16",
+            "config": {"workload": f"causal prefill B={pB} H=16 N=4096 d=128 bf16",
                        "l2": "inputs 512 MB, larger than L2"},
             "roofline": {"bound": "tensor", "achieved": round(p_ach, 1), "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(p_ach / peaks["bf16_tflops"], 4),
@@ -448,6 +448,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
+    ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
+                    help="decode batch (smaller values for profiler captures only)")
+    ap.add_argument("--prefill-batch", type=int, default=PREFILL["B"],
+                    help="prefill batch (smaller values for profiler captures only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -455,10 +459,11 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    cfg = {"workload": "decode B=64 H=16 L=4096 d=128 bf16, all seqlens 4096",
-           "global_batch": DECODE["B"] * world, "seq_len": DECODE["L"],
+    cfg = {"workload": f"decode B={args.decode_batch} H=16 L=4096 d=128 bf16, all seqlens 4096",
+           "global_batch": args.decode_batch * world, "seq_len": DECODE["L"],
            "parallelism": f"replicas{world}" if world > 1 else "single",
-           "l2": "inputs larger than L2 (2.15 GB KV per GPU); no flush"}
+           "l2": f"inputs larger than L2 ({args.decode_batch * 16 * 4096 * 128 * 4 / 1e9:.2f} GB KV "
+                 "per GPU); no flush"}
 
     if args.impl == "reference":
         if rank != 0:
