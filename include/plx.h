@@ -112,6 +112,30 @@ size_t plx_decode_workspace_bytes(int B, int H, int L, int d);
 int plx_decode_num_splits(int B, int H, int L, int d);
 
 /*
+ * plx_decode_noalloc — one bf16 decode step that allocates nothing.
+ * (The paper has no counterpart: this is a deployment variant of plx_decode_ex.)
+ *
+ * For callers that cannot allocate device memory where they decode: a runtime
+ * that reserves all device memory up front and passes kernels only buffers it
+ * owns, or a latency-critical loop that must not risk the device-wide
+ * synchronisation a cudaMalloc or cudaFree can cause.  Same arguments and
+ * result as plx_decode_ex with dtype PLX_BF16, d in {64, 128}; the caller still
+ * passes every input and output.  The split-KV scratch (arrival counters and
+ * partial records) is a fixed 8 MiB array compiled into the library, which every
+ * GPU that loads the library holds until the process exits.  Limits: when the
+ * keys are split, B*H <= 32768 and B*H*splits*(2d+4)*4 bytes <= 8 MiB - 128 KiB
+ * (splits = plx_decode_num_splits); larger sizes return PLX_ERR_WORKSPACE before
+ * anything is launched.  No cudaMalloc, cudaFree or allocating library routine is
+ * called.  The first call on a device looks up the array's device address (make
+ * that first call before any stream capture); every call clears the counters with
+ * an asynchronous memset on `stream`.  All calls share the one array, so calls
+ * that overlap on the GPU (other streams, other threads) race: order them.
+ */
+int plx_decode_noalloc(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                       const int32_t* seqlens, void* out, int B, int H, int L, int d,
+                       void* stream);
+
+/*
  * Per-head RMSNorm (unit weight, eps) followed by rotate-half RoPE (frequencies
  * base^(-2k/d), position = token index) of a projected activation, with the
  * head split folded in: x is bf16 [B, N, H*d] (token-major, as a GEMM writes it),

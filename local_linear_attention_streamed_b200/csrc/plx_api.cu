@@ -90,6 +90,12 @@ int num_sms_or_default() {
 }
 
 }  // namespace
+
+int* status_word_address() {
+  DeviceCache* c = nullptr;
+  return current_device(&c) == PLX_OK ? c->status : nullptr;
+}
+
 }  // namespace plx
 
 using namespace plx;

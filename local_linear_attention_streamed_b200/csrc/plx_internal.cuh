@@ -66,3 +66,8 @@ cudaError_t launch_swap_axes(const void* src, void* dst, int B, int A1, int A2, 
                              cudaStream_t st);
 
 }  // namespace plx
+
+namespace plx {
+// Device address of this device's kernel status word (nullptr if CUDA fails).
+int* status_word_address();
+}  // namespace plx

@@ -27,6 +27,7 @@ SIGNATURES = {
     "plx_decode_ex": (_i, [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_decode_workspace_bytes": (_sz, [_i] * 4),
     "plx_decode_num_splits": (_i, [_i] * 4),
+    "plx_decode_noalloc": (_i, [_vp] * 6 + [_i] * 4 + [_vp]),
     "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
     "plx_layer_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
@@ -122,6 +123,23 @@ def decode(q, r, Kcache, Vcache, seqlens, out=None, workspace=None, stream=None)
                            _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, L, d, _dtype_code(q),
                            ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(rc, "plx_decode_ex")
+    return out
+
+
+def decode_noalloc(q, r, Kcache, Vcache, seqlens, out=None, stream=None):
+    """As decode() for bf16, through plx_decode_noalloc: no device memory is allocated
+    (the library's fixed scratch array is used)."""
+    B, H, L, d = Kcache.shape
+    if q.shape != (B, H, d) or r.shape != (B, H, d) or Vcache.shape != Kcache.shape:
+        raise ValueError("shape mismatch")
+    if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
+        raise ValueError("seqlens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    rc = lib.plx_decode_noalloc(_dev(q, "q"), _dev(r, "r"), _dev(Kcache, "Kcache"),
+                                _dev(Vcache, "Vcache"), _dev(seqlens, "seqlens"), _dev(out, "out"),
+                                B, H, L, d, _stream_ptr(stream))
+    _check(rc, "plx_decode_noalloc")
     return out
 
 
