@@ -1,19 +1,580 @@
-// bf16 Parallax prefill on tcgen05 tensor cores (TMA-staged tiles, TMEM
-// accumulators).  Not built yet: bf16 prefill runs on the SIMT kernel.
+// Causal (or full) Parallax prefill for bf16, d = 128, on sm_100a tensor cores.
+//
+// Per CTA, one 128-query tile at a time (persistent over (b, h, tile), longest
+// causal tiles first).  Warp roles:
+//   warp 0      TMA producer: Q and R tiles, then a ring of 64-key K and V tiles
+//               (128B-swizzled boxes, one mbarrier per stage and direction).
+//   warp 1      TMEM owner and MMA issuer (one elected thread):
+//                 S1 = Q K^T and S2 = R K^T from ONE K tile into TMEM
+//                 (rainbus.top summary, "方法步骤详情": S1 and S2 per KV block
+//                 from one shared instruction stream), double-buffered so that
+//                 the next block's scores overlap this block's softmax;
+//                 O1 += P V and O2 += (w t) V with P and w t read from TMEM and
+//                 V from shared memory ("accumulate O1 and O2 in parallel").
+//   warps 2..5  softmax warpgroup, thread = query row (= TMEM lane): one running
+//               max and one rescale factor shared by both branches (agihunt.info
+//               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
+//               P = bf16(w) and w t as bf16 written back over the scores, and
+//               the epilogue out = ((1 + T/omega) O1 - O2) / omega.
+// TMEM (512 columns): S1/S2 of stage s at 128s and 128s+64 (64 fp32 columns
+// each); O1 at 256 and O2 at 384 (128 fp32 columns each).  P(s) overwrites
+// S1(s) columns 0..31 (bf16 pairs), (w t)_hi overwrites S2(s) columns 0..31, and
+// on the first query tile (whose rows see few keys) (w t)_lo = bf16 of the
+// remainder overwrites S1(s) columns 32..63 and feeds a third value MMA, so that
+// (1 + tbar) O1 - O2, which cancels by up to |t| there, keeps ~16 mantissa bits.
+//
+// The running max is raised only when a block's max exceeds it by more than
+// 2^8 (exact: omega, T, O1 and O2 always share one scale); a raise on a later
+// block rescales that row of O1 and O2 in TMEM after the previous value MMAs
+// completed.  Every wait is bounded in time; a wait that runs out sets the
+// device status word, stops the CTA's loops and frees its TMEM.
 #include "plx_internal.cuh"
 
-namespace plx {
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
-bool prefill_tc_supported(int d) {
-  (void)d;
-  return false;
+#include <math_constants.h>
+
+namespace plx {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kBM = 128;                 // queries per tile
+constexpr int kBN = 64;                  // keys per block
+constexpr int kStages = 4;               // K/V ring depth
+constexpr int kThreads = 192;            // 6 warps
+constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
+constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
+constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
+constexpr uint32_t kHalfKV = kBN * 128;      // one 64-dim half of a K/V block
+constexpr float kLazyTau = 8.f;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on every wait
+
+// TMEM column map.
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColStage = 128, kColO1 = 256, kColO2 = 384;
+
+// Instruction descriptors (kind::f16): D f32 (bits 4-5 = 1), A and B bf16
+// (bits 7-9, 10-12 = 1), A K-major, B K-major (S) or MN-major (bit 16, PV),
+// N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((kD >> 3) << 17) |
+                              ((kBM >> 4) << 24);
+
+struct Smem {
+  // Tiles first (1024-byte aligned for the 128B swizzle).
+  uint8_t q[kQBytes];
+  uint8_t r[kQBytes];
+  uint8_t k[kStages][kKVBytes];
+  uint8_t v[kStages][kKVBytes];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
+  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t o_full, o_empty, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+__device__ __forceinline__ unsigned long long now_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `parity` to complete.  Returns false (and
+// raises the CTA's abort flag and the device timeout status) if it ran out,
+// or false at once if another role already aborted.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                       int* status) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = now_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_test(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (now_ns() - t0 > kWaitNs) {
+        *abort = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used only on the way out (ignores the abort flag).
+__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = now_ns();
+  while (!mbar_test(bar, parity) && now_ns() - t0 < kWaitNs) {
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128B swizzle, sm100 version bits.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // version
+  d |= (uint64_t)2 << 61;  // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
+        "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
+        "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]),
+      "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]),
+      "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]),
+      "r"(v[30]), "r"(v[31]));
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+struct TileInfo {
+  int bh, m, nblk, lo;
+};
+
+__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal) {
+  const int ntile = (N + kBM - 1) / kBM;
+  TileInfo ti;
+  ti.m = ntile - 1 - t / BH;  // longest causal rows first
+  ti.bh = t % BH;
+  const int kmax = causal ? min(N, (ti.m + 1) * kBM) : N;
+  ti.nblk = (kmax + kBN - 1) / kBN;
+  ti.lo = (ti.m == 0);
+  return ti;
+}
+
+struct Params {
+  int B, H, N, causal;
+  __nv_bfloat16* out;
+  int* status;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
+                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = p.B * p.H;
+  const int ntile = (p.N + kBM - 1) / kBM;
+  const int tiles = ntile * BH;
+  volatile int* abort = &sm.abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.pv_done[s], 1);
+    }
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.o_empty, 128);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t kv = 0;
+      int tc = 0;
+      long long k_issued[kStages], v_issued[kStages], q_issued = -1;  // last use index per stage
+      for (int s = 0; s < kStages; ++s) k_issued[s] = v_issued[s] = -1;
+      for (int t = blockIdx.x; t < tiles && !*abort; t += gridDim.x, ++tc) {
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+        const int row0 = ti.bh * p.N;
+        if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
+        mbar_expect_tx(&sm.q_full, 2 * kQBytes);
+        q_issued = tc;
+        for (int h = 0; h < 2; ++h) {
+          tma_load_2d(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+          tma_load_2d(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+        }
+        for (int j = 0; j < ti.nblk; ++j, ++kv) {
+          const int st = kv % kStages;
+          const uint32_t par = ((kv / kStages) & 1) ^ 1;
+          if (!mbar_wait(&sm.k_empty[st], par, abort, p.status)) break;
+          mbar_expect_tx(&sm.k_full[st], kKVBytes);
+          k_issued[st] = kv / kStages;
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.k_full[st], 64 * h, row0 + j * kBN);
+          if (!mbar_wait(&sm.v_empty[st], par, abort, p.status)) break;
+          mbar_expect_tx(&sm.v_full[st], kKVBytes);
+          v_issued[st] = kv / kStages;
+          for (int h = 0; h < 2; ++h)
+            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.v_full[st], 64 * h, row0 + j * kBN);
+        }
+      }
+      // After an abort, let every copy this thread issued land before the CTA
+      // exits (each wait is bounded; consumed stages pass at once).
+      if (*abort) {
+        if (q_issued >= 0) mbar_drain(&sm.q_full, (uint32_t)(q_issued & 1));
+        for (int s = 0; s < kStages; ++s) {
+          if (k_issued[s] >= 0) mbar_drain(&sm.k_full[s], (uint32_t)(k_issued[s] & 1));
+          if (v_issued[s] >= 0) mbar_drain(&sm.v_full[s], (uint32_t)(v_issued[s] & 1));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t kvS = 0, kvV = 0;  // K/V ring positions consumed by S and by PV
+      uint32_t g = 0;             // blocks processed by this CTA (S/P stage counter)
+      int tc = 0;
+      const uint32_t qa = smem_u32(sm.q), ra = smem_u32(sm.r);
+      bool ok = true;
+      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+        if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
+        tc_fence_after();
+        auto issue_S = [&](uint32_t gs, uint32_t kvi) -> bool {
+          const int st = kvi % kStages;
+          if (!mbar_wait(&sm.k_full[st], (kvi / kStages) & 1, abort, p.status)) return false;
+          tc_fence_after();
+          const uint32_t d1 = tmem + (gs & 1) * kColStage + kColS1;
+          const uint32_t d2 = tmem + (gs & 1) * kColStage + kColS2;
+          const uint32_t ka = smem_u32(sm.k[st]);
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
+            const uint32_t koff = (ks >> 2) * kHalfKV + (ks & 3) * 32;
+            const uint64_t bk = sdesc(ka + koff, 16, 1024);
+            mma_ss(d1, sdesc(qa + off, 16, 1024), bk, kIdescS, ks > 0);
+            mma_ss(d2, sdesc(ra + off, 16, 1024), bk, kIdescS, ks > 0);
+          }
+          mma_commit(&sm.s_full[gs & 1]);
+          mma_commit(&sm.k_empty[st]);
+          return true;
+        };
+        const uint32_t g0 = g;
+        if (!(ok = issue_S(g0, kvS++))) break;
+        if (ti.nblk > 1 && !(ok = issue_S(g0 + 1, kvS++))) break;
+        if (ti.nblk <= 2) mma_commit(&sm.q_empty);
+        // The epilogue of the previous tile must have read O before it is overwritten.
+        if (tc > 0 && !(ok = mbar_wait(&sm.o_empty, (tc - 1) & 1, abort, p.status))) break;
+        for (int j = 0; j < ti.nblk; ++j, ++g, ++kvV) {
+          const uint32_t s = g & 1;
+          if (!(ok = mbar_wait(&sm.p_full[s], (g >> 1) & 1, abort, p.status))) break;
+          const int st = kvV % kStages;
+          if (!(ok = mbar_wait(&sm.v_full[st], (kvV / kStages) & 1, abort, p.status))) break;
+          tc_fence_after();
+          const uint32_t va = smem_u32(sm.v[st]);
+          const uint32_t sbase = tmem + s * kColStage;
+#pragma unroll
+          for (int ks = 0; ks < kBN / 16; ++ks) {
+            const uint64_t bv = sdesc(va + ks * 2048, kHalfKV, 1024);
+            const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
+            mma_ts(tmem + kColO1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
+            mma_ts(tmem + kColO2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
+            if (ti.lo) mma_ts(tmem + kColO2, sbase + kColS1 + 32 + ks * 8, bv, kIdescPV, 1u);
+          }
+          mma_commit(&sm.pv_done[s]);
+          mma_commit(&sm.v_empty[st]);
+          if (j + 2 < ti.nblk) {
+            if (!(ok = issue_S(g + 2, kvS++))) break;
+            if (j + 3 == ti.nblk) mma_commit(&sm.q_empty);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&sm.o_full);
+      }
+      // Drain: all MMAs this thread issued complete before TMEM is freed.
+      mma_commit(&sm.drain);
+      mbar_drain(&sm.drain, 0);
+    }
+  } else {
+    // ---------------- softmax / epilogue warpgroup ----------------
+    const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
+    const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+    const float scale = 1.4426950408889634f * rsqrtf((float)kD);
+    uint32_t g = 0;
+    int tc = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
+      const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+      const int i = ti.m * kBM + row;  // query position
+      float m_run = -CUDART_INF_F, omega = 0.f, T = 0.f;
+      for (int j = 0; j < ti.nblk; ++j, ++g) {
+        const uint32_t s = g & 1;
+        if (!(ok = mbar_wait(&sm.s_full[s], (g >> 1) & 1, abort, p.status))) break;
+        tc_fence_after();
+        const uint32_t base = tmem + lane_addr + s * kColStage;
+        uint32_t x[64];
+        tmem_ld32(base + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+        tmem_ld32(base + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+        tc_wait_ld();
+        const int k0 = j * kBN;
+        const bool edge = (p.causal && k0 + kBN - 1 > ti.m * kBM) || (k0 + kBN > p.N);
+        const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          float v = __uint_as_float(x[c]) * scale;
+          if (edge && k0 + c >= kend) v = -CUDART_INF_F;
+          x[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+        float alpha = 1.f;
+        if (mx > m_run + kLazyTau) {
+          alpha = ex2(m_run - mx);  // 0 on the first block (m_run = -inf)
+          m_run = mx;
+          omega *= alpha;
+          T *= alpha;
+        }
+        // Rows whose max rose rescale their part of O1 and O2 once the value
+        // MMAs of the previous block are complete (rare after the first block).
+        const bool need = (j > 0) && (alpha != 1.f);
+        if (__any_sync(0xffffffffu, need)) {
+          const uint32_t gp = g - 1;  // previous block of this tile
+          if (!(ok = mbar_wait(&sm.pv_done[gp & 1], (gp >> 1) & 1, abort, p.status))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c0 = 0; c0 < 256; c0 += 32) {
+            uint32_t o[32];
+            const uint32_t oa = tmem + lane_addr + kColO1 + c0;
+            tmem_ld32(oa, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(oa, o);
+          }
+          tc_wait_st();
+        }
+        float wsum = 0.f, tsum = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t y[32], P[16], PT[16], PL[16];
+          tmem_ld32(base + kColS2 + 32 * hf, y);
+          tc_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float w0 = ex2(__uint_as_float(x[32 * hf + 2 * c]) - m_run);
+            const float w1 = ex2(__uint_as_float(x[32 * hf + 2 * c + 1]) - m_run);
+            const float a0 = w0 * __uint_as_float(y[2 * c]), a1 = w1 * __uint_as_float(y[2 * c + 1]);
+            wsum += w0 + w1;
+            tsum += a0 + a1;
+            P[c] = pack_bf16(w0, w1);
+            const uint32_t hi = pack_bf16(a0, a1);
+            PT[c] = hi;
+            PL[c] = pack_bf16(a0 - __uint_as_float(hi << 16), a1 - __uint_as_float(hi & 0xFFFF0000u));
+          }
+          // S2 columns 32*hf.. are read above before (w t)_hi overwrites S2 columns 16*hf..
+          tmem_st16(base + kColS1 + 16 * hf, P);
+          tmem_st16(base + kColS2 + 16 * hf, PT);
+          if (ti.lo) tmem_st16(base + kColS1 + 32 + 16 * hf, PL);
+        }
+        omega += wsum;
+        T += tsum;
+        tc_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sm.p_full[s]);
+      }
+      if (!ok) break;
+      // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega for this row.
+      if (!(ok = mbar_wait(&sm.o_full, tc & 1, abort, p.status))) break;
+      tc_fence_after();
+      const float inv = 1.f / omega;
+      const float c1 = (1.f + T * inv) * inv;
+      __nv_bfloat16* orow = p.out + ((long long)ti.bh * p.N + i) * kD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kD; c0 += 32) {
+        uint32_t o1[32], o2[32];
+        tmem_ld32(tmem + lane_addr + kColO1 + c0, o1);
+        tmem_ld32(tmem + lane_addr + kColO2 + c0, o2);
+        tc_wait_ld();
+        if (i < p.N) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float v0 = c1 * __uint_as_float(o1[2 * c]) - inv * __uint_as_float(o2[2 * c]);
+            const float v1 = c1 * __uint_as_float(o1[2 * c + 1]) - inv * __uint_as_float(o2[2 * c + 1]);
+            packed[c] = pack_bf16(v0, v1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.o_empty);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D view [rows, 128] of a bf16 [B, H, N, 128] tensor, boxes of 64 dims x box_rows rows.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int d) { return d == kD; }
+
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms) {
-  (void)a;
-  (void)st;
-  (void)num_sms;
-  return cudaErrorNotSupported;
+  const long long rows = (long long)a.B * a.H * a.N;
+  if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
+  CUtensorMap mQ, mR, mK, mV;
+  if (!make_map(&mQ, a.Q, rows, kBM) || !make_map(&mR, a.R, rows, kBM) || !make_map(&mK, a.K, rows, kBN) ||
+      !make_map(&mV, a.V, rows, kBN))
+    return cudaErrorInvalidValue;
+  Params p{a.B, a.H, a.N, a.causal, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
+  const size_t smem = sizeof(Smem) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long tiles = (long long)((a.N + kBM - 1) / kBM) * a.B * a.H;
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  prefill_tc_kernel<<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
+  return cudaGetLastError();
 }
 
 }  // namespace plx

@@ -95,6 +95,22 @@ def test_bf16_prefill_r_zero(plx):
     assert rel_err_rms(got, want) <= BF16_TOL
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_bf16_prefill_rescale_path(plx, causal):
+    """Keys from position 200 on are scaled by 8, so the running max of later
+    rows jumps by far more than 2^8 after their first blocks: the kernels must
+    rescale the partial O1, O2, omega and T exactly."""
+    B, H, N, d = 1, 2, 520, 128
+    specs = synth.prefill_specs(B, H, N, d)
+    dev, ref = small_inputs(13, specs, synth.BF16)
+    dev["K"][:, :, 200:] *= 8
+    ref["K"] = dev["K"].double().cpu().numpy()
+    out = plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=causal)
+    assert plx.get_device_status() == 0
+    want = oracle.prefill_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal=causal)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
 def _sampled_prefill(plx, seed, B, H, N, d, rows):
     specs = synth.prefill_specs(B, H, N, d)
     dev = device_inputs(seed, specs, synth.BF16)
