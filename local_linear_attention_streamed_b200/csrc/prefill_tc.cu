@@ -14,20 +14,28 @@
 //   warps 2..5  softmax warpgroup, thread = query row (= TMEM lane): one running
 //               max and one rescale factor shared by both branches (agihunt.info
 //               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
-//               P = bf16(w) and w t as bf16 written back over the scores, and
+//               P = bf16(w) and bf16(w (t - c)) written back over the scores, and
 //               the epilogue out = ((1 + T/omega) O1 - O2) / omega.
 // TMEM (512 columns): S1/S2 of stage s at 128s and 128s+64 (64 fp32 columns
-// each); O1 at 256 and O2 at 384 (128 fp32 columns each).  P(s) overwrites
-// S1(s) columns 0..31 (bf16 pairs), (w t)_hi overwrites S2(s) columns 0..31, and
-// on the first query tile (whose rows see few keys) (w t)_lo = bf16 of the
-// remainder overwrites S1(s) columns 32..63 and feeds a third value MMA, so that
-// (1 + tbar) O1 - O2, which cancels by up to |t| there, keeps ~16 mantissa bits.
+// each); O1 at 256 and O2 at 384 (128 fp32 columns each).  P(s) = bf16(w)
+// overwrites S1(s) columns 0..31 (bf16 pairs) and bf16(w (t - c)) overwrites
+// S2(s) columns 0..31.
+//
+// Centring.  The output is unchanged when every t_ij of a query is shifted by
+// the same c_i (the pages' key-query difference z_ij = k_j - q_i is one such
+// shift: rho_i . q_i).  The kernel keeps c_i at the running softmax mean of t,
+// so that O2 = sum w (t - c) v and the combine ((1 + T/omega) O1 - O2)/omega
+// stay well conditioned when one key dominates a row and |t| is large; with
+// c = 0 a single bf16 rounding of w t there is amplified by |t| (tens, in
+// trained models and in the rescale test).  c is set from the first block and
+// moved (O2 -= delta O1 in TMEM) only when the running mean drifts by more than
+// kTheta, always before the block's w (t - c) is rounded.
 //
 // The running max is raised only when a block's max exceeds it by more than
-// 2^8 (exact: omega, T, O1 and O2 always share one scale); a raise on a later
-// block rescales that row of O1 and O2 in TMEM after the previous value MMAs
-// completed.  Every wait is bounded in time; a wait that runs out sets the
-// device status word, stops the CTA's loops and frees its TMEM.
+// 2^8 (exact: omega, T, O1 and O2 always share one scale); a raise or a centre
+// move on a later block updates that row of O1 and O2 in TMEM after the
+// previous value MMAs completed.  Every wait is bounded in time; a wait that
+// runs out sets the device status word, stops the CTA's loops and frees its TMEM.
 #include "plx_internal.cuh"
 
 #include <cuda.h>
@@ -48,6 +56,7 @@ constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
 constexpr uint32_t kHalfKV = kBN * 128;      // one 64-dim half of a K/V block
 constexpr float kLazyTau = 8.f;
+constexpr float kTheta = 1.f;  // re-centre t once its running mean drifts this far
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on every wait
 
 // TMEM column map.
@@ -231,7 +240,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 struct TileInfo {
-  int bh, m, nblk, lo;
+  int bh, m, nblk;
 };
 
 __device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal) {
@@ -241,7 +250,6 @@ __device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal) 
   ti.bh = t % BH;
   const int kmax = causal ? min(N, (ti.m + 1) * kBM) : N;
   ti.nblk = (kmax + kBN - 1) / kBN;
-  ti.lo = (ti.m == 0);
   return ti;
 }
 
@@ -387,7 +395,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
             mma_ts(tmem + kColO1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
             mma_ts(tmem + kColO2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
-            if (ti.lo) mma_ts(tmem + kColO2, sbase + kColS1 + 32 + ks * 8, bv, kIdescPV, 1u);
           }
           mma_commit(&sm.pv_done[s]);
           mma_commit(&sm.v_empty[st]);
@@ -414,15 +421,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
       const TileInfo ti = tile_info(t, BH, p.N, p.causal);
       const int i = ti.m * kBM + row;  // query position
-      float m_run = -CUDART_INF_F, omega = 0.f, T = 0.f;
+      // Row state: running max (log2 units), omega = sum w, T = sum w (t - c)
+      // around the row's centre c (see the file comment), all in fp32.
+      float m_run = -CUDART_INF_F, omega = 0.f, T = 0.f, cen = 0.f;
       for (int j = 0; j < ti.nblk; ++j, ++g) {
         const uint32_t s = g & 1;
         if (!(ok = mbar_wait(&sm.s_full[s], (g >> 1) & 1, abort, p.status))) break;
         tc_fence_after();
         const uint32_t base = tmem + lane_addr + s * kColStage;
-        uint32_t x[64];
+        uint32_t x[64], y[64];
         tmem_ld32(base + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(base + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+        tmem_ld32(base + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
+        tmem_ld32(base + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
         tc_wait_ld();
         const int k0 = j * kBN;
         const bool edge = (p.causal && k0 + kBN - 1 > ti.m * kBM) || (k0 + kBN > p.N);
@@ -442,50 +453,64 @@ __global__ void __launch_bounds__(kThreads, 1)
           omega *= alpha;
           T *= alpha;
         }
-        // Rows whose max rose rescale their part of O1 and O2 once the value
-        // MMAs of the previous block are complete (rare after the first block).
-        const bool need = (j > 0) && (alpha != 1.f);
+        float wsum = 0.f, wtsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const float w = ex2(__uint_as_float(x[c]) - m_run);
+          x[c] = __float_as_uint(w);
+          wsum += w;
+          wtsum = fmaf(w, __uint_as_float(y[c]), wtsum);
+        }
+        // Re-centre before this block's w (t - c) is rounded to bf16, on the
+        // first block and whenever the running mean of t has drifted by more
+        // than kTheta from the centre.
+        float Tb = wtsum - cen * wsum;
+        float delta = 0.f;
+        const float tb_new = (T + Tb) / (omega + wsum);
+        if (j == 0 || fabsf(tb_new) > kTheta) {
+          delta = tb_new;
+          cen += delta;
+          T -= delta * omega;
+          Tb -= delta * wsum;
+        }
+        omega += wsum;
+        T += Tb;
+        // Rows whose max rose or whose centre moved update their part of O1 and
+        // O2 (O1 <- alpha O1, O2 <- alpha (O2 - delta O1)) once the value MMAs
+        // of the previous block are complete.
+        const bool need = (j > 0) && (alpha != 1.f || delta != 0.f);
         if (__any_sync(0xffffffffu, need)) {
           const uint32_t gp = g - 1;  // previous block of this tile
           if (!(ok = mbar_wait(&sm.pv_done[gp & 1], (gp >> 1) & 1, abort, p.status))) break;
           tc_fence_after();
+          const float ad = alpha * delta;
 #pragma unroll 1
-          for (int c0 = 0; c0 < 256; c0 += 32) {
-            uint32_t o[32];
-            const uint32_t oa = tmem + lane_addr + kColO1 + c0;
-            tmem_ld32(oa, o);
+          for (int c0 = 0; c0 < kD; c0 += 32) {
+            uint32_t o1[32], o2[32];
+            const uint32_t a1 = tmem + lane_addr + kColO1 + c0, a2 = tmem + lane_addr + kColO2 + c0;
+            tmem_ld32(a1, o1);
+            tmem_ld32(a2, o2);
             tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(oa, o);
+            for (int c = 0; c < 32; ++c) {
+              const float v1 = __uint_as_float(o1[c]);
+              o2[c] = __float_as_uint(alpha * __uint_as_float(o2[c]) - ad * v1);
+              o1[c] = __float_as_uint(alpha * v1);
+            }
+            tmem_st32(a1, o1);
+            tmem_st32(a2, o2);
           }
           tc_wait_st();
         }
-        float wsum = 0.f, tsum = 0.f;
+        uint32_t P[32], PT[32];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t y[32], P[16], PT[16], PL[16];
-          tmem_ld32(base + kColS2 + 32 * hf, y);
-          tc_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float w0 = ex2(__uint_as_float(x[32 * hf + 2 * c]) - m_run);
-            const float w1 = ex2(__uint_as_float(x[32 * hf + 2 * c + 1]) - m_run);
-            const float a0 = w0 * __uint_as_float(y[2 * c]), a1 = w1 * __uint_as_float(y[2 * c + 1]);
-            wsum += w0 + w1;
-            tsum += a0 + a1;
-            P[c] = pack_bf16(w0, w1);
-            const uint32_t hi = pack_bf16(a0, a1);
-            PT[c] = hi;
-            PL[c] = pack_bf16(a0 - __uint_as_float(hi << 16), a1 - __uint_as_float(hi & 0xFFFF0000u));
-          }
-          // S2 columns 32*hf.. are read above before (w t)_hi overwrites S2 columns 16*hf..
-          tmem_st16(base + kColS1 + 16 * hf, P);
-          tmem_st16(base + kColS2 + 16 * hf, PT);
-          if (ti.lo) tmem_st16(base + kColS1 + 32 + 16 * hf, PL);
+        for (int c = 0; c < 32; ++c) {
+          const float w0 = __uint_as_float(x[2 * c]), w1 = __uint_as_float(x[2 * c + 1]);
+          P[c] = pack_bf16(w0, w1);
+          PT[c] = pack_bf16(w0 * (__uint_as_float(y[2 * c]) - cen), w1 * (__uint_as_float(y[2 * c + 1]) - cen));
         }
-        omega += wsum;
-        T += tsum;
+        tmem_st32(base + kColS1, P);
+        tmem_st32(base + kColS2, PT);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[s]);
