@@ -11,7 +11,8 @@
 //                 the next block's scores overlap this block's softmax;
 //                 O1 += P V and O2 += (w t) V with P and w t read from TMEM and
 //                 V from shared memory ("accumulate O1 and O2 in parallel").
-//   warps 2..5  softmax warpgroup, thread = query row (= TMEM lane): one running
+//   warps 2..9  two softmax warpgroups, each thread = one half (32 keys of every
+//               block, 64 output dims) of one query row (= TMEM lane): one running
 //               max and one rescale factor shared by both branches (agihunt.info
 //               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
 //               P = bf16(w) and bf16(w (t - c)) written back over the scores, and
@@ -50,7 +51,7 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
 constexpr int kStages = 4;               // K/V ring depth
-constexpr int kThreads = 192;            // 6 warps
+constexpr int kThreads = 320;            // 10 warps: TMA, MMA, 2 softmax warpgroups
 constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
 constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
@@ -79,6 +80,8 @@ struct Smem {
   uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, o_empty, drain;
+  uint64_t ex_max, ex_sum;  // row exchanges between the two softmax warpgroups
+  float red_max[2][kBM], red_w[2][kBM], red_t[2][kBM];
   uint32_t tmem_base;
   int abort;
 };
@@ -118,12 +121,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase of `parity` to complete.  Returns false (and
-// raises the CTA's abort flag and the device timeout status) if it ran out,
-// or false at once if another role already aborted.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                       int* status) {
-  if (mbar_test(bar, parity)) return true;
+// Slow path of mbar_wait (kept out of line so that the common, already
+// complete case costs one try_wait and no call).
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            int* status) {
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
@@ -136,6 +137,15 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
       }
     }
   }
+}
+
+// Bounded wait for the phase of `parity` to complete.  Returns false (and
+// raises the CTA's abort flag and the device timeout status) if it ran out,
+// or false at once if another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int* status) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort, status);
 }
 
 // Bounded wait used only on the way out (ignores the abort flag).
@@ -234,6 +244,36 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Packed fp32 pairs (two lanes of one 64-bit register): Blackwell's f32x2 ALU.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void uf2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -282,11 +322,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 128);
+      mbar_init(&sm.p_full[s], 256);
       mbar_init(&sm.pv_done[s], 1);
     }
     mbar_init(&sm.o_full, 1);
-    mbar_init(&sm.o_empty, 128);
+    mbar_init(&sm.o_empty, 256);
+    mbar_init(&sm.ex_max, 256);
+    mbar_init(&sm.ex_sum, 256);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -363,13 +405,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t d1 = tmem + (gs & 1) * kColStage + kColS1;
           const uint32_t d2 = tmem + (gs & 1) * kColStage + kColS2;
           const uint32_t ka = smem_u32(sm.k[st]);
+          // All of S1's k-steps, then all of S2's: alternating the A operand and
+          // the accumulator between MMAs costs the tensor pipe a third of its rate.
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
             const uint32_t koff = (ks >> 2) * kHalfKV + (ks & 3) * 32;
-            const uint64_t bk = sdesc(ka + koff, 16, 1024);
-            mma_ss(d1, sdesc(qa + off, 16, 1024), bk, kIdescS, ks > 0);
-            mma_ss(d2, sdesc(ra + off, 16, 1024), bk, kIdescS, ks > 0);
+            mma_ss(d1, sdesc(qa + off, 16, 1024), sdesc(ka + koff, 16, 1024), kIdescS, ks > 0);
+          }
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
+            const uint32_t koff = (ks >> 2) * kHalfKV + (ks & 3) * 32;
+            mma_ss(d2, sdesc(ra + off, 16, 1024), sdesc(ka + koff, 16, 1024), kIdescS, ks > 0);
           }
           mma_commit(&sm.s_full[gs & 1]);
           mma_commit(&sm.k_empty[st]);
@@ -411,11 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(&sm.drain, 0);
     }
   } else {
-    // ---------------- softmax / epilogue warpgroup ----------------
+    // ---------------- softmax / epilogue: two warpgroups ----------------
+    // Warpgroup hf (warps 2..5 -> 0, 6..9 -> 1) owns keys 32hf..32hf+31 of every
+    // block and output dims 64hf..64hf+63; the two threads of a row exchange
+    // their partial max and sums through shared memory, so both keep identical
+    // copies of the row state (m, omega, T, c).
+    const int hf = (warp - 2) >> 2;
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const float scale = 1.4426950408889634f * rsqrtf((float)kD);
-    uint32_t g = 0;
+    uint32_t g = 0;  // blocks processed by this CTA (also the exchange phase)
     int tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
@@ -429,23 +482,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&sm.s_full[s], (g >> 1) & 1, abort, p.status))) break;
         tc_fence_after();
         const uint32_t base = tmem + lane_addr + s * kColStage;
-        uint32_t x[64], y[64];
-        tmem_ld32(base + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tmem_ld32(base + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tmem_ld32(base + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
-        tmem_ld32(base + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
+        uint32_t x[32], y[32];
+        tmem_ld32(base + kColS1 + 32 * hf, x);
+        tmem_ld32(base + kColS2 + 32 * hf, y);
         tc_wait_ld();
-        const int k0 = j * kBN;
-        const bool edge = (p.causal && k0 + kBN - 1 > ti.m * kBM) || (k0 + kBN > p.N);
-        const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
-        float mx = -CUDART_INF_F;
+        const int k0 = j * kBN + 32 * hf;
+        const bool edge = (p.causal && j * kBN + kBN - 1 > ti.m * kBM) || (j * kBN + kBN > p.N);
+        if (edge) {  // block-uniform: only blocks that cross the diagonal or the end
+          const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          float v = __uint_as_float(x[c]) * scale;
-          if (edge && k0 + c >= kend) v = -CUDART_INF_F;
-          x[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          for (int c = 0; c < 32; ++c)
+            if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
         }
+        float rmax = -CUDART_INF_F;
+#pragma unroll
+        for (int c = 0; c < 32; c += 4)
+          rmax = max3(rmax, max3(__uint_as_float(x[c]), __uint_as_float(x[c + 1]), __uint_as_float(x[c + 2])),
+                      __uint_as_float(x[c + 3]));
+        sm.red_max[hf][row] = rmax;
+        mbar_arrive(&sm.ex_max);
+        if (!(ok = mbar_wait(&sm.ex_max, g & 1, abort, p.status))) break;
+        rmax = fmaxf(rmax, sm.red_max[hf ^ 1][row]);
+        const float mx = rmax * scale;
         float alpha = 1.f;
         if (mx > m_run + kLazyTau) {
           alpha = ex2(m_run - mx);  // 0 on the first block (m_run = -inf)
@@ -453,18 +511,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           omega *= alpha;
           T *= alpha;
         }
-        float wsum = 0.f, wtsum = 0.f;
+        // w = 2^(s*scale - m); P = bf16(w) now; a = w (t - c) kept for (w t)'s
+        // bf16 once the centre is settled.
+        const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
+        uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
+        uint32_t P[16];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float w = ex2(__uint_as_float(x[c]) - m_run);
-          x[c] = __float_as_uint(w);
-          wsum += w;
-          wtsum = fmaf(w, __uint_as_float(y[c]), wtsum);
+        for (int c = 0; c < 16; ++c) {
+          float s0, s1;
+          uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sc2, nm2), s0, s1);
+          const float w0 = ex2(s0), w1 = ex2(s1);
+          const uint64_t w2 = f2(w0, w1);
+          const uint64_t a2 = mul2(w2, add2(f2(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1])), nc2));
+          if (c & 1) {
+            ws2b = add2(ws2b, w2);
+            ts2b = add2(ts2b, a2);
+          } else {
+            ws2a = add2(ws2a, w2);
+            ts2a = add2(ts2a, a2);
+          }
+          P[c] = pack_bf16(w0, w1);
+          float a0, a1;
+          uf2(a2, a0, a1);
+          x[2 * c] = __float_as_uint(w0);
+          x[2 * c + 1] = __float_as_uint(w1);
+          y[2 * c] = __float_as_uint(a0);
+          y[2 * c + 1] = __float_as_uint(a1);
         }
+        tmem_st16(base + kColS1 + 16 * hf, P);
+        float lo, hi;
+        uf2(add2(ws2a, ws2b), lo, hi);
+        const float wpart = lo + hi;
+        uf2(add2(ts2a, ts2b), lo, hi);
+        const float tpart = lo + hi;
+        sm.red_w[hf][row] = wpart;
+        sm.red_t[hf][row] = tpart;
+        mbar_arrive(&sm.ex_sum);
+        if (!(ok = mbar_wait(&sm.ex_sum, g & 1, abort, p.status))) break;
+        // Both threads of the row form the same sums (a + b == b + a exactly).
+        const float wsum = wpart + sm.red_w[hf ^ 1][row];
+        float Tb = tpart + sm.red_t[hf ^ 1][row];
         // Re-centre before this block's w (t - c) is rounded to bf16, on the
         // first block and whenever the running mean of t has drifted by more
         // than kTheta from the centre.
-        float Tb = wtsum - cen * wsum;
         float delta = 0.f;
         const float tb_new = (T + Tb) / (omega + wsum);
         if (j == 0 || fabsf(tb_new) > kTheta) {
@@ -477,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         T += Tb;
         // Rows whose max rose or whose centre moved update their part of O1 and
         // O2 (O1 <- alpha O1, O2 <- alpha (O2 - delta O1)) once the value MMAs
-        // of the previous block are complete.
+        // of the previous block are complete; each warpgroup updates its 64 dims.
         const bool need = (j > 0) && (alpha != 1.f || delta != 0.f);
         if (__any_sync(0xffffffffu, need)) {
           const uint32_t gp = g - 1;  // previous block of this tile
@@ -485,7 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float ad = alpha * delta;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kD; c0 += 32) {
+          for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
             uint32_t o1[32], o2[32];
             const uint32_t a1 = tmem + lane_addr + kColO1 + c0, a2 = tmem + lane_addr + kColO2 + c0;
             tmem_ld32(a1, o1);
@@ -502,28 +591,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_wait_st();
         }
-        uint32_t P[32], PT[32];
+        uint32_t PT[16];
+        if (__any_sync(0xffffffffu, delta != 0.f)) {
+          const uint64_t nd2 = f2(-delta, -delta);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float w0 = __uint_as_float(x[2 * c]), w1 = __uint_as_float(x[2 * c + 1]);
-          P[c] = pack_bf16(w0, w1);
-          PT[c] = pack_bf16(w0 * (__uint_as_float(y[2 * c]) - cen), w1 * (__uint_as_float(y[2 * c + 1]) - cen));
+          for (int c = 0; c < 16; ++c) {
+            float a0, a1;
+            uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), nd2,
+                     f2(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1]))),
+                a0, a1);
+            PT[c] = pack_bf16(a0, a1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) PT[c] = pack_bf16(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1]));
         }
-        tmem_st32(base + kColS1, P);
-        tmem_st32(base + kColS2, PT);
+        tmem_st16(base + kColS2 + 16 * hf, PT);
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[s]);
       }
       if (!ok) break;
-      // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega for this row.
+      // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega, dims 64hf.. of this row.
       if (!(ok = mbar_wait(&sm.o_full, tc & 1, abort, p.status))) break;
       tc_fence_after();
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
       __nv_bfloat16* orow = p.out + ((long long)ti.bh * p.N + i) * kD;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kD; c0 += 32) {
+      for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
         uint32_t o1[32], o2[32];
         tmem_ld32(tmem + lane_addr + kColO1 + c0, o1);
         tmem_ld32(tmem + lane_addr + kColO2 + c0, o2);
