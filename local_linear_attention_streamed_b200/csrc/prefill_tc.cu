@@ -77,11 +77,15 @@ struct Smem {
   uint8_t k[kStages][kKVBytes];
   uint8_t v[kStages][kKVBytes];
   uint64_t q_full, q_empty;
-  uint64_t k_full[kStages], k_empty[kStages], v_full[kStages], v_empty[kStages];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  // One full and one empty barrier per K/V stage: K and V of a block land
+  // together, and the stage frees once that block's value MMAs completed.
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2];
   uint64_t o_full, o_empty, drain;
-  uint64_t ex_max, ex_sum;  // row exchanges between the two softmax warpgroups
-  float red_max[2][kBM], red_w[2][kBM], red_t[2][kBM];
+  // Row exchanges between the two softmax warpgroups: per channel, data slots
+  // double-buffered by epoch parity, and a flag holding the last posted epoch.
+  float xch[2][2][2][kBM][4];  // [channel][epoch & 1][warpgroup][row][value]
+  uint32_t xflag[2][2][kBM];   // [channel][warpgroup][row]
   uint32_t tmem_base;
   int abort;
 };
@@ -146,6 +150,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           int* status) {
   if (mbar_test(bar, parity)) return true;
   return mbar_wait_slow(bar, parity, abort, status);
+}
+
+// Pairwise exchange between the two threads that share a query row: write the
+// values, then publish the epoch with release semantics; read the partner's
+// epoch with acquire semantics (bounded in time), then its values.
+__device__ __forceinline__ void flag_post(uint32_t* flag, uint32_t epoch) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(flag)), "r"(epoch) : "memory");
+}
+__device__ __forceinline__ uint32_t flag_peek(const uint32_t* flag) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(flag)) : "memory");
+  return v;
+}
+__device__ __noinline__ bool flag_await_slow(const uint32_t* flag, uint32_t epoch, volatile int* abort,
+                                             int* status) {
+  const unsigned long long t0 = now_ns();
+  for (uint32_t it = 1;; ++it) {
+    if ((int)(flag_peek(flag) - epoch) >= 0) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (now_ns() - t0 > kWaitNs) {
+        *abort = 1;
+        atomicOr(status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool flag_await(const uint32_t* flag, uint32_t epoch, volatile int* abort,
+                                           int* status) {
+  if ((int)(flag_peek(flag) - epoch) >= 0) return true;
+  return flag_await_slow(flag, epoch, abort, status);
 }
 
 // Bounded wait used only on the way out (ignores the abort flag).
@@ -311,24 +347,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = ntile * BH;
   volatile int* abort = &sm.abort;
 
+  for (int x = threadIdx.x; x < 2 * 2 * kBM; x += blockDim.x) (&sm.xflag[0][0][0])[x] = 0u;
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.k_full[s], 1);
-      mbar_init(&sm.k_empty[s], 1);
-      mbar_init(&sm.v_full[s], 1);
-      mbar_init(&sm.v_empty[s], 1);
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 256);
-      mbar_init(&sm.pv_done[s], 1);
     }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, 256);
-    mbar_init(&sm.ex_max, 256);
-    mbar_init(&sm.ex_sum, 256);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -349,8 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t kv = 0;
       int tc = 0;
-      long long k_issued[kStages], v_issued[kStages], q_issued = -1;  // last use index per stage
-      for (int s = 0; s < kStages; ++s) k_issued[s] = v_issued[s] = -1;
+      long long kv_issued[kStages], q_issued = -1;  // last use index per stage
+      for (int s = 0; s < kStages; ++s) kv_issued[s] = -1;
       for (int t = blockIdx.x; t < tiles && !*abort; t += gridDim.x, ++tc) {
         const TileInfo ti = tile_info(t, BH, p.N, p.causal);
         const int row0 = ti.bh * p.N;
@@ -364,16 +396,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < ti.nblk; ++j, ++kv) {
           const int st = kv % kStages;
           const uint32_t par = ((kv / kStages) & 1) ^ 1;
-          if (!mbar_wait(&sm.k_empty[st], par, abort, p.status)) break;
-          mbar_expect_tx(&sm.k_full[st], kKVBytes);
-          k_issued[st] = kv / kStages;
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.k_full[st], 64 * h, row0 + j * kBN);
-          if (!mbar_wait(&sm.v_empty[st], par, abort, p.status)) break;
-          mbar_expect_tx(&sm.v_full[st], kKVBytes);
-          v_issued[st] = kv / kStages;
-          for (int h = 0; h < 2; ++h)
-            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.v_full[st], 64 * h, row0 + j * kBN);
+          if (!mbar_wait(&sm.kv_empty[st], par, abort, p.status)) break;
+          mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
+          kv_issued[st] = kv / kStages;
+          for (int h = 0; h < 2; ++h) {
+            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + j * kBN);
+            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + j * kBN);
+          }
         }
       }
       // After an abort, let every copy this thread issued land before the CTA
@@ -381,8 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort) {
         if (q_issued >= 0) mbar_drain(&sm.q_full, (uint32_t)(q_issued & 1));
         for (int s = 0; s < kStages; ++s) {
-          if (k_issued[s] >= 0) mbar_drain(&sm.k_full[s], (uint32_t)(k_issued[s] & 1));
-          if (v_issued[s] >= 0) mbar_drain(&sm.v_full[s], (uint32_t)(v_issued[s] & 1));
+          if (kv_issued[s] >= 0) mbar_drain(&sm.kv_full[s], (uint32_t)(kv_issued[s] & 1));
         }
       }
     }
@@ -400,27 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         auto issue_S = [&](uint32_t gs, uint32_t kvi) -> bool {
           const int st = kvi % kStages;
-          if (!mbar_wait(&sm.k_full[st], (kvi / kStages) & 1, abort, p.status)) return false;
+          if (!mbar_wait(&sm.kv_full[st], (kvi / kStages) & 1, abort, p.status)) return false;
           tc_fence_after();
           const uint32_t d1 = tmem + (gs & 1) * kColStage + kColS1;
           const uint32_t d2 = tmem + (gs & 1) * kColStage + kColS2;
           const uint32_t ka = smem_u32(sm.k[st]);
-          // All of S1's k-steps, then all of S2's: alternating the A operand and
-          // the accumulator between MMAs costs the tensor pipe a third of its rate.
+          // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
+          // the tensor pipe at the sum of the two GEMMs (issuing all of S1 and
+          // then all of S2 measured about a quarter slower).
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
-            const uint32_t koff = (ks >> 2) * kHalfKV + (ks & 3) * 32;
-            mma_ss(d1, sdesc(qa + off, 16, 1024), sdesc(ka + koff, 16, 1024), kIdescS, ks > 0);
-          }
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
-            const uint32_t koff = (ks >> 2) * kHalfKV + (ks & 3) * 32;
-            mma_ss(d2, sdesc(ra + off, 16, 1024), sdesc(ka + koff, 16, 1024), kIdescS, ks > 0);
+            const uint64_t bk = sdesc(ka + (ks >> 2) * kHalfKV + (ks & 3) * 32, 16, 1024);
+            mma_ss(d1, sdesc(qa + off, 16, 1024), bk, kIdescS, ks > 0);
+            mma_ss(d2, sdesc(ra + off, 16, 1024), bk, kIdescS, ks > 0);
           }
           mma_commit(&sm.s_full[gs & 1]);
-          mma_commit(&sm.k_empty[st]);
           return true;
         };
         const uint32_t g0 = g;
@@ -433,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t s = g & 1;
           if (!(ok = mbar_wait(&sm.p_full[s], (g >> 1) & 1, abort, p.status))) break;
           const int st = kvV % kStages;
-          if (!(ok = mbar_wait(&sm.v_full[st], (kvV / kStages) & 1, abort, p.status))) break;
+          // V of this block arrived with its K (waited on before S of this block).
           tc_fence_after();
           const uint32_t va = smem_u32(sm.v[st]);
           const uint32_t sbase = tmem + s * kColStage;
@@ -444,8 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(tmem + kColO1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
             mma_ts(tmem + kColO2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
           }
-          mma_commit(&sm.pv_done[s]);
-          mma_commit(&sm.v_empty[st]);
+          mma_commit(&sm.kv_empty[st]);
           if (j + 2 < ti.nblk) {
             if (!(ok = issue_S(g + 2, kvS++))) break;
             if (j + 3 == ti.nblk) mma_commit(&sm.q_empty);
@@ -468,7 +490,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const float scale = 1.4426950408889634f * rsqrtf((float)kD);
-    uint32_t g = 0;  // blocks processed by this CTA (also the exchange phase)
+    uint32_t g = 0;     // blocks processed by this CTA (also the exchange epoch)
+    uint32_t redo = 0;  // second-exchange epoch of this row
     int tc = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
@@ -499,58 +522,90 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 32; c += 4)
           rmax = max3(rmax, max3(__uint_as_float(x[c]), __uint_as_float(x[c + 1]), __uint_as_float(x[c + 2])),
                       __uint_as_float(x[c + 3]));
-        sm.red_max[hf][row] = rmax;
-        mbar_arrive(&sm.ex_max);
-        if (!(ok = mbar_wait(&sm.ex_max, g & 1, abort, p.status))) break;
-        rmax = fmaxf(rmax, sm.red_max[hf ^ 1][row]);
-        const float mx = rmax * scale;
-        float alpha = 1.f;
-        if (mx > m_run + kLazyTau) {
-          alpha = ex2(m_run - mx);  // 0 on the first block (m_run = -inf)
-          m_run = mx;
-          omega *= alpha;
-          T *= alpha;
-        }
-        // w = 2^(s*scale - m); P = bf16(w) now; a = w (t - c) kept for (w t)'s
-        // bf16 once the centre is settled.
-        const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
-        uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
+        // w = 2^(s*scale - m_run) with the running max as it stands (the max of
+        // this block is exchanged alongside the sums); a = w (t - c) is kept for
+        // (w t)'s bf16 once the centre is settled.  x <- w, y <- a.
         uint32_t P[16];
+        float wpart = 0.f, tpart = 0.f;
+        auto exp_pass = [&]() {
+          const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
+          uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          float s0, s1;
-          uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sc2, nm2), s0, s1);
-          const float w0 = ex2(s0), w1 = ex2(s1);
-          const uint64_t w2 = f2(w0, w1);
-          const uint64_t a2 = mul2(w2, add2(f2(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1])), nc2));
-          if (c & 1) {
-            ws2b = add2(ws2b, w2);
-            ts2b = add2(ts2b, a2);
-          } else {
-            ws2a = add2(ws2a, w2);
-            ts2a = add2(ts2a, a2);
+          for (int c = 0; c < 16; ++c) {
+            float s0, s1;
+            uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sc2, nm2), s0, s1);
+            const float w0 = ex2(s0), w1 = ex2(s1);
+            const uint64_t w2 = f2(w0, w1);
+            const uint64_t a2 = mul2(w2, add2(f2(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1])), nc2));
+            if (c & 1) {
+              ws2b = add2(ws2b, w2);
+              ts2b = add2(ts2b, a2);
+            } else {
+              ws2a = add2(ws2a, w2);
+              ts2a = add2(ts2a, a2);
+            }
+            P[c] = pack_bf16(w0, w1);
+            float a0, a1;
+            uf2(a2, a0, a1);
+            x[2 * c] = __float_as_uint(w0);
+            x[2 * c + 1] = __float_as_uint(w1);
+            y[2 * c] = __float_as_uint(a0);
+            y[2 * c + 1] = __float_as_uint(a1);
           }
-          P[c] = pack_bf16(w0, w1);
-          float a0, a1;
-          uf2(a2, a0, a1);
-          x[2 * c] = __float_as_uint(w0);
-          x[2 * c + 1] = __float_as_uint(w1);
-          y[2 * c] = __float_as_uint(a0);
-          y[2 * c + 1] = __float_as_uint(a1);
+          float lo, hi;
+          uf2(add2(ws2a, ws2b), lo, hi);
+          wpart = lo + hi;
+          uf2(add2(ts2a, ts2b), lo, hi);
+          tpart = lo + hi;
+        };
+        if (j > 0) exp_pass();
+        // Exchange (max, sum w, sum w (t - c)) with the partner thread of this row.
+        const uint32_t e0 = g + 1;
+        float* mine = sm.xch[0][e0 & 1][hf][row];
+        const float* theirs = sm.xch[0][e0 & 1][hf ^ 1][row];
+        mine[0] = rmax;
+        mine[1] = wpart;
+        mine[2] = tpart;
+        flag_post(&sm.xflag[0][hf][row], e0);
+        if (!(ok = flag_await(&sm.xflag[0][hf ^ 1][row], e0, abort, p.status))) break;
+        const float mx = fmaxf(rmax, theirs[0]) * scale;
+        float pw = theirs[1], pt = theirs[2];
+        float alpha = 1.f;
+        // Partner warps (w and w+4) hold the same 32 rows, so this warp-uniform
+        // decision is the same on both sides of every row.
+        if (__any_sync(0xffffffffu, mx > m_run + kLazyTau)) {
+          // The max rose by more than 2^8 (always on a tile's first block):
+          // rescale the row state and redo this block's exponentials.
+          if (mx > m_run + kLazyTau) {
+            alpha = ex2(m_run - mx);  // 0 on the first block (m_run = -inf)
+            m_run = mx;
+            omega *= alpha;
+            T *= alpha;
+          }
+          tmem_ld32(base + kColS1 + 32 * hf, x);
+          tmem_ld32(base + kColS2 + 32 * hf, y);
+          tc_wait_ld();
+          if (edge) {
+            const int kend = p.causal ? min(i + 1, p.N) : p.N;
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+          }
+          exp_pass();
+          ++redo;
+          float* m1 = sm.xch[1][redo & 1][hf][row];
+          const float* t1 = sm.xch[1][redo & 1][hf ^ 1][row];
+          m1[1] = wpart;
+          m1[2] = tpart;
+          flag_post(&sm.xflag[1][hf][row], redo);
+          if (!(ok = flag_await(&sm.xflag[1][hf ^ 1][row], redo, abort, p.status))) break;
+          pw = t1[1];
+          pt = t1[2];
         }
         tmem_st16(base + kColS1 + 16 * hf, P);
-        float lo, hi;
-        uf2(add2(ws2a, ws2b), lo, hi);
-        const float wpart = lo + hi;
-        uf2(add2(ts2a, ts2b), lo, hi);
-        const float tpart = lo + hi;
-        sm.red_w[hf][row] = wpart;
-        sm.red_t[hf][row] = tpart;
-        mbar_arrive(&sm.ex_sum);
-        if (!(ok = mbar_wait(&sm.ex_sum, g & 1, abort, p.status))) break;
         // Both threads of the row form the same sums (a + b == b + a exactly).
-        const float wsum = wpart + sm.red_w[hf ^ 1][row];
-        float Tb = tpart + sm.red_t[hf ^ 1][row];
+        const float wsum = wpart + pw;
+        float Tb = tpart + pt;
         // Re-centre before this block's w (t - c) is rounded to bf16, on the
         // first block and whenever the running mean of t has drifted by more
         // than kTheta from the centre.
@@ -569,8 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // of the previous block are complete; each warpgroup updates its 64 dims.
         const bool need = (j > 0) && (alpha != 1.f || delta != 0.f);
         if (__any_sync(0xffffffffu, need)) {
-          const uint32_t gp = g - 1;  // previous block of this tile
-          if (!(ok = mbar_wait(&sm.pv_done[gp & 1], (gp >> 1) & 1, abort, p.status))) break;
+          // The previous block's value MMAs completed when its K/V stage was freed
+          // (block counter g equals the K/V ring position).
+          const uint32_t gp = g - 1;
+          if (!(ok = mbar_wait(&sm.kv_empty[gp % kStages], (gp / kStages) & 1, abort, p.status))) break;
           tc_fence_after();
           const float ad = alpha * delta;
 #pragma unroll 1
