@@ -1,7 +1,8 @@
 // Causal (or full) Parallax prefill for bf16, d = 128, on sm_100a tensor cores.
 //
-// Per CTA, one 128-query tile at a time (persistent over (b, h, tile), longest
-// causal tiles first).  Warp roles:
+// Per CTA, one 128-query tile at a time; persistent CTAs take (b, h, tile)
+// work from a global counter in head chunks, longest causal tiles first within
+// a chunk (so a few heads' K/V stay in L2).  Warp roles:
 //   warp 0      TMA producer: Q and R tiles, then a ring of 64-key K and V tiles
 //               (128B-swizzled boxes, one mbarrier per stage and direction).
 //   warp 1      TMEM owner and MMA issuer (one elected thread):
@@ -51,6 +52,7 @@ constexpr int kD = 128;
 constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
 constexpr int kStages = 4;               // K/V ring depth
+constexpr int kTileRing = 4;             // tile indices in flight from producer to consumers
 constexpr int kThreads = 320;            // 10 warps: TMA, MMA, 2 softmax warpgroups
 constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
 constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
@@ -86,6 +88,9 @@ struct Smem {
   // double-buffered by epoch parity, and a flag holding the last posted epoch.
   float xch[2][2][2][kBM][4];  // [channel][epoch & 1][warpgroup][row][value]
   uint32_t xflag[2][2][kBM];   // [channel][warpgroup][row]
+  // Tile indices handed from the producer to the MMA and softmax roles.
+  int tile_ring[kTileRing];
+  uint64_t tile_full[kTileRing], tile_empty[kTileRing];
   uint32_t tmem_base;
   int abort;
 };
@@ -319,18 +324,32 @@ struct TileInfo {
   int bh, m, nblk;
 };
 
-__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal) {
+// Tile t of the schedule: heads are taken in chunks of `ch`; within a chunk
+// the tiles go longest causal rows first across the chunk's heads.  CTAs take
+// tiles in this order from a global counter, so the K/V of a few heads stay in
+// L2 while every tile that reads them runs, and the causal work balances.
+__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, int ch) {
   const int ntile = (N + kBM - 1) / kBM;
+  const int per_chunk = ch * ntile;
+  const int chunk = t / per_chunk;
+  const int nh = min(ch, BH - chunk * ch);
+  const int pos = t - chunk * per_chunk;
   TileInfo ti;
-  ti.m = ntile - 1 - t / BH;  // longest causal rows first
-  ti.bh = t % BH;
+  ti.m = ntile - 1 - pos / nh;
+  ti.bh = chunk * ch + pos % nh;
   const int kmax = causal ? min(N, (ti.m + 1) * kBM) : N;
   ti.nblk = (kmax + kBN - 1) / kBN;
   return ti;
 }
 
+// Dynamic tile scheduler state: the next tile to hand out, and the number of
+// CTAs that finished; the last CTA of a launch resets both for the next one.
+__device__ unsigned int g_tile_next;
+__device__ unsigned int g_cta_done;
+
 struct Params {
   int B, H, N, causal;
+  int chunk_heads;
   __nv_bfloat16* out;
   int* status;
 };
@@ -359,6 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 256);
     }
+    for (int s = 0; s < kTileRing; ++s) {
+      mbar_init(&sm.tile_full[s], 1);
+      mbar_init(&sm.tile_empty[s], 9);  // the MMA thread and one lane of each softmax warp
+    }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, 256);
     mbar_init(&sm.drain, 1);
@@ -383,8 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tc = 0;
       long long kv_issued[kStages], q_issued = -1;  // last use index per stage
       for (int s = 0; s < kStages; ++s) kv_issued[s] = -1;
-      for (int t = blockIdx.x; t < tiles && !*abort; t += gridDim.x, ++tc) {
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+      for (; !*abort; ++tc) {
+        const int slot = tc % kTileRing;
+        if (!mbar_wait(&sm.tile_empty[slot], ((tc / kTileRing) & 1) ^ 1, abort, p.status)) break;
+        const unsigned int nt = atomicAdd(&g_tile_next, 1u);
+        const int t = nt < (unsigned int)tiles ? (int)nt : -1;
+        sm.tile_ring[slot] = t;
+        mbar_arrive(&sm.tile_full[slot]);
+        if (t < 0) break;
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         const int row0 = ti.bh * p.N;
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
@@ -422,8 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tc = 0;
       const uint32_t qa = smem_u32(sm.q), ra = smem_u32(sm.r);
       bool ok = true;
-      for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+      for (; ok; ++tc) {
+        const int slot = tc % kTileRing;
+        if (!(ok = mbar_wait(&sm.tile_full[slot], (tc / kTileRing) & 1, abort, p.status))) break;
+        const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
+        mbar_arrive(&sm.tile_empty[slot]);
+        if (t < 0) break;
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         tc_fence_after();
         auto issue_S = [&](uint32_t gs, uint32_t kvi) -> bool {
@@ -494,8 +529,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t redo = 0;  // second-exchange epoch of this row
     int tc = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++tc) {
-      const TileInfo ti = tile_info(t, BH, p.N, p.causal);
+    for (; ok; ++tc) {
+      const int slot = tc % kTileRing;
+      if (!(ok = mbar_wait(&sm.tile_full[slot], (tc / kTileRing) & 1, abort, p.status))) break;
+      const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tile_empty[slot]);
+      if (t < 0) break;
+      const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
       const int i = ti.m * kBM + row;  // query position
       // Row state: running max (log2 units), omega = sum w, T = sum w (t - c)
       // around the row's centre c (see the file comment), all in fp32.
@@ -702,6 +743,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) {
+    // Every CTA fetched its last tile before this point; the last CTA to get
+    // here leaves the scheduler at zero for the next launch.
+    __threadfence();
+    if (atomicAdd(&g_cta_done, 1u) == gridDim.x - 1) {
+      atomicExch(&g_tile_next, 0u);
+      atomicExch(&g_cta_done, 0u);
+    }
+  }
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
@@ -745,7 +795,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms
   if (!make_map(&mQ, a.Q, rows, kBM) || !make_map(&mR, a.R, rows, kBM) || !make_map(&mK, a.K, rows, kBN) ||
       !make_map(&mV, a.V, rows, kBN))
     return cudaErrorInvalidValue;
-  Params p{a.B, a.H, a.N, a.causal, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
+  const int ntile = (a.N + kBM - 1) / kBM;
+  int ch = (2 * num_sms + ntile - 1) / ntile;  // about two waves of tiles per chunk
+  ch = ch < 1 ? 1 : (ch > a.B * a.H ? a.B * a.H : ch);
+  Params p{a.B, a.H, a.N, a.causal, ch, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
