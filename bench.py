@@ -163,22 +163,34 @@ def timed(fn, steps, warmup, stream, dist=None):
     return start.elapsed_time(end), per
 
 
-def max_over_ranks(x, dist):
+def _reduce_scalar(x, dist, op):
     if dist is None:
         return x
     import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x, dist):
+    """Slowest rank's time: the whole job is done only when every rank is."""
+    return _reduce_scalar(x, dist, None if dist is None else dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(x, dist):
-    if dist is None:
-        return x
-    import torch
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    """Units processed by all ranks together (weak scaling: each rank has its own)."""
+    return _reduce_scalar(x, dist, None if dist is None else dist.ReduceOp.SUM)
+
+
+def rank_seed(base, rank):
+    """Each rank draws its own synthetic inputs."""
+    return base + 1000 * rank
+
+
+def whole_job_rate(units_per_rank, ms_per_rank, dist):
+    """Units per second of the whole job: all ranks' units over the slowest rank's time."""
+    return sum_over_ranks(units_per_rank, dist) / (max_over_ranks(ms_per_rank, dist) * 1e-3)
 
 
 def run_gpu(args, rank, world, dist):
@@ -188,7 +200,7 @@ def run_gpu(args, rank, world, dist):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     peaks, peak_src = load_peaks()
-    seed = 1002 + 1000 * rank
+    seed = rank_seed(1002, rank)
 
     # ---- Decode (headline).
     B, H, L, d = args.decode_batch, DECODE["H"], DECODE["L"], DECODE["d"]
