@@ -45,6 +45,9 @@
 
 #include <math_constants.h>
 
+#include <cstdlib>
+#include <cstring>
+
 namespace plx {
 namespace {
 
@@ -350,6 +353,7 @@ __device__ unsigned int g_cta_done;
 struct Params {
   int B, H, N, causal;
   int chunk_heads;
+  int inject_stall;  // failure-detection test: withhold the first Q/R tile
   __nv_bfloat16* out;
   int* status;
 };
@@ -419,9 +423,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
         q_issued = tc;
-        for (int h = 0; h < 2; ++h) {
-          tma_load_2d(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
-          tma_load_2d(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+        // The failure-detection test withholds the first Q/R tile: its barrier
+        // never completes, the MMA warp's bounded wait runs out and every role
+        // unwinds through the abort path.
+        if (!(p.inject_stall && tc == 0)) {
+          for (int h = 0; h < 2; ++h) {
+            tma_load_2d(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+            tma_load_2d(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+          }
         }
         for (int j = 0; j < ti.nblk; ++j, ++kv) {
           const int st = kv % kStages;
@@ -798,7 +807,11 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms
   const int ntile = (a.N + kBM - 1) / kBM;
   int ch = (2 * num_sms + ntile - 1) / ntile;  // about two waves of tiles per chunk
   ch = ch < 1 ? 1 : (ch > a.B * a.H ? a.B * a.H : ch);
-  Params p{a.B, a.H, a.N, a.causal, ch, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
+  // PLX_FAULT_INJECT=prefill_stall makes the kernel's bounded waits run out
+  // (tests of the timeout status only).
+  const char* fi = getenv("PLX_FAULT_INJECT");
+  const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
+  Params p{a.B, a.H, a.N, a.causal, ch, inject, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
   const size_t smem = sizeof(Smem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

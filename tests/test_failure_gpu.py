@@ -1,0 +1,31 @@
+"""Failure detection on the GPU without a fault.
+
+Every wait in the tcgen05 prefill kernel is bounded in time.  With
+PLX_FAULT_INJECT=prefill_stall the TMA producer withholds the first Q/R tile,
+so a barrier that nothing will complete is waited on: the kernel must give up
+after its limit, report PLX_ERR_TIMEOUT through plx_get_device_status, free
+its resources and leave the context usable (the next prefill is correct).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from local_linear_attention_streamed_b200 import synth
+from _util import BF16_TOL, rel_err_rms, small_inputs, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def test_prefill_timeout_is_reported_and_context_survives(monkeypatch):
+    from local_linear_attention_streamed_b200 import plx
+    specs = synth.prefill_specs(1, 2, 256, 128)
+    dev, ref = small_inputs(31, specs, synth.BF16)
+    assert plx.get_device_status() == 0
+    monkeypatch.setenv("PLX_FAULT_INJECT", "prefill_stall")
+    plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=True)
+    assert plx.get_device_status() == -7  # PLX_ERR_TIMEOUT
+    monkeypatch.delenv("PLX_FAULT_INJECT")
+    out = plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=True)
+    assert plx.get_device_status() == 0
+    want = oracle.prefill_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal=True)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
