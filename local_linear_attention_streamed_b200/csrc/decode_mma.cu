@@ -4,8 +4,10 @@
 // once (8d flops per key against 4d bytes).  The kernel therefore optimises the
 // stream, not the math:
 //
-// * Work unit = (b, h, key chunk).  Persistent CTAs of 4 warps walk the units;
-//   the warps of a CTA take the chunk's 16-key blocks round-robin.
+// * Work unit = (b, h, key chunk).  Persistent CTAs of 4 warps take units
+//   from a global counter (chunk-major, so full chunks first; the last CTA to
+//   finish resets the counter); the warps of a CTA take the chunk's 16-key
+//   blocks round-robin.
 // * K and V are read straight from HBM with coalesced 16-byte non-allocating
 //   loads into registers, one block ahead of the math (software pipeline), so
 //   each warp keeps 8 KB in flight.
@@ -211,7 +213,13 @@ struct Smem {
   float O2[kWarps][D];
   float m[kWarps], omega[kWarps], T[kWarps];
   int last;
+  long long unit;
 };
+
+// Dynamic unit scheduler: the next unit to hand out and the number of CTAs
+// that finished; the last CTA of a launch resets both for the next launch.
+__device__ unsigned long long g_unit_next;
+__device__ unsigned int g_cta_done;
 
 template <int D>
 __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
@@ -227,7 +235,15 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
   const __nv_bfloat16* rall = reinterpret_cast<const __nv_bfloat16*>(a.r);
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
 
-  for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+  // Units in chunk-major order (every sequence's first chunk, then the second,
+  // ...), so that the full-length chunks go first.  Each CTA starts with unit
+  // blockIdx.x; further units come from a global counter, fetched at the start
+  // of the current unit so that the atomic's latency hides behind its stream.
+  long long u = blockIdx.x;
+  while (u < units) {
+    long long next = 0;
+    if (threadIdx.x == 0) next = (long long)gridDim.x + (long long)atomicAdd(&g_unit_next, 1ull);
+    do {  // one unit; `break` leaves it early
     const int c = (int)(u / BH);
     const int bh = (int)(u - (long long)c * BH);
     const int b = bh / a.H;
@@ -237,10 +253,10 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
         for (int x = threadIdx.x; x < D; x += kThreads) out[(long long)bh * D + x] = __float2bfloat16(0.f);
         if (threadIdx.x == 0) atomicOr(a.status, kStatusBadSeqlen);
       }
-      continue;
+      break;
     }
     const int nch = (n + a.chunk - 1) / a.chunk;
-    if (c >= nch) continue;
+    if (c >= nch) break;
     const int kbeg = c * a.chunk;
     const int kend = min(kbeg + a.chunk, n);
 
@@ -326,8 +342,7 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
         float inv = 1.f / omega;
         out[(long long)bh * D + x] = __float2bfloat16_rn(((1.f + T * inv) * o1 - o2) * inv);
       }
-      __syncthreads();  // shared memory is reused by the next unit
-      continue;
+      break;
     }
     // ---- Publish this chunk's partial; the last chunk of (b, h) merges all.
     float* rec = a.partials + ((long long)bh * a.splits + c) * (2 * D + 4);
@@ -367,20 +382,45 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
       }
       if (x == 0) a.counters[bh] = 0;
     }
+    } while (false);
+    __syncthreads();  // shared memory and sm.unit are reused by the next unit
+    if (threadIdx.x == 0) sm.unit = next;
     __syncthreads();
+    u = sm.unit;
+  }
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&g_cta_done, 1u) == gridDim.x - 1) {
+      atomicExch(&g_unit_next, 0ull);
+      atomicExch(&g_cta_done, 0u);
+    }
   }
 }
 
 }  // namespace
 
+// Keys per (b, h) are cut into `splits` chunks.  Fewer, longer chunks stream
+// better (each unit pays a fixed start-up and merge), but the last wave of
+// units should be nearly full: take the fewest splits whose waves over the
+// resident CTAs are at least 97 % used, with chunks of at least 256 keys.
 void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk) {
-  const long long bh = (long long)B * H;
-  const long long resident = (long long)num_sms * 2;  // CTAs the launcher keeps per SM
-  long long S = (16 * resident + bh - 1) / bh;        // about 16 waves of units
-  long long smax = L / 256;                           // chunks of at least 256 keys
-  if (S > smax) S = smax;
-  if (S < 1) S = 1;
-  long long c = (L + S - 1) / S;
+  const double bh = (double)B * H;
+  const double resident = (double)num_sms * 2;  // CTAs the launcher keeps per SM
+  long long smax = L / 256;
+  if (smax < 1) smax = 1;
+  if (smax > 256) smax = 256;
+  long long best = 1;
+  double best_eff = -1.0;
+  for (long long S = 1; S <= smax; ++S) {
+    const double waves = bh * (double)S / resident;
+    const double eff = waves / ceil(waves);
+    if (eff > best_eff + 0.02) {
+      best_eff = eff;
+      best = S;
+    }
+    if (eff >= 0.97) break;
+  }
+  long long c = (L + best - 1) / best;
   c = (c + 63) / 64 * 64;
   *chunk = (int)c;
   *splits = (int)((L + c - 1) / c);

@@ -53,8 +53,9 @@ def test_noalloc_matches_regular_decode_on_two_calls():
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from local_linear_attention_streamed_b200 import plx
-    B, H, L, d = 256, 16, 1024, 128  # 4096 (b, h) x 2 splits of fp32 records > 8 MiB
-    assert plx.lib.plx_decode_num_splits(B, H, L, d) == 2
+    B, H, L, d = 250, 16, 1024, 128  # 4000 (b, h) x 3 splits of fp32 records > 8 MiB
+    S = plx.lib.plx_decode_num_splits(B, H, L, d)
+    assert S > 1 and B * H * S * (2 * d + 4) * 4 > (8 << 20) - (128 << 10)
     small = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
     sl = torch.ones(B, dtype=torch.int32, device="cuda")
     rc = plx.lib.plx_decode_noalloc(small.data_ptr(), small.data_ptr(), small.data_ptr(),
