@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 METRIC = "decode KV GB/s (% HBM peak); causal prefill TFLOP/s (% BF16 peak)"
 DECODE = dict(B=64, H=16, L=4096, d=128)
 PREFILL = dict(B=8, H=16, N=4096, d=128)
+LAYER = dict(B=4, N=8192, D=2048, H=16)
 SWEEP_B = [1, 8, 64, 256, 1024, 2048]
 SWEEP_L = [128, 1024, 4096, 16384, 32768]
 SWEEP_MAX_BYTES = 150e9
@@ -305,10 +306,60 @@ def run_gpu(args, rank, world, dist):
         del pt
         torch.cuda.empty_cache()
 
+    # ---- Full layer (x [4, 8192, 2048], 16 heads of 128).
+    layer = None
+    if not args.no_layer:
+        LB, LN, LD, LH = LAYER["B"], LAYER["N"], LAYER["D"], LAYER["H"]
+        lspecs = synth.layer_specs(LB, LN, LD)
+        lt = {}
+        for name, spec in lspecs.items():
+            lt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(lt[name].data_ptr(), synth.BF16, seed + 3, spec)
+        y = torch.empty_like(lt["x"])
+
+        def lay():
+            plx.layer_forward(lt["x"], lt["WQ"], lt["WK"], lt["WV"], lt["WR"], lt["WO"], LH, out=y)
+
+        lsteps = max(1, args.steps // 4)
+        l_total, l_per = timed(lay, lsteps, 3, stream, dist)
+        if plx.get_device_status() != 0:
+            raise RuntimeError("layer reported a device error")
+        # The attention inside the layer on inputs of the same shape.
+        ad = LD // LH
+        aspecs = synth.prefill_specs(LB, LH, LN, ad)
+        at = {}
+        for name, spec in aspecs.items():
+            at[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(at[name].data_ptr(), synth.BF16, seed + 4, spec)
+        aout = torch.empty_like(at["Q"])
+
+        def att():
+            plx.prefill(at["Q"], at["K"], at["V"], at["R"], causal=True, out=aout)
+
+        a_total, a_per = timed(att, lsteps, 3, stream, dist)
+        l_ms, a_ms = float(np.mean(l_per)), float(np.mean(a_per))
+        aflops = prefill_flops(LB, LH, LN, ad)
+        pflops = 5 * 2.0 * LB * LN * LD * LD  # q, k, v, rho and output projections
+        layer = {
+            "config": {"workload": "layer x[4, 8192, 2048] bf16, 16 heads of 128, causal"},
+            "layer_ms": round(l_ms, 3),
+            "attention_ms": round(a_ms, 3),
+            "attention_tflops": round(aflops / (a_ms * 1e-3) / 1e12, 1),
+            "attention_flops": aflops,
+            "rest_ms": round(l_ms - a_ms, 3),
+            "rest_note": "projections (cuBLAS bf16, 1.37e12 flops), RMSNorm+RoPE, head split/merge",
+            "projection_flops": pflops,
+            "layer_tflops_all": round((aflops + pflops) / (l_ms * 1e-3) / 1e12, 1),
+            "gpu_launches_per_step": {"own_kernels": 6, "cublas_gemms": 5},
+        }
+        del lt, at
+        torch.cuda.empty_cache()
+
     clk.__exit__(None, None, None)
     return {
         "value": round(value, 2), "ms_per_step": round(ms_step, 4), "roofline": roofline,
-        "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "gpu_launches": args.steps,
+        "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "layer": layer,
+        "gpu_launches": args.steps,
         "kernel_ms": kernel_ms,
     }
 
@@ -459,6 +510,7 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
                     help="decode batch (smaller values for profiler captures only)")
@@ -541,7 +593,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
-            "prefill": res["prefill"]}
+            "prefill": res["prefill"], "layer": res["layer"]}
     print(json.dumps(line))
 
 

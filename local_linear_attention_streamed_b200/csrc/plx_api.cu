@@ -221,6 +221,7 @@ int plx_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float 
   if (!x || !y) return PLX_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || H < 1 || !(eps >= 0.f) || !(rope_base > 0.f)) return PLX_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if ((long long)B * N * H * d >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y)) return PLX_ERR_MISALIGNED;
   return launch_qkr_norm_rope(x, y, B, N, H, d, eps, rope_base,
                               reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
@@ -240,6 +241,7 @@ int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void*
   if (!x || !WQ || !WK || !WV || !WR || !WO || !y) return PLX_ERR_INVALID_ARG;
   if (B < 1 || N < 1 || H < 1) return PLX_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if ((long long)B * N * H * d >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(WQ) || !aligned16(WK) || !aligned16(WV) || !aligned16(WR) ||
       !aligned16(WO) || !aligned16(y))
     return PLX_ERR_MISALIGNED;
