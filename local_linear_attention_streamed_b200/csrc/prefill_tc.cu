@@ -459,7 +459,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kvS = 0, kvV = 0;  // K/V ring positions consumed by S and by PV
       uint32_t g = 0;             // blocks processed by this CTA (S/P stage counter)
       int tc = 0;
-      const uint32_t qa = smem_u32(sm.q), ra = smem_u32(sm.r);
+      const uint64_t dQ = sdesc(smem_u32(sm.q), 16, 1024), dR = sdesc(smem_u32(sm.r), 16, 1024);
+      const uint64_t dK0 = sdesc(smem_u32(sm.k[0]), 16, 1024);
+      const uint64_t dV0 = sdesc(smem_u32(sm.v[0]), kHalfKV, 1024);
+      const uint32_t oa1 = tmem + kColO1, oa2 = tmem + kColO2;
       bool ok = true;
       for (; ok; ++tc) {
         const int slot = tc % kTileRing;
@@ -470,22 +473,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         tc_fence_after();
+        // The issuing thread shares its scheduler with two softmax warps, so
+        // every MMA is issued from descriptors built once: a k-step or a stage
+        // only adds a compile-time offset to the start-address field (smem
+        // addresses < 256 KB keep that 14-bit field from carrying).
         auto issue_S = [&](uint32_t gs, uint32_t kvi) -> bool {
-          const int st = kvi % kStages;
+          const uint32_t st = kvi % kStages;
           if (!mbar_wait(&sm.kv_full[st], (kvi / kStages) & 1, abort, p.status)) return false;
           tc_fence_after();
           const uint32_t d1 = tmem + (gs & 1) * kColStage + kColS1;
-          const uint32_t d2 = tmem + (gs & 1) * kColStage + kColS2;
-          const uint32_t ka = smem_u32(sm.k[st]);
+          const uint32_t d2 = d1 + (kColS2 - kColS1);
+          const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
           // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
           // the tensor pipe at the sum of the two GEMMs (issuing all of S1 and
           // then all of S2 measured about a quarter slower).
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t off = (ks >> 2) * kHalfQ + (ks & 3) * 32;
-            const uint64_t bk = sdesc(ka + (ks >> 2) * kHalfKV + (ks & 3) * 32, 16, 1024);
-            mma_ss(d1, sdesc(qa + off, 16, 1024), bk, kIdescS, ks > 0);
-            mma_ss(d2, sdesc(ra + off, 16, 1024), bk, kIdescS, ks > 0);
+            const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
+            const uint64_t koff = (uint64_t)((((ks >> 2) * kHalfKV) + (ks & 3) * 32) >> 4);
+            mma_ss(d1, dQ + off, dk + koff, kIdescS, ks > 0);
+            mma_ss(d2, dR + off, dk + koff, kIdescS, ks > 0);
           }
           mma_commit(&sm.s_full[gs & 1]);
           return true;
@@ -499,17 +506,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < ti.nblk; ++j, ++g, ++kvV) {
           const uint32_t s = g & 1;
           if (!(ok = mbar_wait(&sm.p_full[s], (g >> 1) & 1, abort, p.status))) break;
-          const int st = kvV % kStages;
+          const uint32_t st = kvV % kStages;
           // V of this block arrived with its K (waited on before S of this block).
           tc_fence_after();
-          const uint32_t va = smem_u32(sm.v[st]);
+          const uint64_t dv = dV0 + (uint64_t)(st * (kKVBytes >> 4));
           const uint32_t sbase = tmem + s * kColStage;
+          const uint32_t first = (j == 0) ? 0u : 1u;
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
-            const uint64_t bv = sdesc(va + ks * 2048, kHalfKV, 1024);
-            const uint32_t acc = (j > 0 || ks > 0) ? 1u : 0u;
-            mma_ts(tmem + kColO1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
-            mma_ts(tmem + kColO2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
+            const uint64_t bv = dv + (uint64_t)((ks * 2048) >> 4);
+            const uint32_t acc = ks > 0 ? 1u : first;
+            mma_ts(oa1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
+            mma_ts(oa2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
           }
           mma_commit(&sm.kv_empty[st]);
           if (j + 2 < ti.nblk) {
