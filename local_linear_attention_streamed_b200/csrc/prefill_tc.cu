@@ -5,23 +5,31 @@
 // a chunk (so a few heads' K/V stay in L2).  Warp roles:
 //   warp 0      TMA producer: Q and R tiles, then a ring of 64-key K and V tiles
 //               (128B-swizzled boxes, one mbarrier per stage and direction).
-//   warp 1      TMEM owner and MMA issuer (one elected thread):
+//   warp 1      TMEM owner and score MMA issuer (one elected thread):
 //                 S1 = Q K^T and S2 = R K^T from ONE K tile into TMEM
 //                 (rainbus.top summary, "方法步骤详情": S1 and S2 per KV block
-//                 from one shared instruction stream), double-buffered so that
-//                 the next block's scores overlap this block's softmax;
-//                 O1 += P V and O2 += (w t) V with P and w t read from TMEM and
-//                 V from shared memory ("accumulate O1 and O2 in parallel").
+//                 from one shared instruction stream);
+//   warp 10     value MMA issuer (one elected thread): O1 += P V and
+//                 O2 += (w t) V with P and w t read from TMEM and V from shared
+//                 memory ("accumulate O1 and O2 in parallel").  Two issuing
+//                 threads keep the tensor pipe fed while either one waits on a
+//                 barrier (an MMA issue stalls until the pipe takes it).
 //   warps 2..9  two softmax warpgroups, each thread = one half (32 keys of every
 //               block, 64 output dims) of one query row (= TMEM lane): one running
 //               max and one rescale factor shared by both branches (agihunt.info
 //               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
-//               P = bf16(w) and bf16(w (t - c)) written back over the scores, and
-//               the epilogue out = ((1 + T/omega) O1 - O2) / omega.
-// TMEM (512 columns): S1/S2 of stage s at 128s and 128s+64 (64 fp32 columns
-// each); O1 at 256 and O2 at 384 (128 fp32 columns each).  P(s) = bf16(w)
-// overwrites S1(s) columns 0..31 (bf16 pairs) and bf16(w (t - c)) overwrites
-// S2(s) columns 0..31.
+//               P = bf16(w) and bf16(w (t - c)) into a P buffer, and the
+//               epilogue out = ((1 + T/omega) O1 - O2) / omega.
+// TMEM (512 columns): one S stage (S1 at 0, S2 at 64: 64 fp32 columns each),
+// two P buffers at 128 and 192 (bf16 pairs: bf16(w) in columns 0..31 and
+// bf16(w (t - c)) in 32..63), O1 at 256 and O2 at 384 (128 fp32 columns each).
+// The scores of block g+1 are computed as soon as the softmax has loaded those
+// of block g into registers, and the value MMAs of block g read P buffer g % 2,
+// so the tensor pipe runs ahead of the softmax by a block instead of waiting
+// for it: the two overlap without either one's latency entering the other's
+// period.  Each softmax thread reads the whole row of S1 (its partner's half
+// too) to take the block's row max without an exchange; the row sums are
+// exchanged once per block.
 //
 // Centring.  The output is unchanged when every t_ij of a query is shifted by
 // the same c_i (the pages' key-query difference z_ij = k_j - q_i is one such
@@ -56,17 +64,20 @@ constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
 constexpr int kStages = 4;               // K/V ring depth
 constexpr int kTileRing = 4;             // tile indices in flight from producer to consumers
-constexpr int kThreads = 320;            // 10 warps: TMA, MMA, 2 softmax warpgroups
+constexpr int kThreads = 352;            // 11 warps: TMA, S MMA, 2 softmax warpgroups, PV MMA
+constexpr int kPVWarp = 10;
 constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
 constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
 constexpr uint32_t kHalfKV = kBN * 128;      // one 64-dim half of a K/V block
 constexpr float kLazyTau = 8.f;
-constexpr float kTheta = 1.f;  // re-centre t once its running mean drifts this far
+constexpr float kTheta = 2.f;  // re-centre t once its running mean drifts this far
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on every wait
 
-// TMEM column map.
-constexpr uint32_t kColS1 = 0, kColS2 = 64, kColStage = 128, kColO1 = 256, kColO2 = 384;
+// TMEM column map: the S stage, two P buffers (bf16(w) then bf16(w (t - c))
+// in each), O1 and O2.
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColO1 = 256,
+                   kColO2 = 384;
 
 // Instruction descriptors (kind::f16): D f32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), A K-major, B K-major (S) or MN-major (bit 16, PV),
@@ -85,12 +96,12 @@ struct Smem {
   // One full and one empty barrier per K/V stage: K and V of a block land
   // together, and the stage frees once that block's value MMAs completed.
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full, s_free, p_full[2];
   uint64_t o_full, o_empty, drain;
-  // Row exchanges between the two softmax warpgroups: per channel, data slots
-  // double-buffered by epoch parity, and a flag holding the last posted epoch.
-  float xch[2][2][2][kBM][4];  // [channel][epoch & 1][warpgroup][row][value]
-  uint32_t xflag[2][2][kBM];   // [channel][warpgroup][row]
+  // Row-sum exchange between the two softmax warpgroups, double-buffered by
+  // epoch parity: one 64-bit word per slot holds (sum w, sum w (t - c)), with
+  // the sign bit of sum w (never negative) carrying the epoch tag.
+  unsigned long long xch[2][2][kBM];  // [epoch & 1][warpgroup][row]
   // Tile indices handed from the producer to the MMA and softmax roles.
   int tile_ring[kTileRing];
   uint64_t tile_full[kTileRing], tile_empty[kTileRing];
@@ -160,22 +171,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(bar, parity, abort, status);
 }
 
-// Pairwise exchange between the two threads that share a query row: write the
-// values, then publish the epoch with release semantics; read the partner's
-// epoch with acquire semantics (bounded in time), then its values.
-__device__ __forceinline__ void flag_post(uint32_t* flag, uint32_t epoch) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(flag)), "r"(epoch) : "memory");
+// Pairwise exchange between the two threads that share a query row: each
+// posts one 64-bit word (a single-copy-atomic shared-memory access, so the
+// values and their tag arrive together) and polls the partner's word until
+// its tag matches the epoch (bounded in time).
+__device__ __forceinline__ void xch_post(unsigned long long* slot, unsigned long long v) {
+  asm volatile("st.volatile.shared::cta.u64 [%0], %1;" ::"r"(smem_u32(slot)), "l"(v) : "memory");
 }
-__device__ __forceinline__ uint32_t flag_peek(const uint32_t* flag) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(flag)) : "memory");
+__device__ __forceinline__ unsigned long long xch_peek(const unsigned long long* slot) {
+  unsigned long long v;
+  asm volatile("ld.volatile.shared::cta.u64 %0, [%1];" : "=l"(v) : "r"(smem_u32(slot)) : "memory");
   return v;
 }
-__device__ __noinline__ bool flag_await_slow(const uint32_t* flag, uint32_t epoch, volatile int* abort,
-                                             int* status) {
+__device__ __noinline__ bool xch_await_slow(const unsigned long long* slot, uint32_t tag, unsigned long long* out,
+                                            volatile int* abort, int* status) {
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
-    if ((int)(flag_peek(flag) - epoch) >= 0) return true;
+    const unsigned long long v = xch_peek(slot);
+    if ((uint32_t)(v >> 31 & 1u) == tag) {
+      *out = v;
+      return true;
+    }
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (now_ns() - t0 > kWaitNs) {
@@ -186,10 +202,14 @@ __device__ __noinline__ bool flag_await_slow(const uint32_t* flag, uint32_t epoc
     }
   }
 }
-__device__ __forceinline__ bool flag_await(const uint32_t* flag, uint32_t epoch, volatile int* abort,
-                                           int* status) {
-  if ((int)(flag_peek(flag) - epoch) >= 0) return true;
-  return flag_await_slow(flag, epoch, abort, status);
+__device__ __forceinline__ bool xch_await(const unsigned long long* slot, uint32_t tag, unsigned long long* out,
+                                          volatile int* abort, int* status) {
+  const unsigned long long v = xch_peek(slot);
+  if ((uint32_t)(v >> 31 & 1u) == tag) {
+    *out = v;
+    return true;
+  }
+  return xch_await_slow(slot, tag, out, abort, status);
 }
 
 // Bounded wait used only on the way out (ignores the abort flag).
@@ -370,7 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = ntile * BH;
   volatile int* abort = &sm.abort;
 
-  for (int x = threadIdx.x; x < 2 * 2 * kBM; x += blockDim.x) (&sm.xflag[0][0][0])[x] = 0u;
+  // Slot 1 is first used by epoch 1 (tag 0) and slot 0 by epoch 2 (tag 1):
+  // start each with the other tag.
+  for (int x = threadIdx.x; x < 2 * 2 * kBM; x += blockDim.x)
+    (&sm.xch[0][0][0])[x] = x < 2 * kBM ? 0ull : 0x80000000ull;
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
@@ -378,17 +401,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 256);
-    }
+    mbar_init(&sm.s_full, 1);
+    mbar_init(&sm.s_free, 8);  // one lane of each softmax warp
+    for (int s = 0; s < 2; ++s) mbar_init(&sm.p_full[s], 256);
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(&sm.tile_full[s], 1);
-      mbar_init(&sm.tile_empty[s], 9);  // the MMA thread and one lane of each softmax warp
+      mbar_init(&sm.tile_empty[s], 10);  // the two MMA threads and one lane of each softmax warp
     }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, 256);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, 2);  // one commit from each MMA thread
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -454,13 +476,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- score MMA issuer ----------------
     if (lane == 0) {
-      uint32_t kvS = 0, kvV = 0;  // K/V ring positions consumed by S and by PV
-      uint32_t g = 0;             // blocks processed by this CTA (S/P stage counter)
+      uint32_t g = 0;  // blocks processed by this CTA = K/V ring position = S phase
       int tc = 0;
       const uint64_t dQ = sdesc(smem_u32(sm.q), 16, 1024), dR = sdesc(smem_u32(sm.r), 16, 1024);
       const uint64_t dK0 = sdesc(smem_u32(sm.k[0]), 16, 1024);
+      // Each issuing thread shares its scheduler with two softmax warps, so
+      // every MMA is issued from descriptors built once: a k-step or a stage
+      // only adds a compile-time offset to the start-address field (smem
+      // addresses < 256 KB keep that 14-bit field from carrying).
+      bool ok = true;
+      for (; ok; ++tc) {
+        const int slot = tc % kTileRing;
+        if (!(ok = mbar_wait(&sm.tile_full[slot], (tc / kTileRing) & 1, abort, p.status))) break;
+        const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
+        mbar_arrive(&sm.tile_empty[slot]);
+        if (t < 0) break;
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
+        if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
+        for (int j = 0; j < ti.nblk; ++j, ++g) {
+          // The S stage is free once the softmax has read the previous block's
+          // scores; P buffer g % 2, which the softmax fills once these scores
+          // land, is free once the value MMAs of block g - 2 completed.
+          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
+          if (g > 1) {
+            const uint32_t gq = g - 2;
+            if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
+          }
+          const uint32_t st = g % kStages;
+          if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
+          tc_fence_after();
+          const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
+          // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
+          // the tensor pipe at the sum of the two GEMMs (issuing all of S1 and
+          // then all of S2 measured about a quarter slower).
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
+            const uint64_t koff = (uint64_t)((((ks >> 2) * kHalfKV) + (ks & 3) * 32) >> 4);
+            mma_ss(tmem + kColS1, dQ + off, dk + koff, kIdescS, ks > 0);
+            mma_ss(tmem + kColS2, dR + off, dk + koff, kIdescS, ks > 0);
+          }
+          mma_commit(&sm.s_full);
+          if (j + 1 == ti.nblk) mma_commit(&sm.q_empty);
+        }
+      }
+      // Drain: all MMAs this thread issued complete before TMEM is freed.
+      mma_commit(&sm.drain);
+      mbar_drain(&sm.drain, 0);
+    }
+  } else if (warp == kPVWarp) {
+    // ---------------- value MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t g = 0;
+      int tc = 0;
       const uint64_t dV0 = sdesc(smem_u32(sm.v[0]), kHalfKV, 1024);
       const uint32_t oa1 = tmem + kColO1, oa2 = tmem + kColO2;
       bool ok = true;
@@ -471,79 +541,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.tile_empty[slot]);
         if (t < 0) break;
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
-        if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
-        tc_fence_after();
-        // The issuing thread shares its scheduler with two softmax warps, so
-        // every MMA is issued from descriptors built once: a k-step or a stage
-        // only adds a compile-time offset to the start-address field (smem
-        // addresses < 256 KB keep that 14-bit field from carrying).
-        auto issue_S = [&](uint32_t gs, uint32_t kvi) -> bool {
-          const uint32_t st = kvi % kStages;
-          if (!mbar_wait(&sm.kv_full[st], (kvi / kStages) & 1, abort, p.status)) return false;
-          tc_fence_after();
-          const uint32_t d1 = tmem + (gs & 1) * kColStage + kColS1;
-          const uint32_t d2 = d1 + (kColS2 - kColS1);
-          const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
-          // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
-          // the tensor pipe at the sum of the two GEMMs (issuing all of S1 and
-          // then all of S2 measured about a quarter slower).
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
-            const uint64_t koff = (uint64_t)((((ks >> 2) * kHalfKV) + (ks & 3) * 32) >> 4);
-            mma_ss(d1, dQ + off, dk + koff, kIdescS, ks > 0);
-            mma_ss(d2, dR + off, dk + koff, kIdescS, ks > 0);
-          }
-          mma_commit(&sm.s_full[gs & 1]);
-          return true;
-        };
-        const uint32_t g0 = g;
-        if (!(ok = issue_S(g0, kvS++))) break;
-        if (ti.nblk > 1 && !(ok = issue_S(g0 + 1, kvS++))) break;
-        if (ti.nblk <= 2) mma_commit(&sm.q_empty);
         // The epilogue of the previous tile must have read O before it is overwritten.
         if (tc > 0 && !(ok = mbar_wait(&sm.o_empty, (tc - 1) & 1, abort, p.status))) break;
-        for (int j = 0; j < ti.nblk; ++j, ++g, ++kvV) {
-          const uint32_t s = g & 1;
-          if (!(ok = mbar_wait(&sm.p_full[s], (g >> 1) & 1, abort, p.status))) break;
-          const uint32_t st = kvV % kStages;
-          // V of this block arrived with its K (waited on before S of this block).
+        for (int j = 0; j < ti.nblk; ++j, ++g) {
+          const uint32_t b = g & 1;
+          // P of this block is in TMEM; its scores (so its K) were consumed
+          // before, and V arrived with K.
+          if (!(ok = mbar_wait(&sm.p_full[b], (g >> 1) & 1, abort, p.status))) break;
           tc_fence_after();
+          const uint32_t st = g % kStages;
           const uint64_t dv = dV0 + (uint64_t)(st * (kKVBytes >> 4));
-          const uint32_t sbase = tmem + s * kColStage;
+          const uint32_t pbase = tmem + kColP + b * kColPBuf;
           const uint32_t first = (j == 0) ? 0u : 1u;
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
             const uint64_t bv = dv + (uint64_t)((ks * 2048) >> 4);
             const uint32_t acc = ks > 0 ? 1u : first;
-            mma_ts(oa1, sbase + kColS1 + ks * 8, bv, kIdescPV, acc);
-            mma_ts(oa2, sbase + kColS2 + ks * 8, bv, kIdescPV, acc);
+            mma_ts(oa1, pbase + ks * 8, bv, kIdescPV, acc);
+            mma_ts(oa2, pbase + kColPT + ks * 8, bv, kIdescPV, acc);
           }
+          // Frees the K/V stage and P buffer b.
           mma_commit(&sm.kv_empty[st]);
-          if (j + 2 < ti.nblk) {
-            if (!(ok = issue_S(g + 2, kvS++))) break;
-            if (j + 3 == ti.nblk) mma_commit(&sm.q_empty);
-          }
         }
         if (!ok) break;
         mma_commit(&sm.o_full);
       }
-      // Drain: all MMAs this thread issued complete before TMEM is freed.
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
   } else {
     // ---------------- softmax / epilogue: two warpgroups ----------------
     // Warpgroup hf (warps 2..5 -> 0, 6..9 -> 1) owns keys 32hf..32hf+31 of every
-    // block and output dims 64hf..64hf+63; the two threads of a row exchange
-    // their partial max and sums through shared memory, so both keep identical
-    // copies of the row state (m, omega, T, c).
+    // block and output dims 64hf..64hf+63; both threads of a row take the max
+    // over all 64 scores of a block and exchange their partial sums through
+    // shared memory, so both keep identical copies of the row state
+    // (m, omega, T, c).
     const int hf = (warp - 2) >> 2;
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
     const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
     const float scale = 1.4426950408889634f * rsqrtf((float)kD);
-    uint32_t g = 0;     // blocks processed by this CTA (also the exchange epoch)
-    uint32_t redo = 0;  // second-exchange epoch of this row
+    uint32_t g = 0;  // blocks processed by this CTA (also the exchange epoch)
     int tc = 0;
     bool ok = true;
     for (; ok; ++tc) {
@@ -559,33 +596,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       // around the row's centre c (see the file comment), all in fp32.
       float m_run = -CUDART_INF_F, omega = 0.f, T = 0.f, cen = 0.f;
       for (int j = 0; j < ti.nblk; ++j, ++g) {
-        const uint32_t s = g & 1;
-        if (!(ok = mbar_wait(&sm.s_full[s], (g >> 1) & 1, abort, p.status))) break;
+        if (!(ok = mbar_wait(&sm.s_full, g & 1, abort, p.status))) break;
         tc_fence_after();
-        const uint32_t base = tmem + lane_addr + s * kColStage;
+        const uint32_t sb = tmem + lane_addr;
+        const int kb = j * kBN;
+        const bool edge = (p.causal && kb + kBN - 1 > ti.m * kBM) || (kb + kBN > p.N);
+        const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
         uint32_t x[32], y[32];
-        tmem_ld32(base + kColS1 + 32 * hf, x);
-        tmem_ld32(base + kColS2 + 32 * hf, y);
-        tc_wait_ld();
-        const int k0 = j * kBN + 32 * hf;
-        const bool edge = (p.causal && j * kBN + kBN - 1 > ti.m * kBM) || (j * kBN + kBN > p.N);
-        if (edge) {  // block-uniform: only blocks that cross the diagonal or the end
-          const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
+        float rmax;
+        {
+          // This thread's 32 scores and t values, and the partner half of the
+          // scores for the row max; then the S stage is handed back to the MMA.
+          uint32_t z[32];
+          tmem_ld32(sb + kColS1 + 32 * hf, x);
+          tmem_ld32(sb + kColS1 + 32 * (hf ^ 1), z);
+          tmem_ld32(sb + kColS2 + 32 * hf, y);
+          tc_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free);
+          if (edge) {  // block-uniform: only blocks that cross the diagonal or the end
+            const int k0 = kb + 32 * hf, kz = kb + 32 * (hf ^ 1);
 #pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+            for (int c = 0; c < 32; ++c) {
+              if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+              if (kz + c >= kend) z[c] = __float_as_uint(-CUDART_INF_F);
+            }
+          }
+          // Four independent chains over the 64 scores, then their max.
+          float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            m4[0] = max3(m4[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+            m4[1] = max3(m4[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+            m4[2] = max3(m4[2], __uint_as_float(z[c]), __uint_as_float(z[c + 1]));
+            m4[3] = max3(m4[3], __uint_as_float(z[c + 2]), __uint_as_float(z[c + 3]));
+          }
+          rmax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
         }
-        float rmax = -CUDART_INF_F;
-#pragma unroll
-        for (int c = 0; c < 32; c += 4)
-          rmax = max3(rmax, max3(__uint_as_float(x[c]), __uint_as_float(x[c + 1]), __uint_as_float(x[c + 2])),
-                      __uint_as_float(x[c + 3]));
-        // w = 2^(s*scale - m_run) with the running max as it stands (the max of
-        // this block is exchanged alongside the sums); a = w (t - c) is kept for
-        // (w t)'s bf16 once the centre is settled.  x <- w, y <- a.
+        // Both halves of the row took the max of the same 64 scores, so the
+        // raise decision below is the same on both sides.
+        const float mx = rmax * scale;
+        float alpha = 1.f;
+        if (mx > m_run + kLazyTau) {  // always on a tile's first block (m_run = -inf)
+          alpha = ex2(m_run - mx);    // 0 on the first block
+          m_run = mx;
+          omega *= alpha;
+          T *= alpha;
+        }
+        // w = 2^(s*scale - m_run); a = w (t - c) is kept for bf16(w (t - c))
+        // once the centre is settled.  x <- w, y <- a.
         uint32_t P[16];
-        float wpart = 0.f, tpart = 0.f;
-        auto exp_pass = [&]() {
+        float wpart, tpart;
+        {
           const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
           uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
 #pragma unroll
@@ -615,62 +678,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           wpart = lo + hi;
           uf2(add2(ts2a, ts2b), lo, hi);
           tpart = lo + hi;
-        };
-        if (j > 0) exp_pass();
-        // Exchange (max, sum w, sum w (t - c)) with the partner thread of this row.
-        const uint32_t e0 = g + 1;
-        float* mine = sm.xch[0][e0 & 1][hf][row];
-        const float* theirs = sm.xch[0][e0 & 1][hf ^ 1][row];
-        mine[0] = rmax;
-        mine[1] = wpart;
-        mine[2] = tpart;
-        flag_post(&sm.xflag[0][hf][row], e0);
-        if (!(ok = flag_await(&sm.xflag[0][hf ^ 1][row], e0, abort, p.status))) break;
-        const float mx = fmaxf(rmax, theirs[0]) * scale;
-        float pw = theirs[1], pt = theirs[2];
-        float alpha = 1.f;
-        // Partner warps (w and w+4) hold the same 32 rows, so this warp-uniform
-        // decision is the same on both sides of every row.
-        if (__any_sync(0xffffffffu, mx > m_run + kLazyTau)) {
-          // The max rose by more than 2^8 (always on a tile's first block):
-          // rescale the row state and redo this block's exponentials.
-          if (mx > m_run + kLazyTau) {
-            alpha = ex2(m_run - mx);  // 0 on the first block (m_run = -inf)
-            m_run = mx;
-            omega *= alpha;
-            T *= alpha;
-          }
-          tmem_ld32(base + kColS1 + 32 * hf, x);
-          tmem_ld32(base + kColS2 + 32 * hf, y);
-          tc_wait_ld();
-          if (edge) {
-            const int kend = p.causal ? min(i + 1, p.N) : p.N;
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
-          }
-          exp_pass();
-          ++redo;
-          float* m1 = sm.xch[1][redo & 1][hf][row];
-          const float* t1 = sm.xch[1][redo & 1][hf ^ 1][row];
-          m1[1] = wpart;
-          m1[2] = tpart;
-          flag_post(&sm.xflag[1][hf][row], redo);
-          if (!(ok = flag_await(&sm.xflag[1][hf ^ 1][row], redo, abort, p.status))) break;
-          pw = t1[1];
-          pt = t1[2];
         }
-        tmem_st16(base + kColS1 + 16 * hf, P);
+        // Exchange (sum w, sum w (t - c)) with the partner thread of this row.
+        const uint32_t e0 = g + 1, tag = (e0 >> 1) & 1u;
+        xch_post(&sm.xch[e0 & 1][hf][row],
+                 (unsigned long long)__float_as_uint(tpart) << 32 | __float_as_uint(wpart) | tag << 31);
+        unsigned long long theirs;
+        if (!(ok = xch_await(&sm.xch[e0 & 1][hf ^ 1][row], tag, &theirs, abort, p.status))) break;
         // Both threads of the row form the same sums (a + b == b + a exactly).
-        const float wsum = wpart + pw;
-        float Tb = tpart + pt;
+        const float wsum = wpart + __uint_as_float((uint32_t)theirs & 0x7FFFFFFFu);
+        float Tb = tpart + __uint_as_float((uint32_t)(theirs >> 32));
         // Re-centre before this block's w (t - c) is rounded to bf16, on the
         // first block and whenever the running mean of t has drifted by more
         // than kTheta from the centre.
         float delta = 0.f;
-        const float tb_new = (T + Tb) / (omega + wsum);
-        if (j == 0 || fabsf(tb_new) > kTheta) {
-          delta = tb_new;
+        const float Tn = T + Tb, Wn = omega + wsum;  // Wn > 0: key 0 is visible to every row
+        if (j == 0 || fabsf(Tn) > kTheta * Wn) {
+          delta = Tn / Wn;
           cen += delta;
           T -= delta * omega;
           Tb -= delta * wsum;
@@ -691,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
           for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
             uint32_t o1[32], o2[32];
-            const uint32_t a1 = tmem + lane_addr + kColO1 + c0, a2 = tmem + lane_addr + kColO2 + c0;
+            const uint32_t a1 = sb + kColO1 + c0, a2 = sb + kColO2 + c0;
             tmem_ld32(a1, o1);
             tmem_ld32(a2, o2);
             tc_wait_ld();
@@ -704,8 +728,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(a1, o1);
             tmem_st32(a2, o2);
           }
-          tc_wait_st();
         }
+        // P buffer g % 2 is free: the scores of this block were issued only
+        // after the value MMAs of block g - 2 (its last reader) completed.
+        const uint32_t pb = sb + kColP + (g & 1) * kColPBuf;
+        tmem_st16(pb + 16 * hf, P);
         uint32_t PT[16];
         if (__any_sync(0xffffffffu, delta != 0.f)) {
           const uint64_t nd2 = f2(-delta, -delta);
@@ -721,10 +748,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) PT[c] = pack_bf16(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1]));
         }
-        tmem_st16(base + kColS2 + 16 * hf, PT);
+        tmem_st16(pb + kColPT + 16 * hf, PT);
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[s]);
+        mbar_arrive(&sm.p_full[g & 1]);
       }
       if (!ok) break;
       // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega, dims 64hf.. of this row.
