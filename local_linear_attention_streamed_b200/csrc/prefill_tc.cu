@@ -64,8 +64,13 @@ constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
 constexpr int kStages = 4;               // K/V ring depth
 constexpr int kTileRing = 4;             // tile indices in flight from producer to consumers
-constexpr int kThreads = 352;            // 11 warps: TMA, S MMA, 2 softmax warpgroups, PV MMA
-constexpr int kPVWarp = 10;
+// 12 warps in three warpgroups: {TMA, S MMA, PV MMA, idle} and two softmax
+// warpgroups.  The first gives registers to the other two (setmaxnreg):
+// 128 x 64 + 256 x 216 <= 384 x 168, the registers the block launched with.
+constexpr int kThreads = 384;
+constexpr int kPVWarp = 2;
+constexpr int kFirstSoftmaxWarp = 4;
+constexpr int kRegsControl = 64, kRegsSoftmax = 216;
 constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
 constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
@@ -96,12 +101,15 @@ struct Smem {
   // One full and one empty barrier per K/V stage: K and V of a block land
   // together, and the stage frees once that block's value MMAs completed.
   uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t s_full, s_free, p_full[2];
+  // Block g's scores complete on s_full[g % 2] (the barrier of the softmax
+  // warpgroup that owns the block); its P on p_full[g % 2].
+  uint64_t s_full[2], s_free, p_full[2];
   uint64_t o_full, o_empty, drain;
-  // Row-sum exchange between the two softmax warpgroups, double-buffered by
-  // epoch parity: one 64-bit word per slot holds (sum w, sum w (t - c)), with
-  // the sign bit of sum w (never negative) carrying the epoch tag.
-  unsigned long long xch[2][2][kBM];  // [epoch & 1][warpgroup][row]
+  // Row state handed from the owner of block g to the owner of block g + 1:
+  // (running max, centre, the poster's own sum w, its own sum w (t - c)) in
+  // the state after block g, and the flag holding the last posted g + 1.
+  float4 post[2][kBM];        // [poster's warpgroup][row]
+  uint32_t post_flag[2][kBM];
   // Tile indices handed from the producer to the MMA and softmax roles.
   int tile_ring[kTileRing];
   uint64_t tile_full[kTileRing], tile_empty[kTileRing];
@@ -144,9 +152,10 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Slow path of mbar_wait (kept out of line so that the common, already
-// complete case costs one try_wait and no call).
-__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+// Slow path of mbar_wait.  Inlined like every helper here: the kernel's
+// warpgroups run with different register budgets, and one out-of-line body
+// cannot serve all of them.
+__device__ __forceinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
                                             int* status) {
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
@@ -171,27 +180,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return mbar_wait_slow(bar, parity, abort, status);
 }
 
-// Pairwise exchange between the two threads that share a query row: each
-// posts one 64-bit word (a single-copy-atomic shared-memory access, so the
-// values and their tag arrive together) and polls the partner's word until
-// its tag matches the epoch (bounded in time).
-__device__ __forceinline__ void xch_post(unsigned long long* slot, unsigned long long v) {
-  asm volatile("st.volatile.shared::cta.u64 [%0], %1;" ::"r"(smem_u32(slot)), "l"(v) : "memory");
+// Row-state hand-off between the two softmax warpgroups: the poster writes
+// the values, then publishes its epoch with release semantics; the reader
+// takes the epoch with acquire semantics (bounded in time), then the values.
+__device__ __forceinline__ void flag_post(uint32_t* flag, uint32_t epoch) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(flag)), "r"(epoch) : "memory");
 }
-__device__ __forceinline__ unsigned long long xch_peek(const unsigned long long* slot) {
-  unsigned long long v;
-  asm volatile("ld.volatile.shared::cta.u64 %0, [%1];" : "=l"(v) : "r"(smem_u32(slot)) : "memory");
+__device__ __forceinline__ uint32_t flag_peek(const uint32_t* flag) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(flag)) : "memory");
   return v;
 }
-__device__ __noinline__ bool xch_await_slow(const unsigned long long* slot, uint32_t tag, unsigned long long* out,
-                                            volatile int* abort, int* status) {
+__device__ __forceinline__ bool flag_await_slow(const uint32_t* flag, uint32_t epoch, volatile int* abort,
+                                             int* status) {
   const unsigned long long t0 = now_ns();
   for (uint32_t it = 1;; ++it) {
-    const unsigned long long v = xch_peek(slot);
-    if ((uint32_t)(v >> 31 & 1u) == tag) {
-      *out = v;
-      return true;
-    }
+    if ((int)(flag_peek(flag) - epoch) >= 0) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
       if (now_ns() - t0 > kWaitNs) {
@@ -202,18 +206,14 @@ __device__ __noinline__ bool xch_await_slow(const unsigned long long* slot, uint
     }
   }
 }
-__device__ __forceinline__ bool xch_await(const unsigned long long* slot, uint32_t tag, unsigned long long* out,
-                                          volatile int* abort, int* status) {
-  const unsigned long long v = xch_peek(slot);
-  if ((uint32_t)(v >> 31 & 1u) == tag) {
-    *out = v;
-    return true;
-  }
-  return xch_await_slow(slot, tag, out, abort, status);
+__device__ __forceinline__ bool flag_await(const uint32_t* flag, uint32_t epoch, volatile int* abort,
+                                           int* status) {
+  if ((int)(flag_peek(flag) - epoch) >= 0) return true;
+  return flag_await_slow(flag, epoch, abort, status);
 }
 
 // Bounded wait used only on the way out (ignores the abort flag).
-__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = now_ns();
   while (!mbar_test(bar, parity) && now_ns() - t0 < kWaitNs) {
   }
@@ -280,6 +280,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
         "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]),
         "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]),
         "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
 }
 
@@ -390,10 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tiles = ntile * BH;
   volatile int* abort = &sm.abort;
 
-  // Slot 1 is first used by epoch 1 (tag 0) and slot 0 by epoch 2 (tag 1):
-  // start each with the other tag.
-  for (int x = threadIdx.x; x < 2 * 2 * kBM; x += blockDim.x)
-    (&sm.xch[0][0][0])[x] = x < 2 * kBM ? 0ull : 0x80000000ull;
+  for (int x = threadIdx.x; x < 2 * kBM; x += blockDim.x) (&sm.post_flag[0][0])[x] = 0u;
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
@@ -401,9 +406,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_free, 8);  // one lane of each softmax warp
-    for (int s = 0; s < 2; ++s) mbar_init(&sm.p_full[s], 256);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.p_full[s], 128);  // the owning warpgroup's threads
+    }
+    mbar_init(&sm.s_free, 4);  // one lane of each warp of the owning warpgroup
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(&sm.tile_full[s], 1);
       mbar_init(&sm.tile_empty[s], 10);  // the two MMA threads and one lane of each softmax warp
@@ -425,6 +432,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
+  if (warp < kFirstSoftmaxWarp) {
+  // The control warpgroup hands registers to the softmax warpgroups.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -496,16 +506,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
-          // The S stage is free once the softmax has read the previous block's
-          // scores; P buffer g % 2, which the softmax fills once these scores
-          // land, is free once the value MMAs of block g - 2 completed.
-          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
+          // P buffer g % 2, which the softmax fills once these scores land, is
+          // free once the value MMAs of block g - 2 completed; the S stage is
+          // free once the softmax has read the previous block's scores.  That
+          // last wait is the one on the critical path, so it comes last.
           if (g > 1) {
             const uint32_t gq = g - 2;
             if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
           }
           const uint32_t st = g % kStages;
           if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
+          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
           tc_fence_after();
           const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
           // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
@@ -518,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ss(tmem + kColS1, dQ + off, dk + koff, kIdescS, ks > 0);
             mma_ss(tmem + kColS2, dR + off, dk + koff, kIdescS, ks > 0);
           }
-          mma_commit(&sm.s_full);
+          mma_commit(&sm.s_full[g & 1]);
           if (j + 1 == ti.nblk) mma_commit(&sm.q_empty);
         }
       }
@@ -569,18 +580,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
+  }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // ---------------- softmax / epilogue: two warpgroups ----------------
-    // Warpgroup hf (warps 2..5 -> 0, 6..9 -> 1) owns keys 32hf..32hf+31 of every
-    // block and output dims 64hf..64hf+63; both threads of a row take the max
-    // over all 64 scores of a block and exchange their partial sums through
-    // shared memory, so both keep identical copies of the row state
-    // (m, omega, T, c).
-    const int hf = (warp - 2) >> 2;
+    // Warpgroup wg owns the blocks g with g % 2 == wg: each thread takes the
+    // whole 64-key row of its query (TMEM lane) for those blocks, while the
+    // other warpgroup works on the neighbouring blocks.  The row state passes
+    // from block to block through a post per block: the lazy max m and the
+    // centre c are the same for both warpgroups, and each keeps its own sums
+    // (omega, T) in that state.  The epilogue writes output dims 64wg..64wg+63.
+    const int wg = (warp - kFirstSoftmaxWarp) >> 2;
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
-    const uint32_t lane_addr = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t sb = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     const float scale = 1.4426950408889634f * rsqrtf((float)kD);
-    uint32_t g = 0;  // blocks processed by this CTA (also the exchange epoch)
+    uint32_t gb = 0;  // the CTA's block counter at the current tile's first block
     int tc = 0;
     bool ok = true;
     for (; ok; ++tc) {
@@ -591,68 +605,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&sm.tile_empty[slot]);
       if (t < 0) break;
       const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
-      const int i = ti.m * kBM + row;  // query position
-      // Row state: running max (log2 units), omega = sum w, T = sum w (t - c)
-      // around the row's centre c (see the file comment), all in fp32.
-      float m_run = -CUDART_INF_F, omega = 0.f, T = 0.f, cen = 0.f;
-      for (int j = 0; j < ti.nblk; ++j, ++g) {
-        if (!(ok = mbar_wait(&sm.s_full, g & 1, abort, p.status))) break;
+      const int i = ti.m * kBM + row;                      // query position
+      const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
+      // Row state: running max (log2 units) and centre c (shared), this
+      // warpgroup's omega = sum w and T = sum w (t - c), and the other
+      // warpgroup's sums as last posted (brought to the current state).
+      float m_run = -CUDART_INF_F, cen = 0.f, omega = 0.f, T = 0.f, om_o = 0.f, T_o = 0.f;
+      // Brings this warpgroup's sums from its copy of the state to a posted one
+      // (the max only rises; a raise rescales, then the centre moves).
+      auto adopt = [&](const float4 ps) {
+        if (ps.x > m_run) {
+          const float a = ex2(m_run - ps.x);  // 0 while m_run = -inf
+          omega *= a;
+          T *= a;
+          m_run = ps.x;
+        }
+        T -= (ps.y - cen) * omega;
+        cen = ps.y;
+      };
+      for (int j = ((gb & 1u) == (uint32_t)wg) ? 0 : 1; j < ti.nblk; j += 2) {
+        const uint32_t g = gb + j;
+        if (!(ok = mbar_wait(&sm.s_full[wg], (g >> 1) & 1, abort, p.status))) break;
         tc_fence_after();
-        const uint32_t sb = tmem + lane_addr;
         const int kb = j * kBN;
-        const bool edge = (p.causal && kb + kBN - 1 > ti.m * kBM) || (kb + kBN > p.N);
-        const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
-        uint32_t x[32], y[32];
+        uint32_t x[64], y[64];
+        tmem_ld32(sb + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+        tmem_ld32(sb + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+        tmem_ld32(sb + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
+        tmem_ld32(sb + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free);  // the S stage goes back to the MMA
+        if ((p.causal && kb + kBN - 1 > ti.m * kBM) || kb + kBN > p.N) {
+          // Block-uniform: only blocks that cross the diagonal or the end.
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (kb + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+        }
         float rmax;
         {
-          // This thread's 32 scores and t values, and the partner half of the
-          // scores for the row max; then the S stage is handed back to the MMA.
-          uint32_t z[32];
-          tmem_ld32(sb + kColS1 + 32 * hf, x);
-          tmem_ld32(sb + kColS1 + 32 * (hf ^ 1), z);
-          tmem_ld32(sb + kColS2 + 32 * hf, y);
-          tc_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free);
-          if (edge) {  // block-uniform: only blocks that cross the diagonal or the end
-            const int k0 = kb + 32 * hf, kz = kb + 32 * (hf ^ 1);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              if (k0 + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
-              if (kz + c >= kend) z[c] = __float_as_uint(-CUDART_INF_F);
-            }
-          }
-          // Four independent chains over the 64 scores, then their max.
           float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            m4[0] = max3(m4[0], __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
-            m4[1] = max3(m4[1], __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
-            m4[2] = max3(m4[2], __uint_as_float(z[c]), __uint_as_float(z[c + 1]));
-            m4[3] = max3(m4[3], __uint_as_float(z[c + 2]), __uint_as_float(z[c + 3]));
+          for (int c = 0; c < 64; c += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              m4[q] = max3(m4[q], __uint_as_float(x[c + 2 * q]), __uint_as_float(x[c + 2 * q + 1]));
           }
           rmax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
         }
-        // Both halves of the row took the max of the same 64 scores, so the
-        // raise decision below is the same on both sides.
+        // The state after block g - 1 (the other warpgroup's), except on the
+        // tile's first block.
+        if (j > 0) {
+          if (!(ok = flag_await(&sm.post_flag[wg ^ 1][row], g, abort, p.status))) break;
+          const float4 ps = sm.post[wg ^ 1][row];
+          adopt(ps);
+          om_o = ps.z;
+          T_o = ps.w;
+        }
+        // Raise the max by more than 2^8 only (always on a tile's first block).
         const float mx = rmax * scale;
         float alpha = 1.f;
-        if (mx > m_run + kLazyTau) {  // always on a tile's first block (m_run = -inf)
-          alpha = ex2(m_run - mx);    // 0 on the first block
+        if (mx > m_run + kLazyTau) {
+          alpha = ex2(m_run - mx);  // 0 on the first block
           m_run = mx;
           omega *= alpha;
           T *= alpha;
+          om_o *= alpha;
+          T_o *= alpha;
         }
-        // w = 2^(s*scale - m_run); a = w (t - c) is kept for bf16(w (t - c))
-        // once the centre is settled.  x <- w, y <- a.
-        uint32_t P[16];
-        float wpart, tpart;
+        // w = 2^(s*scale - m_run), a = w (t - c).  x <- w, y <- a.
+        float wb, tb;
         {
           const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
           uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
+          for (int c = 0; c < 32; ++c) {
             float s0, s1;
             uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), sc2, nm2), s0, s1);
             const float w0 = ex2(s0), w1 = ex2(s1);
@@ -665,7 +693,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               ws2a = add2(ws2a, w2);
               ts2a = add2(ts2a, a2);
             }
-            P[c] = pack_bf16(w0, w1);
             float a0, a1;
             uf2(a2, a0, a1);
             x[2 * c] = __float_as_uint(w0);
@@ -675,96 +702,107 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           float lo, hi;
           uf2(add2(ws2a, ws2b), lo, hi);
-          wpart = lo + hi;
+          wb = lo + hi;
           uf2(add2(ts2a, ts2b), lo, hi);
-          tpart = lo + hi;
+          tb = lo + hi;
         }
-        // Exchange (sum w, sum w (t - c)) with the partner thread of this row.
-        const uint32_t e0 = g + 1, tag = (e0 >> 1) & 1u;
-        xch_post(&sm.xch[e0 & 1][hf][row],
-                 (unsigned long long)__float_as_uint(tpart) << 32 | __float_as_uint(wpart) | tag << 31);
-        unsigned long long theirs;
-        if (!(ok = xch_await(&sm.xch[e0 & 1][hf ^ 1][row], tag, &theirs, abort, p.status))) break;
-        // Both threads of the row form the same sums (a + b == b + a exactly).
-        const float wsum = wpart + __uint_as_float((uint32_t)theirs & 0x7FFFFFFFu);
-        float Tb = tpart + __uint_as_float((uint32_t)(theirs >> 32));
         // Re-centre before this block's w (t - c) is rounded to bf16, on the
-        // first block and whenever the running mean of t has drifted by more
-        // than kTheta from the centre.
+        // first block and whenever the running mean of t - c (both warpgroups'
+        // sums through this block) has drifted by more than kTheta.
         float delta = 0.f;
-        const float Tn = T + Tb, Wn = omega + wsum;  // Wn > 0: key 0 is visible to every row
-        if (j == 0 || fabsf(Tn) > kTheta * Wn) {
-          delta = Tn / Wn;
-          cen += delta;
-          T -= delta * omega;
-          Tb -= delta * wsum;
+        {
+          const float Tn = (T + T_o) + tb, Wn = (omega + om_o) + wb;  // Wn > 0: key 0 is visible
+          if (j == 0 || fabsf(Tn) > kTheta * Wn) {
+            const float cn = cen + Tn / Wn;
+            delta = cn - cen;  // the shift as represented
+            cen = cn;
+            T -= delta * omega;
+            T_o -= delta * om_o;
+            tb -= delta * wb;
+          }
         }
-        omega += wsum;
-        T += Tb;
-        // Rows whose max rose or whose centre moved update their part of O1 and
-        // O2 (O1 <- alpha O1, O2 <- alpha (O2 - delta O1)) once the value MMAs
-        // of the previous block are complete; each warpgroup updates its 64 dims.
-        const bool need = (j > 0) && (alpha != 1.f || delta != 0.f);
-        if (__any_sync(0xffffffffu, need)) {
-          // The previous block's value MMAs completed when its K/V stage was freed
-          // (block counter g equals the K/V ring position).
+        omega += wb;
+        T += tb;
+        // Hand the state after this block to the owner of block g + 1.
+        sm.post[wg][row] = make_float4(m_run, cen, omega, T);
+        flag_post(&sm.post_flag[wg][row], g + 1);
+        // Rows whose max rose or whose centre moved update O1 and O2 (all 128
+        // dims: O1 <- alpha O1, O2 <- alpha (O2 - delta O1)) once the value MMAs
+        // of block g - 1 are complete.
+        if (__any_sync(0xffffffffu, j > 0 && (alpha != 1.f || delta != 0.f))) {
+          // The value MMAs of block g - 1 completed when its K/V stage was freed
+          // (the block counter equals the K/V ring position).
           const uint32_t gp = g - 1;
           if (!(ok = mbar_wait(&sm.kv_empty[gp % kStages], (gp / kStages) & 1, abort, p.status))) break;
           tc_fence_after();
           const float ad = alpha * delta;
 #pragma unroll 1
-          for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
-            uint32_t o1[32], o2[32];
+          for (int c0 = 0; c0 < kD; c0 += 16) {
+            uint32_t o1[16], o2[16];
             const uint32_t a1 = sb + kColO1 + c0, a2 = sb + kColO2 + c0;
-            tmem_ld32(a1, o1);
-            tmem_ld32(a2, o2);
+            tmem_ld16(a1, o1);
+            tmem_ld16(a2, o2);
             tc_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 16; ++c) {
               const float v1 = __uint_as_float(o1[c]);
               o2[c] = __float_as_uint(alpha * __uint_as_float(o2[c]) - ad * v1);
               o1[c] = __float_as_uint(alpha * v1);
             }
-            tmem_st32(a1, o1);
-            tmem_st32(a2, o2);
+            tmem_st16(a1, o1);
+            tmem_st16(a2, o2);
+            tc_wait_st();
           }
         }
-        // P buffer g % 2 is free: the scores of this block were issued only
-        // after the value MMAs of block g - 2 (its last reader) completed.
-        const uint32_t pb = sb + kColP + (g & 1) * kColPBuf;
-        tmem_st16(pb + 16 * hf, P);
-        uint32_t PT[16];
-        if (__any_sync(0xffffffffu, delta != 0.f)) {
-          const uint64_t nd2 = f2(-delta, -delta);
+        // P buffer wg (= g % 2) is free: the scores of this block were issued
+        // only after the value MMAs of block g - 2 (its last reader) completed.
+        const uint32_t pb = sb + kColP + (uint32_t)wg * kColPBuf;
+        // bf16(w (t - c)) is a - delta w with the centre settled above.
+        const bool moved = __any_sync(0xffffffffu, delta != 0.f);
+        const uint64_t nd2 = f2(-delta, -delta);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t P[16], PT[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            float a0, a1;
-            uf2(fma2(f2(__uint_as_float(x[2 * c]), __uint_as_float(x[2 * c + 1])), nd2,
-                     f2(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1]))),
-                a0, a1);
+            const int e = 32 * h + 2 * c;
+            P[c] = pack_bf16(__uint_as_float(x[e]), __uint_as_float(x[e + 1]));
+            float a0 = __uint_as_float(y[e]), a1 = __uint_as_float(y[e + 1]);
+            if (moved) uf2(fma2(f2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), nd2, f2(a0, a1)), a0, a1);
             PT[c] = pack_bf16(a0, a1);
           }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 16; ++c) PT[c] = pack_bf16(__uint_as_float(y[2 * c]), __uint_as_float(y[2 * c + 1]));
+          tmem_st16(pb + 16 * h, P);
+          tmem_st16(pb + kColPT + 16 * h, PT);
         }
-        tmem_st16(pb + kColPT + 16 * hf, PT);
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&sm.p_full[g & 1]);
+        mbar_arrive(&sm.p_full[wg]);
       }
       if (!ok) break;
-      // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega, dims 64hf.. of this row.
+      // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega, dims 64wg.. of this row,
+      // with omega and T the sums of both warpgroups in the final state.
+      const int jl = ti.nblk - 1;
+      if (((gb + jl) & 1u) == (uint32_t)wg) {
+        omega += om_o;  // this warpgroup owned the last block
+        T += T_o;
+      } else {
+        if (!(ok = flag_await(&sm.post_flag[wg ^ 1][row], gb + jl + 1, abort, p.status))) break;
+        const float4 ps = sm.post[wg ^ 1][row];
+        adopt(ps);
+        omega += ps.z;
+        T += ps.w;
+      }
+      gb += ti.nblk;
       if (!(ok = mbar_wait(&sm.o_full, tc & 1, abort, p.status))) break;
       tc_fence_after();
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
       __nv_bfloat16* orow = p.out + ((long long)ti.bh * p.N + i) * kD;
 #pragma unroll 1
-      for (int c0 = 64 * hf; c0 < 64 * hf + 64; c0 += 32) {
+      for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 32) {
         uint32_t o1[32], o2[32];
-        tmem_ld32(tmem + lane_addr + kColO1 + c0, o1);
-        tmem_ld32(tmem + lane_addr + kColO2 + c0, o2);
+        tmem_ld32(sb + kColO1 + c0, o1);
+        tmem_ld32(sb + kColO2 + c0, o2);
         tc_wait_ld();
         if (i < p.N) {
           uint32_t packed[16];
