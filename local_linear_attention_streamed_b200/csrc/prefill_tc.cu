@@ -66,11 +66,11 @@ constexpr int kStages = 4;               // K/V ring depth
 constexpr int kTileRing = 4;             // tile indices in flight from producer to consumers
 // 12 warps in three warpgroups: {TMA, S MMA, PV MMA, idle} and two softmax
 // warpgroups.  The first gives registers to the other two (setmaxnreg):
-// 128 x 64 + 256 x 216 <= 384 x 168, the registers the block launched with.
+// 128 x 72 + 256 x 216 = 384 x 168, the registers the block launched with.
 constexpr int kThreads = 384;
 constexpr int kPVWarp = 2;
 constexpr int kFirstSoftmaxWarp = 4;
-constexpr int kRegsControl = 64, kRegsSoftmax = 216;
+constexpr int kRegsControl = 72, kRegsSoftmax = 216;
 constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
 constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
@@ -112,6 +112,7 @@ struct Smem {
   uint32_t post_flag[2][kBM];
   // Tile indices handed from the producer to the MMA and softmax roles.
   int tile_ring[kTileRing];
+  uint32_t s_issued;  // blocks whose scores were issued (all ones: no more)
   uint64_t tile_full[kTileRing], tile_empty[kTileRing];
   uint32_t tmem_base;
   int abort;
@@ -413,11 +414,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.s_free, 4);  // one lane of each warp of the owning warpgroup
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(&sm.tile_full[s], 1);
-      mbar_init(&sm.tile_empty[s], 10);  // the two MMA threads and one lane of each softmax warp
+      mbar_init(&sm.tile_empty[s], 10);  // both MMA threads and one lane of each softmax warp
     }
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, 256);
     mbar_init(&sm.drain, 2);  // one commit from each MMA thread
+    sm.s_issued = 0;
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -492,10 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tc = 0;
       const uint64_t dQ = sdesc(smem_u32(sm.q), 16, 1024), dR = sdesc(smem_u32(sm.r), 16, 1024);
       const uint64_t dK0 = sdesc(smem_u32(sm.k[0]), 16, 1024);
-      // Each issuing thread shares its scheduler with two softmax warps, so
-      // every MMA is issued from descriptors built once: a k-step or a stage
-      // only adds a compile-time offset to the start-address field (smem
-      // addresses < 256 KB keep that 14-bit field from carrying).
       bool ok = true;
       for (; ok; ++tc) {
         const int slot = tc % kTileRing;
@@ -506,22 +504,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
-          // P buffer g % 2, which the softmax fills once these scores land, is
-          // free once the value MMAs of block g - 2 completed; the S stage is
-          // free once the softmax has read the previous block's scores.  That
-          // last wait is the one on the critical path, so it comes last.
-          if (g > 1) {
-            const uint32_t gq = g - 2;
-            if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
-          }
+          // The S stage is free once the softmax has read the previous block's
+          // scores (the wait on the critical path, so it comes first).
+          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
           const uint32_t st = g % kStages;
           if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
-          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
           tc_fence_after();
           const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
-          // S1 and S2 k-steps interleaved: on this per-block sequence that keeps
-          // the tensor pipe at the sum of the two GEMMs (issuing all of S1 and
-          // then all of S2 measured about a quarter slower).
+          // S1 and S2 k-steps interleaved (one B tile feeds both GEMMs); every
+          // MMA comes from the descriptors built once plus a compile-time
+          // offset in the start-address field (shared-memory addresses
+          // < 256 KB keep that 14-bit field from carrying).
 #pragma unroll
           for (int ks = 0; ks < kD / 16; ++ks) {
             const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
@@ -531,14 +524,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&sm.s_full[g & 1]);
           if (j + 1 == ti.nblk) mma_commit(&sm.q_empty);
+          *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) = g + 1;
         }
       }
-      // Drain: all MMAs this thread issued complete before TMEM is freed.
+      // No more scores: the value issuer stops waiting for them.
+      *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) = 0xFFFFFFFFu;
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
   } else if (warp == kPVWarp) {
     // ---------------- value MMA issuer ----------------
+    // The scores of the next blocks are the critical path (the single S stage
+    // frees only when the softmax has loaded the previous block), so the
+    // value MMAs of block k go into the tensor pipe only behind the scores of
+    // block k + 2: issuing stalls while the pipe is full, so issue order is
+    // the order the pipe works in.  (The scores never wait on these values:
+    // the softmax waits for block k's before it overwrites P buffer k % 2.)
     if (lane == 0) {
       uint32_t g = 0;
       int tc = 0;
@@ -556,9 +557,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tc > 0 && !(ok = mbar_wait(&sm.o_empty, (tc - 1) & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
           const uint32_t b = g & 1;
-          // P of this block is in TMEM; its scores (so its K) were consumed
-          // before, and V arrived with K.
           if (!(ok = mbar_wait(&sm.p_full[b], (g >> 1) & 1, abort, p.status))) break;
+          // Behind the scores of block g + 2 (bounded in time like every wait).
+          if ((int)(*reinterpret_cast<volatile uint32_t*>(&sm.s_issued) - (g + 3)) < 0) {
+            const unsigned long long t0 = now_ns();
+            while ((int)(*reinterpret_cast<volatile uint32_t*>(&sm.s_issued) - (g + 3)) < 0 &&
+                   *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) != 0xFFFFFFFFu) {
+              if (*abort) {
+                ok = false;
+                break;
+              }
+              if (now_ns() - t0 > kWaitNs) {
+                *abort = 1;
+                atomicOr(p.status, kStatusTimeout);
+                ok = false;
+                break;
+              }
+              __nanosleep(32);
+            }
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t st = g % kStages;
           const uint64_t dv = dV0 + (uint64_t)(st * (kKVBytes >> 4));
@@ -577,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mma_commit(&sm.o_full);
       }
+      // Drain: all MMAs this thread issued complete before TMEM is freed.
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
@@ -597,13 +616,52 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t gb = 0;  // the CTA's block counter at the current tile's first block
     int tc = 0;
     bool ok = true;
+    // The epilogue out = ((1 + T/omega) O1 - O2) / omega for dims 64wg.. of one
+    // row of tile etc: inv = 1/omega, c1 = (1 + T/omega)/omega.
+    auto epilogue = [&](int etc, __nv_bfloat16* orow, float inv, float c1) -> bool {
+      if (!mbar_wait(&sm.o_full, etc & 1, abort, p.status)) return false;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 32) {
+        uint32_t o1[32], o2[32];
+        tmem_ld32(sb + kColO1 + c0, o1);
+        tmem_ld32(sb + kColO2 + c0, o2);
+        tc_wait_ld();
+        if (orow != nullptr) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float v0 = c1 * __uint_as_float(o1[2 * c]) - inv * __uint_as_float(o2[2 * c]);
+            const float v1 = c1 * __uint_as_float(o1[2 * c + 1]) - inv * __uint_as_float(o2[2 * c + 1]);
+            packed[c] = pack_bf16(v0, v1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.o_empty);
+      return true;
+    };
+    // The warpgroup that did not own a tile's last block defers that tile's
+    // epilogue until it has handled its first block of the next tile (its own
+    // by parity), so the scores keep flowing across the tile boundary.
+    bool epi_pending = false;
+    int epi_tc = 0;
+    __nv_bfloat16* epi_row = nullptr;
+    float epi_inv = 0.f, epi_c1 = 0.f;
     for (; ok; ++tc) {
       const int slot = tc % kTileRing;
       if (!(ok = mbar_wait(&sm.tile_full[slot], (tc / kTileRing) & 1, abort, p.status))) break;
       const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.tile_empty[slot]);
-      if (t < 0) break;
+      if (t < 0) {
+        if (epi_pending) ok = epilogue(epi_tc, epi_row, epi_inv, epi_c1);
+        break;
+      }
       const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
       const int i = ti.m * kBM + row;                      // query position
       const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
@@ -754,8 +812,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_wait_st();
           }
         }
-        // P buffer wg (= g % 2) is free: the scores of this block were issued
-        // only after the value MMAs of block g - 2 (its last reader) completed.
+        // P buffer wg (= g % 2) is free once the value MMAs of block g - 2, its
+        // last reader, completed (the MMA issuer runs them after the scores).
+        if (g >= 2) {
+          const uint32_t gq = g - 2;
+          if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
+          tc_fence_after();
+        }
         const uint32_t pb = sb + kColP + (uint32_t)wg * kColPBuf;
         // bf16(w (t - c)) is a - delta w with the centre settled above.
         const bool moved = __any_sync(0xffffffffu, delta != 0.f);
@@ -777,8 +840,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[wg]);
+        if (epi_pending) {
+          if (!(ok = epilogue(epi_tc, epi_row, epi_inv, epi_c1))) break;
+          epi_pending = false;
+        }
       }
       if (!ok) break;
+      if (epi_pending) {  // not reached: a pending epilogue's next tile starts with this warpgroup
+        if (!(ok = epilogue(epi_tc, epi_row, epi_inv, epi_c1))) break;
+        epi_pending = false;
+      }
       // ---- epilogue: out = ((1 + T/omega) O1 - O2) / omega, dims 64wg.. of this row,
       // with omega and T the sums of both warpgroups in the final state.
       const int jl = ti.nblk - 1;
@@ -792,34 +863,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         omega += ps.z;
         T += ps.w;
       }
+      const bool owner_last = ((gb + ti.nblk - 1) & 1u) == (uint32_t)wg;
       gb += ti.nblk;
-      if (!(ok = mbar_wait(&sm.o_full, tc & 1, abort, p.status))) break;
-      tc_fence_after();
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
-      __nv_bfloat16* orow = p.out + ((long long)ti.bh * p.N + i) * kD;
-#pragma unroll 1
-      for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 32) {
-        uint32_t o1[32], o2[32];
-        tmem_ld32(sb + kColO1 + c0, o1);
-        tmem_ld32(sb + kColO2 + c0, o2);
-        tc_wait_ld();
-        if (i < p.N) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float v0 = c1 * __uint_as_float(o1[2 * c]) - inv * __uint_as_float(o2[2 * c]);
-            const float v1 = c1 * __uint_as_float(o1[2 * c + 1]) - inv * __uint_as_float(o2[2 * c + 1]);
-            packed[c] = pack_bf16(v0, v1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-        }
+      __nv_bfloat16* orow = i < p.N ? p.out + ((long long)ti.bh * p.N + i) * kD : nullptr;
+      if (owner_last) {
+        if (!(ok = epilogue(tc, orow, inv, c1))) break;
+      } else {
+        epi_pending = true;
+        epi_tc = tc;
+        epi_row = orow;
+        epi_inv = inv;
+        epi_c1 = c1;
       }
-      tc_fence_before();
-      mbar_arrive(&sm.o_empty);
     }
   }
   tc_fence_before();
