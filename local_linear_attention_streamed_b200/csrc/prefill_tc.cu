@@ -504,11 +504,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
-          // The S stage is free once the softmax has read the previous block's
-          // scores (the wait on the critical path, so it comes first).
-          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
+          // K of this block (long resident: checked first), then the S stage,
+          // free once the softmax has read the previous block's scores: the
+          // wait on the critical path comes last, right before the issue.
           const uint32_t st = g % kStages;
           if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
+          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
           tc_fence_after();
           const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
           // S1 and S2 k-steps interleaved (one B tile feeds both GEMMs); every
