@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 METRIC = "decode KV GB/s (% HBM peak); causal prefill TFLOP/s (% BF16 peak)"
 DECODE = dict(B=64, H=16, L=4096, d=128)
 PREFILL = dict(B=8, H=16, N=4096, d=128)
+L2_BYTES = 126 * 1024 * 1024  # B200 L2
 LAYER = dict(B=4, N=8192, D=2048, H=16)
 SWEEP_B = [1, 8, 64, 256, 1024, 2048]
 SWEEP_L = [128, 1024, 4096, 16384, 32768]
@@ -231,7 +232,9 @@ def run_gpu(args, rank, world, dist):
     src_hash = kernel_hash("decode_mma.cu")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic_from_profile("decode_bf16_B64_H16_L4096.json", src_hash),
+                # The committed capture is of the default workload; other sizes report none.
+                "traffic": (traffic_from_profile("decode_bf16_B64_H16_L4096.json", src_hash)
+                            if B == DECODE["B"] else None),
                 "peak_source": peak_src, "kernel": "decode_bf16_kernel<128>",
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "frac_of_spec_8000": round(achieved / 8000.0, 4)}
@@ -294,12 +297,14 @@ def run_gpu(args, rank, world, dist):
             "value": round(sum_over_ranks(flops * psteps, dist) / (p_total * 1e-3) / 1e12, 2),
             "ms_per_step": round(p_total / psteps, 3), "steps": psteps,
             "config": {"workload": f"causal prefill B={pB} H=16 N=4096 d=128 bf16",
-                       "l2": "inputs 512 MB, larger than L2"},
+                       "l2": f"inputs {4 * pB * 16 * 4096 * 128 * 2 >> 20} MB"
+                             + (", larger than L2" if 4 * pB * 16 * 4096 * 128 * 2 > L2_BYTES else "")},
             "roofline": {"bound": "tensor", "achieved": round(p_ach, 1), "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": round(p_ach / peaks["bf16_tflops"], 4),
                          "frac_of_sustained": round(p_ach / peaks["bf16_tflops_sustained"], 4),
-                         "traffic": traffic_from_profile("prefill_B8_H16_N4096.json",
-                                                         kernel_hash("prefill_tc.cu", "simt.cu")),
+                         "traffic": (traffic_from_profile("prefill_B8_H16_N4096.json",
+                                                          kernel_hash("prefill_tc.cu", "simt.cu"))
+                                     if pB == PREFILL["B"] else None),
                          "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
             "gpu_launches": psteps,
         }
