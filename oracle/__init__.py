@@ -4,8 +4,8 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 leg may import this package.  The CUDA library never calls it, and it never
 calls the CUDA library.
 """
-from .parallax import decode_ref, parallax_row, prefill_ref, softmax_weights_row
+from .parallax import decode_gqa_ref, decode_ref, parallax_row, prefill_ref, softmax_weights_row
 from .layer import layer_rows_ref, qkr_norm_rope_ref, rmsnorm, rope
 
-__all__ = ["parallax_row", "prefill_ref", "decode_ref", "softmax_weights_row",
+__all__ = ["parallax_row", "prefill_ref", "decode_ref", "decode_gqa_ref", "softmax_weights_row",
            "layer_rows_ref", "qkr_norm_rope_ref", "rmsnorm", "rope"]

@@ -109,6 +109,34 @@ def decode_ref(q, r, Kc, Vc, seqlens, units=None) -> np.ndarray:
     return out.reshape(B, H, d) if full else out
 
 
+def decode_gqa_ref(q, r, Kc, Vc, seqlens, units=None) -> np.ndarray:
+    """Oracle for one decode step with grouped KV heads.
+
+    q, r: [B, H, d]; Kc, Vc: [B, Hkv, L, d] with H a multiple of Hkv; query
+    head h reads KV head h // (H // Hkv) (consecutive query heads share a KV
+    head).  The pages name grouping only as the place where packing the q and
+    rho rows of many heads into one tensor-core tile pays; each head's output
+    is the plain per-query definition over its group's keys.  ``units`` is
+    None (all (b, h)) or a list of (b, h) query heads.
+    """
+    B, H, d = q.shape
+    Hkv = Kc.shape[1]
+    assert H % Hkv == 0
+    G = H // Hkv
+    if units is None:
+        units = [(b, h) for b in range(B) for h in range(H)]
+        full = True
+    else:
+        full = False
+    res = []
+    for (b, h) in units:
+        n = int(seqlens[b])
+        kv = h // G
+        res.append(parallax_row(q[b, h], r[b, h], Kc[b, kv, :n], Vc[b, kv, :n]))
+    out = np.stack(res)
+    return out.reshape(B, H, d) if full else out
+
+
 def softmax_weights_row(q, K) -> np.ndarray:
     """p_j for one query (exposed for the invariant tests on s_ij)."""
     q = np.asarray(q, dtype=np.float64)

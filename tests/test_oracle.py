@@ -29,7 +29,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import decode_ref, parallax_row, prefill_ref
+from oracle import decode_gqa_ref, decode_ref, parallax_row, prefill_ref
 from oracle import layer as olayer
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_examples.json")
@@ -339,6 +339,36 @@ def test_prefill_and_decode_conventions():
                      K, V, seqlens)
     for b in range(B):
         np.testing.assert_allclose(dec[b], full[b, :, seqlens[b] - 1], rtol=0, atol=1e-14)
+
+
+def test_decode_gqa_pins():
+    """Grouped KV heads: query head h reads KV head h // G.
+
+    Pinned to the MHA oracle on the KV heads repeated G times (np.repeat puts
+    the copies of one KV head next to each other), which a head map of
+    h % Hkv would fail; G = 1 is the MHA oracle itself; heads of one group
+    with equal q and rho give equal outputs.
+    """
+    rng = _rng(21)
+    B, Hkv, G, L, d = 2, 3, 4, 11, 8
+    H = Hkv * G
+    q = rng.standard_normal((B, H, d))
+    r = 0.3 * rng.standard_normal((B, H, d))
+    Kc, Vc = rng.standard_normal((B, Hkv, L, d)), rng.standard_normal((B, Hkv, L, d))
+    seqlens = np.array([7, 11])
+    got = decode_gqa_ref(q, r, Kc, Vc, seqlens)
+    want = decode_ref(q, r, np.repeat(Kc, G, axis=1), np.repeat(Vc, G, axis=1), seqlens)
+    np.testing.assert_allclose(got, want, rtol=0, atol=0)
+    wrong = decode_ref(q, r, np.tile(Kc, (1, G, 1, 1)), np.tile(Vc, (1, G, 1, 1)), seqlens)
+    assert np.abs(got - wrong).max() > 1e-3
+    np.testing.assert_allclose(decode_gqa_ref(q[:, :Hkv], r[:, :Hkv], Kc, Vc, seqlens),
+                               decode_ref(q[:, :Hkv], r[:, :Hkv], Kc, Vc, seqlens), rtol=0, atol=0)
+    q2, r2 = q.copy(), r.copy()
+    q2[:, 5], r2[:, 5] = q2[:, 4], r2[:, 4]  # heads 4 and 5 share KV head 1
+    same = decode_gqa_ref(q2, r2, Kc, Vc, seqlens)
+    np.testing.assert_allclose(same[:, 5], same[:, 4], rtol=0, atol=0)
+    picked = decode_gqa_ref(q, r, Kc, Vc, seqlens, units=[(1, 7), (0, 0)])
+    np.testing.assert_allclose(picked, np.stack([got[1, 7], got[0, 0]]), rtol=0, atol=0)
 
 
 # ---------------------------------------------------------------------------
