@@ -113,6 +113,33 @@ size_t plx_decode_workspace_bytes(int B, int H, int L, int d);
 int plx_decode_num_splits(int B, int H, int L, int d);
 
 /*
+ * One bf16 decode step with grouped KV heads: H query heads share Hkv KV heads,
+ * query head h reading KV head h / (H / Hkv) (consecutive query heads form a
+ * group).  The pages' decode packs the q and rho rows into one tensor-core tile
+ * so that one stream of K serves both score products (agihunt.info summary,
+ * decode paragraph); here that tile carries the rows of every head of a group,
+ * so each KV head's cache is read once per step.
+ *
+ * q, r, out: [B, H, d] bf16; Kcache, Vcache: [B, Hkv, L, d] bf16; seqlens:
+ * int32 [B] as for plx_decode (the query of sequence b sees keys
+ * 0..seqlens[b]-1; an entry outside 1..L writes zeros for that sequence and
+ * reports PLX_ERR_BAD_SEQLEN through plx_get_device_status).  d in {64, 128};
+ * H / Hkv in {1, 2, 4, 8} (1 is plx_decode_ex itself), else
+ * PLX_ERR_UNSUPPORTED; H not a multiple of Hkv gives PLX_ERR_INVALID_ARG.
+ * workspace: NULL (library-owned) or at least
+ * plx_decode_gqa_workspace_bytes(B, H, Hkv, L, d) bytes, 256-byte aligned; the
+ * arrival counters are the same library-owned per-device array as
+ * plx_decode_ex's, so decode calls on one device must be ordered.  Pointers
+ * 16-byte aligned (seqlens 4-byte), else PLX_ERR_MISALIGNED.
+ */
+int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                   const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace plx_decode_gqa needs for these sizes (0 if none is needed). */
+size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d);
+
+/*
  * plx_decode_noalloc — one bf16 decode step that allocates nothing.
  * (The paper has no counterpart: this is a deployment variant of plx_decode_ex.)
  *

@@ -7,7 +7,7 @@ does not need the compiled library.  Every compute call goes through
 """
 
 _BINDING_NAMES = {
-    "prefill", "decode", "decode_noalloc", "decode_workspace_bytes", "layer_forward", "qkr_norm_rope",
+    "prefill", "decode", "decode_gqa", "decode_noalloc", "decode_workspace_bytes", "layer_forward", "qkr_norm_rope",
     "get_device_status", "status_string", "PlxError", "lib", "PLX_F32", "PLX_BF16",
 }
 

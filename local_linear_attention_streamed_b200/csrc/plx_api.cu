@@ -210,6 +210,69 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
   return launch_decode_bf16(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
+size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
+  if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return 0;
+  if (H == Hkv) return plx_decode_workspace_bytes(B, H, L, d);
+  int splits = 1, chunk = 0;
+  decode_split_plan(B, Hkv, L, num_sms_or_default(), &splits, &chunk);
+  if (splits <= 1) return 0;
+  return sizeof(float) * (size_t)B * H * (size_t)splits * (size_t)(2 * d + 4);
+}
+
+int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                   const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !r || !Kcache || !Vcache || !seqlens || !out) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return PLX_ERR_INVALID_ARG;
+  const int G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PLX_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if (G == 1)
+    return plx_decode_ex(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, PLX_BF16, workspace,
+                         workspace_bytes, stream);
+  if (!aligned16(q) || !aligned16(r) || !aligned16(Kcache) || !aligned16(Vcache) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H > (1ll << 24) || (long long)B * Hkv * L + 64 >= (1ll << 31))
+    return PLX_ERR_UNSUPPORTED;
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.q = q;
+  a.r = r;
+  a.K = Kcache;
+  a.V = Vcache;
+  a.seqlens = seqlens;
+  a.out = out;
+  a.B = B;
+  a.H = H;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.d = d;
+  a.status = dc->status;
+  decode_split_plan(B, Hkv, L, dc->num_sms, &a.splits, &a.chunk);
+  if (a.splits > 1) {
+    const size_t need = sizeof(float) * (size_t)B * H * (size_t)a.splits * (size_t)(2 * d + 4);
+    if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLX_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    // One arrival counter per (b, KV head), in the same library-owned array
+    // (always left at zero) as the ungrouped decode's.
+    if ((rc = grow(&dc->counters, &dc->counters_bytes, sizeof(int) * (size_t)B * Hkv, st)) != PLX_OK)
+      return rc;
+    a.counters = static_cast<int*>(dc->counters);
+    if (workspace) {
+      a.partials = static_cast<float*>(workspace);
+    } else {
+      if ((rc = grow(&dc->decode_ws, &dc->decode_ws_bytes, need, st)) != PLX_OK) return rc;
+      a.partials = static_cast<float*>(dc->decode_ws);
+    }
+  }
+  return launch_decode_gqa(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
 int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vcache,
                const int32_t* seqlens, void* out, int B, int H, int L, int d) {
   return plx_decode_ex(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, PLX_BF16, nullptr, 0,

@@ -41,8 +41,9 @@ struct DecodeArgs {
   int splits;       // key chunks per (b, h)
   int chunk;        // keys per chunk (multiple of 64)
   float* partials;  // [B*H, splits, 2*d + 4] fp32: (m, omega, T, pad, O1[d], O2[d])
-  int* counters;    // [B*H] arrival counters, zero between calls
+  int* counters;    // [B*H] arrival counters, zero between calls ([B*Hkv] for grouped KV)
   int* status;
+  int Hkv;          // KV heads (grouped-KV decode only; H is a multiple of it)
 };
 
 // SIMT kernels: any d that is a multiple of 32 up to 128, f32 or bf16 storage.
@@ -51,6 +52,10 @@ cudaError_t launch_decode_simt(const DecodeArgs& a, bool bf16, cudaStream_t st);
 
 // bf16 split-KV decode on tensor-core MMAs, d in {64, 128}.
 cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms);
+// bf16 split-KV decode with grouped KV heads (H = G * Hkv, G in {2, 4, 8}),
+// d in {64, 128}: K/V blocks staged by TMA, the q and rho rows of the heads of
+// a group in one MMA tile.
+cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms);
 // Split heuristic shared by the launcher and the workspace-size query.
 void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk);
 

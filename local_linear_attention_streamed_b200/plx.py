@@ -28,6 +28,8 @@ SIGNATURES = {
     "plx_decode_workspace_bytes": (_sz, [_i] * 4),
     "plx_decode_num_splits": (_i, [_i] * 4),
     "plx_decode_noalloc": (_i, [_vp] * 6 + [_i] * 4 + [_vp]),
+    "plx_decode_gqa": (_i, [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]),
+    "plx_decode_gqa_workspace_bytes": (_sz, [_i] * 5),
     "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
     "plx_layer_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
@@ -140,6 +142,27 @@ def decode_noalloc(q, r, Kcache, Vcache, seqlens, out=None, stream=None):
                                 _dev(Vcache, "Vcache"), _dev(seqlens, "seqlens"), _dev(out, "out"),
                                 B, H, L, d, _stream_ptr(stream))
     _check(rc, "plx_decode_noalloc")
+    return out
+
+
+def decode_gqa(q, r, Kcache, Vcache, seqlens, out=None, workspace=None, stream=None):
+    """One bf16 decode step with grouped KV heads: q, r [B, H, d]; caches [B, Hkv, L, d]
+    (query head h reads KV head h // (H // Hkv)); seqlens int32 [B]."""
+    B, Hkv, L, d = Kcache.shape
+    H = q.shape[1]
+    if q.shape != (B, H, d) or r.shape != (B, H, d) or Vcache.shape != Kcache.shape:
+        raise ValueError("shape mismatch")
+    if seqlens.dtype != torch.int32 or seqlens.shape != (B,):
+        raise ValueError("seqlens must be int32 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.plx_decode_gqa(_dev(q, "q"), _dev(r, "r"), _dev(Kcache, "Kcache"), _dev(Vcache, "Vcache"),
+                            _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, Hkv, L, d,
+                            ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(rc, "plx_decode_gqa")
     return out
 
 

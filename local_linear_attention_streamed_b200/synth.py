@@ -198,6 +198,16 @@ def decode_specs(B, H, L, d, rho_sigma=0.25):
     }
 
 
+def decode_gqa_specs(B, H, Hkv, L, d, rho_sigma=0.25):
+    """Grouped KV heads: q, r [B,H,d]; Kcache, Vcache [B,Hkv,L,d] (same distributions as decode)."""
+    return {
+        "q": TensorSpec(TID_Q, (B, H, d), RMS_ROWS),
+        "K": TensorSpec(TID_K, (B, Hkv, L, d), RMS_ROWS),
+        "V": TensorSpec(TID_V, (B, Hkv, L, d), NORMAL, 1.0),
+        "r": TensorSpec(TID_R, (B, H, d), NORMAL, rho_sigma),
+    }
+
+
 def layer_specs(B, N, D):
     """x ~ N(0,1) [B,N,D]; W_Q, W_K, W_V, W_R, W_O ~ N(0, 1/D) stored [in, out]."""
     ws = 1.0 / math.sqrt(D)

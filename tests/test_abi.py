@@ -68,6 +68,20 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.plx_decode_ex(A, A, A, A, A + 2, A, 1, 1, 8, 128, 1, None, 0, None) == -3
 
 
+def test_decode_gqa_rejects_bad_arguments(lib):
+    ok = [A] * 6
+    assert lib.plx_decode_gqa(A, A, A, A, None, A, 1, 8, 2, 64, 128, None, 0, None) == -1
+    assert lib.plx_decode_gqa(*ok, 1, 8, 3, 64, 128, None, 0, None) == -1   # H not a multiple of Hkv
+    assert lib.plx_decode_gqa(*ok, 1, 6, 2, 64, 128, None, 0, None) == -2   # group of 3
+    assert lib.plx_decode_gqa(*ok, 1, 32, 2, 64, 128, None, 0, None) == -2  # group of 16
+    assert lib.plx_decode_gqa(*ok, 1, 8, 2, 64, 96, None, 0, None) == -2
+    assert lib.plx_decode_gqa(A, A, A, A + 8, A, A, 1, 8, 2, 64, 128, None, 0, None) == -3
+    assert lib.plx_decode_gqa_workspace_bytes(1, 8, 3, 64, 128) == 0
+    S = lib.plx_decode_num_splits(1, 2, 8192, 128)
+    assert S > 1
+    assert lib.plx_decode_gqa_workspace_bytes(1, 16, 2, 8192, 128) == 16 * S * (2 * 128 + 4) * 4
+
+
 def test_layer_and_norm_rope_reject_bad_arguments(lib):
     assert lib.plx_qkr_norm_rope(None, A, 1, 8, 2, 128, 1e-6, 1e4, None) == -1
     assert lib.plx_qkr_norm_rope(A, A, 1, 8, 2, 96, 1e-6, 1e4, None) == -2
