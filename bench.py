@@ -7,7 +7,9 @@ on the decode workload B=64, H=16, L=4096, d=128 bf16 (all sequences full),
 one plx_decode launch per step, inputs resident in HBM (2.1 GB of KV, larger
 than the 126 MB L2, so no flush is needed).  The same run measures the causal
 prefill B=8, H=16, N=4096, d=128 bf16 in TFLOP/s (the metric's second half)
-under "prefill".  For N > 1 GPUs (launched by torchrun) every rank runs the
+under "prefill", a layer step (projections, RMSNorm+RoPE, attention) under
+"layer", and the grouped-KV decode B=64, H=32, Hkv=8, L=4096, d=128 in GB/s
+under "decode_gqa".  For N > 1 GPUs (launched by torchrun) every rank runs the
 same per-GPU workload on its own seeded inputs with no data-path collective
 (weak scaling); time is the max over ranks.
 
@@ -35,6 +37,9 @@ if ROOT not in sys.path:
 METRIC = "decode KV GB/s (% HBM peak); causal prefill TFLOP/s (% BF16 peak)"
 DECODE = dict(B=64, H=16, L=4096, d=128)
 PREFILL = dict(B=8, H=16, N=4096, d=128)
+# Grouped KV heads: 32 query heads over 8 KV heads (groups of 4, the grouping of the
+# Llama-3-8B lineage), 1.07 GB of KV.
+DECODE_GQA = dict(B=64, H=32, Hkv=8, L=4096, d=128)
 L2_BYTES = 126 * 1024 * 1024  # B200 L2
 LAYER = dict(B=4, N=8192, D=2048, H=16)
 SWEEP_B = [1, 8, 64, 256, 1024, 2048]
@@ -311,6 +316,46 @@ def run_gpu(args, rank, world, dist):
         del pt
         torch.cuda.empty_cache()
 
+    # ---- Decode with grouped KV heads (the next row of the scope: one KV stream per group).
+    gqa = None
+    if not args.no_gqa:
+        gB, gH, gHkv, gL, gd = (DECODE_GQA[k] for k in ("B", "H", "Hkv", "L", "d"))
+        gspecs = synth.decode_gqa_specs(gB, gH, gHkv, gL, gd)
+        gt = {}
+        for name, spec in gspecs.items():
+            gt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(gt[name].data_ptr(), synth.BF16, seed + 5, spec)
+        gsl = torch.full((gB,), gL, dtype=torch.int32, device=dev)
+        gout = torch.empty_like(gt["q"])
+
+        def gdec():
+            plx.decode_gqa(gt["q"], gt["r"], gt["K"], gt["V"], gsl, out=gout)
+
+        gsteps = max(1, args.steps // 2)
+        g_total, g_per = timed(gdec, gsteps, max(3, args.warmup // 2), stream, dist)
+        if plx.get_device_status() != 0:
+            raise RuntimeError("grouped decode reported a device error")
+        g_total = max_over_ranks(g_total, dist)
+        g_kv = gB * gHkv * gL * gd * 2 * 2
+        g_alg = g_kv + 3 * gB * gH * gd * 2
+        g_kernel_ms = float(np.mean(g_per))
+        g_ach = g_alg / (g_kernel_ms * 1e-3) / 1e9
+        gqa = {
+            "metric": "grouped-KV decode KV GB/s", "unit": "GB/s",
+            "value": round(sum_over_ranks(g_kv * gsteps, dist) / (g_total * 1e-3) / 1e9, 2),
+            "ms_per_step": round(g_total / gsteps, 4), "steps": gsteps,
+            "config": {"workload": f"decode B={gB} H={gH} Hkv={gHkv} (groups of {gH // gHkv}) "
+                                   f"L={gL} d={gd} bf16, all seqlens {gL}",
+                       "l2": f"inputs larger than L2 ({g_kv / 1e9:.2f} GB KV); no flush"},
+            "roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(g_ach / peaks["hbm_gbs"], 4), "traffic": None,
+                         "peak_source": peak_src, "kernel": f"decode_gqa_kernel<{gd}, {gH // gHkv}>",
+                         "algorithmic_bytes_per_launch": g_alg},
+            "gpu_launches": gsteps,
+        }
+        del gt
+        torch.cuda.empty_cache()
+
     # ---- Full layer (x [4, 8192, 2048], 16 heads of 128).
     layer = None
     if not args.no_layer:
@@ -363,7 +408,7 @@ def run_gpu(args, rank, world, dist):
     clk.__exit__(None, None, None)
     return {
         "value": round(value, 2), "ms_per_step": round(ms_step, 4), "roofline": roofline,
-        "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "layer": layer,
+        "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "layer": layer, "decode_gqa": gqa,
         "gpu_launches": args.steps,
         "kernel_ms": kernel_ms,
     }
@@ -515,6 +560,7 @@ def main():
     ap.add_argument("--sweep", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-gqa", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
@@ -598,7 +644,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
-            "prefill": res["prefill"], "layer": res["layer"]}
+            "prefill": res["prefill"], "layer": res["layer"], "decode_gqa": res["decode_gqa"]}
     print(json.dumps(line))
 
 

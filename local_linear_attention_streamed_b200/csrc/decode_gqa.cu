@@ -10,15 +10,17 @@
 //   take units from a global counter (the first one statically).
 // * Warp 4 is a TMA producer: it publishes the units to a small ring and
 //   stages 64-key K and V blocks (128B-swizzled, the layout ldmatrix reads
-//   without bank conflicts) in a 3-stage ring.  HBM is read once per KV head.
-// * Warps 0..3 each own one or two query heads of the group (and, for G = 2, a
-//   half of the keys).  Per 16-key slice: one m16n8k16 MMA per k-step whose A
-//   rows are [q_h0; rho_h0; q_h1; rho_h1] gives S1 and S2 of the warp's heads;
-//   the value MMA V^T x [w_hi, w_lo, wt_hi, wt_lo] per head gives O1 and O2 as
-//   columns (each weight a bf16 hi + lo pair, as in the ungrouped decode).
+//   without bank conflicts) in a 3- or 6-stage ring.  HBM is read once per KV head.
+// * Warps 0..3 each take one 16-key slice of every staged block, for all G
+//   heads of the group, so each K and V byte is read from shared memory once:
+//   one m16n8k16 MMA per k-step whose A rows are [q_0; rho_0; q_1; rho_1; ...]
+//   gives S1 and S2 of every head of the group; the value MMA
+//   V^T x [w_hi, w_lo, wt_hi, wt_lo] per head (two heads per n-tile) gives O1
+//   and O2 as columns, one V fragment feeding every n-tile (each weight a bf16
+//   hi + lo pair, as in the ungrouped decode).
 // * One lazily raised running max per head (raised only when a block's max
 //   exceeds it by more than 2^8), omega = sum w, T = sum w t in fp32.
-// * Partials merge across the key-split warps in shared memory and across the
+// * Partials merge across the four warps in shared memory and across the
 //   chunks of a KV head by the last CTA to finish it (one arrival counter per
 //   (b, KV head) covers the group's heads); it leaves the counter at zero.
 //
@@ -33,10 +35,22 @@
 namespace plx {
 namespace {
 
-constexpr int kConsumerWarps = 4;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + the TMA producer warp
+constexpr int kSlices = 4;  // 16-key slices of a staged block
 constexpr int kBlk = 64;                             // keys per staged block
-constexpr int kStages = 3;
+// Consumer warps: one per (16-key slice, share of the group's heads).  A group
+// of 8 is split into two halves of 4 heads, so that a warp's accumulators
+// (D/16 m-tiles x 2 n-tiles x 4 fp32 per lane) and its serial per-head work
+// stay small; that configuration runs one CTA of 8 consumer warps per SM with
+// a deeper staging ring, the others two CTAs of 4 consumer warps and 3 stages.
+template <int D, int G>
+struct Cfg {
+  static constexpr int kHeadSplits = (G == 8) ? 2 : 1;
+  static constexpr int kHeadsPerWarp = G / kHeadSplits;
+  static constexpr int kConsumerWarps = kSlices * kHeadSplits;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + the TMA producer warp
+  static constexpr int kMinCtas = G == 8 ? 1 : 2;  // = decode_gqa_ctas_per_sm(G)
+  static constexpr int kStages = kMinCtas == 1 ? 6 : 3;
+};
 constexpr int kUnitRing = 4;
 constexpr float kLazyTau = 8.f;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on every wait
@@ -130,8 +144,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // with the 128B swizzle (what a TMA box of 64 bf16 columns writes).
 __device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-template <int D>
+template <int D, int G>
 struct Smem {
+  static constexpr int kStages = Cfg<D, G>::kStages;
   static constexpr int KH = D / 64;  // 64-dim halves per row
   uint8_t k[kStages][KH * 8192];
   uint8_t v[kStages][KH * 8192];
@@ -139,36 +154,47 @@ struct Smem {
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t csync;  // consumer-warp rendezvous (one lane per warp)
   long long unit_ring[kUnitRing];
-  float O1[kConsumerWarps][2][D], O2[kConsumerWarps][2][D];
-  float m[kConsumerWarps][2], omega[kConsumerWarps][2], T[kConsumerWarps][2];
+  // The unit's A tile: row 2j = q and row 2j+1 = rho of the group's head j
+  // (rows past 2G stay zero); rows padded by 16 bytes against bank conflicts.
+  alignas(16) __nv_bfloat16 qr[16][D + 8];
+  // Running merge of the four warps' partials per head of the group.
+  float O1[G][D], O2[G][D];
+  float m[G], omega[G], T[G];
   int last;
   int abort;
 };
 
+// 16-byte vector stores and ldmatrix rows need the A tile 16-byte aligned
+// (its row pitch, 2 (D + 8) bytes, is a multiple of 16).
+using SmemD128G8 = Smem<128, 8>;
+using SmemD128G2 = Smem<128, 2>;
+using SmemD64G8 = Smem<64, 8>;
+using SmemD64G2 = Smem<64, 2>;
+static_assert(offsetof(SmemD128G8, qr) % 16 == 0 && offsetof(SmemD128G2, qr) % 16 == 0 &&
+                  offsetof(SmemD64G8, qr) % 16 == 0 && offsetof(SmemD64G2, qr) % 16 == 0,
+              "A tile alignment");
+
 __device__ unsigned long long g_gqa_unit_next;
 __device__ unsigned int g_gqa_cta_done;
 
-// Per-warp softmax state of one head slot.
-template <int D>
-struct HeadState {
-  float m;          // running max (log2 domain), warp-uniform
-  float omega, T;   // partial sums over this lane's keys (equal in the eight lanes of one t)
-};
 
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(Cfg<D, G>::kThreads, Cfg<D, G>::kMinCtas)
     decode_gqa_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       DecodeArgs a) {
-  constexpr int KH = D / 64;              // 64-dim halves of a row
-  constexpr int KS = D / 16;              // k-steps of the score MMA
-  constexpr int MT = D / 16;              // m-tiles (16 dims) of the value MMA
-  constexpr int HPW = (G == 8) ? 2 : 1;   // query heads per consumer warp
-  constexpr int NHG = G / HPW;            // head groups
-  constexpr int KG = kConsumerWarps / NHG;  // key groups (warps that split a block's keys)
-  static_assert(NHG * KG == kConsumerWarps, "warp split");
+  constexpr int kStages = Cfg<D, G>::kStages;
+  constexpr int KH = D / 64;   // 64-dim halves of a row
+  constexpr int KS = D / 16;   // k-steps of the score MMA
+  constexpr int MT = D / 16;   // m-tiles (16 dims) of the value MMA
+  constexpr int HW = Cfg<D, G>::kHeadsPerWarp;
+  constexpr int NT = HW / 2;   // n-tiles (8 columns = 2 heads) of the value MMA
+  constexpr int kConsumerWarps = Cfg<D, G>::kConsumerWarps;
+  static_assert(G == 2 || G == 4 || G == 8, "group size");
+  static_assert(kBlk / 16 == kSlices, "16-key slices");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem<D>& sm = *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<D, G>& sm =
+      *reinterpret_cast<Smem<D, G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BKV = a.B * a.Hkv;
   const long long units = (long long)BKV * a.splits;
@@ -185,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(&sm.csync, kConsumerWarps);
     sm.abort = 0;
+    for (int x = 0; x < 16 * (D + 8); ++x) (&sm.qr[0][0])[x] = __float2bfloat16(0.f);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -234,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     // ---------------- consumers ----------------
     const int g = lane >> 2, t = lane & 3;
-    const int hg = warp % NHG, kg = warp / NHG;
+    const int sb = warp % kSlices;  // this warp's 16-key slice of every staged block
+    const int h0 = (warp / kSlices) * HW;  // its first head within the group
     const float c_log2 = 1.4426950408889634f / sqrtf((float)D);
     const __nv_bfloat16* qall = reinterpret_cast<const __nv_bfloat16*>(a.q);
     const __nv_bfloat16* rall = reinterpret_cast<const __nv_bfloat16*>(a.r);
@@ -273,187 +301,230 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int nch = (n + a.chunk - 1) / a.chunk;
       const int nblk = (kend - kbeg + kBlk - 1) / kBlk;
 
-      // A fragments: row 2s holds q and row 2s+1 rho of the warp's head slot s.
-      uint32_t aq[KS][2];
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) aq[ks][0] = aq[ks][1] = 0u;
-      if (g < 2 * HPW) {
-        const int h = kvh * G + hg * HPW + (g >> 1);
-        const __nv_bfloat16* src = ((g & 1) ? rall : qall) + ((long long)b * a.H + h) * D;
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          aq[ks][0] = *reinterpret_cast<const uint32_t*>(src + 16 * ks + 2 * t);
-          aq[ks][1] = *reinterpret_cast<const uint32_t*>(src + 16 * ks + 8 + 2 * t);
-        }
+      // The group's q and rho rows into the A tile (the previous unit's readers
+      // finished at its closing rendezvous).
+      for (int x = threadIdx.x; x < 2 * G * (D / 8); x += kConsumerWarps * 32) {
+        const int row = x / (D / 8), col = (x % (D / 8)) * 8;
+        const long long bh = (long long)b * a.H + (long long)kvh * G + (row >> 1);
+        *reinterpret_cast<uint4*>(&sm.qr[row][col]) =
+            *reinterpret_cast<const uint4*>(((row & 1) ? rall : qall) + bh * D + col);
       }
-      float O[MT][4];
+      if (!csync()) break;
+      float O[MT][NT][4];
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f;
-      HeadState<D> hs[HPW];
+      for (int mt = 0; mt < MT; ++mt) {
 #pragma unroll
-      for (int s = 0; s < HPW; ++s) {
-        hs[s].m = -CUDART_INF_F;
-        hs[s].omega = 0.f;
-        hs[s].T = 0.f;
+        for (int nt = 0; nt < NT; ++nt) O[mt][nt][0] = O[mt][nt][1] = O[mt][nt][2] = O[mt][nt][3] = 0.f;
       }
+      // Per head of the warp: running max (warp-uniform) and this lane's partial sums.
+      float hm[HW], hom[HW], hT[HW];
+#pragma unroll
+      for (int j = 0; j < HW; ++j) {
+        hm[j] = -CUDART_INF_F;
+        hom[j] = 0.f;
+        hT[j] = 0.f;
+      }
+      const uint32_t qa = smem_u32(&sm.qr[0][0]);
       bool ok = true;
       for (int i = 0; i < nblk; ++i, ++pos) {
         const int stg = pos % kStages;
         if (!(ok = mbar_wait(&sm.full[stg], (pos / kStages) & 1, abort, a.status))) break;
         const uint32_t kb = smem_u32(sm.k[stg]), vb = smem_u32(sm.v[stg]);
-        for (int sb = kg; sb < kBlk / 16; sb += KG) {
-          const int j0 = kbeg + kBlk * i + 16 * sb;  // first key of this 16-key slice
-          if (j0 >= kend) break;
-          // ---- S = [q; rho; ...] K^T for 16 keys (two n-tiles of 8).
+        const int j0 = kbeg + kBlk * i + 16 * sb;  // first key of this warp's slice
+        if (j0 < kend) {
+          const int mi = lane >> 3;
+          // ---- S = [q_0; rho_0; q_1; ...] K^T for 16 keys (two n-tiles of 8).
           float S[2][4];
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) S[nt][0] = S[nt][1] = S[nt][2] = S[nt][3] = 0.f;
           {
-            const int mi = lane >> 3;
-            const int r = 16 * sb + 8 * (mi >> 1) + (lane & 7);
+            const int ra = 8 * (mi & 1) + (lane & 7);             // A rows of matrices 0..3
+            const int rk = 16 * sb + 8 * (mi >> 1) + (lane & 7);  // K rows (keys)
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
+              uint32_t a0, a1, a2, a3, b00, b01, b10, b11;
+              ldsm_x4(qa + (uint32_t)(ra * (D + 8) + 16 * ks + 8 * (mi >> 1)) * 2u, a0, a1, a2, a3);
               const int d0 = 16 * ks + 8 * (mi & 1);
-              uint32_t b00, b01, b10, b11;
-              ldsm_x4(kb + (uint32_t)((d0 >> 6) * 8192) + swz(r, (d0 & 63) >> 3), b00, b01, b10, b11);
-              mma_bf16(S[0], aq[ks][0], 0u, aq[ks][1], 0u, b00, b01);
-              mma_bf16(S[1], aq[ks][0], 0u, aq[ks][1], 0u, b10, b11);
+              ldsm_x4(kb + (uint32_t)((d0 >> 6) * 8192) + swz(rk, (d0 & 63) >> 3), b00, b01, b10, b11);
+              mma_bf16(S[0], a0, a1, a2, a3, b00, b01);
+              mma_bf16(S[1], a0, a1, a2, a3, b10, b11);
             }
           }
-          // Lane (g, t) holds row g at keys 8nt + 2t + {0, 1}; every lane takes
-          // s1 and s2 of each of the warp's heads at its own keys (e4 = 2nt + e).
-          float s1[HPW][4], s2[HPW][4];
+          // Lane (g, t) holds rows g (S[nt][0..1]) and g + 8 (S[nt][2..3]) at
+          // keys 8nt + 2t + {0, 1}.  Per head j: s1 = row 2j, s2 = row 2j + 1.
+          // Value column n of n-tile nt is head 2nt + n/4, kind n % 4 (w_hi,
+          // w_lo, wt_hi, wt_lo); lane (g, t) supplies column g of every n-tile.
+          uint32_t bw0[NT], bw1[NT];
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float own = S[e4 >> 1][e4 & 1];
-            const bool valid = j0 + 8 * (e4 >> 1) + 2 * t + (e4 & 1) < kend;
+          for (int nt = 0; nt < NT; ++nt) bw0[nt] = bw1[nt] = 0u;
+          // Phase 1 (all heads, no branches): scores at this lane's keys, the
+          // block max and the lazy raise.  Head j of the warp is head h0 + j of
+          // the group: rows 2(h0 + j) and 2(h0 + j) + 1, in S[..][0..1] (rows
+          // 0..7) or S[..][2..3] (rows 8..15).
+          float s1[HW][4], s2[HW][4], alpha[HW];
+          const bool hi_rows = 2 * h0 >= 8;  // a warp's heads never straddle rows 7 | 8 (HW divides 4)
 #pragma unroll
-            for (int s = 0; s < HPW; ++s) {
-              const float x1 = __shfl_sync(0xffffffffu, own, 8 * s + t);
-              const float x2 = __shfl_sync(0xffffffffu, own, 8 * s + 4 + t);
-              s1[s][e4] = valid ? x1 * c_log2 : -CUDART_INF_F;
-              s2[s][e4] = valid ? x2 : 0.f;
-            }
-          }
-          float w[HPW][4];
-#pragma unroll
-          for (int s = 0; s < HPW; ++s) {
-            float ml = fmaxf(fmaxf(s1[s][0], s1[s][1]), fmaxf(s1[s][2], s1[s][3]));
-            ml = fmaxf(ml, __shfl_xor_sync(0xffffffffu, ml, 1));
-            const float mblk = fmaxf(ml, __shfl_xor_sync(0xffffffffu, ml, 2));  // warp-uniform
-            if (mblk > hs[s].m + kLazyTau) {  // also on the slot's first slice (m = -inf)
-              const float alpha = exp2f(hs[s].m - mblk);
-              if ((t >> 1) == s) {  // this lane's value columns 2t, 2t+1 belong to slot t/2
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) O[mt][q] *= alpha;
-                }
-              }
-              hs[s].omega *= alpha;
-              hs[s].T *= alpha;
-              hs[s].m = mblk;
-            }
-#pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) w[s][e4] = exp2f(s1[s][e4] - hs[s].m);
-            hs[s].omega += (w[s][0] + w[s][1]) + (w[s][2] + w[s][3]);
-            hs[s].T += (w[s][0] * s2[s][0] + w[s][1] * s2[s][1]) + (w[s][2] * s2[s][2] + w[s][3] * s2[s][3]);
-          }
-          // ---- [O1 O2] += V^T x [w_hi, w_lo, wt_hi, wt_lo] per head slot:
-          // value column n = 4s + kind comes from the lanes with g = n.
-          uint32_t b0 = 0u, b1 = 0u;
-          if (g < 4 * HPW) {
-            const bool s0 = (g >> 2) == 0;
-            const int kind = g & 3;
-            float x[4];
+          for (int j = 0; j < HW; ++j) {
+            const int src1 = ((2 * (h0 + j)) & 7) * 4 + t, src2 = ((2 * (h0 + j) + 1) & 7) * 4 + t;
 #pragma unroll
             for (int e4 = 0; e4 < 4; ++e4) {
-              const float ww = s0 ? w[0][e4] : w[HPW - 1][e4];
-              const float tt = s0 ? s2[0][e4] : s2[HPW - 1][e4];
-              float v = (kind < 2) ? ww : ww * tt;
-              if (kind & 1) v -= __bfloat162float(__float2bfloat16_rn(v));
-              x[e4] = v;
+              const float own = hi_rows ? S[e4 >> 1][2 + (e4 & 1)] : S[e4 >> 1][e4 & 1];
+              const float x1 = __shfl_sync(0xffffffffu, own, src1);
+              const float x2 = __shfl_sync(0xffffffffu, own, src2);
+              const bool valid = j0 + 8 * (e4 >> 1) + 2 * t + (e4 & 1) < kend;
+              s1[j][e4] = valid ? x1 * c_log2 : -CUDART_INF_F;
+              s2[j][e4] = valid ? x2 : 0.f;
             }
-            b0 = pack_bf16(x[0], x[1]);  // keys 2t, 2t+1
-            b1 = pack_bf16(x[2], x[3]);  // keys 8+2t, 9+2t
           }
-          {
-            const int mi = lane >> 3;
-            const int r = 16 * sb + 8 * (mi >> 1) + (lane & 7);
-            // Keys past the end of the sequence carry zero weight; their V rows
-            // (whatever the cache holds there) are zeroed so that they cannot
-            // turn into NaN in the product.
-            const bool edge = j0 + 16 > kend;
-            const int k0 = j0 + 2 * t, k8 = j0 + 8 + 2 * t;
+          bool raised = false;
 #pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              const int d0 = 16 * mt + 8 * (mi & 1);
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_t(vb + (uint32_t)((d0 >> 6) * 8192) + swz(r, (d0 & 63) >> 3), a0, a1, a2, a3);
-              if (edge) {
-                const uint32_t m0 = (k0 < kend ? 0x0000FFFFu : 0u) | (k0 + 1 < kend ? 0xFFFF0000u : 0u);
-                const uint32_t m8 = (k8 < kend ? 0x0000FFFFu : 0u) | (k8 + 1 < kend ? 0xFFFF0000u : 0u);
-                a0 &= m0;
-                a1 &= m0;
-                a2 &= m8;
-                a3 &= m8;
+          for (int j = 0; j < HW; ++j) {
+            float ml = fmaxf(fmaxf(s1[j][0], s1[j][1]), fmaxf(s1[j][2], s1[j][3]));
+            ml = fmaxf(ml, __shfl_xor_sync(0xffffffffu, ml, 1));
+            const float mblk = fmaxf(ml, __shfl_xor_sync(0xffffffffu, ml, 2));  // warp-uniform
+            const bool up = mblk > hm[j] + kLazyTau;  // also on the head's first slice (m = -inf)
+            alpha[j] = up ? exp2f(hm[j] - mblk) : 1.f;
+            hm[j] = up ? mblk : hm[j];
+            hom[j] *= alpha[j];
+            hT[j] *= alpha[j];
+            raised |= up;
+          }
+          if (raised) {  // warp-uniform; rare after a head's first slice
+            // Columns 2t, 2t+1 of n-tile nt belong to the warp's head 2nt + t/2.
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              const float al = (t >> 1) ? alpha[2 * nt + 1] : alpha[2 * nt];
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) O[mt][nt][q] *= al;
               }
-              mma_bf16(O[mt], a0, a1, a2, a3, b0, b1);
             }
+          }
+          // Phase 2: weights, sums and the value MMA's B fragment.  Value column
+          // n of n-tile nt is head 2nt + n/4, kind n % 4 (w_hi, w_lo, wt_hi,
+          // wt_lo); lane (g, t) supplies column g of every n-tile.
+#pragma unroll
+          for (int j = 0; j < HW; ++j) {
+            float w[4];
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) w[e4] = exp2f(s1[j][e4] - hm[j]);
+            hom[j] += (w[0] + w[1]) + (w[2] + w[3]);
+            hT[j] += (w[0] * s2[j][0] + w[1] * s2[j][1]) + (w[2] * s2[j][2] + w[3] * s2[j][3]);
+            if ((g >> 2) == (j & 1)) {
+              const int kind = g & 3;
+              float x[4];
+#pragma unroll
+              for (int e4 = 0; e4 < 4; ++e4) {
+                float v = (kind < 2) ? w[e4] : w[e4] * s2[j][e4];
+                if (kind & 1) v -= __bfloat162float(__float2bfloat16_rn(v));
+                x[e4] = v;
+              }
+              bw0[j >> 1] = pack_bf16(x[0], x[1]);  // keys 2t, 2t+1
+              bw1[j >> 1] = pack_bf16(x[2], x[3]);  // keys 8+2t, 9+2t
+            }
+          }
+          // ---- [O1 O2] += V^T x weights; one V fragment feeds all n-tiles.
+          const int rv = 16 * sb + 8 * (mi >> 1) + (lane & 7);
+          // Keys past the end of the sequence carry zero weight; their V rows
+          // (whatever the cache holds there) are zeroed so that they cannot
+          // turn into NaN in the product.
+          const bool edge = j0 + 16 > kend;
+          const int k0 = j0 + 2 * t, k8 = j0 + 8 + 2 * t;
+          const uint32_t m0 = (k0 < kend ? 0x0000FFFFu : 0u) | (k0 + 1 < kend ? 0xFFFF0000u : 0u);
+          const uint32_t m8 = (k8 < kend ? 0x0000FFFFu : 0u) | (k8 + 1 < kend ? 0xFFFF0000u : 0u);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const int d0 = 16 * mt + 8 * (mi & 1);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(vb + (uint32_t)((d0 >> 6) * 8192) + swz(rv, (d0 & 63) >> 3), a0, a1, a2, a3);
+            if (edge) {
+              a0 &= m0;
+              a1 &= m0;
+              a2 &= m8;
+              a3 &= m8;
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(O[mt][nt], a0, a1, a2, a3, bw0[nt], bw1[nt]);
           }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[stg]);
       }
       if (!ok) break;
-      // ---- Warp partials to shared memory.
+      // ---- Merge the slice warps' partials of each head, one slice after
+      // another, into shared memory.
 #pragma unroll
-      for (int s = 0; s < HPW; ++s) {
-        float om = hs[s].omega, tt = hs[s].T;
-        om += __shfl_xor_sync(0xffffffffu, om, 1);
-        om += __shfl_xor_sync(0xffffffffu, om, 2);
-        tt += __shfl_xor_sync(0xffffffffu, tt, 1);
-        tt += __shfl_xor_sync(0xffffffffu, tt, 2);
-        if (lane == 0) {
-          sm.m[warp][s] = hs[s].m;
-          sm.omega[warp][s] = om;
-          sm.T[warp][s] = tt;
-        }
+      for (int j = 0; j < HW; ++j) {
+        hom[j] += __shfl_xor_sync(0xffffffffu, hom[j], 1);
+        hom[j] += __shfl_xor_sync(0xffffffffu, hom[j], 2);
+        hT[j] += __shfl_xor_sync(0xffffffffu, hT[j], 1);
+        hT[j] += __shfl_xor_sync(0xffffffffu, hT[j], 2);
       }
-      if ((t >> 1) < HPW) {  // lane t: columns 2t, 2t+1 = slot t/2, O1 (t even) or O2 (t odd), hi + lo
-        float* dst = (t & 1) ? sm.O2[warp][t >> 1] : sm.O1[warp][t >> 1];
+      for (int w2 = 0; w2 < kSlices && ok; ++w2) {
+        if (sb == w2) {
+          // Lane (g, t): columns 2t, 2t+1 of n-tile nt = the warp's head
+          // 2nt + t/2, O1 (t even) or O2 (t odd) as a hi + lo pair, dims
+          // 16mt + g and + 8.
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          dst[16 * mt + g] = O[mt][0] + O[mt][1];
-          dst[16 * mt + 8 + g] = O[mt][2] + O[mt][3];
-        }
-      }
-      if (!csync()) break;
-      // ---- Merge the key groups per head; finish or publish the chunk's partials.
-      const int x = threadIdx.x;  // 0..127: output dim
-#pragma unroll 1
-      for (int hh = 0; hh < G; ++hh) {
-        const int hgg = hh / HPW, s = hh % HPW;
-        float M = -CUDART_INF_F;
+          for (int nt = 0; nt < NT; ++nt) {
+            const int jl = 2 * nt + (t >> 1);
+            const int h = h0 + jl;
+            const float mh = (t >> 1) ? hm[2 * nt + 1] : hm[2 * nt];
+            float* dst = (t & 1) ? sm.O2[h] : sm.O1[h];
+            float so = 1.f, ss = 0.f;
+            if (w2 > 0) {
+              const float M = fmaxf(sm.m[h], mh);
+              ss = (sm.m[h] == -CUDART_INF_F) ? 0.f : exp2f(sm.m[h] - M);
+              so = (mh == -CUDART_INF_F) ? 0.f : exp2f(mh - M);
+            }
 #pragma unroll
-        for (int kk = 0; kk < KG; ++kk) M = fmaxf(M, sm.m[hgg + NHG * kk][s]);
-        float om = 0.f, TT = 0.f, o1 = 0.f, o2 = 0.f;
+            for (int mt = 0; mt < MT; ++mt) {
+              const float v0 = O[mt][nt][0] + O[mt][nt][1], v8 = O[mt][nt][2] + O[mt][nt][3];
+              float* p0 = dst + 16 * mt + g;
+              p0[0] = w2 > 0 ? so * v0 + ss * p0[0] : v0;
+              p0[8] = w2 > 0 ? so * v8 + ss * p0[8] : v8;
+            }
+          }
+          __syncwarp();
+          if (lane < HW) {
+            const int h = h0 + lane;
+            float mh = hm[0], oh = hom[0], th = hT[0];
 #pragma unroll
-        for (int kk = 0; kk < KG; ++kk) {
-          const int w2 = hgg + NHG * kk;
-          const float sc = (sm.m[w2][s] == -CUDART_INF_F) ? 0.f : exp2f(sm.m[w2][s] - M);
-          om += sc * sm.omega[w2][s];
-          TT += sc * sm.T[w2][s];
-          if (x < D) {
-            o1 += sc * sm.O1[w2][s][x];
-            o2 += sc * sm.O2[w2][s][x];
+            for (int j = 1; j < HW; ++j) {
+              if (lane == j) {
+                mh = hm[j];
+                oh = hom[j];
+                th = hT[j];
+              }
+            }
+            if (w2 == 0) {
+              sm.m[h] = mh;
+              sm.omega[h] = oh;
+              sm.T[h] = th;
+            } else {
+              const float M = fmaxf(sm.m[h], mh);
+              const float ss = (sm.m[h] == -CUDART_INF_F) ? 0.f : exp2f(sm.m[h] - M);
+              const float so = (mh == -CUDART_INF_F) ? 0.f : exp2f(mh - M);
+              sm.omega[h] = ss * sm.omega[h] + so * oh;
+              sm.T[h] = ss * sm.T[h] + so * th;
+              sm.m[h] = M;
+            }
           }
         }
+        ok = csync();
+      }
+      if (!ok) break;
+      // ---- Finish or publish the chunk's partials (thread x owns dim x).
+      const int x = threadIdx.x;
+#pragma unroll 1
+      for (int hh = 0; hh < G; ++hh) {
+        const float M = sm.m[hh], om = sm.omega[hh], TT = sm.T[hh];
         const long long bh = (long long)b * a.H + (long long)kvh * G + hh;
         if (nch == 1) {
           if (x < D) {
             const float inv = 1.f / om;
-            out[bh * D + x] = __float2bfloat16_rn(((1.f + TT * inv) * o1 - o2) * inv);
+            out[bh * D + x] = __float2bfloat16_rn(((1.f + TT * inv) * sm.O1[hh][x] - sm.O2[hh][x]) * inv);
           }
         } else {
           float* rec = a.partials + (bh * a.splits + c) * (2 * D + 4);
@@ -463,8 +534,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             rec[2] = TT;
           }
           if (x < D) {
-            rec[4 + x] = o1;
-            rec[4 + D + x] = o2;
+            rec[4 + x] = sm.O1[hh][x];
+            rec[4 + D + x] = sm.O2[hh][x];
           }
         }
       }
@@ -545,18 +616,19 @@ bool make_cache_map(CUtensorMap* m, const void* base, long long rows, int d) {
 template <int D, int G>
 cudaError_t launch_gqa(const DecodeArgs& a, const CUtensorMap& mK, const CUtensorMap& mV, cudaStream_t st,
                        int num_sms) {
-  const size_t smem = sizeof(Smem<D>) + 1024;
+  const size_t smem = sizeof(Smem<D, G>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D, G>, kThreads, smem);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D, G>, Cfg<D, G>::kThreads,
+                                                    smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   const long long units = (long long)a.B * a.Hkv * a.splits;
   long long grid = (long long)num_sms * per_sm;
   if (grid > units) grid = units;
-  decode_gqa_kernel<D, G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, a);
+  decode_gqa_kernel<D, G><<<(unsigned)grid, Cfg<D, G>::kThreads, smem, st>>>(mK, mV, a);
   return cudaGetLastError();
 }
 

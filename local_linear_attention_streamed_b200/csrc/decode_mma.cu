@@ -403,9 +403,9 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
 // better (each unit pays a fixed start-up and merge), but the last wave of
 // units should be nearly full: take the fewest splits whose waves over the
 // resident CTAs are at least 97 % used, with chunks of at least 256 keys.
-void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk) {
+void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk, int ctas_per_sm) {
   const double bh = (double)B * H;
-  const double resident = (double)num_sms * 2;  // CTAs the launcher keeps per SM
+  const double resident = (double)num_sms * ctas_per_sm;  // CTAs the launcher keeps per SM
   long long smax = L / 256;
   if (smax < 1) smax = 1;
   if (smax > 256) smax = 256;

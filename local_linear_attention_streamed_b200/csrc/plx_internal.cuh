@@ -56,8 +56,11 @@ cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms
 // d in {64, 128}: K/V blocks staged by TMA, the q and rho rows of the heads of
 // a group in one MMA tile.
 cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms);
-// Split heuristic shared by the launcher and the workspace-size query.
-void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk);
+// Split heuristic shared by the launcher and the workspace-size query;
+// ctas_per_sm is how many CTAs of the decode kernel an SM holds.
+void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk, int ctas_per_sm = 2);
+// CTAs per SM of the grouped-KV decode kernel for group size G.
+inline int decode_gqa_ctas_per_sm(int G) { return G == 8 ? 1 : 2; }
 
 // bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
 bool prefill_tc_supported(int d);

@@ -116,9 +116,11 @@ def test_gqa_bad_seqlen_reports_and_zeroes(plx):
     assert rel_err_rms(o[0], want) <= BF16_TOL
 
 
-def test_gqa_full_size_sampled(plx):
-    """Grouped decode at the bench's grouped workload: B=64, H=32, Hkv=4, L=4096, d=128."""
-    B, H, Hkv, L, d = 64, 32, 4, 4096, 128
+@pytest.mark.parametrize("H,Hkv", [(32, 8), (64, 8)])
+def test_gqa_full_size_sampled(plx, H, Hkv):
+    """Grouped decode at full size (B=64, L=4096, d=128, ragged lengths): groups of 4
+    (the bench's grouped workload) and of 8."""
+    B, L, d = 64, 4096, 128
     G = H // Hkv
     seed = 1005
     specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
