@@ -37,6 +37,8 @@ if ROOT not in sys.path:
 METRIC = "decode KV GB/s (% HBM peak); causal prefill TFLOP/s (% BF16 peak)"
 DECODE = dict(B=64, H=16, L=4096, d=128)
 PREFILL = dict(B=8, H=16, N=4096, d=128)
+# The compute-matched variant (head dim halved, twice the heads, same width).
+PREFILL_D64 = dict(B=8, H=32, N=4096, d=64)
 # Grouped KV heads: 32 query heads over 8 KV heads (groups of 4, the grouping of the
 # Llama-3-8B lineage), 1.07 GB of KV.
 DECODE_GQA = dict(B=64, H=32, Hkv=8, L=4096, d=128)
@@ -314,6 +316,32 @@ def run_gpu(args, rank, world, dist):
             "gpu_launches": psteps,
         }
         del pt
+        torch.cuda.empty_cache()
+        # Head dim 64 at the same width (same Q, K, V, R bytes).
+        qB, qH, qN, qd = (PREFILL_D64[k] for k in ("B", "H", "N", "d"))
+        qspecs = synth.prefill_specs(qB, qH, qN, qd)
+        qt = {}
+        for name, spec in qspecs.items():
+            qt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(qt[name].data_ptr(), synth.BF16, seed + 6, spec)
+        qout = torch.empty_like(qt["Q"])
+
+        def pre64():
+            plx.prefill(qt["Q"], qt["K"], qt["V"], qt["R"], causal=True, out=qout)
+
+        q_total, q_per = timed(pre64, psteps, max(3, args.warmup // 2), stream, dist)
+        if plx.get_device_status() != 0:
+            raise RuntimeError("prefill (d = 64) reported a device error")
+        q_total = max_over_ranks(q_total, dist)
+        qflops = prefill_flops(qB, qH, qN, qd)
+        q_ach = qflops / (float(np.mean(q_per)) * 1e-3) / 1e12
+        prefill["d64"] = {
+            "workload": f"causal prefill B={qB} H={qH} N={qN} d={qd} bf16 (head dim halved, same width)",
+            "value": round(sum_over_ranks(qflops * psteps, dist) / (q_total * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(q_total / psteps, 3),
+            "kernel_tflops": round(q_ach, 1), "frac": round(q_ach / peaks["bf16_tflops"], 4),
+        }
+        del qt
         torch.cuda.empty_cache()
 
     # ---- Decode with grouped KV heads (the next row of the scope: one KV stream per group).

@@ -1,4 +1,4 @@
-// Causal (or full) Parallax prefill for bf16, d = 128, on sm_100a tensor cores.
+// Causal (or full) Parallax prefill for bf16, d in {64, 128}, on sm_100a tensor cores.
 //
 // Per CTA, one 128-query tile at a time; persistent CTAs take (b, h, tile)
 // work from a global counter in head chunks, longest causal tiles first within
@@ -59,7 +59,6 @@
 namespace plx {
 namespace {
 
-constexpr int kD = 128;
 constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
 constexpr int kStages = 4;               // K/V ring depth
@@ -71,27 +70,38 @@ constexpr int kThreads = 384;
 constexpr int kPVWarp = 2;
 constexpr int kFirstSoftmaxWarp = 4;
 constexpr int kRegsControl = 72, kRegsSoftmax = 216;
-constexpr uint32_t kQBytes = kBM * kD * 2;   // 32 KiB (Q tile, also R tile)
-constexpr uint32_t kKVBytes = kBN * kD * 2;  // 16 KiB (one K or V block)
 constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128 B rows)
 constexpr uint32_t kHalfKV = kBN * 128;      // one 64-dim half of a K/V block
 constexpr float kLazyTau = 8.f;
-constexpr float kTheta = 2.f;  // re-centre t once its running mean drifts this far
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s bound on every wait
 
 // TMEM column map: the S stage, two P buffers (bf16(w) then bf16(w (t - c))
-// in each), O1 and O2.
-constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColO1 = 256,
-                   kColO2 = 384;
+// in each), O1 (D columns from 256) and O2 (after O1).
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColO1 = 256;
 
 // Instruction descriptors (kind::f16): D f32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), A K-major, B K-major (S) or MN-major (bit 16, PV),
 // N >> 3 at bits 17-22, M >> 4 at bits 24-28.
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kBN >> 3) << 17) | ((kBM >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((kD >> 3) << 17) |
-                              ((kBM >> 4) << 24);
+// Head dimension D in {64, 128}: the tile sizes, the value MMA's N and O2's columns.
+template <int D>
+struct Dims {
+  static constexpr int kHalves = D / 64;                // 64-dim halves (TMA boxes) per row
+  static constexpr uint32_t kQBytes = kBM * D * 2;      // Q tile (also R tile)
+  static constexpr uint32_t kKVBytes = kBN * D * 2;     // one K or V block
+  static constexpr uint32_t kColO2 = kColO1 + D;
+  // Re-centre t once its running mean drifts this far (section "Centring"
+  // above).  2 at D = 128: 1.7 % on the rescale test, and 8 % faster than 1
+  // (fewer O passes).  At D = 64 the rescale test gives 2.7 % (causal) with
+  // 2 and 2.2 % (all keys) with 1, 1.8 % and 2.0 % with 0.5.
+  static constexpr float kTheta = D == 128 ? 2.f : 0.5f;
+  static constexpr uint32_t kIdescPV =
+      (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((D >> 3) << 17) | ((kBM >> 4) << 24);
+};
 
+template <int D>
 struct Smem {
+  static constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
   // Tiles first (1024-byte aligned for the 128B swizzle).
   uint8_t q[kQBytes];
   uint8_t r[kQBytes];
@@ -387,12 +397,17 @@ struct Params {
   int* status;
 };
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
+  constexpr uint32_t kColO2 = Dims<D>::kColO2, kIdescPV = Dims<D>::kIdescPV;
+  constexpr int kHalves = Dims<D>::kHalves;
+  Smem<D>& sm =
+      *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
   const int ntile = (p.N + kBM - 1) / kBM;
@@ -461,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // never completes, the MMA warp's bounded wait runs out and every role
         // unwinds through the abort path.
         if (!(p.inject_stall && tc == 0)) {
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kHalves; ++h) {
             tma_load_2d(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
             tma_load_2d(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
           }
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&sm.kv_empty[st], par, abort, p.status)) break;
           mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
           kv_issued[st] = kv / kStages;
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < kHalves; ++h) {
             tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + j * kBN);
             tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + j * kBN);
           }
@@ -517,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // offset in the start-address field (shared-memory addresses
           // < 256 KB keep that 14-bit field from carrying).
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
+          for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
             const uint64_t koff = (uint64_t)((((ks >> 2) * kHalfKV) + (ks & 3) * 32) >> 4);
             mma_ss(tmem + kColS1, dQ + off, dk + koff, kIdescS, ks > 0);
@@ -613,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int wg = (warp - kFirstSoftmaxWarp) >> 2;
     const int row = 32 * (warp & 3) + lane;  // TMEM lane == query row within the tile
     const uint32_t sb = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    const float scale = 1.4426950408889634f * rsqrtf((float)kD);
+    const float scale = 1.4426950408889634f * rsqrtf((float)D);
     uint32_t gb = 0;  // the CTA's block counter at the current tile's first block
     int tc = 0;
     bool ok = true;
@@ -623,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!mbar_wait(&sm.o_full, etc & 1, abort, p.status)) return false;
       tc_fence_after();
 #pragma unroll 1
-      for (int c0 = 64 * wg; c0 < 64 * wg + 64; c0 += 32) {
+      for (int c0 = (D / 2) * wg; c0 < (D / 2) * wg + D / 2; c0 += 32) {
         uint32_t o1[32], o2[32];
         tmem_ld32(sb + kColO1 + c0, o1);
         tmem_ld32(sb + kColO2 + c0, o2);
@@ -771,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float delta = 0.f;
         {
           const float Tn = (T + T_o) + tb, Wn = (omega + om_o) + wb;  // Wn > 0: key 0 is visible
-          if (j == 0 || fabsf(Tn) > kTheta * Wn) {
+          if (j == 0 || fabsf(Tn) > Dims<D>::kTheta * Wn) {
             const float cn = cen + Tn / Wn;
             delta = cn - cen;  // the shift as represented
             cen = cn;
@@ -796,7 +811,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const float ad = alpha * delta;
 #pragma unroll 1
-          for (int c0 = 0; c0 < kD; c0 += 16) {
+          for (int c0 = 0; c0 < D; c0 += 16) {
             uint32_t o1[16], o2[16];
             const uint32_t a1 = sb + kColO1 + c0, a2 = sb + kColO2 + c0;
             tmem_ld16(a1, o1);
@@ -868,7 +883,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       gb += ti.nblk;
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
-      __nv_bfloat16* orow = i < p.N ? p.out + ((long long)ti.bh * p.N + i) * kD : nullptr;
+      __nv_bfloat16* orow = i < p.N ? p.out + ((long long)ti.bh * p.N + i) * D : nullptr;
       if (owner_last) {
         if (!(ok = epilogue(tc, orow, inv, c1))) break;
       } else {
@@ -911,11 +926,11 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 // 2-D view [rows, 128] of a bf16 [B, H, N, 128] tensor, boxes of 64 dims x box_rows rows.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
+bool make_map(CUtensorMap* m, const void* base, long long rows, int box_rows, int d) {
   auto enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
   cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
@@ -926,14 +941,15 @@ bool make_map(CUtensorMap* m, const void* base, long long rows, int box_rows) {
 
 }  // namespace
 
-bool prefill_tc_supported(int d) { return d == kD; }
+namespace {
 
-cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms) {
+template <int D>
+cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   const long long rows = (long long)a.B * a.H * a.N;
   if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
   CUtensorMap mQ, mR, mK, mV;
-  if (!make_map(&mQ, a.Q, rows, kBM) || !make_map(&mR, a.R, rows, kBM) || !make_map(&mK, a.K, rows, kBN) ||
-      !make_map(&mV, a.V, rows, kBN))
+  if (!make_map(&mQ, a.Q, rows, kBM, D) || !make_map(&mR, a.R, rows, kBM, D) || !make_map(&mK, a.K, rows, kBN, D) ||
+      !make_map(&mV, a.V, rows, kBN, D))
     return cudaErrorInvalidValue;
   const int ntile = (a.N + kBM - 1) / kBM;
   int ch = (2 * num_sms + ntile - 1) / ntile;  // about two waves of tiles per chunk
@@ -943,13 +959,24 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
   Params p{a.B, a.H, a.N, a.causal, ch, inject, reinterpret_cast<__nv_bfloat16*>(a.out), a.status};
-  const size_t smem = sizeof(Smem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(Smem<D>) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)((a.N + kBM - 1) / kBM) * a.B * a.H;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  prefill_tc_kernel<<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
+  prefill_tc_kernel<D><<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int d) { return d == 64 || d == 128; }
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms) {
+  if (a.d == 128) return launch_d<128>(a, st, num_sms);
+  if (a.d == 64) return launch_d<64>(a, st, num_sms);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace plx

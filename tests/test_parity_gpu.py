@@ -83,7 +83,8 @@ def test_fp32_shapes(plx, N, d, causal):
 
 
 @pytest.mark.parametrize("N,d,causal", [(1, 128, True), (100, 128, True), (300, 128, True),
-                                        (300, 128, False), (257, 64, True), (513, 128, True)])
+                                        (300, 128, False), (257, 64, True), (513, 128, True),
+                                        (1, 64, True), (300, 64, False), (513, 64, True)])
 def test_bf16_prefill_small(plx, N, d, causal):
     got, want = _prefill_case(plx, 11, 2, 3, N, d, synth.BF16, causal, qk_dist=synth.RMS_ROWS)
     assert rel_err_rms(got, want) <= BF16_TOL
@@ -95,12 +96,13 @@ def test_bf16_prefill_r_zero(plx):
     assert rel_err_rms(got, want) <= BF16_TOL
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
-def test_bf16_prefill_rescale_path(plx, causal):
+def test_bf16_prefill_rescale_path(plx, causal, d):
     """Keys from position 200 on are scaled by 8, so the running max of later
     rows jumps by far more than 2^8 after their first blocks: the kernels must
     rescale the partial O1, O2, omega and T exactly."""
-    B, H, N, d = 1, 2, 520, 128
+    B, H, N = 1, 2, 520
     specs = synth.prefill_specs(B, H, N, d)
     dev, ref = small_inputs(13, specs, synth.BF16)
     dev["K"][:, :, 200:] *= 8
@@ -126,6 +128,18 @@ def _sampled_prefill(plx, seed, B, H, N, d, rows):
         want.append(oracle.parallax_row(q, r, K, V))
         got.append(out[b, h, i].double().cpu().numpy())
     return np.stack(got), np.stack(want), out
+
+
+def test_prefill_compute_matched_d64_sampled(plx):
+    """Head dim halved at the same width (the pages' compute-matched control):
+    causal prefill B=8, H=32, N=4096, d=64 bf16, sampled rows across tiles."""
+    B, H, N, d = 8, 32, 4096, 64
+    rng = np.random.default_rng(4)
+    rows = [(0, 0, 0), (7, 31, N - 1), (3, 17, 127), (5, 2, 128)] + \
+        [(int(rng.integers(B)), int(rng.integers(H)), int(rng.integers(N))) for _ in range(8)]
+    got, want, out = _sampled_prefill(plx, 1006, B, H, N, d, rows)
+    assert rel_err_rms(got, want) <= BF16_TOL
+    assert torch.isfinite(out).all()
 
 
 def test_config_prefill_full_size_sampled(plx):
