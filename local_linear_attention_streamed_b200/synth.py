@@ -54,6 +54,7 @@ BF16 = 1
 
 # Tensor ids: one independent stream per tensor of a workload.
 TID_Q, TID_K, TID_V, TID_R, TID_SEQLENS = 1, 2, 3, 4, 5
+TID_DO = 6
 TID_X, TID_WQ, TID_WK, TID_WV, TID_WR, TID_WO = 11, 12, 13, 14, 15, 16
 
 
@@ -196,6 +197,13 @@ def decode_specs(B, H, L, d, rho_sigma=0.25):
         "V": TensorSpec(TID_V, (B, H, L, d), NORMAL, 1.0),
         "r": TensorSpec(TID_R, (B, H, d), NORMAL, rho_sigma),
     }
+
+
+def backward_specs(B, H, N, d, qk_dist=RMS_ROWS, rho_sigma=0.25):
+    """prefill_specs plus the output gradient dO ~ N(0, 1), all [B, H, N, d]."""
+    specs = prefill_specs(B, H, N, d, qk_dist=qk_dist, rho_sigma=rho_sigma)
+    specs["dO"] = TensorSpec(TID_DO, (B, H, N, d), NORMAL, 1.0)
+    return specs
 
 
 def decode_gqa_specs(B, H, Hkv, L, d, rho_sigma=0.25):
