@@ -9,7 +9,8 @@ than the 126 MB L2, so no flush is needed).  The same run measures the causal
 prefill B=8, H=16, N=4096, d=128 bf16 in TFLOP/s (the metric's second half)
 under "prefill", a layer step (projections, RMSNorm+RoPE, attention) under
 "layer", and the grouped-KV decode B=64, H=32, Hkv=8, L=4096, d=128 in GB/s
-under "decode_gqa".  For N > 1 GPUs (launched by torchrun) every rank runs the
+under "decode_gqa", and the training forward plus backward pass of the
+prefill workload under "prefill.backward".  For N > 1 GPUs (launched by torchrun) every rank runs the
 same per-GPU workload on its own seeded inputs with no data-path collective
 (weak scaling); time is the max over ranks.
 
@@ -68,6 +69,13 @@ def decode_bytes(seqlens, H, d):
 def prefill_flops(B, H, N, d, causal=True):
     pairs = N * (N + 1) // 2 if causal else N * N
     return 8.0 * d * pairs * B * H
+
+
+def backward_flops(B, H, N, d, causal=True):
+    """Algorithmic flops of the backward pass: eight GEMMs per visible pair
+    (S, T, dA = dO V^T, dV, dK from dl and from dt, dQ, dR), 2 d flops each."""
+    pairs = N * (N + 1) // 2 if causal else N * N
+    return 16.0 * d * pairs * B * H
 
 
 def prefill_bytes(B, H, N, d):
@@ -344,6 +352,54 @@ def run_gpu(args, rank, world, dist):
         del qt
         torch.cuda.empty_cache()
 
+        # Training: forward that saves the backward's inputs, then the backward
+        # pass (three launches: statistics, dK/dV, dQ/dR) on the same workload.
+        if not args.no_backward:
+            bspecs = synth.backward_specs(pB, pH, pN, pd)
+            bt = {}
+            for name, spec in bspecs.items():
+                bt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+                synth.device_fill(bt[name].data_ptr(), synth.BF16, seed + 7, spec)
+            saved = plx.prefill_train(bt["Q"], bt["K"], bt["V"], bt["R"], True)
+            grads = tuple(torch.empty_like(bt["Q"]) for _ in range(4))
+            bws = torch.empty(plx.prefill_bwd_workspace_bytes(pB, pH, pN, pd) // 4, dtype=torch.float32,
+                              device=dev)
+
+            def trn():
+                plx.prefill_train(bt["Q"], bt["K"], bt["V"], bt["R"], True)
+
+            def bwd():
+                plx.prefill_backward(bt["Q"], bt["K"], bt["V"], bt["R"], *saved, bt["dO"], True, grads=grads,
+                                     workspace=bws)
+
+            t_total, t_per = timed(trn, psteps, max(3, args.warmup // 2), stream, dist)
+            b_total, b_per = timed(bwd, psteps, max(3, args.warmup // 2), stream, dist)
+            if plx.get_device_status() != 0:
+                raise RuntimeError("backward reported a device error")
+            b_total = max_over_ranks(b_total, dist)
+            bflops = backward_flops(pB, pH, pN, pd)
+            b_ach = bflops / (float(np.mean(b_per)) * 1e-3) / 1e12
+            t_ms = float(np.mean(t_per))
+            prefill["backward"] = {
+                "workload": f"causal prefill backward B={pB} H={pH} N={pN} d={pd} bf16 "
+                            "(dQ, dK, dV, dR from dO and the training forward's out, vbar, lse, tbar)",
+                "metric": "backward TFLOP/s", "unit": "TFLOP/s",
+                "value": round(sum_over_ranks(bflops * psteps, dist) / (b_total * 1e-3) / 1e12, 2),
+                "ms_per_step": round(b_total / psteps, 3), "steps": psteps,
+                "achieved": round(b_ach, 1), "frac": round(b_ach / peaks["bf16_tflops"], 4),
+                "frac_of_sustained": round(b_ach / peaks["bf16_tflops_sustained"], 4),
+                "algorithmic_flops_per_step": bflops,
+                "executed_mma_flops_per_step": bflops * 11.0 / 8.0,
+                "flops_note": "algorithmic = 8 GEMMs per visible pair; the two kernels issue 11 "
+                              "(the scores are recomputed in the dQ/dR kernel)",
+                "gpu_launches_per_step": 3,
+                "train_forward_ms": round(t_ms, 3),
+                "train_forward_tflops": round(flops / (t_ms * 1e-3) / 1e12, 1),
+                "train_step_ms": round(t_ms + float(np.mean(b_per)), 3),
+            }
+            del bt, saved, grads, bws
+            torch.cuda.empty_cache()
+
     # ---- Decode with grouped KV heads (the next row of the scope: one KV stream per group).
     gqa = None
     if not args.no_gqa:
@@ -589,6 +645,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-gqa", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],

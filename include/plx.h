@@ -65,6 +65,10 @@ typedef enum { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
 #define PLX_ERR_TIMEOUT (-7)      /* device-reported: a bounded wait gave up (tests force
                                      it with the environment PLX_FAULT_INJECT=prefill_stall) */
 
+/* Name of the CUDA error behind this thread's last PLX_ERR_CUDA from a kernel
+ * launch ("no error" if there was none).  Static string. */
+const char* plx_last_cuda_error(void);
+
 /* Supported shapes: bf16 with d in {64, 128}; f32 with d a multiple of 32 and
  * d <= 128.  B, H, N, L >= 1. */
 
@@ -78,6 +82,51 @@ int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void
 /* As plx_prefill with an explicit element type and stream. */
 int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, void* out,
                    int B, int H, int N, int d, int causal, int dtype, void* stream);
+
+/*
+ * Training forward: the causal (or full) bf16 prefill of plx_prefill_ex that
+ * also saves what plx_prefill_bwd needs, per query row i of head (b, h):
+ *   vbar[b,h,i,:] = sum_j p_ij v_j                 (fp32 [B, H, N, d]),
+ *   lse[b,h,i]    = log sum_j exp(q_i . k_j / sqrt(d))  (fp32 [B, H, N], natural log),
+ *   tbar[b,h,i]   = sum_j p_ij (rho_i . k_j)       (fp32 [B, H, N]),
+ * with p_ij the softmax weights over the visible keys ("Parallax: Parameterized
+ * Local Linear Attention for Language Modeling": the softmax weights and the
+ * probe scores of the rainbus.top summary's forward steps; vbar and tbar are
+ * the weighted means that centre the covariance of the gist.science summary's
+ * "Mecanismo central").  out as plx_prefill_ex.  d in {64, 128}, else
+ * PLX_ERR_UNSUPPORTED.  All pointers device memory, caller-owned; Q, K, V, R,
+ * out and vbar 16-byte aligned, lse and tbar 4-byte aligned, else
+ * PLX_ERR_MISALIGNED.
+ * Asynchronous on `stream`.
+ */
+int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R, void* out,
+                      void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
+                      void* stream);
+
+/* Bytes of the statistics workspace plx_prefill_bwd needs:
+ * 16 * B * H * (N rounded up to a multiple of 128); 0 for invalid sizes. */
+size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * Backward pass of the prefill: the gradients dQ, dK, dV, dR (bf16, each
+ * [B, H, N, d], overwritten) of sum(out * dO) for one causal (or full) bf16
+ * prefill, given its inputs Q, K, V, R, the output gradient dO and the tensors
+ * plx_prefill_train saved (out, vbar, lse, tbar).  The pages train the layer
+ * but print no backward pass: these are the exact gradients of the forward
+ * definition (per query i, out_i = sum_j p_ij (1 - t_ij + tbar_i) v_j with
+ * t_ij = rho_i . k_j), computed on tensor cores with fp32 accumulation and
+ * bf16 rounding of the per-pair weights before each gradient MMA.
+ * workspace: device memory of plx_prefill_bwd_workspace_bytes(B, H, N, d)
+ * bytes, 16-byte aligned, no initial contents, or NULL for a library-owned
+ * one (grown on demand, per device; calls on one device must then be ordered).
+ * d in {64, 128}, else PLX_ERR_UNSUPPORTED; tensors 16-byte aligned, lse and
+ * tbar 4-byte aligned, else PLX_ERR_MISALIGNED; a short workspace gives
+ * PLX_ERR_WORKSPACE.  Three kernel launches, asynchronous on `stream`.
+ */
+int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                    const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                    void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * One decode step with split-KV: every (b, h) streams its cache rows

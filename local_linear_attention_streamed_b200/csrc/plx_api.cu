@@ -4,6 +4,7 @@
 
 #include <cublas_v2.h>
 
+#include <cstdio>
 #include <mutex>
 
 #include "../../include/plx.h"
@@ -26,6 +27,8 @@ struct DeviceCache {
   size_t counters_bytes = 0;
   void* layer_ws = nullptr;
   size_t layer_ws_bytes = 0;
+  void* bwd_ws = nullptr;  // per-row statistics of the prefill backward pass
+  size_t bwd_ws_bytes = 0;
   cublasHandle_t cublas = nullptr;
 };
 
@@ -35,6 +38,16 @@ DeviceCache g_dev[kMaxDevices];
 int current_device(DeviceCache** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
+  // Binds the device's primary context to this thread: the tensor-map encoder
+  // (a driver call) fails in a thread whose context is not yet current, e.g.
+  // an autograd worker that has made no runtime call of its own.
+  if (cudaSetDevice(dev) != cudaSuccess) return PLX_ERR_CUDA;
+  // Launch failures are read back with cudaGetLastError, which also returns a
+  // non-sticky error that an earlier runtime call of this thread left unread
+  // (another library's, e.g. on an autograd worker thread).  Drop it here so
+  // that only this call's own launches are judged; a sticky error (a faulted
+  // context) comes back from the launch itself.
+  (void)cudaGetLastError();
   DeviceCache& c = g_dev[dev];
   if (!c.init) {
     if (cudaDeviceGetAttribute(&c.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -48,6 +61,16 @@ int current_device(DeviceCache** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The CUDA error behind this thread's last PLX_ERR_CUDA from a launch
+// (plx_last_cuda_error reports it).
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+
+int cuda_rc(cudaError_t e) {
+  if (e == cudaSuccess) return PLX_OK;
+  t_last_cuda = e;
+  return PLX_ERR_CUDA;
+}
 
 
 // Shapes each kernel family supports.
@@ -104,6 +127,13 @@ extern "C" {
 
 int plx_abi_version(void) { return PLX_ABI_VERSION; }
 
+const char* plx_last_cuda_error(void) {
+  thread_local char buf[160];
+  const char* where = bwd_last_failure();
+  snprintf(buf, sizeof buf, "%s%s%s", cudaGetErrorString(t_last_cuda), where[0] ? " at " : "", where);
+  return buf;
+}
+
 const char* plx_status_string(int code) {
   switch (code) {
     case PLX_OK: return "ok";
@@ -138,12 +168,69 @@ int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, v
   } else {
     e = launch_prefill_simt(a, dtype == PLX_BF16, st);
   }
-  return e == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return cuda_rc(e);
 }
 
 int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
                 int H, int N, int d, int causal) {
   return plx_prefill_ex(Q, K, V, R, out, B, H, N, d, causal, PLX_BF16, nullptr);
+}
+
+int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R, void* out,
+                      void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
+                      void* stream) {
+  if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(R) || !aligned16(out) ||
+      !aligned16(vbar) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(tbar) & 3u))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  PrefillArgs a{Q, K, V, R, out, B, H, N, d, causal ? 1 : 0, dc->status};
+  a.vbar = vbar;
+  a.lse = lse;
+  a.tbar = tbar;
+  return cuda_rc(launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream), dc->num_sms));
+}
+
+size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
+  return 16 * (size_t)B * H * bwd_padded_rows(N);
+}
+
+int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                    const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                    void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar || !dO || !dQ || !dK || !dV || !dR)
+    return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
+  const void* t16[] = {Q, K, V, R, out, vbar, dO, dQ, dK, dV, dR};
+  for (const void* t : t16)
+    if (!aligned16(t)) return PLX_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(tbar) & 3u))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H * (long long)bwd_padded_rows(N) >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
+  const size_t need = plx_prefill_bwd_workspace_bytes(B, H, N, d);
+  if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
+  if (workspace && !aligned16(workspace)) return PLX_ERR_MISALIGNED;
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  BwdArgs a{Q, K, V, R, out, vbar, dO, lse, tbar, dQ, dK, dV, dR, B, H, N, d, causal ? 1 : 0, workspace,
+            dc->status};
+  if (!workspace) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = grow(&dc->bwd_ws, &dc->bwd_ws_bytes, need, st)) != PLX_OK) return rc;
+    a.stats = dc->bwd_ws;
+    return cuda_rc(launch_prefill_bwd(a, st));
+  }
+  return cuda_rc(launch_prefill_bwd(a, st));
 }
 
 int plx_decode_num_splits(int B, int H, int L, int d) {
@@ -188,7 +275,7 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
   a.d = d;
   a.status = dc->status;
   if (dtype == PLX_F32) {
-    return launch_decode_simt(a, false, st) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+    return cuda_rc(launch_decode_simt(a, false, st));
   }
   size_t need = decode_ws_layout(B, H, L, d, dc->num_sms, &a.splits, &a.chunk);
   if (need > 0) {
@@ -207,7 +294,7 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
       a.partials = static_cast<float*>(dc->decode_ws);
     }
   }
-  return launch_decode_bf16(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return cuda_rc(launch_decode_bf16(a, st, dc->num_sms));
 }
 
 size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
@@ -270,7 +357,7 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
       a.partials = static_cast<float*>(dc->decode_ws);
     }
   }
-  return launch_decode_gqa(a, st, dc->num_sms) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return cuda_rc(launch_decode_gqa(a, st, dc->num_sms));
 }
 
 int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vcache,
@@ -286,10 +373,8 @@ int plx_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float 
   if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
   if ((long long)B * N * H * d >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(y)) return PLX_ERR_MISALIGNED;
-  return launch_qkr_norm_rope(x, y, B, N, H, d, eps, rope_base,
-                              reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? PLX_OK
-             : PLX_ERR_CUDA;
+  return cuda_rc(launch_qkr_norm_rope(x, y, B, N, H, d, eps, rope_base,
+                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t plx_layer_workspace_bytes(int B, int N, int H, int d) {

@@ -28,6 +28,11 @@ struct PrefillArgs {
   int B, H, N, d;
   int causal;
   int* status;
+  // Optional (tensor-core path only): softmax mean of v [rows, d] and the
+  // per-row lse and tbar [rows], all fp32, for the backward pass.
+  void* vbar = nullptr;
+  float* lse = nullptr;
+  float* tbar = nullptr;
 };
 
 struct DecodeArgs {
@@ -65,6 +70,32 @@ inline int decode_gqa_ctas_per_sm(int G) { return G == 8 ? 1 : 2; }
 // bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
 bool prefill_tc_supported(int d);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms);
+
+// Backward pass of the bf16 tensor-core prefill (d in {64, 128}): gradients of
+// Q, K, V, R from the output gradient dO and the forward's out, vbar, lse and
+// tbar.  `stats` is a workspace of B * H * bwd_padded_rows(N) float4.
+struct BwdArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const void* R;
+  const void* out;
+  const void* vbar;
+  const void* dO;
+  const float* lse;
+  const float* tbar;
+  void* dQ;
+  void* dK;
+  void* dV;
+  void* dR;
+  int B, H, N, d, causal;
+  void* stats;
+  int* status;
+};
+size_t bwd_padded_rows(int N);
+// The step of this thread's last failed backward launch ("" if none).
+const char* bwd_last_failure();
+cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st);
 
 // Per-head RMSNorm + RoPE with the head split folded in.
 cudaError_t launch_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,

@@ -14,6 +14,7 @@ import torch
 
 PLX_F32 = 0
 PLX_BF16 = 1
+PLX_ERR_CUDA = -4
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libplx.so")
@@ -33,15 +34,22 @@ SIGNATURES = {
     "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
     "plx_layer_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
+    "plx_prefill_train": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
+    "plx_prefill_bwd_workspace_bytes": (_sz, [_i] * 4),
+    "plx_prefill_bwd": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_get_device_status": (_i, [_vp]),
     "plx_status_string": (ctypes.c_char_p, [_i]),
+    "plx_last_cuda_error": (ctypes.c_char_p, []),
     "plx_abi_version": (_i, []),
 }
 
 
 class PlxError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        msg = f"{where}: {status_string(code)} (code {code})"
+        if code == PLX_ERR_CUDA:
+            msg += f": {lib.plx_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -103,6 +111,87 @@ def prefill(Q, K, V, R, causal: bool = True, out=None, stream=None):
                             B, H, N, d, int(bool(causal)), _dtype_code(Q), _stream_ptr(stream))
     _check(rc, "plx_prefill_ex")
     return out
+
+
+def prefill_train(Q, K, V, R, causal: bool = True, stream=None):
+    """bf16 prefill that also saves the backward pass's inputs.
+
+    Returns (out, vbar, lse, tbar): out bf16 [B, H, N, d], vbar fp32
+    [B, H, N, d], lse and tbar fp32 [B, H, N] (see plx_prefill_train in
+    include/plx.h).
+    """
+    B, H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("R", R)):
+        if t.shape != Q.shape or t.dtype != Q.dtype:
+            raise ValueError(f"{n} must match Q in shape and dtype")
+    if Q.dtype != torch.bfloat16:
+        raise TypeError("prefill_train takes bf16 tensors")
+    out = torch.empty_like(Q)
+    vbar = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    tbar = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    rc = lib.plx_prefill_train(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                               _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, N, d,
+                               int(bool(causal)), _stream_ptr(stream))
+    _check(rc, "plx_prefill_train")
+    return out, vbar, lse, tbar
+
+
+def prefill_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib.plx_prefill_bwd_workspace_bytes(B, H, N, d))
+
+
+def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, grads=None,
+                     workspace=None, stream=None):
+    """Gradients (dQ, dK, dV, dR) of sum(out * dO) for one bf16 prefill.
+
+    ``out, vbar, lse, tbar`` are what prefill_train returned for the same
+    inputs; ``grads`` optionally gives the four output tensors.
+    """
+    B, H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("R", R), ("out", out), ("dO", dO)):
+        if t.shape != Q.shape or t.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be bf16 of Q's shape")
+    if vbar.shape != Q.shape or vbar.dtype != torch.float32:
+        raise ValueError("vbar must be fp32 of Q's shape")
+    for n, t in (("lse", lse), ("tbar", tbar)):
+        if t.shape != (B, H, N) or t.dtype != torch.float32:
+            raise ValueError(f"{n} must be fp32 [B, H, N]")
+    if grads is None:
+        grads = tuple(torch.empty_like(Q) for _ in range(4))
+    dQ, dK, dV, dR = grads
+    ws, wsb = (0, 0) if workspace is None else (_dev(workspace, "workspace"),
+                                                workspace.numel() * workspace.element_size())
+    rc = lib.plx_prefill_bwd(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                             _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), _dev(dO, "dO"),
+                             _dev(dQ, "dQ"), _dev(dK, "dK"), _dev(dV, "dV"), _dev(dR, "dR"),
+                             B, H, N, d, int(bool(causal)), ws, wsb, _stream_ptr(stream))
+    _check(rc, "plx_prefill_bwd")
+    return dQ, dK, dV, dR
+
+
+class ParallaxAttention(torch.autograd.Function):
+    """Autograd wrapper: forward = prefill_train, backward = prefill_backward (bf16)."""
+
+    @staticmethod
+    def forward(ctx, Q, K, V, R, causal=True):
+        Q, K, V, R = (t.contiguous() for t in (Q, K, V, R))
+        out, vbar, lse, tbar = prefill_train(Q, K, V, R, causal)
+        ctx.save_for_backward(Q, K, V, R, out, vbar, lse, tbar)
+        ctx.causal = causal
+        return out
+
+    @staticmethod
+    def backward(ctx, dO):
+        Q, K, V, R, out, vbar, lse, tbar = ctx.saved_tensors
+        dQ, dK, dV, dR = prefill_backward(Q, K, V, R, out, vbar, lse, tbar,
+                                          dO.contiguous().to(torch.bfloat16), ctx.causal)
+        return dQ, dK, dV, dR, None
+
+
+def parallax_attention(Q, K, V, R, causal: bool = True):
+    """Differentiable bf16 Parallax attention over [B, H, N, d] (d in {64, 128})."""
+    return ParallaxAttention.apply(Q, K, V, R, causal)
 
 
 def decode_workspace_bytes(B: int, H: int, L: int, d: int) -> int:

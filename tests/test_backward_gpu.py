@@ -1,0 +1,185 @@
+"""GPU parity of the training forward (saved statistics) and of the backward
+pass, through the C ABI, against the float64 oracle on the same seeded inputs.
+
+Bars.  The training forward's out is the inference kernel's out bit for bit;
+vbar (fp32, from the bf16 weights of the value MMAs) is held to the forward's
+bf16 bar (max |g - o| / RMS of the row <= 2e-2); lse and tbar are fp32 results
+of fp32 sums over bf16 inputs (bar 1e-4 of max(1, |lse|) and 1e-3 of
+max(1, RMS(t))).  Each whole gradient tensor is held to a relative Frobenius
+error <= GRAD_TOL and a largest elementwise error
+max_e |g - o| / max(|o_e|, RMS(o)) <= GRAD_MAX_TOL (derived in tests/_util.py
+and checked attainable in tests/test_backward_bound.py).  The backward kernels
+are checked twice: given the oracle's saved tensors (their own error alone),
+and after the training forward (the composition a user runs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from local_linear_attention_streamed_b200 import synth
+from _util import (BF16_TOL, GRAD_MAX_TOL, GRAD_TOL, device_inputs, rel_err_elem, rel_err_fro, rel_err_rms,
+                   small_inputs, to_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def plx():
+    from local_linear_attention_streamed_b200 import plx as mod
+    assert torch.cuda.is_available()
+    return mod
+
+
+def _check_grads(grads, want, where=""):
+    for name, g, w in zip(("dQ", "dK", "dV", "dR"), grads, want):
+        assert torch.isfinite(g).all(), (name, where)
+        gf = to_f64(g).reshape(w.shape)
+        if not np.any(w):
+            # A single visible key: out = v_0 whatever q, k and rho are, so
+            # dQ, dK and dR are exactly zero; the kernels leave the fp32
+            # rounding residue of dA - F (inputs are O(1)).
+            assert np.max(np.abs(gf)) <= 1e-3, (name, where)
+            continue
+        fro, emax = rel_err_fro(gf, w), rel_err_elem(gf, w)
+        assert fro <= GRAD_TOL and emax <= GRAD_MAX_TOL, (name, where, fro, emax)
+
+
+def _case(plx, seed, B, H, N, d, causal):
+    specs = synth.backward_specs(B, H, N, d)
+    dev, ref = small_inputs(seed, specs, synth.BF16)
+    out, vbar, lse, tbar = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], causal)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], out, vbar, lse, tbar, dev["dO"], causal)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    return dev, ref, (out, vbar, lse, tbar), grads
+
+
+@pytest.mark.parametrize("N,d,causal", [(320, 128, True), (200, 64, False), (1, 128, True)])
+def test_train_forward_saved_statistics(plx, N, d, causal):
+    B, H = 2, 3
+    dev, ref, (out, vbar, lse, tbar), _ = _case(plx, 300 + N, B, H, N, d, causal)
+    plain = plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=causal)
+    assert torch.equal(out, plain)
+    w_vbar, w_lse, w_tbar = oracle.prefill_stats_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal)
+    assert rel_err_rms(to_f64(vbar), w_vbar) <= BF16_TOL
+    assert np.max(np.abs(to_f64(lse) - w_lse) / np.maximum(1.0, np.abs(w_lse))) <= 1e-4
+    t_rms = np.sqrt(np.mean((ref["R"] * ref["K"]).sum(-1) ** 2)) * np.sqrt(N)
+    assert np.max(np.abs(to_f64(tbar) - w_tbar)) <= 1e-3 * max(1.0, t_rms)
+
+
+CASES = [(64, 128, True), (200, 128, True), (320, 128, False), (384, 128, True),
+         (256, 64, True), (200, 64, False), (130, 64, True), (1, 128, True), (1, 64, False)]
+
+
+@pytest.mark.parametrize("N,d,causal", CASES)
+def test_backward_kernels_match_oracle(plx, N, d, causal):
+    """The backward kernels alone, fed the oracle's saved tensors (out rounded
+    to bf16 as the forward stores it): every element of dQ, dK, dV, dR over
+    several 64/128-row tiles, ragged tails (N not a multiple of 64 or 128), a
+    single key, causal and full."""
+    B, H = 1, 2
+    specs = synth.backward_specs(B, H, N, d)
+    dev, ref = small_inputs(500 + N + d, specs, synth.BF16)
+    vbar, lse, tbar = oracle.prefill_stats_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal)
+    out = oracle.prefill_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal=causal)
+    cuda = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dt).cuda()
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], cuda(out, torch.bfloat16),
+                                 cuda(vbar, torch.float32), cuda(lse, torch.float32), cuda(tbar, torch.float32),
+                                 dev["dO"], causal)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], causal)
+    _check_grads(grads, want)
+
+
+@pytest.mark.parametrize("N,d,causal", CASES)
+def test_train_forward_then_backward_matches_oracle(plx, N, d, causal):
+    """The composition a user runs: training forward, then the backward pass."""
+    B, H = 1, 2
+    _, ref, _, grads = _case(plx, 500 + N + d, B, H, N, d, causal)
+    want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], causal)
+    _check_grads(grads, want)
+
+
+def test_backward_caller_workspace_and_autograd(plx):
+    B, H, N, d = 1, 2, 192, 128
+    specs = synth.backward_specs(B, H, N, d)
+    dev, ref = small_inputs(77, specs, synth.BF16)
+    ws = torch.empty(plx.prefill_bwd_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32, device="cuda")
+    out, vbar, lse, tbar = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    g1 = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], out, vbar, lse, tbar, dev["dO"], True,
+                              workspace=ws)
+    leaves = [dev[n].clone().requires_grad_(True) for n in "QKVR"]
+    o2 = plx.parallax_attention(*leaves, causal=True)
+    o2.backward(dev["dO"])
+    assert torch.equal(o2.detach(), out)
+    for a, leaf in zip(g1, leaves):
+        assert torch.equal(a, leaf.grad)
+
+
+def test_backward_rejects_bad_arguments(plx):
+    B, H, N, d = 1, 1, 64, 96
+    x = torch.zeros((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    vb = torch.zeros((B, H, N, d), dtype=torch.float32, device="cuda")
+    s = torch.zeros((B, H, N), dtype=torch.float32, device="cuda")
+    with pytest.raises(plx.PlxError) as e:
+        plx.prefill_backward(x, x, x, x, x, vb, s, s, x, True)
+    assert e.value.code == -2
+    d = 128
+    x = torch.zeros((B, H, N, d), dtype=torch.bfloat16, device="cuda")
+    vb = torch.zeros((B, H, N, d), dtype=torch.float32, device="cuda")
+    ws = torch.empty(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(plx.PlxError) as e:
+        plx.prefill_backward(x, x, x, x, x, vb, s, s, x, True, workspace=ws)
+    assert e.value.code == -5
+
+
+def test_backward_full_size_heads(plx):
+    """Causal B=8, H=16, N=4096, d=128 (the prefill workload), in the launch
+    configuration the benchmark times; two whole heads (heads are independent)
+    compared element by element with the oracle run on those heads alone."""
+    B, H, N, d = 8, 16, 4096, 128
+    seed = 1010
+    specs = synth.backward_specs(B, H, N, d)
+    dev = device_inputs(seed, specs, synth.BF16)
+    out, vbar, lse, tbar = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], out, vbar, lse, tbar, dev["dO"], True)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    for g in grads:
+        assert torch.isfinite(g).all()
+    for (b, h) in [(0, 0), (7, 13)]:
+        row0 = (b * H + h) * N
+        head = {n: synth.host_rows_f64(seed, specs[n], synth.BF16, row0, N).reshape(1, 1, N, d)
+                for n in ("Q", "K", "V", "R", "dO")}
+        want = oracle.parallax_backward_ref(head["Q"], head["K"], head["V"], head["R"], head["dO"], True)
+        _check_grads([g[b, h] for g in grads], [w[0, 0] for w in want], where=(b, h))
+
+
+def test_calls_from_a_fresh_thread(plx):
+    """The library binds the device's context in every call, so a thread that
+    has made no CUDA call of its own (an autograd worker, a data loader) can
+    call it after another thread did (the tensor maps need a current context)."""
+    import threading
+    B, H, N, d = 1, 2, 128, 128
+    dev, _ = small_inputs(88, synth.backward_specs(B, H, N, d), synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    first = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+    res = {}
+
+    def work():
+        try:
+            res["g"] = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+            res["o"] = plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=True)
+            torch.cuda.synchronize()
+        except Exception as e:  # reported below
+            res["e"] = e
+
+    t = threading.Thread(target=work)
+    t.start()
+    t.join()
+    assert "e" not in res, res.get("e")
+    for a, b in zip(first, res["g"]):
+        assert torch.equal(a, b)
+    assert torch.equal(res["o"], saved[0])
