@@ -19,20 +19,23 @@
 // costs no precision.
 //
 // Three launches:
-//  1. prep: per query row, the statistics (lse in log2 units, 1 + tbar, D,
-//     D - F) from the forward's saved lse, tbar, vbar (fp32: D from a bf16
+//  1. prep: per query row, the statistics (-lse in log2 units, 1 + tbar, D,
+//     F - D) from the forward's saved lse, tbar, vbar (fp32: D from a bf16
 //     vbar would carry its rounding into every dt and dl of the row) and out,
-//     into a per-head padded workspace (padding rows give p = 0).
+//     into a per-head padded workspace (padding rows give p = 0), laid out
+//     by 64-row blocks as four arrays of 64 floats (one 1 KB copy per block).
 //  2. dK/dV: one CTA per 128-key block of a head.  K and V stay in shared
-//     memory; 64-query blocks stream through a two-stage ring (Q and R stacked
-//     as one 128-row operand, dO, the 64 rows' statistics).  Per block:
+//     memory; 64-query blocks stream through a three-stage ring (Q and R
+//     stacked as one 128-row operand, and dO).  Per block:
 //       [S^T | T^T] = K [Q; R]^T   (one N = 128 MMA: keys are M, so Q and R
 //                                   share it as the B operand)
 //       dA^T        = V dO^T
-//     the elementwise warps turn the scores into a^T, dl^T/sqrt(d) and dt^T
-//     (bf16, shared memory, K-major), then
-//       dV += a^T dO,   dK += [dl^T | dt^T] [Q; R]   (one K = 128 MMA)
-//     accumulate in TMEM for the whole key block.
+//     the elementwise warps turn the scores into a^T (bf16, shared memory,
+//     K-major) and dl^T/sqrt(d), dt^T (bf16 pairs in TMEM), then
+//       dV += a^T dO,   dK += [dl^T | dt^T] [Q; R]   (one K = 128 MMA, A in TMEM)
+//     accumulate in TMEM for the whole key block.  A stage is held until the
+//     block's gradient MMAs complete, so the third stage lets the loads of
+//     block i + 2 overlap block i's elementwise step and gradient MMAs.
 //  3. dQ/dR: one CTA per 128-query block; 64-key blocks stream through a
 //     three-stage ring.  Per block S = Q K^T, T = R K^T, dA = dO V^T; the
 //     elementwise warps write dl/sqrt(d) and dt as bf16 into TMEM, and
@@ -43,7 +46,7 @@
 // gradient is written once, in bf16, with no atomics and no fp32 workspace.
 //
 // Warp roles in both kernels: warp 0 TMA producer, warp 1 TMEM owner and MMA
-// issuer (one elected thread), warps 4..11 two elementwise warpgroups that
+// issuer (one elected thread), warps 4..19 four elementwise warpgroups that
 // split each block's columns (every TMEM lane is read by one warp of each).
 // Every wait is bounded in time; one that runs out sets the device status
 // word and the CTA's abort flag, and every role unwinds.
@@ -56,7 +59,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 384;
+// Four elementwise warpgroups, each taking 16 of a block's 64 columns for every
+// TMEM lane: the per-pair arithmetic is latency-bound, so more warps per
+// scheduler hide more of it.
+constexpr int kEwGroups = 4;
+constexpr int kEwCols = 64 / kEwGroups;  // columns per elementwise thread
+constexpr int kThreads = 128 * (1 + kEwGroups);
 constexpr int kFirstEwWarp = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -77,21 +85,27 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
 // 1. Per-row statistics.
 // ---------------------------------------------------------------------------
 
-// stats[bh * Npad + i] = (lse_i log2(e), 1 + tbar_i, D_i, D_i - F_i) for i < N;
-// (+inf, 1, 0, 0) for the padding rows i in [N, Npad).  One warp per row.
+// Float index of statistic k (0..3) of row i of head bh: 64-row blocks of
+// four 64-float arrays.
+__host__ __device__ __forceinline__ size_t stat_index(int bh, int Npad, int i, int k) {
+  return ((size_t)bh * (Npad / 64) + (size_t)(i / 64)) * 256 + (size_t)k * 64 + (size_t)(i % 64);
+}
+
+// Statistics of row i: (-lse_i log2(e), 1 + tbar_i, D_i, F_i - D_i) for i < N;
+// (-inf, 1, 0, 0) for the padding rows i in [N, Npad).  One warp per row.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ out,
                                                        const float* __restrict__ vbar,
                                                        const __nv_bfloat16* __restrict__ dO,
                                                        const float* __restrict__ lse,
                                                        const float* __restrict__ tbar,
-                                                       float4* __restrict__ stats, int BH, int N, int Npad,
+                                                       float* __restrict__ stats, int BH, int N, int Npad,
                                                        int d) {
   const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= (long long)BH * Npad) return;
   const int bh = (int)(r / Npad), i = (int)(r % Npad);
   if (i >= N) {
-    if (lane == 0) stats[r] = make_float4(CUDART_INF_F, 1.f, 0.f, 0.f);
+    if (lane < 4) stats[stat_index(bh, Npad, i, lane)] = lane == 0 ? -CUDART_INF_F : (lane == 1 ? 1.f : 0.f);
     return;
   }
   const long long g = (long long)bh * N + i;
@@ -108,16 +122,36 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
     dv += __shfl_xor_sync(0xffffffffu, dv, o);
     df += __shfl_xor_sync(0xffffffffu, df, o);
   }
-  if (lane == 0) stats[r] = make_float4(lse[g] * kLog2e, 1.f + tbar[g], dv, dv - df);
+  const float v = lane == 0 ? -lse[g] * kLog2e : (lane == 1 ? 1.f + tbar[g] : (lane == 2 ? dv : df - dv));
+  if (lane < 4) stats[stat_index(bh, Npad, i, lane)] = v;
 }
 
 struct BwdParams {
   int B, H, N, Npad, causal;
-  const float4* stats;
+  int chunk_heads;  // heads whose blocks are launched together (L2 reuse of their tiles)
+  const float* stats;
   __nv_bfloat16* g0;  // dV (key-block kernel) or dQ (query-block kernel)
   __nv_bfloat16* g1;  // dK or dR
   int* status;
 };
+
+// Block t of the launch order: heads in chunks of `ch`, and within a chunk the
+// blocks with the most causal work first (rank 0 = most), across the chunk's
+// heads.  Blocks start roughly in index order, so the few heads whose blocks
+// run at one time keep their streamed tiles in L2 for all of those blocks.
+struct BlockOrder {
+  int bh, rank;
+};
+__device__ __forceinline__ BlockOrder block_order(int t, int BH, int nblk, int ch) {
+  const int per_chunk = ch * nblk;
+  const int chunk = t / per_chunk;
+  const int nh = min(ch, BH - chunk * ch);
+  const int pos = t - chunk * per_chunk;
+  BlockOrder o;
+  o.rank = pos / nh;
+  o.bh = chunk * ch + pos % nh;
+  return o;
+}
 
 // Bounded wait taken by a whole warp: every lane leaves with the same answer,
 // so the warp-collective TMEM accesses that follow are reached by all or none.
@@ -126,38 +160,60 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Elementwise step shared by both kernels, for two neighbouring (query, key)
-// pairs: scores s (raw q . k), probe scores t, dA = dO . v and the query
-// statistics st = (lse log2 e, 1 + tbar, D, D - F); `keep` clears masked
-// pairs.  Returns p (1 - t + tbar), p (D - dA) and p (u (dA - D) + D - F) / sqrt(d).
-struct Grad3 {
-  float a, dt, dl;
+// pairs at once in packed f32x2 arithmetic: raw scores s = q . k, probe scores
+// t, dA = dO . v, and the pairs' statistics nl = -lse log2 e, c0 = 1 + tbar,
+// dd = D, fd = F - D; keep0/keep1 clear masked pairs.  With p the softmax
+// weight, u = c0 - t and x = D - dA, it packs bf16 pairs of
+//   a = p u,   dt = p x,   dl = p (D - F - u x) / sqrt(d) = p (u (dA - D) + D - F) / sqrt(d).
+struct GradPairs {
+  uint32_t a, dt, dl;
 };
-__device__ __forceinline__ Grad3 grad_elem(float s, float t, float da, float4 st, float scale2, float isd,
-                                           bool keep) {
-  const float pr = keep ? ex2(fmaf(s, scale2, -st.x)) : 0.f;
-  const float u = st.y - t;   // 1 + tbar - t
-  const float x = st.z - da;  // D - dA
-  Grad3 g;
-  g.a = pr * u;
-  g.dt = pr * x;
-  g.dl = (pr * isd) * fmaf(-u, x, st.w);
+__device__ __forceinline__ uint32_t pack2(uint64_t v) {
+  float lo, hi;
+  uf2(v, lo, hi);
+  return pack_bf16(lo, hi);
+}
+__device__ __forceinline__ GradPairs grad_pairs(uint32_t s0, uint32_t s1, uint32_t t0, uint32_t t1, uint32_t a0,
+                                                uint32_t a1, uint64_t nl, uint64_t c0, uint64_t dd, uint64_t fd,
+                                                uint64_t sc2, uint64_t nisd2, bool keep0, bool keep1) {
+  const uint64_t m1 = f2(-1.f, -1.f);
+  float e0, e1;
+  uf2(fma2(f2(__uint_as_float(s0), __uint_as_float(s1)), sc2, nl), e0, e1);
+  float p0 = ex2(e0), p1 = ex2(e1);
+  p0 = keep0 ? p0 : 0.f;
+  p1 = keep1 ? p1 : 0.f;
+  const uint64_t p2 = f2(p0, p1);
+  const uint64_t u2 = fma2(f2(__uint_as_float(t0), __uint_as_float(t1)), m1, c0);
+  const uint64_t x2 = fma2(f2(__uint_as_float(a0), __uint_as_float(a1)), m1, dd);
+  GradPairs g;
+  g.a = pack2(mul2(p2, u2));
+  g.dt = pack2(mul2(p2, x2));
+  // u x - (D - F) = u x + fd; times -p / sqrt(d).
+  g.dl = pack2(mul2(mul2(p2, nisd2), fma2(u2, x2, fd)));
   return g;
 }
 
-// Writes 32 bf16 values (16 packed pairs) as 16-byte chunks c0..c0+3 of a
-// 128B-swizzled row.
-__device__ __forceinline__ void st_row_chunks(uint8_t* tile, int row, int c0, const uint32_t (&v)[16]) {
+// Writes 8 * NC bf16 values (4 * NC packed pairs) as 16-byte chunks
+// c0..c0+NC-1 of a 128B-swizzled row.
+template <int NC>
+__device__ __forceinline__ void st_row_chunks(uint8_t* tile, int row, int c0, const uint32_t (&v)[4 * NC]) {
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
+  for (int j = 0; j < NC; ++j)
     *reinterpret_cast<uint4*>(tile + sw128(row, c0 + j)) = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
-// Loads D fp32 TMEM columns of this thread's lane from `taddr` and stores them
-// as a bf16 row at dst (nullptr: load only, every lane takes part).
-template <int D>
+// 8 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]));
+}
+
+// Loads NC fp32 TMEM columns of this thread's lane from `taddr` and stores
+// them as bf16 at dst (nullptr: load only, every lane takes part).
+template <int NC>
 __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, __nv_bfloat16* dst) {
 #pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
+  for (int c0 = 0; c0 < NC; c0 += 32) {
     uint32_t v[32];
     tmem_ld32(taddr + c0, v);
     tc_wait_ld();
@@ -177,7 +233,7 @@ __device__ __forceinline__ void tmem_row_to_global(uint32_t taddr, __nv_bfloat16
 // ---------------------------------------------------------------------------
 constexpr int kKB = 128;  // keys per CTA (MMA M)
 constexpr int kQB = 64;   // queries per streamed block
-constexpr int kQStages = 2;
+constexpr int kQStages = 3;
 
 template <int D>
 struct KvSmem {
@@ -187,9 +243,7 @@ struct KvSmem {
   uint8_t v[kHalves][kKB * 128];
   uint8_t qr[kQStages][kHalves][2 * kQB * 128];  // per half: Q rows 0..63, then R rows 0..63
   uint8_t dout[kQStages][kHalves][kQB * 128];
-  uint8_t a[kKB * 128];     // a^T [128 keys][64 queries] bf16, K-major
-  uint8_t g[2][kKB * 128];  // dl^T / sqrt(d) and dt^T, the two K-chunks of one operand
-  float4 stats[kQStages][kQB];
+  uint8_t a[kKB * 128];  // a^T [128 keys][64 queries] bf16, K-major
   uint64_t kv_full, q_full[kQStages], q_empty[kQStages];
   uint64_t s_full, s_free, p_full, ag_free, done, drain;
   uint32_t tmem_base;
@@ -204,13 +258,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   using Sm = KvSmem<D>;
   constexpr int kHalves = D / 64;
-  // TMEM columns: dV and dK accumulators, then the score stage.
-  constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColT = 2 * D + 64, kColDA = 2 * D + 128;
+  // TMEM columns: dV and dK accumulators, the score stage, then the bf16
+  // pairs of dl^T / sqrt(d) (32 columns) and dt^T (32): the A operand of dK.
+  constexpr uint32_t kColDV = 0, kColDK = D, kColS = 2 * D, kColT = 2 * D + 64, kColDA = 2 * D + 128,
+                     kColG = 2 * D + 192;
   Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
-  // Key blocks in order of their query count (causal: block 0 sees every query).
-  const int kb = blockIdx.x / BH, bh = blockIdx.x % BH;
+  // Key block 0 sees every query (causal): rank r is key block r.
+  const BlockOrder bo = block_order(blockIdx.x, BH, (p.N + kKB - 1) / kKB, p.chunk_heads);
+  const int kb = bo.rank, bh = bo.bh;
   const int nqb = (p.N + kQB - 1) / kQB;
   const int q0 = p.causal ? (kb * kKB) / kQB : 0;
   const int nq = nqb - q0;  // >= 1: key block kb starts below N
@@ -223,8 +280,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.q_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_free, 8);   // lane 0 of each elementwise warp
-    mbar_init(&sm.p_full, 256);  // every elementwise thread
+    mbar_init(&sm.s_free, 4 * kEwGroups);    // lane 0 of each elementwise warp
+    mbar_init(&sm.p_full, 128 * kEwGroups);  // every elementwise thread
     mbar_init(&sm.ag_free, 1);
     mbar_init(&sm.done, 1);
     mbar_init(&sm.drain, 1);
@@ -251,11 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sm.k[h], &tmK, &sm.kv_full, 64 * h, krow);
         tma_load_2d(sm.v[h], &tmV, &sm.kv_full, 64 * h, krow);
       }
-      int last_use[kQStages] = {-1, -1};
+      int last_use[kQStages] = {-1, -1, -1};
       for (int i = 0; i < nq && !*abort; ++i) {
-        const int st = i & 1, u = i >> 1;
+        const int st = i % kQStages, u = i / kQStages;
         if (u > 0 && !mbar_wait(&sm.q_empty[st], (u - 1) & 1, abort, p.status)) break;
-        mbar_expect_tx(&sm.q_full[st], 3 * kQB * D * 2 + kQB * 16);
+        mbar_expect_tx(&sm.q_full[st], 3 * kQB * D * 2);
         last_use[st] = u;
         const int qrow = bh * p.N + (q0 + i) * kQB;
         for (int h = 0; h < kHalves; ++h) {
@@ -263,8 +320,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sm.qr[st][h] + kQB * 128, &tmR, &sm.q_full[st], 64 * h, qrow);
           tma_load_2d(sm.dout[st][h], &tmdO, &sm.q_full[st], 64 * h, qrow);
         }
-        bulk_load(sm.stats[st], p.stats + (size_t)bh * p.Npad + (size_t)(q0 + i) * kQB, kQB * 16,
-                  &sm.q_full[st]);
       }
       if (*abort) {  // let every copy issued here land before the CTA exits
         mbar_drain(&sm.kv_full, 0);
@@ -278,9 +333,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block i - 1 (their operands are written while block i's scores run).
     if (lane == 0) {
       const uint64_t aK = sdesc(smem_u32(sm.k[0]), 16, 1024), aV = sdesc(smem_u32(sm.v[0]), 16, 1024);
-      const uint64_t aA = sdesc(smem_u32(sm.a), 16, 1024), aG = sdesc(smem_u32(sm.g[0]), 16, 1024);
+      const uint64_t aA = sdesc(smem_u32(sm.a), 16, 1024);
       auto issue_grads = [&](int b) {
-        const int st = b & 1;
+        const int st = b % kQStages;
         // dO and [Q; R] as MN-major B operands: 64-dim halves apart by LBO,
         // 8-row groups by 1024 bytes, 16 rows (one K step) by 2048.
         const uint64_t bdo = sdesc(smem_u32(sm.dout[st][0]), kQB * 128, 1024);
@@ -291,15 +346,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                  (b > 0 || ks > 0) ? 1u : 0u);
 #pragma unroll
         for (int ks = 0; ks < 2 * kQB / 16; ++ks)
-          mma_ss(tmem + kColDK, aG + (uint64_t)((((ks >> 2) * kKB * 128) + (ks & 3) * 32) >> 4),
-                 bqr + (uint64_t)((ks * 2048) >> 4), idesc(D, 1), (b > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tmem + kColDK, tmem + kColG + ks * 8, bqr + (uint64_t)((ks * 2048) >> 4), idesc(D, 1),
+                 (b > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&sm.ag_free);
         mma_commit(&sm.q_empty[st]);
       };
       bool ok = mbar_wait(&sm.kv_full, 0, abort, p.status);
       for (int i = 0; ok && i < nq; ++i) {
-        const int st = i & 1;
-        if (!(ok = mbar_wait(&sm.q_full[st], (i >> 1) & 1, abort, p.status))) break;
+        const int st = i % kQStages;
+        if (!(ok = mbar_wait(&sm.q_full[st], (i / kQStages) & 1, abort, p.status))) break;
         if (i > 0 && !(ok = mbar_wait(&sm.s_free, (i - 1) & 1, abort, p.status))) break;
         tc_fence_after();
         const uint64_t bqr = sdesc(smem_u32(sm.qr[st][0]), 16, 1024);
@@ -332,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kFirstEwWarp) {
     // ---------------- elementwise warpgroups ----------------
-    // Thread = one key (TMEM lane) x 32 of the block's 64 queries (wg picks the half).
+    // Thread = one key (TMEM lane) x 16 of the block's 64 queries (wg picks which).
     const int wg = (warp - kFirstEwWarp) >> 2, quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t lb = tmem + ((uint32_t)(32 * quarter) << 16);
@@ -340,49 +395,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float isd = rsqrtf((float)D), scale2 = kLog2e * isd;
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
-      const int st = i & 1;
-      if (!(ok = warp_wait(&sm.q_full[st], (i >> 1) & 1, abort, p.status))) break;
       if (!(ok = warp_wait(&sm.s_full, i & 1, abort, p.status))) break;
       tc_fence_after();
-      uint32_t s[32], t[32], da[32];
-      tmem_ld32(lb + kColS + 32 * wg, s);
-      tmem_ld32(lb + kColT + 32 * wg, t);
-      tmem_ld32(lb + kColDA + 32 * wg, da);
+      uint32_t s[kEwCols], t[kEwCols], da[kEwCols];
+      tmem_ld16(lb + kColS + kEwCols * wg, s);
+      tmem_ld16(lb + kColT + kEwCols * wg, t);
+      tmem_ld16(lb + kColDA + kEwCols * wg, da);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free);
-      const int i0 = (q0 + i) * kQB + 32 * wg;  // query of column 0
+      const int i0 = (q0 + i) * kQB + kEwCols * wg;  // query of column 0
       // Masks only where some pair of the warp is masked: the causal diagonal
       // (query before key) and queries past N.
-      const bool edge = __any_sync(0xffffffffu, (p.causal && i0 < kk) || i0 + 31 >= p.N);
-      const float4* sts = sm.stats[st] + 32 * wg;
-      uint32_t pa[16], pl[16], pt[16];
+      const bool edge = __any_sync(0xffffffffu, (p.causal && i0 < kk) || i0 + kEwCols - 1 >= p.N);
+      // The statistics of this thread's 16 queries (read by every lane: cached).
+      const float* sts = p.stats + stat_index(bh, p.Npad, (q0 + i) * kQB, 0) + kEwCols * wg;
+      const uint64_t sc2 = f2(scale2, scale2), nisd2 = f2(-isd, -isd);
+      uint32_t pa[kEwCols / 2], pl[kEwCols / 2], pt[kEwCols / 2];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int e = 2 * c;
-        const bool k0 = !edge || ((!p.causal || i0 + e >= kk) && i0 + e < p.N);
-        const bool k1 = !edge || ((!p.causal || i0 + e + 1 >= kk) && i0 + e + 1 < p.N);
-        const Grad3 g0 = grad_elem(__uint_as_float(s[e]), __uint_as_float(t[e]), __uint_as_float(da[e]), sts[e],
-                                   scale2, isd, k0);
-        const Grad3 g1 = grad_elem(__uint_as_float(s[e + 1]), __uint_as_float(t[e + 1]),
-                                   __uint_as_float(da[e + 1]), sts[e + 1], scale2, isd, k1);
-        pa[c] = pack_bf16(g0.a, g1.a);
-        pl[c] = pack_bf16(g0.dl, g1.dl);
-        pt[c] = pack_bf16(g0.dt, g1.dt);
+      for (int c4 = 0; c4 < kEwCols / 4; ++c4) {
+        // Statistics of four consecutive queries (broadcast loads).
+        const float4 L = __ldg(reinterpret_cast<const float4*>(sts + 4 * c4));
+        const float4 C = __ldg(reinterpret_cast<const float4*>(sts + 64 + 4 * c4));
+        const float4 Dv = __ldg(reinterpret_cast<const float4*>(sts + 128 + 4 * c4));
+        const float4 Fd = __ldg(reinterpret_cast<const float4*>(sts + 192 + 4 * c4));
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = 4 * c4 + 2 * h;
+          const bool k0 = !edge || ((!p.causal || i0 + e >= kk) && i0 + e < p.N);
+          const bool k1 = !edge || ((!p.causal || i0 + e + 1 >= kk) && i0 + e + 1 < p.N);
+          const GradPairs g = grad_pairs(
+              s[e], s[e + 1], t[e], t[e + 1], da[e], da[e + 1], h ? f2(L.z, L.w) : f2(L.x, L.y),
+              h ? f2(C.z, C.w) : f2(C.x, C.y), h ? f2(Dv.z, Dv.w) : f2(Dv.x, Dv.y),
+              h ? f2(Fd.z, Fd.w) : f2(Fd.x, Fd.y), sc2, nisd2, k0, k1);
+          pa[2 * c4 + h] = g.a;
+          pl[2 * c4 + h] = g.dl;
+          pt[2 * c4 + h] = g.dt;
+        }
       }
-      // The tiles are free once the gradient MMAs of block i - 1 completed.
-      if (i > 0 && !(ok = warp_wait(&sm.ag_free, (i - 1) & 1, abort, p.status))) break;
-      st_row_chunks(sm.a, row, 4 * wg, pa);
-      st_row_chunks(sm.g[0], row, 4 * wg, pl);
-      st_row_chunks(sm.g[1], row, 4 * wg, pt);
+      // The operands are free once the gradient MMAs of block i - 1 completed.
+      if (i > 0) {
+        if (!(ok = warp_wait(&sm.ag_free, (i - 1) & 1, abort, p.status))) break;
+        tc_fence_after();
+      }
+      st_row_chunks<kEwCols / 8>(sm.a, row, (kEwCols / 8) * wg, pa);
+      tmem_st8(lb + kColG + (kEwCols / 2) * wg, pl);
+      tmem_st8(lb + kColG + 32 + (kEwCols / 2) * wg, pt);
       fence_async_smem();
+      tc_wait_st();
+      tc_fence_before();
       mbar_arrive(&sm.p_full);
     }
     if (ok && warp_wait(&sm.done, 0, abort, p.status)) {
       tc_fence_after();
-      __nv_bfloat16* dst = kk < p.N ? (wg == 0 ? p.g0 : p.g1) + ((long long)bh * p.N + kk) * D : nullptr;
-      tmem_row_to_global<D>(lb + (wg == 0 ? kColDV : kColDK), dst);
+      // Warpgroups 0, 1: the two halves of dV; 2, 3: of dK.
+      const int half = (wg & 1) * (D / 2);
+      __nv_bfloat16* dst = kk < p.N ? (wg < 2 ? p.g0 : p.g1) + ((long long)bh * p.N + kk) * D + half : nullptr;
+      tmem_row_to_global<D / 2>(lb + (wg < 2 ? kColDV : kColDK) + half, dst);
     }
   }
   tc_fence_before();
@@ -430,8 +500,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int BH = p.B * p.H;
   const int nmb = (p.N + kQM - 1) / kQM;
-  // Query blocks with the most keys first.
-  const int m = nmb - 1 - (int)(blockIdx.x / BH), bh = blockIdx.x % BH;
+  // The last query block sees every key (causal): rank r is query block nmb - 1 - r.
+  const BlockOrder bo = block_order(blockIdx.x, BH, nmb, p.chunk_heads);
+  const int m = nmb - 1 - bo.rank, bh = bo.bh;
   const int nk = p.causal ? (min(m * kQM + kQM - 1, p.N - 1) / kKN + 1) : (p.N + kKN - 1) / kKN;
   volatile int* abort = &sm.abort;
 
@@ -442,8 +513,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_empty[s], 1);
     }
     mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.s_free, 8);
-    mbar_init(&sm.p_full, 256);
+    mbar_init(&sm.s_free, 4 * kEwGroups);
+    mbar_init(&sm.p_full, 128 * kEwGroups);
     mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.done, 1);
     mbar_init(&sm.drain, 1);
@@ -542,55 +613,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kFirstEwWarp) {
     // ---------------- elementwise warpgroups ----------------
-    // Thread = one query (TMEM lane) x 32 of the block's 64 keys (wg picks the half).
+    // Thread = one query (TMEM lane) x 16 of the block's 64 keys (wg picks which).
     const int wg = (warp - kFirstEwWarp) >> 2, quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t lb = tmem + ((uint32_t)(32 * quarter) << 16);
     const int i = m * kQM + row;  // query position
-    const float4 sv = p.stats[(size_t)bh * p.Npad + (size_t)i];
     const float isd = rsqrtf((float)D), scale2 = kLog2e * isd;
+    // This query's statistics, as f32x2 pairs for the packed arithmetic.
+    const float* sp = p.stats + stat_index(bh, p.Npad, i, 0);
+    const uint64_t nl2 = f2(sp[0], sp[0]), c02 = f2(sp[64], sp[64]), dd2 = f2(sp[128], sp[128]),
+                   fd2 = f2(sp[192], sp[192]);
+    const uint64_t sc2 = f2(scale2, scale2), nisd2 = f2(-isd, -isd);
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       if (!(ok = warp_wait(&sm.s_full, j & 1, abort, p.status))) break;
       tc_fence_after();
-      uint32_t s[32], t[32], da[32];
-      tmem_ld32(lb + kColS + 32 * wg, s);
-      tmem_ld32(lb + kColT + 32 * wg, t);
-      tmem_ld32(lb + kColDA + 32 * wg, da);
+      uint32_t s[kEwCols], t[kEwCols], da[kEwCols];
+      tmem_ld16(lb + kColS + kEwCols * wg, s);
+      tmem_ld16(lb + kColT + kEwCols * wg, t);
+      tmem_ld16(lb + kColDA + kEwCols * wg, da);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free);
-      const int k0 = j * kKN + 32 * wg;  // key of column 0
-      const bool edge = __any_sync(0xffffffffu, (p.causal && k0 + 31 > i) || k0 + 31 >= p.N);
-      uint32_t pl[16], pt[16];
+      const int k0 = j * kKN + kEwCols * wg;  // key of column 0
+      const bool edge = __any_sync(0xffffffffu, (p.causal && k0 + kEwCols - 1 > i) || k0 + kEwCols - 1 >= p.N);
+      uint32_t pl[kEwCols / 2], pt[kEwCols / 2];
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < kEwCols / 2; ++c) {
         const int e = 2 * c;
         const bool keep0 = !edge || ((!p.causal || k0 + e <= i) && k0 + e < p.N);
         const bool keep1 = !edge || ((!p.causal || k0 + e + 1 <= i) && k0 + e + 1 < p.N);
-        const Grad3 g0 = grad_elem(__uint_as_float(s[e]), __uint_as_float(t[e]), __uint_as_float(da[e]), sv,
-                                   scale2, isd, keep0);
-        const Grad3 g1 = grad_elem(__uint_as_float(s[e + 1]), __uint_as_float(t[e + 1]),
-                                   __uint_as_float(da[e + 1]), sv, scale2, isd, keep1);
-        pl[c] = pack_bf16(g0.dl, g1.dl);
-        pt[c] = pack_bf16(g0.dt, g1.dt);
+        const GradPairs g = grad_pairs(s[e], s[e + 1], t[e], t[e + 1], da[e], da[e + 1], nl2, c02, dd2, fd2, sc2,
+                                       nisd2, keep0, keep1);
+        pl[c] = g.dl;
+        pt[c] = g.dt;
       }
       // The bf16 buffer is free once the gradient MMAs of block j - 1 completed.
       if (j > 0) {
         if (!(ok = warp_wait(&sm.pv_done, (j - 1) & 1, abort, p.status))) break;
         tc_fence_after();
       }
-      tmem_st16(lb + kColP + 16 * wg, pl);
-      tmem_st16(lb + kColP + 32 + 16 * wg, pt);
+      tmem_st8(lb + kColP + (kEwCols / 2) * wg, pl);
+      tmem_st8(lb + kColP + 32 + (kEwCols / 2) * wg, pt);
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&sm.p_full);
     }
     if (ok && warp_wait(&sm.done, 0, abort, p.status)) {
       tc_fence_after();
-      __nv_bfloat16* dst = i < p.N ? (wg == 0 ? p.g0 : p.g1) + ((long long)bh * p.N + i) * D : nullptr;
-      tmem_row_to_global<D>(lb + (wg == 0 ? kColDQ : kColDR), dst);
+      // Warpgroups 0, 1: the two halves of dQ; 2, 3: of dR.
+      const int half = (wg & 1) * (D / 2);
+      __nv_bfloat16* dst = i < p.N ? (wg < 2 ? p.g0 : p.g1) + ((long long)bh * p.N + i) * D + half : nullptr;
+      tmem_row_to_global<D / 2>(lb + (wg < 2 ? kColDQ : kColDR) + half, dst);
     }
   }
   tc_fence_before();
@@ -611,7 +686,7 @@ cudaError_t fail_at(const char* where, cudaError_t e) {
 }
 
 template <int D>
-cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
+cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   const long long rows = (long long)a.B * a.H * a.N;
   if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
   const int BH = a.B * a.H;
@@ -623,7 +698,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
       !make_map(&mR128, a.R, rows, kQM, D) || !make_map(&mO128, a.dO, rows, kQM, D) ||
       !make_map(&mK64, a.K, rows, kKN, D) || !make_map(&mV64, a.V, rows, kKN, D))
     return fail_at("tensor map", cudaErrorInvalidValue);
-  float4* stats = reinterpret_cast<float4*>(a.stats);
+  float* stats = reinterpret_cast<float*>(a.stats);
   const long long srows = (long long)BH * Npad;
   bwd_prep_kernel<<<(unsigned)((srows + 7) / 8), 256, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(a.out), reinterpret_cast<const float*>(a.vbar),
@@ -631,7 +706,10 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail_at("statistics kernel", e);
   const int nblk = (a.N + 127) / 128;  // 128-key blocks = 128-query blocks
-  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
+  // About two waves of blocks per chunk of heads.
+  int ch = (2 * num_sms + nblk - 1) / nblk;
+  ch = ch < 1 ? 1 : (ch > BH ? BH : ch);
+  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
                reinterpret_cast<__nv_bfloat16*>(a.dK), a.status};
   size_t smem = sizeof(KvSmem<D>) + 1024;
   if ((e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
@@ -639,7 +717,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st) {
     return fail_at("dK/dV shared-memory attribute", e);
   bwd_dkv_kernel<D><<<BH * nblk, kThreads, smem, st>>>(mQ64, mR64, mO64, mK128, mV128, pk);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail_at("dK/dV kernel", e);
-  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
+  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
                reinterpret_cast<__nv_bfloat16*>(a.dR), a.status};
   // At least 116 KB so that one CTA (and its 512 TMEM columns) holds an SM.
   smem = sizeof(QSmem<D>) + 1024;
@@ -658,9 +736,9 @@ size_t bwd_padded_rows(int N) { return ((size_t)N + 127) / 128 * 128; }
 
 const char* bwd_last_failure() { return t_bwd_fail; }
 
-cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st) {
-  if (a.d == 128) return launch_bwd_d<128>(a, st);
-  if (a.d == 64) return launch_bwd_d<64>(a, st);
+cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st, int num_sms) {
+  if (a.d == 128) return launch_bwd_d<128>(a, st, num_sms);
+  if (a.d == 64) return launch_bwd_d<64>(a, st, num_sms);
   return cudaErrorInvalidValue;
 }
 
