@@ -78,6 +78,14 @@ def backward_flops(B, H, N, d, causal=True):
     return 16.0 * d * pairs * B * H
 
 
+def backward_bytes(B, H, N, d):
+    """Bytes the backward pass must move once: Q, K, V, R, dO, out (bf16), vbar
+    (fp32), lse and tbar read; dQ, dK, dV, dR written; the statistics
+    workspace (16 B per row) written and read."""
+    rows = B * H * N
+    return rows * d * (6 * 2 + 4 + 4 * 2) + rows * (2 * 4 + 2 * 16)
+
+
 def prefill_bytes(B, H, N, d):
     return 5 * B * H * N * d * 2
 
@@ -318,7 +326,7 @@ def run_gpu(args, rank, world, dist):
                          "unit": "TFLOP/s", "frac": round(p_ach / peaks["bf16_tflops"], 4),
                          "frac_of_sustained": round(p_ach / peaks["bf16_tflops_sustained"], 4),
                          "traffic": (traffic_from_profile("prefill_B8_H16_N4096.json",
-                                                          kernel_hash("prefill_tc.cu", "simt.cu"))
+                                                          kernel_hash("prefill_tc.cu", "sm100.cuh"))
                                      if pB == PREFILL["B"] else None),
                          "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
             "gpu_launches": psteps,
@@ -393,6 +401,10 @@ def run_gpu(args, rank, world, dist):
                 "flops_note": "algorithmic = 8 GEMMs per visible pair; the two kernels issue 11 "
                               "(the scores are recomputed in the dQ/dR kernel)",
                 "gpu_launches_per_step": 3,
+                "traffic_per_step": (traffic_from_profile("backward_B8_H16_N4096.json",
+                                                          kernel_hash("backward_tc.cu", "sm100.cuh"))
+                                     if pB == PREFILL["B"] else None),
+                "algorithmic_bytes_per_step": backward_bytes(pB, pH, pN, pd),
                 "train_forward_ms": round(t_ms, 3),
                 "train_forward_tflops": round(flops / (t_ms * 1e-3) / 1e12, 1),
                 "train_step_ms": round(t_ms + float(np.mean(b_per)), 3),
