@@ -31,6 +31,10 @@ Readings of the pages adopted here (the pages print no layout or mask rule):
 scores are scaled by 1/sqrt(d) and the probe term is not scaled; the causal
 mask lets query i see keys j <= i; a decode query at KV length n sees keys
 0..n-1; Q, K, V, R are [B, H, N, d] and all heads have their own K and V.
+Sliding window (the pages list kernels combining Parallax with sliding-window
+sparsity as future work, rainbus.top "未来方向"; they fix no rule): with a
+window of W keys, query i sees keys max(0, i - W + 1)..i, and a decode query
+at KV length n sees keys max(0, n - W)..n-1.
 """
 from __future__ import annotations
 
@@ -65,35 +69,43 @@ def parallax_row(q: np.ndarray, rho: np.ndarray, K: np.ndarray, V: np.ndarray) -
     return vbar - correction
 
 
-def prefill_ref(Q, K, V, R, causal: bool = True, rows=None) -> np.ndarray:
+def visible_keys(i: int, N: int, causal: bool, window=None):
+    """[lo, hi) of the keys query i sees: j <= i when causal, and j > i - window
+    when a window is given (a window implies the causal mask)."""
+    if window is not None:
+        return max(0, i - int(window) + 1), i + 1
+    return 0, (i + 1 if causal else N)
+
+
+def prefill_ref(Q, K, V, R, causal: bool = True, rows=None, window=None) -> np.ndarray:
     """Oracle for a prefill.
 
     Q, K, V, R: float64 arrays [B, H, N, d].  ``rows`` is None (every output
     row) or an iterable of (b, h, i) triples; the result is then [len(rows), d]
-    in the same order.
+    in the same order.  ``window`` (None or W >= 1) restricts query i to its
+    last W keys (causal).
     """
     B, H, N, d = Q.shape
     if rows is None:
-        out = np.empty((B, H, N, d), dtype=np.float64)
-        for b in range(B):
-            for h in range(H):
-                for i in range(N):
-                    n = i + 1 if causal else N
-                    out[b, h, i] = parallax_row(Q[b, h, i], R[b, h, i], K[b, h, :n], V[b, h, :n])
-        return out
+        rows_iter = [(b, h, i) for b in range(B) for h in range(H) for i in range(N)]
+    else:
+        rows_iter = list(rows)
     res = []
-    for (b, h, i) in rows:
-        n = i + 1 if causal else N
-        res.append(parallax_row(Q[b, h, i], R[b, h, i], K[b, h, :n], V[b, h, :n]))
+    for (b, h, i) in rows_iter:
+        lo, hi = visible_keys(i, N, causal, window)
+        res.append(parallax_row(Q[b, h, i], R[b, h, i], K[b, h, lo:hi], V[b, h, lo:hi]))
+    if rows is None:
+        return np.stack(res).reshape(B, H, N, d)
     return np.stack(res) if res else np.zeros((0, d))
 
 
-def decode_ref(q, r, Kc, Vc, seqlens, units=None) -> np.ndarray:
+def decode_ref(q, r, Kc, Vc, seqlens, units=None, window=None) -> np.ndarray:
     """Oracle for one decode step.
 
     q, r: [B, H, d]; Kc, Vc: [B, H, L, d]; seqlens: [B] ints in 1..L.  The
     query of sequence b sits at position seqlens[b]-1 and sees keys
-    0..seqlens[b]-1.  ``units`` is None (all (b, h)) or a list of (b, h).
+    0..seqlens[b]-1 (with a window W: the last W of them).  ``units`` is None
+    (all (b, h)) or a list of (b, h).
     """
     B, H, d = q.shape
     if units is None:
@@ -104,7 +116,8 @@ def decode_ref(q, r, Kc, Vc, seqlens, units=None) -> np.ndarray:
     res = []
     for (b, h) in units:
         n = int(seqlens[b])
-        res.append(parallax_row(q[b, h], r[b, h], Kc[b, h, :n], Vc[b, h, :n]))
+        lo = 0 if window is None else max(0, n - int(window))
+        res.append(parallax_row(q[b, h], r[b, h], Kc[b, h, lo:n], Vc[b, h, lo:n]))
     out = np.stack(res)
     return out.reshape(B, H, d) if full else out
 
