@@ -9,8 +9,9 @@ than the 126 MB L2, so no flush is needed).  The same run measures the causal
 prefill B=8, H=16, N=4096, d=128 bf16 in TFLOP/s (the metric's second half)
 under "prefill", a layer step (projections, RMSNorm+RoPE, attention) under
 "layer", and the grouped-KV decode B=64, H=32, Hkv=8, L=4096, d=128 in GB/s
-under "decode_gqa", and the training forward plus backward pass of the
-prefill workload under "prefill.backward".  For N > 1 GPUs (launched by torchrun) every rank runs the
+under "decode_gqa", the training forward plus backward pass of the
+prefill workload under "prefill.backward", and sliding windows of 1024 keys on
+the prefill and decode workloads under "window".  For N > 1 GPUs (launched by torchrun) every rank runs the
 same per-GPU workload on its own seeded inputs with no data-path collective
 (weak scaling); time is the max over ranks.
 
@@ -40,6 +41,7 @@ DECODE = dict(B=64, H=16, L=4096, d=128)
 PREFILL = dict(B=8, H=16, N=4096, d=128)
 # The compute-matched variant (head dim halved, twice the heads, same width).
 PREFILL_D64 = dict(B=8, H=32, N=4096, d=64)
+WINDOW = 1024  # sliding-window length of the window lines
 # Grouped KV heads: 32 query heads over 8 KV heads (groups of 4, the grouping of the
 # Llama-3-8B lineage), 1.07 GB of KV.
 DECODE_GQA = dict(B=64, H=32, Hkv=8, L=4096, d=128)
@@ -69,6 +71,10 @@ def decode_bytes(seqlens, H, d):
 def prefill_flops(B, H, N, d, causal=True):
     pairs = N * (N + 1) // 2 if causal else N * N
     return 8.0 * d * pairs * B * H
+
+
+def lib_ws_window(plx, B, H, Hkv, L, d, W):
+    return int(plx.lib.plx_decode_window_workspace_bytes(B, H, Hkv, L, d, W))
 
 
 def backward_flops(B, H, N, d, causal=True):
@@ -413,6 +419,63 @@ def run_gpu(args, rank, world, dist):
             torch.cuda.empty_cache()
 
     # ---- Decode with grouped KV heads (the next row of the scope: one KV stream per group).
+    # ---- Sliding-window variants (a window of 1024 keys on the prefill and decode workloads).
+    win = None
+    if not args.no_window:
+        W = WINDOW
+        wB, wH, wN, wd = args.prefill_batch, PREFILL["H"], PREFILL["N"], PREFILL["d"]
+        wspecs = synth.prefill_specs(wB, wH, wN, wd)
+        wt = {}
+        for name, spec in wspecs.items():
+            wt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(wt[name].data_ptr(), synth.BF16, seed + 8, spec)
+        wout = torch.empty_like(wt["Q"])
+
+        def wpre():
+            plx.prefill_window(wt["Q"], wt["K"], wt["V"], wt["R"], W, out=wout)
+
+        wsteps = max(1, args.steps // 2)
+        w_total, w_per = timed(wpre, wsteps, max(3, args.warmup // 2), stream, dist)
+        pairs = (W * (W + 1) // 2 + (wN - W) * W) * wB * wH
+        wflops = 8.0 * wd * pairs
+        w_ach = wflops / (float(np.mean(w_per)) * 1e-3) / 1e12
+        del wt, wout
+        dB, dH, dL, dd = args.decode_batch, DECODE["H"], DECODE["L"], DECODE["d"]
+        dspecs = synth.decode_specs(dB, dH, dL, dd)
+        dt_ = {}
+        for name, spec in dspecs.items():
+            dt_[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(dt_[name].data_ptr(), synth.BF16, seed + 9, spec)
+        dsl = torch.full((dB,), dL, dtype=torch.int32, device=dev)
+        dout = torch.empty_like(dt_["q"])
+        dws = torch.empty(max(16, lib_ws_window(plx, dB, dH, dH, dL, dd, W)), dtype=torch.uint8, device=dev)
+
+        def wdec():
+            plx.decode_window(dt_["q"], dt_["r"], dt_["K"], dt_["V"], dsl, W, out=dout, workspace=dws)
+
+        d_total, d_per = timed(wdec, args.steps, args.warmup, stream, dist)
+        dbytes = dB * dH * min(W, dL) * dd * 2 * 2 + 3 * dB * dH * dd * 2
+        if plx.get_device_status() != 0:
+            raise RuntimeError("window kernels reported a device error")
+        win = {
+            "window": W,
+            "prefill": {
+                "workload": f"sliding-window prefill W={W} B={wB} H={wH} N={wN} d={wd} bf16",
+                "value": round(sum_over_ranks(wflops * wsteps, dist) / (max_over_ranks(w_total, dist) * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "kernel_tflops": round(w_ach, 1), "frac": round(w_ach / peaks["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": wflops,
+            },
+            "decode": {
+                "workload": f"sliding-window decode W={W} B={dB} H={dH} L={dL} d={dd} bf16 (all lengths {dL})",
+                "value": round(sum_over_ranks(dbytes * args.steps, dist) / (max_over_ranks(d_total, dist) * 1e-3) / 1e9, 1),
+                "unit": "GB/s", "kernel_gbs": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9, 1),
+                "frac": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                "algorithmic_bytes_per_launch": dbytes,
+            },
+        }
+        del dt_, dout, dws
+        torch.cuda.empty_cache()
+
     gqa = None
     if not args.no_gqa:
         gB, gH, gHkv, gL, gd = (DECODE_GQA[k] for k in ("B", "H", "Hkv", "L", "d"))
@@ -505,6 +568,7 @@ def run_gpu(args, rank, world, dist):
     return {
         "value": round(value, 2), "ms_per_step": round(ms_step, 4), "roofline": roofline,
         "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "layer": layer, "decode_gqa": gqa,
+        "window": win,
         "gpu_launches": args.steps,
         "kernel_ms": kernel_ms,
     }
@@ -658,6 +722,7 @@ def main():
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-gqa", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-window", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
@@ -741,7 +806,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": cfg, "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
-            "prefill": res["prefill"], "layer": res["layer"], "decode_gqa": res["decode_gqa"]}
+            "prefill": res["prefill"], "layer": res["layer"], "decode_gqa": res["decode_gqa"],
+            "window": res["window"]}
     print(json.dumps(line))
 
 

@@ -84,6 +84,30 @@ int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, v
                    int B, int H, int N, int d, int causal, int dtype, void* stream);
 
 /*
+ * Sliding-window causal prefill: query i sees keys max(0, i - window + 1)..i
+ * (the pages list kernels combining Parallax with sliding-window sparsity as
+ * future work: rainbus.top "未来方向"; the rule is this build's reading).
+ * Layout, dtypes, head dims and errors as plx_prefill_ex; window >= 1 (a window
+ * of N or more keys is the causal prefill), else PLX_ERR_INVALID_ARG.
+ */
+int plx_prefill_window(const void* Q, const void* K, const void* V, const void* R, void* out,
+                       int B, int H, int N, int d, int window, int dtype, void* stream);
+
+/*
+ * Sliding-window decode step: the query of sequence b sees its last `window`
+ * keys, max(0, seqlens[b] - window)..seqlens[b]-1.  Hkv == H is the decode of
+ * plx_decode_ex (bf16 or fp32); Hkv < H is the grouped-KV decode of
+ * plx_decode_gqa (bf16 only, else PLX_ERR_UNSUPPORTED).  Workspace: at least
+ * plx_decode_window_workspace_bytes(B, H, Hkv, L, d, window) bytes, or NULL;
+ * other arguments and errors as those two calls; window >= 1 (window >= L is
+ * the full decode), else PLX_ERR_INVALID_ARG.
+ */
+int plx_decode_window(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                      const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
+                      int window, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+size_t plx_decode_window_workspace_bytes(int B, int H, int Hkv, int L, int d, int window);
+
+/*
  * Training forward: the causal (or full) bf16 prefill of plx_prefill_ex that
  * also saves what plx_prefill_bwd needs, per query row i of head (b, h):
  *   vbar[b,h,i,:] = sum_j p_ij v_j                 (fp32 [B, H, N, d]),

@@ -234,7 +234,9 @@ __global__ void __launch_bounds__(Cfg<D, G>::kThreads, Cfg<D, G>::kMinCtas)
         const int c = (int)(u / BKV);
         const int bkv = (int)(u - (long long)c * BKV);
         const int n = a.seqlens[bkv / a.Hkv];
-        const int kbeg = c * a.chunk;
+        // Keys lo..n-1 (lo > 0 only with a sliding window), cut into chunks.
+        const int lo = (a.window > 0 && n > a.window) ? n - a.window : 0;
+        const int kbeg = lo + c * a.chunk;
         const int nblk = (n >= 1 && n <= a.L && kbeg < n) ? (min(kbeg + a.chunk, n) - kbeg + kBlk - 1) / kBlk : 0;
         const int row0 = bkv * a.L + kbeg;  // < 2^31 (checked by the launcher)
         bool ok = true;
@@ -295,10 +297,11 @@ __global__ void __launch_bounds__(Cfg<D, G>::kThreads, Cfg<D, G>::kMinCtas)
         }
         continue;
       }
-      const int kbeg = c * a.chunk;
+      const int lo = (a.window > 0 && n > a.window) ? n - a.window : 0;
+      const int kbeg = lo + c * a.chunk;
       if (kbeg >= n) continue;
       const int kend = min(kbeg + a.chunk, n);
-      const int nch = (n + a.chunk - 1) / a.chunk;
+      const int nch = (n - lo + a.chunk - 1) / a.chunk;
       const int nblk = (kend - kbeg + kBlk - 1) / kBlk;
 
       // The group's q and rho rows into the A tile (the previous unit's readers

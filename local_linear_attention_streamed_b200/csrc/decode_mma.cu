@@ -255,9 +255,11 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
       }
       break;
     }
-    const int nch = (n + a.chunk - 1) / a.chunk;
+    // Keys lo..n-1 (lo > 0 only with a sliding window), cut into chunks.
+    const int lo = a.window > 0 ? max(0, n - a.window) : 0;
+    const int nch = (n - lo + a.chunk - 1) / a.chunk;
     if (c >= nch) break;
-    const int kbeg = c * a.chunk;
+    const int kbeg = lo + c * a.chunk;
     const int kend = min(kbeg + a.chunk, n);
 
     // A fragments of [q ; rho]: row g (0 = q, 1 = rho), contraction dims of

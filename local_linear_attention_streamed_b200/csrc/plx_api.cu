@@ -148,8 +148,8 @@ const char* plx_status_string(int code) {
   }
 }
 
-int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
-                   int H, int N, int d, int causal, int dtype, void* stream) {
+static int prefill_impl(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                        int N, int d, int causal, int window, int dtype, void* stream) {
   if (!Q || !K || !V || !R || !out) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
@@ -161,6 +161,7 @@ int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, v
   DeviceCache* dc = nullptr;
   if ((rc = current_device(&dc)) != PLX_OK) return rc;
   PrefillArgs a{Q, K, V, R, out, B, H, N, d, causal ? 1 : 0, dc->status};
+  a.window = window < N ? window : 0;  // a window of N or more keys is the causal prefill
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == PLX_BF16 && prefill_tc_supported(d)) {
@@ -169,6 +170,17 @@ int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, v
     e = launch_prefill_simt(a, dtype == PLX_BF16, st);
   }
   return cuda_rc(e);
+}
+
+int plx_prefill_ex(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
+                   int H, int N, int d, int causal, int dtype, void* stream) {
+  return prefill_impl(Q, K, V, R, out, B, H, N, d, causal, 0, dtype, stream);
+}
+
+int plx_prefill_window(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
+                       int H, int N, int d, int window, int dtype, void* stream) {
+  if (window < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_impl(Q, K, V, R, out, B, H, N, d, 1, window, dtype, stream);
 }
 
 int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
@@ -228,9 +240,9 @@ int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, 
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = grow(&dc->bwd_ws, &dc->bwd_ws_bytes, need, st)) != PLX_OK) return rc;
     a.stats = dc->bwd_ws;
-    return cuda_rc(launch_prefill_bwd(a, st));
+    return cuda_rc(launch_prefill_bwd(a, st, dc->num_sms));
   }
-  return cuda_rc(launch_prefill_bwd(a, st));
+  return cuda_rc(launch_prefill_bwd(a, st, dc->num_sms));
 }
 
 int plx_decode_num_splits(int B, int H, int L, int d) {
@@ -247,9 +259,9 @@ size_t plx_decode_workspace_bytes(int B, int H, int L, int d) {
   return decode_ws_layout(B, H, L, d, num_sms_or_default(), &splits, &chunk);
 }
 
-int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
-                  const int32_t* seqlens, void* out, int B, int H, int L, int d, int dtype,
-                  void* workspace, size_t workspace_bytes, void* stream) {
+static int decode_impl(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                       const int32_t* seqlens, void* out, int B, int H, int L, int d, int window, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !r || !Kcache || !Vcache || !seqlens || !out) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || L < 1 || d < 1) return PLX_ERR_INVALID_ARG;
   if (dtype != PLX_F32 && dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
@@ -274,10 +286,12 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
   a.L = L;
   a.d = d;
   a.status = dc->status;
+  a.window = window < L ? window : 0;
   if (dtype == PLX_F32) {
     return cuda_rc(launch_decode_simt(a, false, st));
   }
-  size_t need = decode_ws_layout(B, H, L, d, dc->num_sms, &a.splits, &a.chunk);
+  // The split plan covers the keys one query can see (the window, when set).
+  size_t need = decode_ws_layout(B, H, a.window > 0 ? a.window : L, d, dc->num_sms, &a.splits, &a.chunk);
   if (need > 0) {
     if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLX_ERR_MISALIGNED;
@@ -297,6 +311,13 @@ int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* 
   return cuda_rc(launch_decode_bf16(a, st, dc->num_sms));
 }
 
+int plx_decode_ex(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                  const int32_t* seqlens, void* out, int B, int H, int L, int d, int dtype,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, 0, dtype, workspace, workspace_bytes,
+                     stream);
+}
+
 size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
   if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return 0;
   if (H == Hkv) return plx_decode_workspace_bytes(B, H, L, d);
@@ -306,17 +327,17 @@ size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
   return sizeof(float) * (size_t)B * H * (size_t)splits * (size_t)(2 * d + 4);
 }
 
-int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void* Vcache,
-                   const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
-                   void* workspace, size_t workspace_bytes, void* stream) {
+static int decode_gqa_impl(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                           const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d, int window,
+                           void* workspace, size_t workspace_bytes, void* stream) {
   if (!q || !r || !Kcache || !Vcache || !seqlens || !out) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return PLX_ERR_INVALID_ARG;
   const int G = H / Hkv;
   if (G != 1 && G != 2 && G != 4 && G != 8) return PLX_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
   if (G == 1)
-    return plx_decode_ex(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, PLX_BF16, workspace,
-                         workspace_bytes, stream);
+    return decode_impl(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, window, PLX_BF16, workspace,
+                       workspace_bytes, stream);
   if (!aligned16(q) || !aligned16(r) || !aligned16(Kcache) || !aligned16(Vcache) ||
       !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_MISALIGNED;
@@ -339,7 +360,9 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
   a.L = L;
   a.d = d;
   a.status = dc->status;
-  decode_split_plan(B, Hkv, L, dc->num_sms, &a.splits, &a.chunk, decode_gqa_ctas_per_sm(G));
+  a.window = window < L ? window : 0;
+  decode_split_plan(B, Hkv, a.window > 0 ? a.window : L, dc->num_sms, &a.splits, &a.chunk,
+                    decode_gqa_ctas_per_sm(G));
   if (a.splits > 1) {
     const size_t need = sizeof(float) * (size_t)B * H * (size_t)a.splits * (size_t)(2 * d + 4);
     if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
@@ -358,6 +381,31 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
     }
   }
   return cuda_rc(launch_decode_gqa(a, st, dc->num_sms));
+}
+
+int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                   const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_gqa_impl(q, r, Kcache, Vcache, seqlens, out, B, H, Hkv, L, d, 0, workspace, workspace_bytes,
+                         stream);
+}
+
+size_t plx_decode_window_workspace_bytes(int B, int H, int Hkv, int L, int d, int window) {
+  if (window < 1) return 0;
+  const int Leff = window < L ? window : L;
+  return Hkv == H ? plx_decode_workspace_bytes(B, H, Leff, d) : plx_decode_gqa_workspace_bytes(B, H, Hkv, Leff, d);
+}
+
+int plx_decode_window(const void* q, const void* r, const void* Kcache, const void* Vcache,
+                      const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d, int window,
+                      int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (window < 1 || Hkv < 1) return PLX_ERR_INVALID_ARG;
+  if (Hkv == H)
+    return decode_impl(q, r, Kcache, Vcache, seqlens, out, B, H, L, d, window, dtype, workspace, workspace_bytes,
+                       stream);
+  if (dtype != PLX_BF16) return PLX_ERR_UNSUPPORTED;
+  return decode_gqa_impl(q, r, Kcache, Vcache, seqlens, out, B, H, Hkv, L, d, window, workspace, workspace_bytes,
+                         stream);
 }
 
 int plx_decode(const void* q, const void* r, const void* Kcache, const void* Vcache,

@@ -33,6 +33,7 @@ struct PrefillArgs {
   void* vbar = nullptr;
   float* lse = nullptr;
   float* tbar = nullptr;
+  int window = 0;  // sliding window: query i sees keys i - window + 1 .. i (0: none; implies causal)
 };
 
 struct DecodeArgs {
@@ -49,6 +50,7 @@ struct DecodeArgs {
   int* counters;    // [B*H] arrival counters, zero between calls ([B*Hkv] for grouped KV)
   int* status;
   int Hkv;          // KV heads (grouped-KV decode only; H is a multiple of it)
+  int window;       // sliding window: the last `window` keys of each sequence (0: all)
 };
 
 // SIMT kernels: any d that is a multiple of 32 up to 128, f32 or bf16 storage.
@@ -95,7 +97,7 @@ struct BwdArgs {
 size_t bwd_padded_rows(int N);
 // The step of this thread's last failed backward launch ("" if none).
 const char* bwd_last_failure();
-cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st);
+cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st, int num_sms);
 
 // Per-head RMSNorm + RoPE with the head split folded in.
 cudaError_t launch_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,

@@ -127,14 +127,14 @@ struct Smem {
 using namespace sm100;
 
 struct TileInfo {
-  int bh, m, nblk;
+  int bh, m, j0, nblk;  // key blocks j0 .. j0 + nblk - 1
 };
 
 // Tile t of the schedule: heads are taken in chunks of `ch`; within a chunk
 // the tiles go longest causal rows first across the chunk's heads.  CTAs take
 // tiles in this order from a global counter, so the K/V of a few heads stay in
 // L2 while every tile that reads them runs, and the causal work balances.
-__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, int ch) {
+__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, int ch, int window) {
   const int ntile = (N + kBM - 1) / kBM;
   const int per_chunk = ch * ntile;
   const int chunk = t / per_chunk;
@@ -144,7 +144,9 @@ __device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, 
   ti.m = ntile - 1 - pos / nh;
   ti.bh = chunk * ch + pos % nh;
   const int kmax = causal ? min(N, (ti.m + 1) * kBM) : N;
-  ti.nblk = (kmax + kBN - 1) / kBN;
+  // A sliding window of W keys: the tile's first query sees keys from m kBM - W + 1.
+  ti.j0 = window > 0 ? max(0, ti.m * kBM - window + 1) / kBN : 0;
+  ti.nblk = (kmax + kBN - 1) / kBN - ti.j0;
   return ti;
 }
 
@@ -155,6 +157,7 @@ __device__ unsigned int g_cta_done;
 
 struct Params {
   int B, H, N, causal;
+  int window;  // sliding window of keys per query (0: none)
   int chunk_heads;
   int inject_stall;  // failure-detection test: withhold the first Q/R tile
   __nv_bfloat16* out;
@@ -167,12 +170,15 @@ struct Params {
   float* tbar;
 };
 
-template <int D>
+// kWin: the sliding-window variant (the causal and full prefills compile
+// without any of its per-row logic).
+template <int D, bool kWin>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int window = kWin ? p.window : 0;
   constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
   constexpr uint32_t kColO2 = Dims<D>::kColO2, kIdescPV = Dims<D>::kIdescPV;
   constexpr int kHalves = Dims<D>::kHalves;
@@ -237,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.tile_ring[slot] = t;
         mbar_arrive(&sm.tile_full[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
         const int row0 = ti.bh * p.N;
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
@@ -258,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
           kv_issued[st] = kv / kStages;
           for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + j * kBN);
-            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + j * kBN);
+            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + (ti.j0 + j) * kBN);
+            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + (ti.j0 + j) * kBN);
           }
         }
       }
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
         mbar_arrive(&sm.tile_empty[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
           // K of this block (long resident: checked first), then the S stage,
@@ -338,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
         mbar_arrive(&sm.tile_empty[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
         // The epilogue of the previous tile must have read O before it is overwritten.
         if (tc > 0 && !(ok = mbar_wait(&sm.o_empty, (tc - 1) & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
@@ -456,9 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (epi_pending) ok = epilogue(epi_tc, epi_row, epi_vrow, epi_inv, epi_c1);
         break;
       }
-      const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads);
+      const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
       const int i = ti.m * kBM + row;                      // query position
       const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
+      const int kbeg = i - window + 1;                    // and, with a window, keys >= kbeg
       // Row state: running max (log2 units) and centre c (shared), this
       // warpgroup's omega = sum w and T = sum w (t - c), and the other
       // warpgroup's sums as last posted (brought to the current state).
@@ -479,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t g = gb + j;
         if (!(ok = mbar_wait(&sm.s_full[wg], (g >> 1) & 1, abort, p.status))) break;
         tc_fence_after();
-        const int kb = j * kBN;
+        const int kb = (ti.j0 + j) * kBN;
         uint32_t x[64], y[64];
         tmem_ld32(sb + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(sb + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
@@ -489,11 +496,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free);  // the S stage goes back to the MMA
-        if ((p.causal && kb + kBN - 1 > ti.m * kBM) || kb + kBN > p.N) {
-          // Block-uniform: only blocks that cross the diagonal or the end.
+        if ((p.causal && kb + kBN - 1 > ti.m * kBM) || kb + kBN > p.N ||
+            (kWin && kb < ti.m * kBM + kBM - window)) {
+          // Block-uniform: only blocks that cross the diagonal, the end or the
+          // window's start.
+          if constexpr (kWin) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (kb + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+            for (int c = 0; c < 64; ++c)
+              if (kb + c >= kend || kb + c < kbeg) x[c] = __float_as_uint(-CUDART_INF_F);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+              if (kb + c >= kend) x[c] = __float_as_uint(-CUDART_INF_F);
+          }
         }
         float rmax;
         {
@@ -529,7 +544,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // w = 2^(s*scale - m_run), a = w (t - c).  x <- w, y <- a.
         float wb, tb;
         {
-          const uint64_t sc2 = f2(scale, scale), nm2 = f2(-m_run, -m_run), nc2 = f2(-cen, -cen);
+          // A row that has seen no key yet (only with a window) keeps m_run =
+          // -inf and gets w = 2^(-inf) = 0 from the reference 0.
+          const float mref = (kWin && m_run == -CUDART_INF_F) ? 0.f : m_run;
+          const uint64_t sc2 = f2(scale, scale), nm2 = f2(-mref, -mref), nc2 = f2(-cen, -cen);
           uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -563,8 +581,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // sums through this block) has drifted by more than kTheta.
         float delta = 0.f;
         {
-          const float Tn = (T + T_o) + tb, Wn = (omega + om_o) + wb;  // Wn > 0: key 0 is visible
-          if (j == 0 || fabsf(Tn) > Dims<D>::kTheta * Wn) {
+          // The centre is set by the row's first block with weight (the tile's
+          // first block unless a window hides it) and moved on drift.  A window
+          // that starts inside the previous block left that first estimate
+          // from a few keys: the row's second block re-centres unconditionally.
+          // Rows of short windows see few keys, so they track the mean more
+          // closely (drift 0.5 below 256 keys: 1.6 % on a 37-key window where
+          // the causal kernel's threshold gives 3.7 %); from 256 keys on the
+          // causal threshold holds (1.5-1.9 % at 256..1024) and moves O less.
+          const float Wp = omega + om_o;
+          const float Tn = (T + T_o) + tb, Wn = Wp + wb;
+          bool recentre;
+          if constexpr (kWin) {
+            const bool second = kbeg > kb - kBN && kbeg < kb;
+            const float theta = window >= 256 ? Dims<D>::kTheta : 0.5f;
+            recentre = Wn > 0.f && (Wp == 0.f || second || fabsf(Tn) > theta * Wn);
+          } else {
+            recentre = j == 0 || fabsf(Tn) > Dims<D>::kTheta * Wn;  // key 0 is visible: Wn > 0
+          }
+          if (recentre) {
             const float cn = cen + Tn / Wn;
             delta = cn - cen;  // the shift as represented
             cen = cn;
@@ -719,15 +754,15 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   // (tests of the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
-  Params p{a.B,      a.H,    a.N, a.causal, ch, inject, reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
+  Params p{a.B,      a.H,    a.N, a.causal, a.window, ch, inject, reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
            reinterpret_cast<float*>(a.vbar), a.lse, a.tbar};
   const size_t smem = sizeof(Smem<D>) + 1024;
-  cudaError_t e =
-      cudaFuncSetAttribute(prefill_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = a.window > 0 ? prefill_tc_kernel<D, true> : prefill_tc_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)((a.N + kBM - 1) / kBM) * a.B * a.H;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  prefill_tc_kernel<D><<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
+  kernel<<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
   return cudaGetLastError();
 }
 

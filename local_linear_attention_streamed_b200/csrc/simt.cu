@@ -173,7 +173,9 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_simt_kernel(PrefillArgs a
 
   int last_row = min(row0 + kRowsPerCta, a.N) - 1;
   int kend = a.causal ? last_row + 1 : a.N;
-  for (int k0 = 0; k0 < kend; k0 += kChunk) {
+  // With a sliding window the tile's first row sees keys from row0 - window + 1.
+  const int kfirst = a.window > 0 ? max(0, row0 - a.window + 1) / kChunk * kChunk : 0;
+  for (int k0 = kfirst; k0 < kend; k0 += kChunk) {
     __syncthreads();
     stage_kv<BF16>(Ks, Vs, a.K, a.V, base, k0, a.N, d);
     __syncthreads();
@@ -183,8 +185,9 @@ __global__ void __launch_bounds__(kWarps * 32) prefill_simt_kernel(PrefillArgs a
       int i = row0 + lr;
       if (i >= a.N) continue;
       if (a.causal && k0 > i) continue;
+      if (a.window > 0 && k0 + kChunk <= i - a.window + 1) continue;
       int key = k0 + lane;
-      bool valid = key < a.N && (!a.causal || key <= i);
+      bool valid = key < a.N && (!a.causal || key <= i) && (a.window <= 0 || key > i - a.window);
       row_update(s[r], Qs + lr * d, Rs + lr * d, Ks, Vs, d, valid, inv_sqrt_d, lane);
     }
   }
@@ -222,11 +225,12 @@ __global__ void __launch_bounds__(32) decode_simt_kernel(DecodeArgs a) {
   const float inv_sqrt_d = 1.f / sqrtf((float)d);
   RowState s;
   s.init();
-  for (int k0 = 0; k0 < n; k0 += kChunk) {
+  const int lo = (a.window > 0 && n > a.window) ? n - a.window : 0;  // sliding window
+  for (int k0 = lo / kChunk * kChunk; k0 < n; k0 += kChunk) {
     __syncwarp();
     stage_kv<BF16>(Ks, Vs, a.K, a.V, base, k0, n, d);
     __syncwarp();
-    row_update(s, Qs, Rs, Ks, Vs, d, k0 + lane < n, inv_sqrt_d, lane);
+    row_update(s, Qs, Rs, Ks, Vs, d, k0 + lane < n && k0 + lane >= lo, inv_sqrt_d, lane);
   }
   row_finish<BF16>(s, a.out, qoff, d, lane);
 }

@@ -34,6 +34,9 @@ SIGNATURES = {
     "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
     "plx_layer_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
+    "plx_prefill_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
+    "plx_decode_window": (_i, [_vp] * 6 + [_i] * 7 + [_vp, _sz, _vp]),
+    "plx_decode_window_workspace_bytes": (_sz, [_i] * 6),
     "plx_prefill_train": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
     "plx_prefill_bwd_workspace_bytes": (_sz, [_i] * 4),
     "plx_prefill_bwd": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
@@ -110,6 +113,38 @@ def prefill(Q, K, V, R, causal: bool = True, out=None, stream=None):
     rc = lib.plx_prefill_ex(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
                             B, H, N, d, int(bool(causal)), _dtype_code(Q), _stream_ptr(stream))
     _check(rc, "plx_prefill_ex")
+    return out
+
+
+def prefill_window(Q, K, V, R, window: int, out=None, stream=None):
+    """Sliding-window causal prefill (query i sees its last `window` keys); returns out."""
+    B, H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("R", R)):
+        if t.shape != Q.shape or t.dtype != Q.dtype:
+            raise ValueError(f"{n} must match Q in shape and dtype")
+    if out is None:
+        out = torch.empty_like(Q)
+    rc = lib.plx_prefill_window(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                B, H, N, d, int(window), _dtype_code(Q), _stream_ptr(stream))
+    _check(rc, "plx_prefill_window")
+    return out
+
+
+def decode_window(q, r, Kcache, Vcache, seqlens, window: int, out=None, workspace=None, stream=None):
+    """Sliding-window decode step: each query sees the last `window` keys of its sequence.
+
+    Kcache/Vcache are [B, Hkv, L, d] with H a multiple of Hkv (Hkv == H: one KV head per head).
+    """
+    B, H, d = q.shape
+    Hkv, L = Kcache.shape[1], Kcache.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws, wsb = (0, 0) if workspace is None else (_dev(workspace, "workspace"),
+                                                workspace.numel() * workspace.element_size())
+    rc = lib.plx_decode_window(_dev(q, "q"), _dev(r, "r"), _dev(Kcache, "Kcache"), _dev(Vcache, "Vcache"),
+                               _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, Hkv, L, d, int(window),
+                               _dtype_code(q), ws, wsb, _stream_ptr(stream))
+    _check(rc, "plx_decode_window")
     return out
 
 
