@@ -464,6 +464,9 @@ def run_gpu(args, rank, world, dist):
                 "value": round(sum_over_ranks(wflops * wsteps, dist) / (max_over_ranks(w_total, dist) * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "kernel_tflops": round(w_ach, 1), "frac": round(w_ach / peaks["bf16_tflops"], 4),
                 "algorithmic_flops_per_launch": wflops,
+                "traffic": (traffic_from_profile("prefill_window_B8_H16_N4096_W1024.json",
+                                                 kernel_hash("prefill_tc.cu", "sm100.cuh"))
+                            if wB == PREFILL["B"] else None),
             },
             "decode": {
                 "workload": f"sliding-window decode W={W} B={dB} H={dH} L={dL} d={dd} bf16 (all lengths {dL})",
@@ -471,6 +474,8 @@ def run_gpu(args, rank, world, dist):
                 "unit": "GB/s", "kernel_gbs": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9, 1),
                 "frac": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                 "algorithmic_bytes_per_launch": dbytes,
+                "traffic": (traffic_from_profile("decode_window_B64_H16_L4096_W1024.json", kernel_hash("decode_mma.cu"))
+                            if dB == DECODE["B"] else None),
             },
         }
         del dt_, dout, dws
