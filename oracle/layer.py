@@ -90,3 +90,66 @@ def qkr_norm_rope_ref(x, W, H: int) -> np.ndarray:
     d = D // H
     y = (x @ W).reshape(B, N, H, d).transpose(0, 2, 1, 3)
     return rope(rmsnorm(y), np.arange(N)[None, None, :])
+
+
+# ---------------------------------------------------------------------------
+# fp8 linear layers.  The pages' pretraining runs the linear layers in dynamic
+# fp8 (rainbus.top, 复现评估: dynamic fp8 for the linear layers, bf16 for the
+# LM head).  Reading: "dynamic" = one scale per tensor per call, s = max|a| /
+# 448 (the largest e4m3 value), every operand of a linear (the activation and
+# the weight) rounded to e4m3 (round to nearest, ties to even) after division
+# by its scale, products accumulated exactly, the sum scaled back by s_a s_w.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3(a: np.ndarray) -> np.ndarray:
+    """Round to the nearest float8 e4m3 value (ties to even); |a| <= 448 expected."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float64))
+    return t.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def fp8_per_tensor(a: np.ndarray):
+    """Dynamic per-tensor e4m3 quantisation: returns (e4m3 codes as float64, scale)."""
+    a = np.asarray(a, dtype=np.float64)
+    amax = float(np.max(np.abs(a)))
+    s = amax / E4M3_MAX if amax > 0 else 1.0
+    return e4m3(a / s), s
+
+
+def fp8_linear(a: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """a @ W with both operands quantised per tensor to e4m3 (exact accumulation)."""
+    qa, sa = fp8_per_tensor(a)
+    qw, sw = fp8_per_tensor(W)
+    return (qa @ qw) * (sa * sw)
+
+
+def layer_fp8_ref(x, WQ, WK, WV, WR, WO, H: int, linear=fp8_linear) -> np.ndarray:
+    """The whole layer output [B, N, D] with fp8 linears (float64 elsewhere).
+
+    The scale of the attention output (the input of W_O) depends on every
+    token of the batch, so this oracle computes all rows.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    B, N, D = x.shape
+    d = D // H
+    x2 = x.reshape(B * N, D)
+    pos = np.arange(N)[None, None, :]
+
+    def heads(y):
+        return y.reshape(B, N, H, d).transpose(0, 2, 1, 3)
+
+    q = rope(rmsnorm(heads(linear(x2, WQ))), pos)
+    k = rope(rmsnorm(heads(linear(x2, WK))), pos)
+    v = heads(linear(x2, WV))
+    r = rope(rmsnorm(heads(linear(x2, WR))), pos)
+    o = np.empty((B, H, N, d))
+    for b in range(B):
+        for h in range(H):
+            for t in range(N):
+                o[b, h, t] = parallax_row(q[b, h, t], r[b, h, t], k[b, h, :t + 1], v[b, h, :t + 1])
+    merged = o.transpose(0, 2, 1, 3).reshape(B * N, D)
+    return linear(merged, WO).reshape(B, N, D)
