@@ -566,6 +566,22 @@ def run_gpu(args, rank, world, dist):
             "layer_tflops_all": round((aflops + pflops) / (l_ms * 1e-3) / 1e12, 1),
             "gpu_launches_per_step": {"own_kernels": 6, "cublas_gemms": 5},
         }
+
+        # The same layer with its five linears in dynamic fp8 (per-tensor e4m3).
+        def lay8():
+            plx.layer_forward_fp8(lt["x"], lt["WQ"], lt["WK"], lt["WV"], lt["WR"], lt["WO"], LH, out=y)
+
+        f_total, f_per = timed(lay8, lsteps, 3, stream, dist)
+        if plx.get_device_status() != 0:
+            raise RuntimeError("fp8 layer reported a device error")
+        f_ms = float(np.mean(f_per))
+        layer["fp8_linears"] = {
+            "layer_ms": round(f_ms, 3),
+            "rest_ms": round(f_ms - a_ms, 3),
+            "note": "x, the weights and the attention output quantised per tensor to e4m3 every call "
+                    "(|max| reductions and quantisers: own kernels), e4m3 GEMMs through cuBLASLt",
+            "gpu_launches_per_step": {"own_kernels": 6 + 14, "cublaslt_gemms": 5},
+        }
         del lt, at
         torch.cuda.empty_cache()
 

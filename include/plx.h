@@ -262,6 +262,24 @@ int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void*
                       const void* WR, const void* WO, void* y, int B, int N, int H, int d,
                       void* workspace, size_t workspace_bytes, void* stream);
 
+/* The scratch plx_layer_forward_fp8 needs, in bytes (includes a 32 MB GEMM workspace). */
+size_t plx_layer_fp8_workspace_bytes(int B, int N, int H, int d);
+
+/*
+ * The layer of plx_layer_forward with its five linears in dynamic fp8, as the
+ * pages pretrain it (rainbus.top reproduction notes: dynamic fp8 for the
+ * linear layers): per call and per tensor, s = max|a| / 448 for the input x,
+ * each weight and the merged attention output; each operand rounded to e4m3
+ * (nearest, ties to even) after division by its scale; e4m3 GEMMs with fp32
+ * accumulation, scaled by s_a s_w, written as bf16.  Norms, RoPE and attention
+ * as plx_layer_forward (bf16 tensor-core prefill, so d in {64, 128}).
+ * B*N must be a multiple of 16 and H*d of 32, else PLX_ERR_UNSUPPORTED.
+ * workspace: plx_layer_fp8_workspace_bytes() bytes, 256-byte aligned, or NULL.
+ */
+int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const void* WV,
+                          const void* WR, const void* WO, void* y, int B, int N, int H, int d,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
 /*
  * Waits for `stream`, then reads and clears this device's kernel status word.
  * Returns PLX_OK, or the first device-reported error since the last read

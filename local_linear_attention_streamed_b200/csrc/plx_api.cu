@@ -2,6 +2,7 @@
 // kernel selection, library-owned workspaces and the per-device status word.
 #include "plx_internal.cuh"
 
+#include <cublasLt.h>
 #include <cublas_v2.h>
 
 #include <cstdio>
@@ -30,6 +31,7 @@ struct DeviceCache {
   void* bwd_ws = nullptr;  // per-row statistics of the prefill backward pass
   size_t bwd_ws_bytes = 0;
   cublasHandle_t cublas = nullptr;
+  cublasLtHandle_t cublas_lt = nullptr;  // fp8 GEMMs of the fp8 layer
 };
 
 std::mutex g_mu;
@@ -98,6 +100,8 @@ int grow(void** ptr, size_t* bytes, size_t need, cudaStream_t st) {
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+constexpr size_t kLtWorkspace = 32u << 20;  // cuBLASLt workspace of the fp8 GEMMs
 
 // Bytes of partial records a split decode needs (0 when keys are not split).
 size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk) {
@@ -493,6 +497,90 @@ int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void*
   if (cublasGemmEx(dc->cublas, CUBLAS_OP_N, CUBLAS_OP_N, D, (int)M, D, &one, WO, CUDA_R_16BF, D,
                    proj[0], CUDA_R_16BF, D, &zero, y, CUDA_R_16BF, D, CUBLAS_COMPUTE_32F,
                    CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS)
+    return PLX_ERR_CUDA;
+  return PLX_OK;
+}
+
+size_t plx_layer_fp8_workspace_bytes(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return 0;
+  const size_t M = (size_t)B * N, D = (size_t)H * d;
+  // bf16 buffers of the bf16 layer, two e4m3 activations, five e4m3 weights,
+  // the scales, and the GEMM's workspace.
+  return plx_layer_workspace_bytes(B, N, H, d) + 2 * round_up(M * D, 256) + 5 * round_up(D * D, 256) + 256 +
+         kLtWorkspace;
+}
+
+int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const void* WV, const void* WR,
+                          const void* WO, void* y, int B, int N, int H, int d, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  if (!x || !WQ || !WK || !WV || !WR || !WO || !y) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1) return PLX_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if ((long long)B * N * H * d >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
+  if (((long long)B * N) % 16 != 0) return PLX_ERR_UNSUPPORTED;  // fp8 GEMM operand alignment
+  if (!aligned16(x) || !aligned16(WQ) || !aligned16(WK) || !aligned16(WV) || !aligned16(WR) ||
+      !aligned16(WO) || !aligned16(y))
+    return PLX_ERR_MISALIGNED;
+  DeviceCache* dc = nullptr;
+  int rc = current_device(&dc);
+  if (rc != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t need = plx_layer_fp8_workspace_bytes(B, N, H, d);
+  char* ws = nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (workspace) {
+    if (workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return PLX_ERR_MISALIGNED;
+    ws = static_cast<char*>(workspace);
+  } else {
+    if ((rc = grow(&dc->layer_ws, &dc->layer_ws_bytes, need, st)) != PLX_OK) return rc;
+    ws = static_cast<char*>(dc->layer_ws);
+  }
+  if (!dc->cublas_lt) {
+    if (cublasLtCreate(&dc->cublas_lt) != CUBLAS_STATUS_SUCCESS) {
+      dc->cublas_lt = nullptr;
+      return PLX_ERR_CUDA;
+    }
+  }
+  const int D = H * d;
+  const long long M = (long long)B * N;
+  const size_t t = round_up((size_t)M * D * 2, 256);
+  void* proj[4] = {ws, ws + t, ws + 2 * t, ws + 3 * t};
+  void* head[4] = {ws + 4 * t, ws + 5 * t, ws + 6 * t, ws + 7 * t};
+  void* attn = ws + 8 * t;
+  char* p8 = ws + 9 * t;
+  void* x8 = p8;
+  void* a8 = p8 + round_up((size_t)M * D, 256);
+  char* w8 = p8 + 2 * round_up((size_t)M * D, 256);
+  const size_t wsz = round_up((size_t)D * D, 256);
+  unsigned* amax = reinterpret_cast<unsigned*>(w8 + 5 * wsz);  // 7 words: x, W_Q..W_R, W_O, attention
+  float* scale = reinterpret_cast<float*>(amax + 8);           // 7 scales
+  void* lt_ws = w8 + 5 * wsz + 256;
+  const void* W[5] = {WQ, WK, WV, WR, WO};
+  if (cudaMemsetAsync(amax, 0, 8 * sizeof(unsigned), st) != cudaSuccess) return PLX_ERR_CUDA;
+  cudaError_t e = launch_amax(x, (size_t)M * D, amax, st);
+  for (int i = 0; i < 5 && e == cudaSuccess; ++i) e = launch_amax(W[i], (size_t)D * D, amax + 1 + i, st);
+  if (e == cudaSuccess) e = launch_quant(x, (size_t)M * D, amax, x8, scale, st);
+  for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+    e = launch_quant_t(W[i], D, D, amax + 1 + i, w8 + i * wsz, scale + 1 + i, st);
+  if (e != cudaSuccess) return cuda_rc(e);
+  for (int i = 0; i < 4; ++i)
+    if (fp8_gemm(dc->cublas_lt, w8 + i * wsz, x8, proj[i], D, D, M, scale + 1 + i, scale, lt_ws, kLtWorkspace,
+                 st) != 0)
+      return PLX_ERR_CUDA;
+  const float eps = 1e-6f, base = 10000.f;
+  if (launch_qkr_norm_rope(proj[0], head[0], B, N, H, d, eps, base, st) != cudaSuccess ||
+      launch_qkr_norm_rope(proj[1], head[1], B, N, H, d, eps, base, st) != cudaSuccess ||
+      launch_swap_axes(proj[2], head[2], B, N, H, d, st) != cudaSuccess ||
+      launch_qkr_norm_rope(proj[3], head[3], B, N, H, d, eps, base, st) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  PrefillArgs a{head[0], head[1], head[2], head[3], attn, B, H, N, d, 1, dc->status};
+  if ((e = launch_prefill_tc(a, st, dc->num_sms)) != cudaSuccess) return cuda_rc(e);
+  if (launch_swap_axes(attn, proj[0], B, H, N, d, st) != cudaSuccess) return PLX_ERR_CUDA;
+  if ((e = launch_amax(proj[0], (size_t)M * D, amax + 6, st)) != cudaSuccess ||
+      (e = launch_quant(proj[0], (size_t)M * D, amax + 6, a8, scale + 6, st)) != cudaSuccess)
+    return cuda_rc(e);
+  if (fp8_gemm(dc->cublas_lt, w8 + 4 * wsz, a8, y, D, D, M, scale + 5, scale + 6, lt_ws, kLtWorkspace, st) != 0)
     return PLX_ERR_CUDA;
   return PLX_OK;
 }

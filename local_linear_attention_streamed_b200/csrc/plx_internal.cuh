@@ -99,6 +99,19 @@ size_t bwd_padded_rows(int N);
 const char* bwd_last_failure();
 cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st, int num_sms);
 
+// Dynamic per-tensor fp8 (e4m3) linears: |max| reduction into float bits
+// (*amax_bits zeroed first), quantisation (s = max/448, written to *scale),
+// quantisation with a transpose of a [rows, cols] weight, and the e4m3 GEMM
+// Y[M, Dout] = X8[M, Din] Wt8[Dout, Din]^T sX sW in bf16 through cuBLASLt
+// (returns 0 on success).  Sizes are multiples of 32; pointers 16-byte aligned.
+cudaError_t launch_amax(const void* x, size_t n, unsigned* amax_bits, cudaStream_t st);
+cudaError_t launch_quant(const void* x, size_t n, const unsigned* amax_bits, void* out, float* scale,
+                         cudaStream_t st);
+cudaError_t launch_quant_t(const void* W, int rows, int cols, const unsigned* amax_bits, void* Wt, float* scale,
+                           cudaStream_t st);
+int fp8_gemm(void* lt_handle, const void* Wt8, const void* X8, void* Y, int Dout, int Din, long long M,
+             const float* sW, const float* sX, void* ws, size_t ws_bytes, cudaStream_t st);
+
 // Per-head RMSNorm + RoPE with the head split folded in.
 cudaError_t launch_qkr_norm_rope(const void* x, void* y, int B, int N, int H, int d, float eps,
                                  float base, cudaStream_t st);

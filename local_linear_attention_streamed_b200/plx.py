@@ -34,6 +34,8 @@ SIGNATURES = {
     "plx_qkr_norm_rope": (_i, [_vp, _vp] + [_i] * 4 + [_f, _f, _vp]),
     "plx_layer_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
+    "plx_layer_fp8_workspace_bytes": (_sz, [_i] * 4),
+    "plx_layer_forward_fp8": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
     "plx_prefill_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_decode_window": (_i, [_vp] * 6 + [_i] * 7 + [_vp, _sz, _vp]),
     "plx_decode_window_workspace_bytes": (_sz, [_i] * 6),
@@ -315,6 +317,22 @@ def layer_forward(x, WQ, WK, WV, WR, WO, H: int, out=None, workspace=None, strea
                                _dev(WR, "WR"), _dev(WO, "WO"), _dev(out, "out"), B, N, H, d,
                                ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(rc, "plx_layer_forward")
+    return out
+
+
+def layer_forward_fp8(x, WQ, WK, WV, WR, WO, H: int, out=None, workspace=None, stream=None):
+    """The layer of layer_forward with its five linears in dynamic per-tensor fp8 (e4m3)."""
+    B, N, D = x.shape
+    d = D // H
+    if out is None:
+        out = torch.empty_like(x)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.plx_layer_forward_fp8(_dev(x, "x"), _dev(WQ, "WQ"), _dev(WK, "WK"), _dev(WV, "WV"),
+                                   _dev(WR, "WR"), _dev(WO, "WO"), _dev(out, "out"), B, N, H, d,
+                                   ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(rc, "plx_layer_forward_fp8")
     return out
 
 

@@ -101,3 +101,12 @@ def rel_err_fro(got: np.ndarray, ref: np.ndarray) -> float:
 # 3e-2 at N = 384 to 6.6e-2 for a whole N = 4096 head: GRAD_MAX_TOL bounds it.
 GRAD_TOL = 1e-2
 GRAD_MAX_TOL = 1e-1
+
+# Layer with fp8 linears, against the float64 layer with the same per-tensor
+# e4m3 quantisation: relative Frobenius error over the whole output.  The GPU
+# also stores its intermediates in bf16 (projections, normalised heads, the
+# attention output), and a bf16 rounding upstream flips e4m3 rounding decisions
+# downstream: the float64 layer rounded to bf16 at exactly those points is
+# 2.0-2.1e-2 away from the oracle (tests/test_fp8_layer_bound.py), while
+# leaving the linears unquantised is 8.4-8.8e-2 away.
+FP8_LAYER_TOL = 5e-2
