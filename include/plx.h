@@ -273,7 +273,7 @@ size_t plx_layer_fp8_workspace_bytes(int B, int N, int H, int d);
  * (nearest, ties to even) after division by its scale; e4m3 GEMMs with fp32
  * accumulation, scaled by s_a s_w, written as bf16.  Norms, RoPE and attention
  * as plx_layer_forward (bf16 tensor-core prefill, so d in {64, 128}).
- * B*N must be a multiple of 16 and H*d of 32, else PLX_ERR_UNSUPPORTED.
+ * B*N must be a multiple of 16 and H*d of 64, else PLX_ERR_UNSUPPORTED.
  * workspace: plx_layer_fp8_workspace_bytes() bytes, 256-byte aligned, or NULL.
  */
 int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const void* WV,

@@ -27,11 +27,21 @@ __device__ __forceinline__ float scale_of(const unsigned* amax_bits) {
   return amax > 0.f ? amax / kE4m3Max : 1.f;
 }
 
+// Up to five tensors of one launch (blockIdx.y picks one).
+struct Tensors5 {
+  const __nv_bfloat16* x[5];
+  unsigned* amax_bits[5];
+  __nv_fp8_e4m3* out[5];
+  float* scale[5];
+};
+
 // max |x| over n bf16 values (n a multiple of 8, x 16-byte aligned) into
 // *amax_bits, as float bits: non-negative floats order like their bit
 // patterns, so an unsigned atomicMax reduces them (*amax_bits starts at 0).
-__global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restrict__ x, size_t n,
-                                                   unsigned* __restrict__ amax_bits) {
+// One atomic per block after a warp and a block reduction.
+__global__ void __launch_bounds__(256) amax_kernel(Tensors5 t, size_t n) {
+  const __nv_bfloat16* __restrict__ x = t.x[blockIdx.y];
+  __shared__ float wmax[8];
   float m = 0.f;
   const size_t stride = (size_t)gridDim.x * blockDim.x * 8;
   for (size_t i = ((size_t)blockIdx.x * blockDim.x + threadIdx.x) * 8; i < n; i += stride) {
@@ -45,7 +55,13 @@ __global__ void __launch_bounds__(256) amax_kernel(const __nv_bfloat16* __restri
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, wmax[w]);
+    atomicMax(t.amax_bits[blockIdx.y], __float_as_uint(m));
+  }
 }
 
 // out[i] = e4m3(x[i] / s), s from *amax_bits; block 0 publishes s.
@@ -69,49 +85,80 @@ __global__ void __launch_bounds__(256) quant_kernel(const __nv_bfloat16* __restr
   }
 }
 
-// Wt[c][r] = e4m3(W[r][c] / s) for W [rows][cols] bf16: 32 x 32 tiles through
-// shared memory (rows and cols multiples of 32).
-__global__ void __launch_bounds__(256) quant_t_kernel(const __nv_bfloat16* __restrict__ W, int rows, int cols,
-                                                      const unsigned* __restrict__ amax_bits,
-                                                      __nv_fp8_e4m3* __restrict__ Wt, float* __restrict__ scale) {
-  __shared__ float tile[32][33];
-  const float s = scale_of(amax_bits);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && threadIdx.y == 0) *scale = s;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  for (int y = threadIdx.y; y < 32; y += 8)
-    tile[y][threadIdx.x] = __bfloat162float(W[(size_t)(r0 + y) * cols + c0 + threadIdx.x]);
+// Wt[c][r] = e4m3(W[r][c] / s) for W [rows][cols] bf16 (blockIdx.z picks the
+// tensor): 64 x 64 tiles through shared memory, 16-byte loads and 4-byte
+// stores (rows and cols multiples of 64).
+__global__ void __launch_bounds__(256) quant_t_kernel(Tensors5 t, int rows, int cols) {
+  __shared__ float tile[64][65];
+  const int z = blockIdx.z;
+  const float s = scale_of(t.amax_bits[z]);
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *t.scale[z] = s;
+  const __nv_bfloat16* __restrict__ W = t.x[z];
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int idx = threadIdx.x + 256 * k, r = idx >> 3, c8 = (idx & 7) * 8;
+    const uint4 v = *reinterpret_cast<const uint4*>(W + (size_t)(r0 + r) * cols + c0 + c8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+      tile[r][c8 + 2 * j] = f.x;
+      tile[r][c8 + 2 * j + 1] = f.y;
+    }
+  }
   __syncthreads();
-  for (int y = threadIdx.y; y < 32; y += 8) {
-    const float v = tile[threadIdx.x][y];
-    reinterpret_cast<uint8_t*>(Wt)[(size_t)(c0 + y) * rows + r0 + threadIdx.x] =
-        __nv_cvt_float_to_fp8(__fdiv_rn(v, s), __NV_SATFINITE, __NV_E4M3);
+  uint8_t* __restrict__ out = reinterpret_cast<uint8_t*>(t.out[z]);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int idx = threadIdx.x + 256 * k, oc = idx >> 4, r4 = (idx & 15) * 4;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      packed |= (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(tile[r4 + e][oc], s), __NV_SATFINITE, __NV_E4M3)
+                << (8 * e);
+    *reinterpret_cast<uint32_t*>(out + (size_t)(c0 + oc) * rows + r0 + r4) = packed;
   }
 }
 
 int grid_for(size_t n) {
   const size_t blocks = (n / 8 + 255) / 256;
-  return (int)(blocks < 4096 ? (blocks > 0 ? blocks : 1) : 4096);
+  return (int)(blocks < 1184 ? (blocks > 0 ? blocks : 1) : 1184);  // 8 blocks per SM at most
 }
 
 }  // namespace
 
-cudaError_t launch_amax(const void* x, size_t n, unsigned* amax_bits, cudaStream_t st) {
-  amax_kernel<<<grid_for(n), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), n, amax_bits);
+cudaError_t launch_amax(const void* const* x, int count, size_t n, unsigned* amax_bits, cudaStream_t st) {
+  if (count < 1 || count > 5) return cudaErrorInvalidValue;
+  Tensors5 t{};
+  for (int i = 0; i < count; ++i) {
+    t.x[i] = reinterpret_cast<const __nv_bfloat16*>(x[i]);
+    t.amax_bits[i] = amax_bits + i;
+  }
+  amax_kernel<<<dim3(grid_for(n), count), 256, 0, st>>>(t, n);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant(const void* x, size_t n, const unsigned* amax_bits, void* out, float* scale,
                          cudaStream_t st) {
-  quant_kernel<<<grid_for(n), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), n, amax_bits,
+  // Streaming conversion: enough blocks to keep every SM's memory pipe busy.
+  const size_t blocks = (n / 8 + 255) / 256;
+  quant_kernel<<<(int)(blocks < 4096 ? (blocks > 0 ? blocks : 1) : 4096), 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(x), n, amax_bits,
                                             reinterpret_cast<__nv_fp8_e4m3*>(out), scale);
   return cudaGetLastError();
 }
 
-cudaError_t launch_quant_t(const void* W, int rows, int cols, const unsigned* amax_bits, void* Wt, float* scale,
-                           cudaStream_t st) {
-  dim3 grid(cols / 32, rows / 32), block(32, 8);
-  quant_t_kernel<<<grid, block, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(W), rows, cols, amax_bits,
-                                         reinterpret_cast<__nv_fp8_e4m3*>(Wt), scale);
+cudaError_t launch_quant_t(const void* const* W, int count, int rows, int cols, const unsigned* amax_bits,
+                           void* Wt, size_t wt_stride, float* scale, cudaStream_t st) {
+  if (count < 1 || count > 5 || rows % 64 != 0 || cols % 64 != 0) return cudaErrorInvalidValue;
+  Tensors5 t{};
+  for (int i = 0; i < count; ++i) {
+    t.x[i] = reinterpret_cast<const __nv_bfloat16*>(W[i]);
+    t.amax_bits[i] = const_cast<unsigned*>(amax_bits) + i;
+    t.out[i] = reinterpret_cast<__nv_fp8_e4m3*>(static_cast<char*>(Wt) + i * wt_stride);
+    t.scale[i] = scale + i;
+  }
+  quant_t_kernel<<<dim3(cols / 64, rows / 64, count), 256, 0, st>>>(t, rows, cols);
   return cudaGetLastError();
 }
 

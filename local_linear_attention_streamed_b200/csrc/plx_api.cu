@@ -517,7 +517,7 @@ int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const v
   if (B < 1 || N < 1 || H < 1) return PLX_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
   if ((long long)B * N * H * d >= (1ll << 31)) return PLX_ERR_UNSUPPORTED;
-  if (((long long)B * N) % 16 != 0) return PLX_ERR_UNSUPPORTED;  // fp8 GEMM operand alignment
+  if (((long long)B * N) % 16 != 0 || (H * d) % 64 != 0) return PLX_ERR_UNSUPPORTED;  // fp8 operand tiles
   if (!aligned16(x) || !aligned16(WQ) || !aligned16(WK) || !aligned16(WV) || !aligned16(WR) ||
       !aligned16(WO) || !aligned16(y))
     return PLX_ERR_MISALIGNED;
@@ -558,11 +558,10 @@ int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const v
   void* lt_ws = w8 + 5 * wsz + 256;
   const void* W[5] = {WQ, WK, WV, WR, WO};
   if (cudaMemsetAsync(amax, 0, 8 * sizeof(unsigned), st) != cudaSuccess) return PLX_ERR_CUDA;
-  cudaError_t e = launch_amax(x, (size_t)M * D, amax, st);
-  for (int i = 0; i < 5 && e == cudaSuccess; ++i) e = launch_amax(W[i], (size_t)D * D, amax + 1 + i, st);
+  cudaError_t e = launch_amax(&x, 1, (size_t)M * D, amax, st);
+  if (e == cudaSuccess) e = launch_amax(W, 5, (size_t)D * D, amax + 1, st);
   if (e == cudaSuccess) e = launch_quant(x, (size_t)M * D, amax, x8, scale, st);
-  for (int i = 0; i < 5 && e == cudaSuccess; ++i)
-    e = launch_quant_t(W[i], D, D, amax + 1 + i, w8 + i * wsz, scale + 1 + i, st);
+  if (e == cudaSuccess) e = launch_quant_t(W, 5, D, D, amax + 1, w8, wsz, scale + 1, st);
   if (e != cudaSuccess) return cuda_rc(e);
   for (int i = 0; i < 4; ++i)
     if (fp8_gemm(dc->cublas_lt, w8 + i * wsz, x8, proj[i], D, D, M, scale + 1 + i, scale, lt_ws, kLtWorkspace,
@@ -577,7 +576,8 @@ int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const v
   PrefillArgs a{head[0], head[1], head[2], head[3], attn, B, H, N, d, 1, dc->status};
   if ((e = launch_prefill_tc(a, st, dc->num_sms)) != cudaSuccess) return cuda_rc(e);
   if (launch_swap_axes(attn, proj[0], B, H, N, d, st) != cudaSuccess) return PLX_ERR_CUDA;
-  if ((e = launch_amax(proj[0], (size_t)M * D, amax + 6, st)) != cudaSuccess ||
+  const void* merged = proj[0];
+  if ((e = launch_amax(&merged, 1, (size_t)M * D, amax + 6, st)) != cudaSuccess ||
       (e = launch_quant(proj[0], (size_t)M * D, amax + 6, a8, scale + 6, st)) != cudaSuccess)
     return cuda_rc(e);
   if (fp8_gemm(dc->cublas_lt, w8 + 4 * wsz, a8, y, D, D, M, scale + 5, scale + 6, lt_ws, kLtWorkspace, st) != 0)

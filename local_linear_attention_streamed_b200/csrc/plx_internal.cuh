@@ -99,16 +99,18 @@ size_t bwd_padded_rows(int N);
 const char* bwd_last_failure();
 cudaError_t launch_prefill_bwd(const BwdArgs& a, cudaStream_t st, int num_sms);
 
-// Dynamic per-tensor fp8 (e4m3) linears: |max| reduction into float bits
-// (*amax_bits zeroed first), quantisation (s = max/448, written to *scale),
-// quantisation with a transpose of a [rows, cols] weight, and the e4m3 GEMM
-// Y[M, Dout] = X8[M, Din] Wt8[Dout, Din]^T sX sW in bf16 through cuBLASLt
-// (returns 0 on success).  Sizes are multiples of 32; pointers 16-byte aligned.
-cudaError_t launch_amax(const void* x, size_t n, unsigned* amax_bits, cudaStream_t st);
+// Dynamic per-tensor fp8 (e4m3) linears: |max| reductions of `count` (<= 5)
+// tensors of n values each into amax_bits[0..count) (zeroed first),
+// quantisation (s = max/448, written to *scale), quantisation with a
+// transpose of `count` [rows, cols] weights into Wt + i * wt_stride (scales to
+// scale[i]), and the e4m3 GEMM Y[M, Dout] = X8[M, Din] Wt8[Dout, Din]^T sX sW
+// in bf16 through cuBLASLt (returns 0 on success).  Sizes are multiples of 64;
+// pointers 16-byte aligned.
+cudaError_t launch_amax(const void* const* x, int count, size_t n, unsigned* amax_bits, cudaStream_t st);
 cudaError_t launch_quant(const void* x, size_t n, const unsigned* amax_bits, void* out, float* scale,
                          cudaStream_t st);
-cudaError_t launch_quant_t(const void* W, int rows, int cols, const unsigned* amax_bits, void* Wt, float* scale,
-                           cudaStream_t st);
+cudaError_t launch_quant_t(const void* const* W, int count, int rows, int cols, const unsigned* amax_bits,
+                           void* Wt, size_t wt_stride, float* scale, cudaStream_t st);
 int fp8_gemm(void* lt_handle, const void* Wt8, const void* X8, void* Y, int Dout, int Din, long long M,
              const float* sW, const float* sX, void* ws, size_t ws_bytes, cudaStream_t st);
 
