@@ -245,7 +245,7 @@ struct KvSmem {
   uint8_t dout[kQStages][kHalves][kQB * 128];
   uint8_t a[kKB * 128];  // a^T [128 keys][64 queries] bf16, K-major
   uint64_t kv_full, q_full[kQStages], q_empty[kQStages];
-  uint64_t s_full, s_free, p_full, ag_free, done, drain;
+  uint64_t s_full, s_free, p_full, ag_free, done, drain, drain_g;
   uint32_t tmem_base;
   int abort;
 };
@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.ag_free, 1);
     mbar_init(&sm.done, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_g, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -320,6 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sm.qr[st][h] + kQB * 128, &tmR, &sm.q_full[st], 64 * h, qrow);
           tma_load_2d(sm.dout[st][h], &tmdO, &sm.q_full[st], 64 * h, qrow);
         }
+        // The block's statistics (1 KB, read by every elementwise thread)
+        // into L1 ahead of use.
+        const float* stp = p.stats + stat_index(bh, p.Npad, (q0 + i) * kQB, 0);
+#pragma unroll
+        for (int l = 0; l < 8; ++l) asm volatile("prefetch.global.L1 [%0];" ::"l"(stp + 32 * l));
       }
       if (*abort) {  // let every copy issued here land before the CTA exits
         mbar_drain(&sm.kv_full, 0);
@@ -327,10 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_use[s] >= 0) mbar_drain(&sm.q_full[s], (uint32_t)(last_use[s] & 1));
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    // Order in the tensor pipe: scores of block i, then the gradient MMAs of
-    // block i - 1 (their operands are written while block i's scores run).
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers ----------------
+    // Warp 1 issues the scores of every block, warp 2 its gradient MMAs: an
+    // issue returns only once the tensor pipe has taken the MMA, so one
+    // thread for both would hold the gradients of block i behind the scores
+    // of block i + 1 (and those behind the wait for block i + 1's operands).
     if (lane == 0) {
       const uint64_t aK = sdesc(smem_u32(sm.k[0]), 16, 1024), aV = sdesc(smem_u32(sm.v[0]), 16, 1024);
       const uint64_t aA = sdesc(smem_u32(sm.a), 16, 1024);
@@ -351,39 +359,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&sm.ag_free);
         mma_commit(&sm.q_empty[st]);
       };
-      bool ok = mbar_wait(&sm.kv_full, 0, abort, p.status);
-      for (int i = 0; ok && i < nq; ++i) {
-        const int st = i % kQStages;
-        if (!(ok = mbar_wait(&sm.q_full[st], (i / kQStages) & 1, abort, p.status))) break;
-        if (i > 0 && !(ok = mbar_wait(&sm.s_free, (i - 1) & 1, abort, p.status))) break;
-        tc_fence_after();
-        const uint64_t bqr = sdesc(smem_u32(sm.qr[st][0]), 16, 1024);
-        const uint64_t bdo = sdesc(smem_u32(sm.dout[st][0]), 16, 1024);
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t ka = (ks >> 2) * (kKB * 128) + (ks & 3) * 32;
-          mma_ss(tmem + kColS, aK + (uint64_t)(ka >> 4),
-                 bqr + (uint64_t)((((ks >> 2) * 2 * kQB * 128) + (ks & 3) * 32) >> 4), idesc(2 * kQB, 0),
-                 ks > 0 ? 1u : 0u);
-          mma_ss(tmem + kColDA, aV + (uint64_t)(ka >> 4),
-                 bdo + (uint64_t)((((ks >> 2) * kQB * 128) + (ks & 3) * 32) >> 4), idesc(kQB, 0),
-                 ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&sm.s_full);
-        if (i > 0) {
-          if (!(ok = mbar_wait(&sm.p_full, (i - 1) & 1, abort, p.status))) break;
+      if (warp == 1) {
+        bool ok = mbar_wait(&sm.kv_full, 0, abort, p.status);
+        for (int i = 0; ok && i < nq; ++i) {
+          const int st = i % kQStages;
+          if (!(ok = mbar_wait(&sm.q_full[st], (i / kQStages) & 1, abort, p.status))) break;
+          if (i > 0 && !(ok = mbar_wait(&sm.s_free, (i - 1) & 1, abort, p.status))) break;
           tc_fence_after();
-          issue_grads(i - 1);
+          const uint64_t bqr = sdesc(smem_u32(sm.qr[st][0]), 16, 1024);
+          const uint64_t bdo = sdesc(smem_u32(sm.dout[st][0]), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const uint32_t ka = (ks >> 2) * (kKB * 128) + (ks & 3) * 32;
+            mma_ss(tmem + kColS, aK + (uint64_t)(ka >> 4),
+                   bqr + (uint64_t)((((ks >> 2) * 2 * kQB * 128) + (ks & 3) * 32) >> 4), idesc(2 * kQB, 0),
+                   ks > 0 ? 1u : 0u);
+            mma_ss(tmem + kColDA, aV + (uint64_t)(ka >> 4),
+                   bdo + (uint64_t)((((ks >> 2) * kQB * 128) + (ks & 3) * 32) >> 4), idesc(kQB, 0),
+                   ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.s_full);
         }
+        // Every MMA issued here completes before TMEM is freed.
+        mma_commit(&sm.drain);
+        mbar_drain(&sm.drain, 0);
+      } else {
+        bool ok = true;
+        for (int i = 0; ok && i < nq; ++i) {
+          if (!(ok = mbar_wait(&sm.p_full, i & 1, abort, p.status))) break;
+          tc_fence_after();
+          issue_grads(i);
+        }
+        if (ok) mma_commit(&sm.done);
+        mma_commit(&sm.drain_g);
+        mbar_drain(&sm.drain_g, 0);
       }
-      if (ok && mbar_wait(&sm.p_full, (nq - 1) & 1, abort, p.status)) {
-        tc_fence_after();
-        issue_grads(nq - 1);
-        mma_commit(&sm.done);
-      }
-      // Every MMA issued here completes before TMEM is freed.
-      mma_commit(&sm.drain);
-      mbar_drain(&sm.drain, 0);
     }
   } else if (warp >= kFirstEwWarp) {
     // ---------------- elementwise warpgroups ----------------
@@ -480,7 +490,7 @@ struct QSmem {
   uint8_t k[kKVStages][kHalves][kKN * 128];
   uint8_t v[kKVStages][kHalves][kKN * 128];
   uint64_t q_full, kv_full[kKVStages], kv_empty[kKVStages];
-  uint64_t s_full, s_free, p_full, pv_done, done, drain;
+  uint64_t s_full, s_free, p_full, pv_done, done, drain, drain_g;
   uint32_t tmem_base;
   int abort;
 };
@@ -518,6 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.pv_done, 1);
     mbar_init(&sm.done, 1);
     mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain_g, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -560,8 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_use[s] >= 0) mbar_drain(&sm.kv_full[s], (uint32_t)(last_use[s] & 1));
       }
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == 2) {
+    // ---------------- MMA issuers: scores (warp 1) and gradients (warp 2) ----------------
     if (lane == 0) {
       const uint64_t aQ = sdesc(smem_u32(sm.q[0]), 16, 1024), aR = sdesc(smem_u32(sm.r[0]), 16, 1024);
       const uint64_t aO = sdesc(smem_u32(sm.dout[0]), 16, 1024);
@@ -579,6 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&sm.kv_empty[st]);
         mma_commit(&sm.pv_done);
       };
+      if (warp == 1) {
       bool ok = mbar_wait(&sm.q_full, 0, abort, p.status);
       for (int j = 0; ok && j < nk; ++j) {
         const int st = j % kKVStages;
@@ -597,19 +609,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + kColDA, aO + ao, bv + bo, idesc(kKN, 0), acc);
         }
         mma_commit(&sm.s_full);
-        if (j > 0) {
-          if (!(ok = mbar_wait(&sm.p_full, (j - 1) & 1, abort, p.status))) break;
-          tc_fence_after();
-          issue_grads(j - 1);
-        }
-      }
-      if (ok && mbar_wait(&sm.p_full, (nk - 1) & 1, abort, p.status)) {
-        tc_fence_after();
-        issue_grads(nk - 1);
-        mma_commit(&sm.done);
       }
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
+      } else {
+        bool ok = true;
+        for (int j = 0; ok && j < nk; ++j) {
+          if (!(ok = mbar_wait(&sm.p_full, j & 1, abort, p.status))) break;
+          tc_fence_after();
+          issue_grads(j);
+        }
+        if (ok) mma_commit(&sm.done);
+        mma_commit(&sm.drain_g);
+        mbar_drain(&sm.drain_g, 0);
+      }
     }
   } else if (warp >= kFirstEwWarp) {
     // ---------------- elementwise warpgroups ----------------
