@@ -54,6 +54,9 @@
 
 #include <math_constants.h>
 
+#include <cstdlib>
+#include <cstring>
+
 namespace plx {
 namespace {
 
@@ -128,6 +131,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 
 struct BwdParams {
   int B, H, N, Npad, causal;
+  int inject_stall;  // failure-detection test: CTA 0 of the dK/dV kernel never loads its K/V
   int chunk_heads;  // heads whose blocks are launched together (L2 reuse of their tiles)
   const float* stats;
   __nv_bfloat16* g0;  // dV (key-block kernel) or dQ (query-block kernel)
@@ -304,10 +308,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       const int krow = bh * p.N + kb * kKB;
-      mbar_expect_tx(&sm.kv_full, 2 * kKB * D * 2);
-      for (int h = 0; h < kHalves; ++h) {
-        tma_load_2d(sm.k[h], &tmK, &sm.kv_full, 64 * h, krow);
-        tma_load_2d(sm.v[h], &tmV, &sm.kv_full, 64 * h, krow);
+      // The failure-detection test withholds CTA 0's K/V: the score issuer's
+      // bounded wait runs out and every role unwinds through the abort path.
+      if (!(p.inject_stall && blockIdx.x == 0)) {
+        mbar_expect_tx(&sm.kv_full, 2 * kKB * D * 2);
+        for (int h = 0; h < kHalves; ++h) {
+          tma_load_2d(sm.k[h], &tmK, &sm.kv_full, 64 * h, krow);
+          tma_load_2d(sm.v[h], &tmV, &sm.kv_full, 64 * h, krow);
+        }
       }
       int last_use[kQStages] = {-1, -1, -1};
       for (int i = 0; i < nq && !*abort; ++i) {
@@ -722,7 +730,11 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   // About two waves of blocks per chunk of heads.
   int ch = (2 * num_sms + nblk - 1) / nblk;
   ch = ch < 1 ? 1 : (ch > BH ? BH : ch);
-  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
+  // PLX_FAULT_INJECT=bwd_stall makes one CTA's bounded waits run out (tests of
+  // the timeout status only).
+  const char* fi = getenv("PLX_FAULT_INJECT");
+  const int inject = (fi != nullptr && strcmp(fi, "bwd_stall") == 0) ? 1 : 0;
+  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, inject, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
                reinterpret_cast<__nv_bfloat16*>(a.dK), a.status};
   size_t smem = sizeof(KvSmem<D>) + 1024;
   if ((e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
@@ -730,7 +742,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
     return fail_at("dK/dV shared-memory attribute", e);
   bwd_dkv_kernel<D><<<BH * nblk, kThreads, smem, st>>>(mQ64, mR64, mO64, mK128, mV128, pk);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail_at("dK/dV kernel", e);
-  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
+  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, 0, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
                reinterpret_cast<__nv_bfloat16*>(a.dR), a.status};
   // At least 116 KB so that one CTA (and its 512 TMEM columns) holds an SM.
   smem = sizeof(QSmem<D>) + 1024;

@@ -29,3 +29,24 @@ def test_prefill_timeout_is_reported_and_context_survives(monkeypatch):
     assert plx.get_device_status() == 0
     want = oracle.prefill_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal=True)
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
+def test_backward_timeout_is_reported_and_context_survives(monkeypatch):
+    """PLX_FAULT_INJECT=bwd_stall: one CTA of the dK/dV kernel never receives its
+    K/V tiles; its bounded waits run out, the status word reports the timeout,
+    and the next backward call on the same context is correct."""
+    from local_linear_attention_streamed_b200 import plx
+    from _util import GRAD_TOL, rel_err_fro
+    B, H, N, d = 1, 2, 192, 128
+    dev, ref = small_inputs(32, synth.backward_specs(B, H, N, d), synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    assert plx.get_device_status() == 0
+    monkeypatch.setenv("PLX_FAULT_INJECT", "bwd_stall")
+    plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+    assert plx.get_device_status() == -7  # PLX_ERR_TIMEOUT
+    monkeypatch.delenv("PLX_FAULT_INJECT")
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+    assert plx.get_device_status() == 0
+    want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], True)
+    for g, w in zip(grads, want):
+        assert rel_err_fro(to_f64(g), w) <= GRAD_TOL
