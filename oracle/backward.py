@@ -23,14 +23,24 @@ import numpy as np
 import torch
 
 
-def _forward_torch(Q, K, V, R, causal: bool):
+def _hidden_keys(N: int, causal: bool, window=None) -> np.ndarray:
+    """[N, N] boolean, True where query i may not see key j: j > i when
+    causal, and j <= i - window with a sliding window (which implies causal)."""
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    hidden = (j > i) if (causal or window is not None) else np.zeros((N, N), dtype=bool)
+    if window is not None:
+        hidden |= j <= i - int(window)
+    return hidden
+
+
+def _forward_torch(Q, K, V, R, causal: bool, window=None):
     """Plain float64 forward over [..., N, d] tensors (all rows at once)."""
     d = Q.shape[-1]
     N = Q.shape[-2]
     S = Q @ K.transpose(-1, -2) / np.sqrt(d)
-    if causal:
-        mask = torch.ones(N, N, dtype=torch.bool).triu(1)
-        S = S.masked_fill(mask, float("-inf"))
+    if causal or window is not None:
+        S = S.masked_fill(torch.from_numpy(_hidden_keys(N, causal, window)), float("-inf"))
     P = torch.softmax(S, dim=-1)
     kbar = P @ K
     vbar = P @ V
@@ -42,14 +52,14 @@ def _forward_torch(Q, K, V, R, causal: bool):
     return vbar - corr
 
 
-def parallax_forward_ref(Q, K, V, R, causal: bool = True) -> np.ndarray:
+def parallax_forward_ref(Q, K, V, R, causal: bool = True, window=None) -> np.ndarray:
     """Forward output from the same statement (float64), for cross-checks."""
     t = [torch.from_numpy(np.asarray(x, dtype=np.float64)) for x in (Q, K, V, R)]
     with torch.no_grad():
-        return _forward_torch(*t, causal).numpy()
+        return _forward_torch(*t, causal, window).numpy()
 
 
-def prefill_stats_ref(Q, K, V, R, causal: bool = True):
+def prefill_stats_ref(Q, K, V, R, causal: bool = True, window=None):
     """What a training forward saves, per query row (float64), for [B, H, N, d] inputs.
 
     Returns (vbar [B,H,N,d], lse [B,H,N], tbar [B,H,N]): the softmax mean of the
@@ -61,8 +71,8 @@ def prefill_stats_ref(Q, K, V, R, causal: bool = True):
     Q, K, V, R = (np.asarray(x, dtype=np.float64) for x in (Q, K, V, R))
     N, d = Q.shape[-2], Q.shape[-1]
     S = Q @ np.swapaxes(K, -1, -2) / np.sqrt(d)
-    if causal:
-        S = np.where(np.triu(np.ones((N, N), dtype=bool), 1), -np.inf, S)
+    if causal or window is not None:
+        S = np.where(_hidden_keys(N, causal, window), -np.inf, S)
     smax = S.max(axis=-1, keepdims=True)
     W = np.exp(S - smax)
     omega = W.sum(axis=-1, keepdims=True)
@@ -73,9 +83,10 @@ def prefill_stats_ref(Q, K, V, R, causal: bool = True):
     return vbar, lse, tbar
 
 
-def parallax_backward_ref(Q, K, V, R, dO, causal: bool = True):
-    """Gradients (dQ, dK, dV, dR) of sum(out * dO) for inputs [B, H, N, d] (float64)."""
+def parallax_backward_ref(Q, K, V, R, dO, causal: bool = True, window=None):
+    """Gradients (dQ, dK, dV, dR) of sum(out * dO) for inputs [B, H, N, d] (float64);
+    ``window`` (None or W >= 1) restricts query i to its last W keys."""
     t = [torch.from_numpy(np.asarray(x, dtype=np.float64)).requires_grad_(True) for x in (Q, K, V, R)]
-    out = _forward_torch(*t, causal)
+    out = _forward_torch(*t, causal, window)
     out.backward(torch.from_numpy(np.asarray(dO, dtype=np.float64)))
     return tuple(x.grad.numpy() for x in t)

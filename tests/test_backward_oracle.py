@@ -188,3 +188,29 @@ def test_kernel_pair_formulas_reproduce_gradients(causal):
 def test_oracle_runs_on_cpu_only():
     assert not any(isinstance(x, torch.Tensor) and x.is_cuda for x in
                    oracle.parallax_backward_ref(*_inputs(81, N=3, d=2), True))
+
+
+@pytest.mark.parametrize("W", [1, 3, 6])
+def test_window_statement_and_gradients(W):
+    """With a sliding window the statement equals the row oracle's window, and
+    its gradients match central differences of that row oracle."""
+    Q, K, V, R, dO = _inputs(91, N=7)
+    np.testing.assert_allclose(oracle.parallax_forward_ref(Q, K, V, R, True, window=W),
+                               oracle.prefill_ref(Q, K, V, R, window=W), rtol=0, atol=1e-12)
+    got = oracle.parallax_backward_ref(Q, K, V, R, dO, True, window=W)
+    xs = [Q.copy(), K.copy(), V.copy(), R.copy()]
+    h = 1e-6
+    for a in range(4):
+        g = np.zeros_like(xs[a])
+        for idx in np.ndindex(xs[a].shape):
+            old = xs[a][idx]
+            xs[a][idx] = old + h
+            fp = np.sum(oracle.prefill_ref(*xs, window=W) * dO)
+            xs[a][idx] = old - h
+            fm = np.sum(oracle.prefill_ref(*xs, window=W) * dO)
+            xs[a][idx] = old
+            g[idx] = (fp - fm) / (2 * h)
+        assert np.max(np.abs(got[a] - g)) < 1e-7 * max(1.0, np.max(np.abs(g)))
+    vb, lse, tb = oracle.prefill_stats_ref(Q, K, V, R, True, window=W)
+    if W == 1:
+        np.testing.assert_allclose(vb, V, rtol=0, atol=1e-14)
