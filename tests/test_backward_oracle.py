@@ -73,7 +73,7 @@ def test_planted_mistake_in_statement_is_caught(monkeypatch):
     Q, K, V, R, dO = _inputs(11)
     want = _fd_grads(Q, K, V, R, dO, True)
     orig = bwd._forward_torch
-    monkeypatch.setattr(bwd, "_forward_torch", lambda q, k, v, r, c: orig(q, k, v, r, c) + 0.05 * q * r)
+    monkeypatch.setattr(bwd, "_forward_torch", lambda q, k, v, r, *a: orig(q, k, v, r, *a) + 0.05 * q * r)
     got = oracle.parallax_backward_ref(Q, K, V, R, dO, True)
     assert np.max(np.abs(got[0] - want[0])) > 1e-3
 
