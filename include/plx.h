@@ -127,6 +127,13 @@ int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R
                       void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
                       void* stream);
 
+/* plx_prefill_train for the sliding-window prefill of plx_prefill_window
+ * (query i sees keys i - window + 1 .. i): the statistics are those of the
+ * windowed softmax.  window >= 1, else PLX_ERR_INVALID_ARG. */
+int plx_prefill_train_window(const void* Q, const void* K, const void* V, const void* R, void* out,
+                             void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int window,
+                             void* stream);
+
 /* Bytes of the statistics workspace plx_prefill_bwd needs:
  * 16 * B * H * (N rounded up to a multiple of 128); 0 for invalid sizes. */
 size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d);
@@ -151,6 +158,14 @@ int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, 
                     const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
                     void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* plx_prefill_bwd for a sliding-window prefill (the tensors plx_prefill_train_window
+ * saved): key j takes gradient only from queries j .. j + window - 1.
+ * window >= 1, else PLX_ERR_INVALID_ARG; workspace as plx_prefill_bwd. */
+int plx_prefill_bwd_window(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                           const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                           void* dK, void* dV, void* dR, int B, int H, int N, int d, int window,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * One decode step with split-KV: every (b, h) streams its cache rows

@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 
 struct BwdParams {
   int B, H, N, Npad, causal;
+  int window;        // sliding window (0: none): query i saw keys i - window + 1 .. i
   int inject_stall;  // failure-detection test: CTA 0 of the dK/dV kernel never loads its K/V
   int chunk_heads;  // heads whose blocks are launched together (L2 reuse of their tiles)
   const float* stats;
@@ -274,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kb = bo.rank, bh = bo.bh;
   const int nqb = (p.N + kQB - 1) / kQB;
   const int q0 = p.causal ? (kb * kKB) / kQB : 0;
-  const int nq = nqb - q0;  // >= 1: key block kb starts below N
+  // With a window, the block's last key is seen by queries up to kb kKB + kKB - 1 + window - 1.
+  const int qend = p.window > 0 ? min(nqb, (kb * kKB + kKB + p.window - 2) / kQB + 1) : nqb;
+  const int nq = qend - q0;  // >= 1: key block kb starts below N
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
@@ -426,7 +429,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = (q0 + i) * kQB + kEwCols * wg;  // query of column 0
       // Masks only where some pair of the warp is masked: the causal diagonal
       // (query before key) and queries past N.
-      const bool edge = __any_sync(0xffffffffu, (p.causal && i0 < kk) || i0 + kEwCols - 1 >= p.N);
+      const bool edge = __any_sync(0xffffffffu, (p.causal && i0 < kk) || i0 + kEwCols - 1 >= p.N ||
+                                                    (p.window > 0 && i0 + kEwCols - 1 >= kk + p.window));
       // The statistics of this thread's 16 queries (read by every lane: cached).
       const float* sts = p.stats + stat_index(bh, p.Npad, (q0 + i) * kQB, 0) + kEwCols * wg;
       const uint64_t sc2 = f2(scale2, scale2), nisd2 = f2(-isd, -isd);
@@ -441,8 +445,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int e = 4 * c4 + 2 * h;
-          const bool k0 = !edge || ((!p.causal || i0 + e >= kk) && i0 + e < p.N);
-          const bool k1 = !edge || ((!p.causal || i0 + e + 1 >= kk) && i0 + e + 1 < p.N);
+          const bool k0 = !edge || ((!p.causal || i0 + e >= kk) && i0 + e < p.N &&
+                                    (p.window <= 0 || i0 + e < kk + p.window));
+          const bool k1 = !edge || ((!p.causal || i0 + e + 1 >= kk) && i0 + e + 1 < p.N &&
+                                    (p.window <= 0 || i0 + e + 1 < kk + p.window));
           const GradPairs g = grad_pairs(
               s[e], s[e + 1], t[e], t[e + 1], da[e], da[e + 1], h ? f2(L.z, L.w) : f2(L.x, L.y),
               h ? f2(C.z, C.w) : f2(C.x, C.y), h ? f2(Dv.z, Dv.w) : f2(Dv.x, Dv.y),
@@ -521,7 +527,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The last query block sees every key (causal): rank r is query block nmb - 1 - r.
   const BlockOrder bo = block_order(blockIdx.x, BH, nmb, p.chunk_heads);
   const int m = nmb - 1 - bo.rank, bh = bo.bh;
-  const int nk = p.causal ? (min(m * kQM + kQM - 1, p.N - 1) / kKN + 1) : (p.N + kKN - 1) / kKN;
+  // Key blocks j0 .. j0 + nk - 1 (a window hides the keys before m kQM - window + 1).
+  const int j0 = p.window > 0 ? max(0, m * kQM - p.window + 1) / kKN : 0;
+  const int nk = (p.causal ? (min(m * kQM + kQM - 1, p.N - 1) / kKN + 1) : (p.N + kKN - 1) / kKN) - j0;
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u > 0 && !mbar_wait(&sm.kv_empty[st], (u - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.kv_full[st], 2 * kKN * D * 2);
         last_use[st] = u;
-        const int krow = bh * p.N + j * kKN;
+        const int krow = bh * p.N + (j0 + j) * kKN;
         for (int h = 0; h < kHalves; ++h) {
           tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], 64 * h, krow);
           tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], 64 * h, krow);
@@ -657,14 +665,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free);
-      const int k0 = j * kKN + kEwCols * wg;  // key of column 0
-      const bool edge = __any_sync(0xffffffffu, (p.causal && k0 + kEwCols - 1 > i) || k0 + kEwCols - 1 >= p.N);
+      const int k0 = (j0 + j) * kKN + kEwCols * wg;  // key of column 0
+      const bool edge = __any_sync(0xffffffffu, (p.causal && k0 + kEwCols - 1 > i) || k0 + kEwCols - 1 >= p.N ||
+                                                    (p.window > 0 && k0 <= i - p.window));
       uint32_t pl[kEwCols / 2], pt[kEwCols / 2];
 #pragma unroll
       for (int c = 0; c < kEwCols / 2; ++c) {
         const int e = 2 * c;
-        const bool keep0 = !edge || ((!p.causal || k0 + e <= i) && k0 + e < p.N);
-        const bool keep1 = !edge || ((!p.causal || k0 + e + 1 <= i) && k0 + e + 1 < p.N);
+        const bool keep0 = !edge || ((!p.causal || k0 + e <= i) && k0 + e < p.N &&
+                                     (p.window <= 0 || k0 + e > i - p.window));
+        const bool keep1 = !edge || ((!p.causal || k0 + e + 1 <= i) && k0 + e + 1 < p.N &&
+                                     (p.window <= 0 || k0 + e + 1 > i - p.window));
         const GradPairs g = grad_pairs(s[e], s[e + 1], t[e], t[e + 1], da[e], da[e + 1], nl2, c02, dd2, fd2, sc2,
                                        nisd2, keep0, keep1);
         pl[c] = g.dl;
@@ -734,7 +745,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   // the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "bwd_stall") == 0) ? 1 : 0;
-  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, inject, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
+  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, a.window, inject, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
                reinterpret_cast<__nv_bfloat16*>(a.dK), a.status};
   size_t smem = sizeof(KvSmem<D>) + 1024;
   if ((e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
@@ -742,7 +753,7 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
     return fail_at("dK/dV shared-memory attribute", e);
   bwd_dkv_kernel<D><<<BH * nblk, kThreads, smem, st>>>(mQ64, mR64, mO64, mK128, mV128, pk);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail_at("dK/dV kernel", e);
-  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, 0, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
+  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, a.window, 0, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
                reinterpret_cast<__nv_bfloat16*>(a.dR), a.status};
   // At least 116 KB so that one CTA (and its 512 TMEM columns) holds an SM.
   smem = sizeof(QSmem<D>) + 1024;

@@ -192,9 +192,9 @@ int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void
   return plx_prefill_ex(Q, K, V, R, out, B, H, N, d, causal, PLX_BF16, nullptr);
 }
 
-int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R, void* out,
-                      void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
-                      void* stream) {
+static int prefill_train_impl(const void* Q, const void* K, const void* V, const void* R, void* out,
+                              void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
+                              int window, void* stream) {
   if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
   if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
@@ -209,7 +209,21 @@ int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R
   a.vbar = vbar;
   a.lse = lse;
   a.tbar = tbar;
+  a.window = window < N ? window : 0;
   return cuda_rc(launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream), dc->num_sms));
+}
+
+int plx_prefill_train(const void* Q, const void* K, const void* V, const void* R, void* out,
+                      void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
+                      void* stream) {
+  return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, causal, 0, stream);
+}
+
+int plx_prefill_train_window(const void* Q, const void* K, const void* V, const void* R, void* out,
+                             void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int window,
+                             void* stream) {
+  if (window < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, 1, window, stream);
 }
 
 size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d) {
@@ -217,10 +231,10 @@ size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d) {
   return 16 * (size_t)B * H * bwd_padded_rows(N);
 }
 
-int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, const void* out,
-                    const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
-                    void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+static int prefill_bwd_impl(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                            const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                            void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal, int window,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar || !dO || !dQ || !dK || !dV || !dR)
     return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
@@ -240,6 +254,7 @@ int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   BwdArgs a{Q, K, V, R, out, vbar, dO, lse, tbar, dQ, dK, dV, dR, B, H, N, d, causal ? 1 : 0, workspace,
             dc->status};
+  a.window = window < N ? window : 0;
   if (!workspace) {
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = grow(&dc->bwd_ws, &dc->bwd_ws_bytes, need, st)) != PLX_OK) return rc;
@@ -247,6 +262,23 @@ int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, 
     return cuda_rc(launch_prefill_bwd(a, st, dc->num_sms));
   }
   return cuda_rc(launch_prefill_bwd(a, st, dc->num_sms));
+}
+
+int plx_prefill_bwd(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                    const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                    void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, causal, 0, workspace,
+                          workspace_bytes, stream);
+}
+
+int plx_prefill_bwd_window(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                           const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
+                           void* dK, void* dV, void* dR, int B, int H, int N, int d, int window,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (window < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, 1, window, workspace,
+                          workspace_bytes, stream);
 }
 
 int plx_decode_num_splits(int B, int H, int L, int d) {

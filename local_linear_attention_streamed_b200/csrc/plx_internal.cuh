@@ -93,6 +93,7 @@ struct BwdArgs {
   int B, H, N, d, causal;
   void* stats;
   int* status;
+  int window = 0;  // sliding window of the forward (0: none; implies causal)
 };
 size_t bwd_padded_rows(int N);
 // The step of this thread's last failed backward launch ("" if none).

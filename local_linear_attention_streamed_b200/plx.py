@@ -42,6 +42,8 @@ SIGNATURES = {
     "plx_prefill_train": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
     "plx_prefill_bwd_workspace_bytes": (_sz, [_i] * 4),
     "plx_prefill_bwd": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
+    "plx_prefill_train_window": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
+    "plx_prefill_bwd_window": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_get_device_status": (_i, [_vp]),
     "plx_status_string": (ctypes.c_char_p, [_i]),
     "plx_last_cuda_error": (ctypes.c_char_p, []),
@@ -150,8 +152,9 @@ def decode_window(q, r, Kcache, Vcache, seqlens, window: int, out=None, workspac
     return out
 
 
-def prefill_train(Q, K, V, R, causal: bool = True, stream=None):
-    """bf16 prefill that also saves the backward pass's inputs.
+def prefill_train(Q, K, V, R, causal: bool = True, stream=None, window=None):
+    """bf16 prefill that also saves the backward pass's inputs (``window``:
+    the sliding-window prefill of prefill_window).
 
     Returns (out, vbar, lse, tbar): out bf16 [B, H, N, d], vbar fp32
     [B, H, N, d], lse and tbar fp32 [B, H, N] (see plx_prefill_train in
@@ -167,10 +170,16 @@ def prefill_train(Q, K, V, R, causal: bool = True, stream=None):
     vbar = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     tbar = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
-    rc = lib.plx_prefill_train(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
-                               _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, N, d,
-                               int(bool(causal)), _stream_ptr(stream))
-    _check(rc, "plx_prefill_train")
+    if window is None:
+        rc = lib.plx_prefill_train(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                   _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, N, d,
+                                   int(bool(causal)), _stream_ptr(stream))
+        _check(rc, "plx_prefill_train")
+    else:
+        rc = lib.plx_prefill_train_window(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"),
+                                          _dev(out, "out"), _dev(vbar, "vbar"), _dev(lse, "lse"),
+                                          _dev(tbar, "tbar"), B, H, N, d, int(window), _stream_ptr(stream))
+        _check(rc, "plx_prefill_train_window")
     return out, vbar, lse, tbar
 
 
@@ -179,7 +188,7 @@ def prefill_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, grads=None,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, window=None):
     """Gradients (dQ, dK, dV, dR) of sum(out * dO) for one bf16 prefill.
 
     ``out, vbar, lse, tbar`` are what prefill_train returned for the same
@@ -199,11 +208,15 @@ def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, 
     dQ, dK, dV, dR = grads
     ws, wsb = (0, 0) if workspace is None else (_dev(workspace, "workspace"),
                                                 workspace.numel() * workspace.element_size())
-    rc = lib.plx_prefill_bwd(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
-                             _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), _dev(dO, "dO"),
-                             _dev(dQ, "dQ"), _dev(dK, "dK"), _dev(dV, "dV"), _dev(dR, "dR"),
-                             B, H, N, d, int(bool(causal)), ws, wsb, _stream_ptr(stream))
-    _check(rc, "plx_prefill_bwd")
+    args = (_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"), _dev(vbar, "vbar"),
+            _dev(lse, "lse"), _dev(tbar, "tbar"), _dev(dO, "dO"), _dev(dQ, "dQ"), _dev(dK, "dK"),
+            _dev(dV, "dV"), _dev(dR, "dR"), B, H, N, d)
+    if window is None:
+        rc = lib.plx_prefill_bwd(*args, int(bool(causal)), ws, wsb, _stream_ptr(stream))
+        _check(rc, "plx_prefill_bwd")
+    else:
+        rc = lib.plx_prefill_bwd_window(*args, int(window), ws, wsb, _stream_ptr(stream))
+        _check(rc, "plx_prefill_bwd_window")
     return dQ, dK, dV, dR
 
 
@@ -211,24 +224,26 @@ class ParallaxAttention(torch.autograd.Function):
     """Autograd wrapper: forward = prefill_train, backward = prefill_backward (bf16)."""
 
     @staticmethod
-    def forward(ctx, Q, K, V, R, causal=True):
+    def forward(ctx, Q, K, V, R, causal=True, window=None):
         Q, K, V, R = (t.contiguous() for t in (Q, K, V, R))
-        out, vbar, lse, tbar = prefill_train(Q, K, V, R, causal)
+        out, vbar, lse, tbar = prefill_train(Q, K, V, R, causal, window=window)
         ctx.save_for_backward(Q, K, V, R, out, vbar, lse, tbar)
         ctx.causal = causal
+        ctx.window = window
         return out
 
     @staticmethod
     def backward(ctx, dO):
         Q, K, V, R, out, vbar, lse, tbar = ctx.saved_tensors
         dQ, dK, dV, dR = prefill_backward(Q, K, V, R, out, vbar, lse, tbar,
-                                          dO.contiguous().to(torch.bfloat16), ctx.causal)
-        return dQ, dK, dV, dR, None
+                                          dO.contiguous().to(torch.bfloat16), ctx.causal, window=ctx.window)
+        return dQ, dK, dV, dR, None, None
 
 
-def parallax_attention(Q, K, V, R, causal: bool = True):
-    """Differentiable bf16 Parallax attention over [B, H, N, d] (d in {64, 128})."""
-    return ParallaxAttention.apply(Q, K, V, R, causal)
+def parallax_attention(Q, K, V, R, causal: bool = True, window=None):
+    """Differentiable bf16 Parallax attention over [B, H, N, d] (d in {64, 128});
+    ``window`` (None or W >= 1) makes it the sliding-window prefill."""
+    return ParallaxAttention.apply(Q, K, V, R, causal, window)
 
 
 def decode_workspace_bytes(B: int, H: int, L: int, d: int) -> int:

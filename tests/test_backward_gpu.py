@@ -183,3 +183,20 @@ def test_calls_from_a_fresh_thread(plx):
     for a, b in zip(first, res["g"]):
         assert torch.equal(a, b)
     assert torch.equal(res["o"], saved[0])
+
+
+@pytest.mark.parametrize("N,d,W", [(300, 128, 37), (300, 128, 100), (320, 128, 200), (260, 64, 64),
+                                   (200, 64, 150), (130, 128, 1)])
+def test_window_backward_matches_oracle(plx, N, d, W):
+    """Sliding-window training forward then backward: every gradient element,
+    windows shorter and longer than the 64/128-row blocks, ragged N."""
+    B, H = 1, 2
+    dev, ref = small_inputs(600 + N + W, synth.backward_specs(B, H, N, d), synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True, window=W)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True, window=W)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    out_w = plx.prefill_window(dev["Q"], dev["K"], dev["V"], dev["R"], W)
+    assert torch.equal(saved[0], out_w)
+    want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], True, window=W)
+    _check_grads(grads, want, where=W)
