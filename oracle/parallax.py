@@ -35,6 +35,9 @@ Sliding window (the pages list kernels combining Parallax with sliding-window
 sparsity as future work, rainbus.top "未来方向"; they fix no rule): with a
 window of W keys, query i sees keys max(0, i - W + 1)..i, and a decode query
 at KV length n sees keys max(0, n - W)..n-1.
+Block sparsity (the same list; no rule either): a boolean mask over (tile of
+128 queries, block of 64 keys) pairs; query i sees key j when j <= i and the
+pair (i // 128, j // 64) is active.
 """
 from __future__ import annotations
 
@@ -75,6 +78,34 @@ def visible_keys(i: int, N: int, causal: bool, window=None):
     if window is not None:
         return max(0, i - int(window) + 1), i + 1
     return 0, (i + 1 if causal else N)
+
+
+BLOCK_Q, BLOCK_K = 128, 64  # query tile and key block of the block-sparse mask
+
+
+def sparse_visible_keys(i: int, block_mask) -> np.ndarray:
+    """Indices of the keys query i sees under a block mask [tiles, key blocks] (causal)."""
+    t = i // BLOCK_Q
+    keys = [j for j in range(i + 1) if block_mask[t, j // BLOCK_K]]
+    return np.asarray(keys, dtype=np.int64)
+
+
+def prefill_block_sparse_ref(Q, K, V, R, block_mask, rows=None) -> np.ndarray:
+    """Oracle for a block-sparse causal prefill (mask shared by all heads).
+
+    block_mask: bool [ceil(N/128), ceil(N/64)].  Every query must see at least
+    one key (the tile's own diagonal block active).  ``rows`` as prefill_ref.
+    """
+    B, H, N, d = Q.shape
+    rows_iter = ([(b, h, i) for b in range(B) for h in range(H) for i in range(N)] if rows is None
+                 else list(rows))
+    res = []
+    for (b, h, i) in rows_iter:
+        ks = sparse_visible_keys(i, block_mask)
+        res.append(parallax_row(Q[b, h, i], R[b, h, i], K[b, h, ks], V[b, h, ks]))
+    if rows is None:
+        return np.stack(res).reshape(B, H, N, d)
+    return np.stack(res) if res else np.zeros((0, d))
 
 
 def prefill_ref(Q, K, V, R, causal: bool = True, rows=None, window=None) -> np.ndarray:

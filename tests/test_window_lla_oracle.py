@@ -121,3 +121,52 @@ def test_lla_prefill_ref_shapes_and_rows():
     out, Rs = oracle.lla_prefill_ref(Q, K, V, 0.5, causal=True)
     assert out.shape == V.shape and Rs.shape == Q.shape
     np.testing.assert_allclose(out, oracle.prefill_ref(Q, K, V, Rs, causal=True), rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse reading: mask over (128-query tile, 64-key block) pairs.
+# ---------------------------------------------------------------------------
+
+def _sparse_inputs(seed, N=300, d=4):
+    rng = _rng(seed)
+    return tuple(rng.standard_normal((1, 2, N, d)) for _ in range(3)) + (0.5 * rng.standard_normal((1, 2, N, d)),)
+
+
+def _mask(N, active):
+    nt, nkb = (N + 127) // 128, (N + 63) // 64
+    m = np.zeros((nt, nkb), dtype=bool)
+    for t in range(nt):
+        for kb in range(nkb):
+            m[t, kb] = active(t, kb)
+    return m
+
+
+def test_block_sparse_all_active_is_causal():
+    Q, K, V, R = _sparse_inputs(20)
+    m = _mask(300, lambda t, kb: True)
+    np.testing.assert_allclose(oracle.prefill_block_sparse_ref(Q, K, V, R, m),
+                               oracle.prefill_ref(Q, K, V, R, causal=True), rtol=0, atol=1e-13)
+
+
+def test_block_sparse_diagonal_blocks_only_is_a_per_tile_prefill():
+    """Only each tile's own two key blocks: every tile is an independent causal
+    prefill of its 128 positions."""
+    Q, K, V, R = _sparse_inputs(21)
+    N = 300
+    m = _mask(N, lambda t, kb: kb // 2 == t)
+    got = oracle.prefill_block_sparse_ref(Q, K, V, R, m)
+    for t in range(3):
+        lo, hi = 128 * t, min(N, 128 * t + 128)
+        sub = [x[:, :, lo:hi] for x in (Q, K, V, R)]
+        np.testing.assert_allclose(got[:, :, lo:hi], oracle.prefill_ref(*sub, causal=True), rtol=0, atol=1e-13)
+
+
+def test_block_sparse_rows_see_exactly_their_blocks():
+    """A strided pattern: each visible-key set is the causal keys of the active blocks."""
+    Q, K, V, R = _sparse_inputs(22)
+    m = _mask(300, lambda t, kb: kb // 2 == t or kb % 3 == 0)
+    got = oracle.prefill_block_sparse_ref(Q, K, V, R, m, rows=[(0, 1, 200), (0, 0, 299)])
+    for row, (b, h, i) in zip(got, [(0, 1, 200), (0, 0, 299)]):
+        ks = [j for j in range(i + 1) if (j // 64) // 2 == i // 128 or (j // 64) % 3 == 0]
+        np.testing.assert_allclose(row, oracle.parallax_row(Q[b, h, i], R[b, h, i], K[b, h, ks], V[b, h, ks]),
+                                   rtol=0, atol=1e-13)
