@@ -453,6 +453,29 @@ def run_gpu(args, rank, world, dist):
         def wdec():
             plx.decode_window(dt_["q"], dt_["r"], dt_["K"], dt_["V"], dsl, W, out=dout, workspace=dws)
 
+        # Block-sparse prefill on the same inputs shape: every 128-query tile sees
+        # its diagonal blocks, the 16 key blocks (1024 keys) before them and the
+        # first 2 blocks.
+        nt, nkb = (wN + 127) // 128, (wN + 63) // 64
+        bmask = np.array([[kb < 2 or 2 * t - 16 <= kb or kb // 2 == t for kb in range(nkb)] for t in range(nt)])
+        wt2 = {}
+        for name, spec in wspecs.items():
+            wt2[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(wt2[name].data_ptr(), synth.BF16, seed + 10, spec)
+        sout = torch.empty_like(wt2["Q"])
+
+        def spre():
+            plx.prefill_block_sparse(wt2["Q"], wt2["K"], wt2["V"], wt2["R"], bmask, out=sout)
+
+        s_total, s_per = timed(spre, wsteps, max(3, args.warmup // 2), stream, dist)
+        spairs = 0
+        for i in range(wN):
+            t = i // 128
+            full = i // 64  # blocks strictly before key block of i are whole; i's own block is partial
+            spairs += int(np.sum(bmask[t, :full])) * 64 + (i % 64 + 1)
+        sflops = 8.0 * wd * spairs * wB * wH
+        s_ach = sflops / (float(np.mean(s_per)) * 1e-3) / 1e12
+        del wt2, sout
         d_total, d_per = timed(wdec, args.steps, args.warmup, stream, dist)
         dbytes = dB * dH * min(W, dL) * dd * 2 * 2 + 3 * dB * dH * dd * 2
         if plx.get_device_status() != 0:
@@ -467,6 +490,13 @@ def run_gpu(args, rank, world, dist):
                 "traffic": (traffic_from_profile("prefill_window_B8_H16_N4096_W1024.json",
                                                  kernel_hash("prefill_tc.cu", "sm100.cuh"))
                             if wB == PREFILL["B"] else None),
+            },
+            "block_sparse_prefill": {
+                "workload": f"block-sparse prefill B={wB} H={wH} N={wN} d={wd} bf16: per 128-query tile its "
+                            "diagonal blocks, the 16 64-key blocks before them and the first 2 blocks",
+                "value": round(sum_over_ranks(sflops * wsteps, dist) / (max_over_ranks(s_total, dist) * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "kernel_tflops": round(s_ach, 1), "frac": round(s_ach / peaks["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": sflops,
             },
             "decode": {
                 "workload": f"sliding-window decode W={W} B={dB} H={dH} L={dL} d={dd} bf16 (all lengths {dL})",

@@ -94,6 +94,20 @@ int plx_prefill_window(const void* Q, const void* K, const void* V, const void* 
                        int B, int H, int N, int d, int window, int dtype, void* stream);
 
 /*
+ * Block-sparse causal prefill, bf16, d in {64, 128}: query i sees key j when
+ * j <= i and block_mask[i / 128][j / 64] is non-zero (the pages list
+ * block-sparse kernels as future work: rainbus.top "未来方向"; the rule is
+ * this build's reading).  block_mask: HOST array of ceil(N/128) x ceil(N/64)
+ * bytes, row-major, shared by all heads; copied during the call.  Each tile's
+ * own diagonal blocks (2m and 2m+1 where they exist) must be active, else
+ * PLX_ERR_INVALID_ARG; blocks above the diagonal are ignored.  The block lists
+ * live in a library-owned device buffer: calls on one device must be ordered.
+ * Other arguments and errors as plx_prefill_ex.
+ */
+int plx_prefill_block_sparse(const void* Q, const void* K, const void* V, const void* R, void* out,
+                             int B, int H, int N, int d, const uint8_t* block_mask, void* stream);
+
+/*
  * Sliding-window decode step: the query of sequence b sees its last `window`
  * keys, max(0, seqlens[b] - window)..seqlens[b]-1.  Hkv == H is the decode of
  * plx_decode_ex (bf16 or fp32); Hkv < H is the grouped-KV decode of

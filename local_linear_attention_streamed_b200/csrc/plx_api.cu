@@ -5,8 +5,10 @@
 #include <cublasLt.h>
 #include <cublas_v2.h>
 
+#include <algorithm>
 #include <cstdio>
 #include <mutex>
+#include <vector>
 
 #include "../../include/plx.h"
 
@@ -30,6 +32,8 @@ struct DeviceCache {
   size_t layer_ws_bytes = 0;
   void* bwd_ws = nullptr;  // per-row statistics of the prefill backward pass
   size_t bwd_ws_bytes = 0;
+  void* sparse_ws = nullptr;  // block lists of the block-sparse prefill
+  size_t sparse_ws_bytes = 0;
   cublasHandle_t cublas = nullptr;
   cublasLtHandle_t cublas_lt = nullptr;  // fp8 GEMMs of the fp8 layer
 };
@@ -185,6 +189,46 @@ int plx_prefill_window(const void* Q, const void* K, const void* V, const void* 
                        int H, int N, int d, int window, int dtype, void* stream) {
   if (window < 1) return PLX_ERR_INVALID_ARG;
   return prefill_impl(Q, K, V, R, out, B, H, N, d, 1, window, dtype, stream);
+}
+
+int plx_prefill_block_sparse(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
+                             int H, int N, int d, const uint8_t* block_mask, void* stream) {
+  if (!Q || !K || !V || !R || !out || !block_mask) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(R) || !aligned16(out))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  // The mask as lists of active key blocks per tile (blocks above a tile's
+  // diagonal hold no visible key and are dropped); every row must see its
+  // own key, so each tile's diagonal blocks must be active.
+  const int ntile = (N + 127) / 128, nkb = (N + 63) / 64;
+  std::vector<int> list;
+  list.reserve((size_t)ntile + 1 + (size_t)ntile * 2);
+  list.resize((size_t)ntile + 1);
+  for (int m = 0; m < ntile; ++m) {
+    list[m] = (int)(list.size() - (ntile + 1));
+    const int last = std::min(nkb - 1, 2 * m + 1);
+    for (int kb = 0; kb <= last; ++kb) {
+      const bool on = block_mask[(size_t)m * nkb + kb] != 0;
+      if (kb >= 2 * m && !on) return PLX_ERR_INVALID_ARG;  // a diagonal block is off
+      if (on) list.push_back(kb);
+    }
+  }
+  list[ntile] = (int)(list.size() - (ntile + 1));
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = list.size() * sizeof(int);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if ((rc = grow(&dc->sparse_ws, &dc->sparse_ws_bytes, bytes, st)) != PLX_OK) return rc;
+  if (cudaMemcpyAsync(dc->sparse_ws, list.data(), bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  PrefillArgs a{Q, K, V, R, out, B, H, N, d, 1, dc->status};
+  a.blk_ptr = static_cast<const int*>(dc->sparse_ws);
+  a.blk_idx = a.blk_ptr + ntile + 1;
+  return cuda_rc(launch_prefill_tc(a, st, dc->num_sms));
 }
 
 int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void* out, int B,

@@ -34,6 +34,10 @@ struct PrefillArgs {
   float* lse = nullptr;
   float* tbar = nullptr;
   int window = 0;  // sliding window: query i sees keys i - window + 1 .. i (0: none; implies causal)
+  // Block-sparse causal prefill (tensor-core path; device CSR over 128-query
+  // tiles of ascending 64-key block indices), or null.
+  const int* blk_ptr = nullptr;
+  const int* blk_idx = nullptr;
 };
 
 struct DecodeArgs {

@@ -127,14 +127,15 @@ struct Smem {
 using namespace sm100;
 
 struct TileInfo {
-  int bh, m, j0, nblk;  // key blocks j0 .. j0 + nblk - 1
+  int bh, m, j0, nblk;  // key blocks j0 .. j0 + nblk - 1 (block-sparse: list entries j0 .. j0 + nblk - 1)
 };
 
 // Tile t of the schedule: heads are taken in chunks of `ch`; within a chunk
 // the tiles go longest causal rows first across the chunk's heads.  CTAs take
 // tiles in this order from a global counter, so the K/V of a few heads stay in
 // L2 while every tile that reads them runs, and the causal work balances.
-__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, int ch, int window) {
+__device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, int ch, int window,
+                                              const int* blk_ptr) {
   const int ntile = (N + kBM - 1) / kBM;
   const int per_chunk = ch * ntile;
   const int chunk = t / per_chunk;
@@ -144,6 +145,12 @@ __device__ __forceinline__ TileInfo tile_info(int t, int BH, int N, int causal, 
   ti.m = ntile - 1 - pos / nh;
   ti.bh = chunk * ch + pos % nh;
   const int kmax = causal ? min(N, (ti.m + 1) * kBM) : N;
+  if (blk_ptr != nullptr) {
+    // Block-sparse: the tile's active key blocks are a list (CSR row m).
+    ti.j0 = blk_ptr[ti.m];
+    ti.nblk = blk_ptr[ti.m + 1] - ti.j0;
+    return ti;
+  }
   // A sliding window of W keys: the tile's first query sees keys from m kBM - W + 1.
   ti.j0 = window > 0 ? max(0, ti.m * kBM - window + 1) / kBN : 0;
   ti.nblk = (kmax + kBN - 1) / kBN - ti.j0;
@@ -158,6 +165,10 @@ __device__ unsigned int g_cta_done;
 struct Params {
   int B, H, N, causal;
   int window;  // sliding window of keys per query (0: none)
+  // Block-sparse (else null): per 128-query tile m, the active 64-key blocks
+  // blk_idx[blk_ptr[m] .. blk_ptr[m + 1]), ascending, on or below the diagonal.
+  const int* blk_ptr;
+  const int* blk_idx;
   int chunk_heads;
   int inject_stall;  // failure-detection test: withhold the first Q/R tile
   __nv_bfloat16* out;
@@ -170,15 +181,22 @@ struct Params {
   float* tbar;
 };
 
-// kWin: the sliding-window variant (the causal and full prefills compile
-// without any of its per-row logic).
-template <int D, bool kWin>
+// kMode: 0 causal or full, 1 sliding window, 2 block-sparse.  The causal and
+// full prefills compile without any of the other variants' per-row logic.
+template <int D, int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  constexpr bool kWin = kMode == 1, kSparse = kMode == 2;
+  // Rows that may see no key in a block (window or block sparsity) need the
+  // guards for an empty running max.
+  constexpr bool kRobust = kMode != 0;
   const int window = kWin ? p.window : 0;
+  const int* blk_ptr = kSparse ? p.blk_ptr : nullptr;
+  // The key block of the tile's j-th iteration.
+  auto kblock = [&](const TileInfo& ti, int j) { return kSparse ? p.blk_idx[ti.j0 + j] : ti.j0 + j; };
   constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
   constexpr uint32_t kColO2 = Dims<D>::kColO2, kIdescPV = Dims<D>::kIdescPV;
   constexpr int kHalves = Dims<D>::kHalves;
@@ -243,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.tile_ring[slot] = t;
         mbar_arrive(&sm.tile_full[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         const int row0 = ti.bh * p.N;
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
@@ -264,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
           kv_issued[st] = kv / kStages;
           for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + (ti.j0 + j) * kBN);
-            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + (ti.j0 + j) * kBN);
+            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + kblock(ti, j) * kBN);
+            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + kblock(ti, j) * kBN);
           }
         }
       }
@@ -292,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
         mbar_arrive(&sm.tile_empty[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
           // K of this block (long resident: checked first), then the S stage,
@@ -344,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = *reinterpret_cast<volatile int*>(&sm.tile_ring[slot]);
         mbar_arrive(&sm.tile_empty[slot]);
         if (t < 0) break;
-        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
+        const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         // The epilogue of the previous tile must have read O before it is overwritten.
         if (tc > 0 && !(ok = mbar_wait(&sm.o_empty, (tc - 1) & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
@@ -462,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (epi_pending) ok = epilogue(epi_tc, epi_row, epi_vrow, epi_inv, epi_c1);
         break;
       }
-      const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window);
+      const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
       const int i = ti.m * kBM + row;                      // query position
       const int kend = p.causal ? min(i + 1, p.N) : p.N;  // keys < kend are visible
       const int kbeg = i - window + 1;                    // and, with a window, keys >= kbeg
@@ -486,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t g = gb + j;
         if (!(ok = mbar_wait(&sm.s_full[wg], (g >> 1) & 1, abort, p.status))) break;
         tc_fence_after();
-        const int kb = (ti.j0 + j) * kBN;
+        const int kb = kblock(ti, j) * kBN;
         uint32_t x[64], y[64];
         tmem_ld32(sb + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(sb + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
@@ -546,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           // A row that has seen no key yet (only with a window) keeps m_run =
           // -inf and gets w = 2^(-inf) = 0 from the reference 0.
-          const float mref = (kWin && m_run == -CUDART_INF_F) ? 0.f : m_run;
+          const float mref = (kRobust && m_run == -CUDART_INF_F) ? 0.f : m_run;
           const uint64_t sc2 = f2(scale, scale), nm2 = f2(-mref, -mref), nc2 = f2(-cen, -cen);
           uint64_t ws2a = f2(0.f, 0.f), ts2a = f2(0.f, 0.f), ws2b = ws2a, ts2b = ts2a;
 #pragma unroll
@@ -596,6 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool second = kbeg > kb - kBN && kbeg < kb;
             const float theta = window >= 256 ? Dims<D>::kTheta : 0.5f;
             recentre = Wn > 0.f && (Wp == 0.f || second || fabsf(Tn) > theta * Wn);
+          } else if constexpr (kSparse) {
+            // Rows of a sparse tile may start from a partial (diagonal) block.
+            recentre = Wn > 0.f && (Wp == 0.f || fabsf(Tn) > 0.5f * Wn);
           } else {
             recentre = j == 0 || fabsf(Tn) > Dims<D>::kTheta * Wn;  // key 0 is visible: Wn > 0
           }
@@ -754,10 +775,12 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   // (tests of the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
-  Params p{a.B,      a.H,    a.N, a.causal, a.window, ch, inject, reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
+  Params p{a.B,      a.H,    a.N, a.causal, a.window, a.blk_ptr, a.blk_idx, ch, inject,
+           reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
            reinterpret_cast<float*>(a.vbar), a.lse, a.tbar};
   const size_t smem = sizeof(Smem<D>) + 1024;
-  auto kernel = a.window > 0 ? prefill_tc_kernel<D, true> : prefill_tc_kernel<D, false>;
+  auto kernel = a.blk_ptr != nullptr ? prefill_tc_kernel<D, 2>
+                : (a.window > 0 ? prefill_tc_kernel<D, 1> : prefill_tc_kernel<D, 0>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)((a.N + kBM - 1) / kBM) * a.B * a.H;

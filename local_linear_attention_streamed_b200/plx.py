@@ -37,6 +37,7 @@ SIGNATURES = {
     "plx_layer_fp8_workspace_bytes": (_sz, [_i] * 4),
     "plx_layer_forward_fp8": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
     "plx_prefill_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
+    "plx_prefill_block_sparse": (_i, [_vp] * 5 + [_i] * 4 + [_vp, _vp]),
     "plx_decode_window": (_i, [_vp] * 6 + [_i] * 7 + [_vp, _sz, _vp]),
     "plx_decode_window_workspace_bytes": (_sz, [_i] * 6),
     "plx_prefill_train": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
@@ -131,6 +132,25 @@ def prefill_window(Q, K, V, R, window: int, out=None, stream=None):
     rc = lib.plx_prefill_window(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
                                 B, H, N, d, int(window), _dtype_code(Q), _stream_ptr(stream))
     _check(rc, "plx_prefill_window")
+    return out
+
+
+def prefill_block_sparse(Q, K, V, R, block_mask, out=None, stream=None):
+    """Block-sparse causal prefill: ``block_mask`` is a host array [ceil(N/128), ceil(N/64)]
+    (truthy = the 64-key block is visible to the 128-query tile); returns out."""
+    import numpy as np
+    B, H, N, d = Q.shape
+    for n, t in (("K", K), ("V", V), ("R", R)):
+        if t.shape != Q.shape or t.dtype != Q.dtype:
+            raise ValueError(f"{n} must match Q in shape and dtype")
+    m = np.ascontiguousarray(np.asarray(block_mask).astype(np.uint8))
+    if m.shape != ((N + 127) // 128, (N + 63) // 64):
+        raise ValueError("block_mask must be [ceil(N/128), ceil(N/64)]")
+    if out is None:
+        out = torch.empty_like(Q)
+    rc = lib.plx_prefill_block_sparse(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                      B, H, N, d, m.ctypes.data, _stream_ptr(stream))
+    _check(rc, "plx_prefill_block_sparse")
     return out
 
 

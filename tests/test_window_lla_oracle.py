@@ -16,6 +16,10 @@ parameterises; gist.science, "Mecanismo central"):
     function of the keys are reproduced exactly at the query (the defining
     property of a local-linear fit), which softmax attention does not do;
   * lambda -> infinity gives softmax attention (rho* -> 0).
+
+Block sparsity (a mask over 128-query tiles and 64-key blocks): all blocks
+active is causal, diagonal blocks only is a per-tile causal prefill, and rows
+of a strided pattern see exactly the causal keys of their active blocks.
 """
 import math
 
