@@ -130,6 +130,21 @@ def prefill_ref(Q, K, V, R, causal: bool = True, rows=None, window=None) -> np.n
     return np.stack(res) if res else np.zeros((0, d))
 
 
+def prefill_gqa_ref(Q, K, V, R, causal: bool = True) -> np.ndarray:
+    """Oracle for a prefill with grouped KV heads: Q, R [B, H, N, d]; K, V
+    [B, Hkv, N, d]; query head h reads KV head h // (H // Hkv)."""
+    B, H, N, d = Q.shape
+    G = H // K.shape[1]
+    out = np.empty((B, H, N, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            kv = h // G
+            for i in range(N):
+                lo, hi = visible_keys(i, N, causal)
+                out[b, h, i] = parallax_row(Q[b, h, i], R[b, h, i], K[b, kv, lo:hi], V[b, kv, lo:hi])
+    return out
+
+
 def decode_ref(q, r, Kc, Vc, seqlens, units=None, window=None) -> np.ndarray:
     """Oracle for one decode step.
 

@@ -452,3 +452,25 @@ def test_layer_row_matches_head_oracle():
     o = prefill_ref(q, k, v, r, causal=True)
     y = o.transpose(0, 2, 1, 3).reshape(B, N, D) @ W[4]
     np.testing.assert_allclose(got[0], y[0, 9], rtol=0, atol=1e-12)
+
+
+def test_prefill_gqa_pins():
+    """Grouped KV heads in the prefill: equal to the ungrouped oracle with each
+    KV head repeated for its query heads (np.repeat, not the oracle's index
+    map), G = 1 is the ungrouped prefill, and swapping two KV heads permutes
+    the output groups."""
+    from oracle import prefill_gqa_ref
+    rng = _rng(30)
+    B, H, Hkv, N, d = 2, 6, 2, 9, 4
+    Q, R = rng.standard_normal((B, H, N, d)), rng.standard_normal((B, H, N, d))
+    K, V = rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hkv, N, d))
+    G = H // Hkv
+    for causal in (True, False):
+        want = prefill_ref(Q, np.repeat(K, G, axis=1), np.repeat(V, G, axis=1), R, causal=causal)
+        np.testing.assert_allclose(prefill_gqa_ref(Q, K, V, R, causal), want, rtol=0, atol=1e-13)
+    K1, V1 = rng.standard_normal((B, H, N, d)), rng.standard_normal((B, H, N, d))
+    np.testing.assert_allclose(prefill_gqa_ref(Q, K1, V1, R), prefill_ref(Q, K1, V1, R), rtol=0, atol=0)
+    # Reversing the KV heads hands the first group of query heads the last KV head.
+    sw = prefill_gqa_ref(Q, K[:, ::-1].copy(), V[:, ::-1].copy(), R)
+    np.testing.assert_allclose(sw[:, :G], prefill_gqa_ref(Q[:, :G], K[:, -1:], V[:, -1:], R[:, :G]),
+                               rtol=0, atol=1e-13)
