@@ -94,6 +94,17 @@ int plx_prefill_window(const void* Q, const void* K, const void* V, const void* 
                        int B, int H, int N, int d, int window, int dtype, void* stream);
 
 /*
+ * Causal (or full) bf16 prefill with grouped KV heads: Q, R, out [B, H, N, d];
+ * K, V [B, Hkv, N, d] with H a multiple of Hkv; query head h reads KV head
+ * h / (H / Hkv) (consecutive query heads share one).  The pages place Parallax
+ * in a Qwen-3 architecture (rainbus.top reproduction notes), whose attention
+ * groups KV heads.  d in {64, 128}, else PLX_ERR_UNSUPPORTED; H not a multiple
+ * of Hkv gives PLX_ERR_INVALID_ARG.  Other arguments as plx_prefill_ex.
+ */
+int plx_prefill_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                    int Hkv, int N, int d, int causal, void* stream);
+
+/*
  * Block-sparse causal prefill, bf16, d in {64, 128}: query i sees key j when
  * j <= i and block_mask[i / 128][j / 64] is non-zero (the pages list
  * block-sparse kernels as future work: rainbus.top "未来方向"; the rule is

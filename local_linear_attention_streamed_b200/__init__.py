@@ -10,7 +10,7 @@ _BINDING_NAMES = {
     "prefill", "decode", "decode_gqa", "decode_noalloc", "decode_workspace_bytes", "layer_forward", "qkr_norm_rope",
     "get_device_status", "status_string", "PlxError", "lib", "PLX_F32", "PLX_BF16",
     "prefill_train", "prefill_backward", "prefill_bwd_workspace_bytes", "parallax_attention",
-    "ParallaxAttention", "prefill_window", "decode_window", "layer_forward_fp8", "prefill_block_sparse",
+    "ParallaxAttention", "prefill_window", "decode_window", "layer_forward_fp8", "prefill_block_sparse", "prefill_gqa",
 }
 
 

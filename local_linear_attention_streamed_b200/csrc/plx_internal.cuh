@@ -38,6 +38,9 @@ struct PrefillArgs {
   // tiles of ascending 64-key block indices), or null.
   const int* blk_ptr = nullptr;
   const int* blk_idx = nullptr;
+  // Grouped KV heads (tensor-core path): K and V are [B, Hkv, N, d] and query
+  // head h reads KV head h / (H / Hkv); 0 means Hkv = H.
+  int Hkv = 0;
 };
 
 struct DecodeArgs {

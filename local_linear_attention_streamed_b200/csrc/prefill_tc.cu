@@ -164,6 +164,7 @@ __device__ unsigned int g_cta_done;
 
 struct Params {
   int B, H, N, causal;
+  int Hkv;     // KV heads (H: one per head); query head h reads KV head h / (H / Hkv)
   int window;  // sliding window of keys per query (0: none)
   // Block-sparse (else null): per 128-query tile m, the active 64-key blocks
   // blk_idx[blk_ptr[m] .. blk_ptr[m + 1]), ascending, on or below the diagonal.
@@ -263,6 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t < 0) break;
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         const int row0 = ti.bh * p.N;
+        // Grouped KV heads: consecutive query heads share one K/V head.
+        const int kvrow0 = ((ti.bh / p.H) * p.Hkv + (ti.bh % p.H) / (p.H / p.Hkv)) * p.N;
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
         q_issued = tc;
@@ -282,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
           kv_issued[st] = kv / kStages;
           for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, row0 + kblock(ti, j) * kBN);
-            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, row0 + kblock(ti, j) * kBN);
+            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
+            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
           }
         }
       }
@@ -763,10 +766,11 @@ namespace {
 template <int D>
 cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   const long long rows = (long long)a.B * a.H * a.N;
+  const long long kv_rows = (long long)a.B * (a.Hkv > 0 ? a.Hkv : a.H) * a.N;
   if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
   CUtensorMap mQ, mR, mK, mV;
-  if (!make_map(&mQ, a.Q, rows, kBM, D) || !make_map(&mR, a.R, rows, kBM, D) || !make_map(&mK, a.K, rows, kBN, D) ||
-      !make_map(&mV, a.V, rows, kBN, D))
+  if (!make_map(&mQ, a.Q, rows, kBM, D) || !make_map(&mR, a.R, rows, kBM, D) ||
+      !make_map(&mK, a.K, kv_rows, kBN, D) || !make_map(&mV, a.V, kv_rows, kBN, D))
     return cudaErrorInvalidValue;
   const int ntile = (a.N + kBM - 1) / kBM;
   int ch = (2 * num_sms + ntile - 1) / ntile;  // about two waves of tiles per chunk
@@ -775,7 +779,7 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   // (tests of the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
-  Params p{a.B,      a.H,    a.N, a.causal, a.window, a.blk_ptr, a.blk_idx, ch, inject,
+  Params p{a.B,      a.H,    a.N, a.causal, a.Hkv > 0 ? a.Hkv : a.H, a.window, a.blk_ptr, a.blk_idx, ch, inject,
            reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
            reinterpret_cast<float*>(a.vbar), a.lse, a.tbar};
   const size_t smem = sizeof(Smem<D>) + 1024;

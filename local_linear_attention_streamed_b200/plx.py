@@ -38,6 +38,7 @@ SIGNATURES = {
     "plx_layer_forward_fp8": (_i, [_vp] * 7 + [_i] * 4 + [_vp, _sz, _vp]),
     "plx_prefill_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_prefill_block_sparse": (_i, [_vp] * 5 + [_i] * 4 + [_vp, _vp]),
+    "plx_prefill_gqa": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_decode_window": (_i, [_vp] * 6 + [_i] * 7 + [_vp, _sz, _vp]),
     "plx_decode_window_workspace_bytes": (_sz, [_i] * 6),
     "plx_prefill_train": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
@@ -132,6 +133,20 @@ def prefill_window(Q, K, V, R, window: int, out=None, stream=None):
     rc = lib.plx_prefill_window(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
                                 B, H, N, d, int(window), _dtype_code(Q), _stream_ptr(stream))
     _check(rc, "plx_prefill_window")
+    return out
+
+
+def prefill_gqa(Q, K, V, R, causal: bool = True, out=None, stream=None):
+    """bf16 prefill with grouped KV heads: Q, R [B, H, N, d]; K, V [B, Hkv, N, d]."""
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    if K.shape != (B, Hkv, N, d) or V.shape != K.shape or R.shape != Q.shape:
+        raise ValueError("K, V must be [B, Hkv, N, d] and R like Q")
+    if out is None:
+        out = torch.empty_like(Q)
+    rc = lib.plx_prefill_gqa(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                             B, H, Hkv, N, d, int(bool(causal)), _stream_ptr(stream))
+    _check(rc, "plx_prefill_gqa")
     return out
 
 

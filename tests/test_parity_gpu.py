@@ -340,3 +340,30 @@ def test_config_layer_full_size_sampled(plx):
         got.append(np.stack([y[b, t].double().cpu().numpy() for (_, t) in rb]))
     assert rel_err_rms(np.concatenate(got), np.concatenate(want)) <= LAYER_TOL
     assert torch.isfinite(y).all()
+
+
+# ---------------------------------------------------------------------------
+# Prefill with grouped KV heads.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+@pytest.mark.parametrize("N,d,causal", [(300, 128, True), (200, 64, True), (130, 128, False)])
+def test_prefill_gqa(plx, G, N, d, causal):
+    B, Hkv = 2, 2
+    H = G * Hkv
+    specs = synth.prefill_specs(B, H, N, d)
+    specs["K"] = synth.TensorSpec(synth.TID_K, (B, Hkv, N, d), specs["K"].dist, specs["K"].sigma)
+    specs["V"] = synth.TensorSpec(synth.TID_V, (B, Hkv, N, d), specs["V"].dist, specs["V"].sigma)
+    dev, ref = small_inputs(1200 + G + N, specs, synth.BF16)
+    out = plx.prefill_gqa(dev["Q"], dev["K"], dev["V"], dev["R"], causal=causal)
+    assert plx.get_device_status() == 0
+    want = oracle.prefill_gqa_ref(ref["Q"], ref["K"], ref["V"], ref["R"], causal)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
+def test_prefill_gqa_ungrouped_is_prefill(plx):
+    B, H, N, d = 1, 4, 256, 128
+    dev, _ = small_inputs(1210, synth.prefill_specs(B, H, N, d), synth.BF16)
+    a = plx.prefill_gqa(dev["Q"], dev["K"], dev["V"], dev["R"], causal=True)
+    b = plx.prefill(dev["Q"], dev["K"], dev["V"], dev["R"], causal=True)
+    assert torch.equal(a, b)
