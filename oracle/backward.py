@@ -35,7 +35,15 @@ def _hidden_keys(N: int, causal: bool, window=None) -> np.ndarray:
 
 
 def _forward_torch(Q, K, V, R, causal: bool, window=None):
-    """Plain float64 forward over [..., N, d] tensors (all rows at once)."""
+    """Plain float64 forward over [..., N, d] tensors (all rows at once).
+
+    K and V may have fewer heads than Q (grouped KV heads: query head h reads
+    KV head h // (H // Hkv)); they are repeated across each group, so the
+    gradients of K and V sum over the group's query heads."""
+    if K.dim() == 4 and K.shape[1] != Q.shape[1]:
+        G = Q.shape[1] // K.shape[1]
+        K = torch.repeat_interleave(K, G, dim=1)
+        V = torch.repeat_interleave(V, G, dim=1)
     d = Q.shape[-1]
     N = Q.shape[-2]
     S = Q @ K.transpose(-1, -2) / np.sqrt(d)

@@ -214,3 +214,28 @@ def test_window_statement_and_gradients(W):
     vb, lse, tb = oracle.prefill_stats_ref(Q, K, V, R, True, window=W)
     if W == 1:
         np.testing.assert_allclose(vb, V, rtol=0, atol=1e-14)
+
+
+def test_grouped_kv_gradients_match_finite_differences():
+    """Grouped KV heads (two query heads per KV head): the gradients of K and V
+    sum over the group; checked against central differences of the grouped
+    row oracle."""
+    rng = np.random.default_rng(101)
+    B, H, Hkv, N, d = 1, 4, 2, 5, 3
+    Q, R, dO = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    K, V = rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hkv, N, d))
+    got = oracle.parallax_backward_ref(Q, K, V, R, dO, True)
+    assert got[1].shape == K.shape and got[2].shape == V.shape
+    xs = [Q.copy(), K.copy(), V.copy(), R.copy()]
+    h = 1e-6
+    for a in range(4):
+        g = np.zeros_like(xs[a])
+        for idx in np.ndindex(xs[a].shape):
+            old = xs[a][idx]
+            xs[a][idx] = old + h
+            fp = np.sum(oracle.prefill_gqa_ref(*xs, True) * dO)
+            xs[a][idx] = old - h
+            fm = np.sum(oracle.prefill_gqa_ref(*xs, True) * dO)
+            xs[a][idx] = old
+            g[idx] = (fp - fm) / (2 * h)
+        assert np.max(np.abs(got[a] - g)) < 1e-7 * max(1.0, np.max(np.abs(g)))
