@@ -159,6 +159,14 @@ int plx_prefill_train_window(const void* Q, const void* K, const void* V, const 
                              void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int window,
                              void* stream);
 
+/* plx_prefill_train with grouped KV heads, as plx_prefill_gqa: K and V are
+ * [B, Hkv, N, d] and query head h reads KV head h / (H / Hkv); Q, R, out, vbar,
+ * lse and tbar keep H heads.  Hkv >= 1 dividing H, else PLX_ERR_INVALID_ARG;
+ * Hkv = H is plx_prefill_train.  Causal or full. */
+int plx_prefill_train_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, void* vbar,
+                          float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal,
+                          void* stream);
+
 /* Bytes of the statistics workspace plx_prefill_bwd needs:
  * 16 * B * H * (N rounded up to a multiple of 128); 0 for invalid sizes. */
 size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d);
@@ -191,6 +199,18 @@ int plx_prefill_bwd_window(const void* Q, const void* K, const void* V, const vo
                            const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
                            void* dK, void* dV, void* dR, int B, int H, int N, int d, int window,
                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* plx_prefill_bwd for the grouped-KV prefill of plx_prefill_train_gqa: K, V,
+ * dK and dV are [B, Hkv, N, d]; Q, R, dQ, dR, out, vbar, dO, lse and tbar have
+ * H heads.  KV head g is shared by query heads g G .. g G + G - 1 of its batch
+ * (G = H / Hkv), so dK and dV of a KV head sum the contributions of those G
+ * query heads (one CTA per 128-key block of a KV head accumulates all of them
+ * in TMEM; no atomics, no second pass).  Hkv >= 1 dividing H, else
+ * PLX_ERR_INVALID_ARG; workspace as plx_prefill_bwd (sized by H). */
+int plx_prefill_bwd_gqa(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                        const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ, void* dK,
+                        void* dV, void* dR, int B, int H, int Hkv, int N, int d, int causal, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /*
  * One decode step with split-KV: every (b, h) streams its cache rows

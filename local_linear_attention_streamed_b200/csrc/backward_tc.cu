@@ -131,6 +131,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 
 struct BwdParams {
   int B, H, N, Npad, causal;
+  int Hkv;           // KV heads (H a multiple of it): query head h read KV head h / (H / Hkv)
   int window;        // sliding window (0: none): query i saw keys i - window + 1 .. i
   int inject_stall;  // failure-detection test: CTA 0 of the dK/dV kernel never loads its K/V
   int chunk_heads;  // heads whose blocks are launched together (L2 reuse of their tiles)
@@ -269,15 +270,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                      kColG = 2 * D + 192;
   Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.B * p.H;
-  // Key block 0 sees every query (causal): rank r is key block r.
-  const BlockOrder bo = block_order(blockIdx.x, BH, (p.N + kKB - 1) / kKB, p.chunk_heads);
+  // One CTA per key block of a KV head (bh indexes KV heads); its gradients
+  // sum over the query blocks of every query head of the head's group, taken
+  // head by head: step i is query block q0 + i % nq1 of group member i / nq1.
+  const int G = p.H / p.Hkv;
+  const BlockOrder bo = block_order(blockIdx.x, p.B * p.Hkv, (p.N + kKB - 1) / kKB, p.chunk_heads);
   const int kb = bo.rank, bh = bo.bh;
+  const int qbh0 = (bh / p.Hkv) * p.H + (bh % p.Hkv) * G;  // first query head of the group
   const int nqb = (p.N + kQB - 1) / kQB;
   const int q0 = p.causal ? (kb * kKB) / kQB : 0;
   // With a window, the block's last key is seen by queries up to kb kKB + kKB - 1 + window - 1.
   const int qend = p.window > 0 ? min(nqb, (kb * kKB + kKB + p.window - 2) / kQB + 1) : nqb;
-  const int nq = qend - q0;  // >= 1: key block kb starts below N
+  const int nq1 = qend - q0;  // >= 1: key block kb starts below N
+  const int nq = G * nq1;
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
@@ -321,12 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       int last_use[kQStages] = {-1, -1, -1};
-      for (int i = 0; i < nq && !*abort; ++i) {
+      int qh = qbh0, qb = q0;  // query head and block of step i
+      for (int i = 0; i < nq && !*abort; ++i, qb = qb + 1 < qend ? qb + 1 : (++qh, q0)) {
         const int st = i % kQStages, u = i / kQStages;
         if (u > 0 && !mbar_wait(&sm.q_empty[st], (u - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full[st], 3 * kQB * D * 2);
         last_use[st] = u;
-        const int qrow = bh * p.N + (q0 + i) * kQB;
+        const int qrow = qh * p.N + qb * kQB;
         for (int h = 0; h < kHalves; ++h) {
           tma_load_2d(sm.qr[st][h], &tmQ, &sm.q_full[st], 64 * h, qrow);
           tma_load_2d(sm.qr[st][h] + kQB * 128, &tmR, &sm.q_full[st], 64 * h, qrow);
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // The block's statistics (1 KB, read by every elementwise thread)
         // into L1 ahead of use.
-        const float* stp = p.stats + stat_index(bh, p.Npad, (q0 + i) * kQB, 0);
+        const float* stp = p.stats + stat_index(qh, p.Npad, qb * kQB, 0);
 #pragma unroll
         for (int l = 0; l < 8; ++l) asm volatile("prefetch.global.L1 [%0];" ::"l"(stp + 32 * l));
       }
@@ -415,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kk = kb * kKB + row;  // key position
     const float isd = rsqrtf((float)D), scale2 = kLog2e * isd;
     bool ok = true;
-    for (int i = 0; i < nq; ++i) {
+    int qh = qbh0, qb = q0;  // query head and block of step i
+    for (int i = 0; i < nq; ++i, qb = qb + 1 < qend ? qb + 1 : (++qh, q0)) {
       if (!(ok = warp_wait(&sm.s_full, i & 1, abort, p.status))) break;
       tc_fence_after();
       uint32_t s[kEwCols], t[kEwCols], da[kEwCols];
@@ -426,13 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free);
-      const int i0 = (q0 + i) * kQB + kEwCols * wg;  // query of column 0
+      const int i0 = qb * kQB + kEwCols * wg;  // query of column 0
       // Masks only where some pair of the warp is masked: the causal diagonal
       // (query before key) and queries past N.
       const bool edge = __any_sync(0xffffffffu, (p.causal && i0 < kk) || i0 + kEwCols - 1 >= p.N ||
                                                     (p.window > 0 && i0 + kEwCols - 1 >= kk + p.window));
       // The statistics of this thread's 16 queries (read by every lane: cached).
-      const float* sts = p.stats + stat_index(bh, p.Npad, (q0 + i) * kQB, 0) + kEwCols * wg;
+      const float* sts = p.stats + stat_index(qh, p.Npad, qb * kQB, 0) + kEwCols * wg;
       const uint64_t sc2 = f2(scale2, scale2), nisd2 = f2(-isd, -isd);
       uint32_t pa[kEwCols / 2], pl[kEwCols / 2], pt[kEwCols / 2];
 #pragma unroll
@@ -527,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The last query block sees every key (causal): rank r is query block nmb - 1 - r.
   const BlockOrder bo = block_order(blockIdx.x, BH, nmb, p.chunk_heads);
   const int m = nmb - 1 - bo.rank, bh = bo.bh;
+  const int kvbh = (bh / p.H) * p.Hkv + (bh % p.H) / (p.H / p.Hkv);  // the KV head this query head reads
   // Key blocks j0 .. j0 + nk - 1 (a window hides the keys before m kQM - window + 1).
   const int j0 = p.window > 0 ? max(0, m * kQM - p.window + 1) / kKN : 0;
   const int nk = (p.causal ? (min(m * kQM + kQM - 1, p.N - 1) / kKN + 1) : (p.N + kKN - 1) / kKN) - j0;
@@ -575,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u > 0 && !mbar_wait(&sm.kv_empty[st], (u - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.kv_full[st], 2 * kKN * D * 2);
         last_use[st] = u;
-        const int krow = bh * p.N + (j0 + j) * kKN;
+        const int krow = kvbh * p.N + (j0 + j) * kKN;
         for (int h = 0; h < kHalves; ++h) {
           tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], 64 * h, krow);
           tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], 64 * h, krow);
@@ -722,13 +730,15 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   const long long rows = (long long)a.B * a.H * a.N;
   if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
   const int BH = a.B * a.H;
+  const int Hkv = a.Hkv > 0 ? a.Hkv : a.H;
+  const long long kv_rows = (long long)a.B * Hkv * a.N;
   const int Npad = (int)bwd_padded_rows(a.N);
   CUtensorMap mQ64, mR64, mO64, mK128, mV128, mQ128, mR128, mO128, mK64, mV64;
   if (!make_map(&mQ64, a.Q, rows, kQB, D) || !make_map(&mR64, a.R, rows, kQB, D) ||
-      !make_map(&mO64, a.dO, rows, kQB, D) || !make_map(&mK128, a.K, rows, kKB, D) ||
-      !make_map(&mV128, a.V, rows, kKB, D) || !make_map(&mQ128, a.Q, rows, kQM, D) ||
+      !make_map(&mO64, a.dO, rows, kQB, D) || !make_map(&mK128, a.K, kv_rows, kKB, D) ||
+      !make_map(&mV128, a.V, kv_rows, kKB, D) || !make_map(&mQ128, a.Q, rows, kQM, D) ||
       !make_map(&mR128, a.R, rows, kQM, D) || !make_map(&mO128, a.dO, rows, kQM, D) ||
-      !make_map(&mK64, a.K, rows, kKN, D) || !make_map(&mV64, a.V, rows, kKN, D))
+      !make_map(&mK64, a.K, kv_rows, kKN, D) || !make_map(&mV64, a.V, kv_rows, kKN, D))
     return fail_at("tensor map", cudaErrorInvalidValue);
   float* stats = reinterpret_cast<float*>(a.stats);
   const long long srows = (long long)BH * Npad;
@@ -741,19 +751,21 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   // About two waves of blocks per chunk of heads.
   int ch = (2 * num_sms + nblk - 1) / nblk;
   ch = ch < 1 ? 1 : (ch > BH ? BH : ch);
+  const int BHkv = a.B * Hkv;
+  const int chkv = ch > BHkv ? BHkv : ch;
   // PLX_FAULT_INJECT=bwd_stall makes one CTA's bounded waits run out (tests of
   // the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "bwd_stall") == 0) ? 1 : 0;
-  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, a.window, inject, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
+  BwdParams pk{a.B, a.H, a.N, Npad, a.causal, Hkv, a.window, inject, chkv, stats, reinterpret_cast<__nv_bfloat16*>(a.dV),
                reinterpret_cast<__nv_bfloat16*>(a.dK), a.status};
   size_t smem = sizeof(KvSmem<D>) + 1024;
   if ((e = cudaFuncSetAttribute(bwd_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
       cudaSuccess)
     return fail_at("dK/dV shared-memory attribute", e);
-  bwd_dkv_kernel<D><<<BH * nblk, kThreads, smem, st>>>(mQ64, mR64, mO64, mK128, mV128, pk);
+  bwd_dkv_kernel<D><<<BHkv * nblk, kThreads, smem, st>>>(mQ64, mR64, mO64, mK128, mV128, pk);
   if ((e = cudaGetLastError()) != cudaSuccess) return fail_at("dK/dV kernel", e);
-  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, a.window, 0, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
+  BwdParams pq{a.B, a.H, a.N, Npad, a.causal, Hkv, a.window, 0, ch, stats, reinterpret_cast<__nv_bfloat16*>(a.dQ),
                reinterpret_cast<__nv_bfloat16*>(a.dR), a.status};
   // At least 116 KB so that one CTA (and its 512 TMEM columns) holds an SM.
   smem = sizeof(QSmem<D>) + 1024;

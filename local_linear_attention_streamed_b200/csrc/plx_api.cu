@@ -254,9 +254,10 @@ int plx_prefill(const void* Q, const void* K, const void* V, const void* R, void
 
 static int prefill_train_impl(const void* Q, const void* K, const void* V, const void* R, void* out,
                               void* vbar, float* lse, float* tbar, int B, int H, int N, int d, int causal,
-                              int window, void* stream) {
+                              int window, void* stream, int Hkv = 0) {
   if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (Hkv != 0 && (Hkv < 1 || H % Hkv != 0)) return PLX_ERR_INVALID_ARG;
   if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(R) || !aligned16(out) ||
       !aligned16(vbar) || (reinterpret_cast<uintptr_t>(lse) & 3u) || (reinterpret_cast<uintptr_t>(tbar) & 3u))
@@ -270,6 +271,7 @@ static int prefill_train_impl(const void* Q, const void* K, const void* V, const
   a.lse = lse;
   a.tbar = tbar;
   a.window = window < N ? window : 0;
+  a.Hkv = Hkv > 0 ? Hkv : H;
   return cuda_rc(launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream), dc->num_sms));
 }
 
@@ -286,6 +288,13 @@ int plx_prefill_train_window(const void* Q, const void* K, const void* V, const 
   return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, 1, window, stream);
 }
 
+int plx_prefill_train_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, void* vbar,
+                          float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal,
+                          void* stream) {
+  if (Hkv < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, causal, 0, stream, Hkv);
+}
+
 size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || d < 1) return 0;
   return 16 * (size_t)B * H * bwd_padded_rows(N);
@@ -294,10 +303,11 @@ size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d) {
 static int prefill_bwd_impl(const void* Q, const void* K, const void* V, const void* R, const void* out,
                             const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ,
                             void* dK, void* dV, void* dR, int B, int H, int N, int d, int causal, int window,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+                            void* workspace, size_t workspace_bytes, void* stream, int Hkv = 0) {
   if (!Q || !K || !V || !R || !out || !vbar || !lse || !tbar || !dO || !dQ || !dK || !dV || !dR)
     return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || d < 1) return PLX_ERR_INVALID_ARG;
+  if (Hkv != 0 && (Hkv < 1 || H % Hkv != 0)) return PLX_ERR_INVALID_ARG;
   if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
   const void* t16[] = {Q, K, V, R, out, vbar, dO, dQ, dK, dV, dR};
   for (const void* t : t16)
@@ -315,6 +325,7 @@ static int prefill_bwd_impl(const void* Q, const void* K, const void* V, const v
   BwdArgs a{Q, K, V, R, out, vbar, dO, lse, tbar, dQ, dK, dV, dR, B, H, N, d, causal ? 1 : 0, workspace,
             dc->status};
   a.window = window < N ? window : 0;
+  a.Hkv = Hkv > 0 ? Hkv : H;
   if (!workspace) {
     std::lock_guard<std::mutex> lk(g_mu);
     if ((rc = grow(&dc->bwd_ws, &dc->bwd_ws_bytes, need, st)) != PLX_OK) return rc;
@@ -339,6 +350,15 @@ int plx_prefill_bwd_window(const void* Q, const void* K, const void* V, const vo
   if (window < 1) return PLX_ERR_INVALID_ARG;
   return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, 1, window, workspace,
                           workspace_bytes, stream);
+}
+
+int plx_prefill_bwd_gqa(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                        const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ, void* dK,
+                        void* dV, void* dR, int B, int H, int Hkv, int N, int d, int causal, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  if (Hkv < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, causal, 0, workspace,
+                          workspace_bytes, stream, Hkv);
 }
 
 int plx_decode_num_splits(int B, int H, int L, int d) {

@@ -101,6 +101,7 @@ struct BwdArgs {
   void* stats;
   int* status;
   int window = 0;  // sliding window of the forward (0: none; implies causal)
+  int Hkv = 0;     // KV heads of K, V, dK, dV (0: H); H a multiple of it
 };
 size_t bwd_padded_rows(int N);
 // The step of this thread's last failed backward launch ("" if none).

@@ -46,6 +46,8 @@ SIGNATURES = {
     "plx_prefill_bwd": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_prefill_train_window": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
     "plx_prefill_bwd_window": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
+    "plx_prefill_train_gqa": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
+    "plx_prefill_bwd_gqa": (_i, [_vp] * 13 + [_i] * 6 + [_vp, _sz, _vp]),
     "plx_get_device_status": (_i, [_vp]),
     "plx_status_string": (ctypes.c_char_p, [_i]),
     "plx_last_cuda_error": (ctypes.c_char_p, []),
@@ -187,25 +189,46 @@ def decode_window(q, r, Kcache, Vcache, seqlens, window: int, out=None, workspac
     return out
 
 
+def _kv_heads(Q, K, V, window):
+    """KV heads of K and V ([B, Hkv, N, d], H a multiple of Hkv); grouping and
+    a window are not combined."""
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    if K.shape != (B, Hkv, N, d) or V.shape != K.shape or Hkv < 1 or H % Hkv:
+        raise ValueError("K, V must be [B, Hkv, N, d] with H a multiple of Hkv")
+    if Hkv != H and window is not None:
+        raise ValueError("grouped KV heads take no window")
+    return Hkv
+
+
 def prefill_train(Q, K, V, R, causal: bool = True, stream=None, window=None):
     """bf16 prefill that also saves the backward pass's inputs (``window``:
-    the sliding-window prefill of prefill_window).
+    the sliding-window prefill of prefill_window).  K and V may have fewer
+    heads than Q (grouped KV heads, as prefill_gqa).
 
     Returns (out, vbar, lse, tbar): out bf16 [B, H, N, d], vbar fp32
     [B, H, N, d], lse and tbar fp32 [B, H, N] (see plx_prefill_train in
     include/plx.h).
     """
     B, H, N, d = Q.shape
+    Hkv = _kv_heads(Q, K, V, window)
     for n, t in (("K", K), ("V", V), ("R", R)):
-        if t.shape != Q.shape or t.dtype != Q.dtype:
-            raise ValueError(f"{n} must match Q in shape and dtype")
+        if t.dtype != Q.dtype:
+            raise ValueError(f"{n} must match Q's dtype")
+    if R.shape != Q.shape:
+        raise ValueError("R must match Q's shape")
     if Q.dtype != torch.bfloat16:
         raise TypeError("prefill_train takes bf16 tensors")
     out = torch.empty_like(Q)
     vbar = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     tbar = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
-    if window is None:
+    if Hkv != H:
+        rc = lib.plx_prefill_train_gqa(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                       _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, Hkv, N, d,
+                                       int(bool(causal)), _stream_ptr(stream))
+        _check(rc, "plx_prefill_train_gqa")
+    elif window is None:
         rc = lib.plx_prefill_train(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
                                    _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, N, d,
                                    int(bool(causal)), _stream_ptr(stream))
@@ -227,10 +250,16 @@ def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, 
     """Gradients (dQ, dK, dV, dR) of sum(out * dO) for one bf16 prefill.
 
     ``out, vbar, lse, tbar`` are what prefill_train returned for the same
-    inputs; ``grads`` optionally gives the four output tensors.
+    inputs; ``grads`` optionally gives the four output tensors.  With grouped
+    KV heads (K, V [B, Hkv, N, d]) dK and dV have K's shape: each sums over
+    its group's query heads.
     """
     B, H, N, d = Q.shape
-    for n, t in (("K", K), ("V", V), ("R", R), ("out", out), ("dO", dO)):
+    Hkv = _kv_heads(Q, K, V, window)
+    for n, t in (("K", K), ("V", V)):
+        if t.dtype != torch.bfloat16:
+            raise ValueError(f"{n} must be bf16")
+    for n, t in (("R", R), ("out", out), ("dO", dO)):
         if t.shape != Q.shape or t.dtype != torch.bfloat16:
             raise ValueError(f"{n} must be bf16 of Q's shape")
     if vbar.shape != Q.shape or vbar.dtype != torch.float32:
@@ -239,14 +268,17 @@ def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, 
         if t.shape != (B, H, N) or t.dtype != torch.float32:
             raise ValueError(f"{n} must be fp32 [B, H, N]")
     if grads is None:
-        grads = tuple(torch.empty_like(Q) for _ in range(4))
+        grads = (torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V), torch.empty_like(Q))
     dQ, dK, dV, dR = grads
     ws, wsb = (0, 0) if workspace is None else (_dev(workspace, "workspace"),
                                                 workspace.numel() * workspace.element_size())
     args = (_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"), _dev(vbar, "vbar"),
             _dev(lse, "lse"), _dev(tbar, "tbar"), _dev(dO, "dO"), _dev(dQ, "dQ"), _dev(dK, "dK"),
             _dev(dV, "dV"), _dev(dR, "dR"), B, H, N, d)
-    if window is None:
+    if Hkv != H:
+        rc = lib.plx_prefill_bwd_gqa(*args[:14], H, Hkv, N, d, int(bool(causal)), ws, wsb, _stream_ptr(stream))
+        _check(rc, "plx_prefill_bwd_gqa")
+    elif window is None:
         rc = lib.plx_prefill_bwd(*args, int(bool(causal)), ws, wsb, _stream_ptr(stream))
         _check(rc, "plx_prefill_bwd")
     else:
@@ -277,7 +309,8 @@ class ParallaxAttention(torch.autograd.Function):
 
 def parallax_attention(Q, K, V, R, causal: bool = True, window=None):
     """Differentiable bf16 Parallax attention over [B, H, N, d] (d in {64, 128});
-    ``window`` (None or W >= 1) makes it the sliding-window prefill."""
+    ``window`` (None or W >= 1) makes it the sliding-window prefill; K and V
+    may have fewer heads (grouped KV heads, no window)."""
     return ParallaxAttention.apply(Q, K, V, R, causal, window)
 
 

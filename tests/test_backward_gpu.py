@@ -200,3 +200,79 @@ def test_window_backward_matches_oracle(plx, N, d, W):
     assert torch.equal(saved[0], out_w)
     want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], True, window=W)
     _check_grads(grads, want, where=W)
+
+
+def _gqa_specs(B, H, Hkv, N, d):
+    specs = synth.backward_specs(B, H, N, d)
+    for n, tid in (("K", synth.TID_K), ("V", synth.TID_V)):
+        specs[n] = synth.TensorSpec(tid, (B, Hkv, N, d), specs[n].dist, specs[n].sigma)
+    return specs
+
+
+@pytest.mark.parametrize("G,N,d,causal", [(2, 200, 128, True), (4, 320, 128, True), (8, 130, 128, False),
+                                          (4, 256, 64, True), (2, 200, 64, False), (8, 1, 128, True)])
+def test_gqa_train_then_backward_matches_oracle(plx, G, N, d, causal):
+    """Grouped KV heads (query head h reads KV head h / G): the training
+    forward's out equals the grouped inference prefill bit for bit, and every
+    element of dQ, dR (per query head) and of dK, dV (per KV head, summed over
+    the group's query heads) meets the gradient bars; ragged N, causal and full."""
+    B, Hkv = 2, 2
+    H = G * Hkv
+    dev, ref = small_inputs(1400 + 10 * G + N + d, _gqa_specs(B, H, Hkv, N, d), synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], causal)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], causal)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    assert torch.equal(saved[0], plx.prefill_gqa(dev["Q"], dev["K"], dev["V"], dev["R"], causal=causal))
+    assert grads[1].shape == dev["K"].shape and grads[2].shape == dev["V"].shape
+    want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], causal)
+    _check_grads(grads, want, where=G)
+
+
+def test_gqa_autograd_matches_direct_calls(plx):
+    B, H, Hkv, N, d = 1, 8, 2, 192, 128
+    dev, _ = small_inputs(1450, _gqa_specs(B, H, Hkv, N, d), synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    g1 = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+    leaves = [dev[n].clone().requires_grad_(True) for n in "QKVR"]
+    o2 = plx.parallax_attention(*leaves, causal=True)
+    o2.backward(dev["dO"])
+    assert torch.equal(o2.detach(), saved[0])
+    for a, leaf in zip(g1, leaves):
+        assert torch.equal(a, leaf.grad)
+
+
+def test_gqa_backward_rejects_bad_groups(plx):
+    B, N, d = 1, 64, 128
+    q = torch.zeros((B, 6, N, d), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((B, 4, N, d), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ValueError):
+        plx.prefill_train(q, kv, kv, q, True)
+    with pytest.raises(ValueError):
+        plx.prefill_train(q, kv[:, :3], kv[:, :3], q, True, window=16)
+
+
+def test_gqa_backward_full_size_group(plx):
+    """B=2, H=32, Hkv=8, N=4096, d=128 causal: the whole group of KV head
+    (1, 5) (its four query heads' dQ, dR and the head's dK, dV) compared element
+    by element with the oracle run on that group alone."""
+    B, H, Hkv, N, d = 2, 32, 8, 4096, 128
+    G = H // Hkv
+    seed = 1460
+    specs = _gqa_specs(B, H, Hkv, N, d)
+    dev = device_inputs(seed, specs, synth.BF16)
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    for g in grads:
+        assert torch.isfinite(g).all()
+    b, hk = 1, 5
+    qrows = lambda n: synth.host_rows_f64(seed, specs[n], synth.BF16, (b * H + hk * G) * N, G * N).reshape(1, G, N, d)
+    krows = lambda n: synth.host_rows_f64(seed, specs[n], synth.BF16, (b * Hkv + hk) * N, N).reshape(1, 1, N, d)
+    head = {n: qrows(n) for n in ("Q", "R", "dO")}
+    head.update({n: krows(n) for n in ("K", "V")})
+    want = oracle.parallax_backward_ref(head["Q"], head["K"], head["V"], head["R"], head["dO"], True)
+    got = [grads[0][b, hk * G:(hk + 1) * G], grads[1][b, hk:hk + 1], grads[2][b, hk:hk + 1],
+           grads[3][b, hk * G:(hk + 1) * G]]
+    _check_grads(got, [w[0] for w in want], where=(b, hk))
