@@ -418,6 +418,57 @@ def run_gpu(args, rank, world, dist):
             del bt, saved, grads, bws
             torch.cuda.empty_cache()
 
+        # Grouped KV heads on the same query workload (G = 4): forward, and
+        # the training forward plus backward.
+        if not args.no_gqa:
+            gHkv = pH // 4
+            gspecs = synth.backward_specs(pB, pH, pN, pd)
+            for n, tid in (("K", synth.TID_K), ("V", synth.TID_V)):
+                gspecs[n] = synth.TensorSpec(tid, (pB, gHkv, pN, pd), gspecs[n].dist, gspecs[n].sigma)
+            gt = {}
+            for name, spec in gspecs.items():
+                gt[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+                synth.device_fill(gt[name].data_ptr(), synth.BF16, seed + 8, spec)
+            gout = torch.empty_like(gt["Q"])
+
+            def gfwd():
+                plx.prefill_gqa(gt["Q"], gt["K"], gt["V"], gt["R"], True, out=gout)
+
+            gf_total, gf_per = timed(gfwd, psteps, max(3, args.warmup // 2), stream, dist)
+            gf_total = max_over_ranks(gf_total, dist)
+            entry = {
+                "workload": f"causal prefill B={pB} H={pH} Hkv={gHkv} N={pN} d={pd} bf16 (grouped KV heads, G=4)",
+                "value": round(sum_over_ranks(flops * psteps, dist) / (gf_total * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "ms_per_step": round(gf_total / psteps, 3),
+                "kernel_tflops": round(flops / (float(np.mean(gf_per)) * 1e-3) / 1e12, 1),
+            }
+            if not args.no_backward:
+                gsaved = plx.prefill_train(gt["Q"], gt["K"], gt["V"], gt["R"], True)
+                ggrads = (torch.empty_like(gt["Q"]), torch.empty_like(gt["K"]), torch.empty_like(gt["V"]),
+                          torch.empty_like(gt["Q"]))
+                gws = torch.empty(plx.prefill_bwd_workspace_bytes(pB, pH, pN, pd) // 4, dtype=torch.float32,
+                                  device=dev)
+
+                def gbwd():
+                    plx.prefill_backward(gt["Q"], gt["K"], gt["V"], gt["R"], *gsaved, gt["dO"], True,
+                                         grads=ggrads, workspace=gws)
+
+                gb_total, gb_per = timed(gbwd, psteps, max(3, args.warmup // 2), stream, dist)
+                gb_total = max_over_ranks(gb_total, dist)
+                gbflops = backward_flops(pB, pH, pN, pd)
+                entry["backward"] = {
+                    "value": round(sum_over_ranks(gbflops * psteps, dist) / (gb_total * 1e-3) / 1e12, 2),
+                    "unit": "TFLOP/s", "ms_per_step": round(gb_total / psteps, 3),
+                    "kernel_tflops": round(gbflops / (float(np.mean(gb_per)) * 1e-3) / 1e12, 1),
+                    "gpu_launches_per_step": 3,
+                }
+                del gsaved, ggrads, gws
+            if plx.get_device_status() != 0:
+                raise RuntimeError("grouped-KV prefill reported a device error")
+            prefill["gqa"] = entry
+            del gt, gout
+            torch.cuda.empty_cache()
+
     # ---- Decode with grouped KV heads (the next row of the scope: one KV stream per group).
     # ---- Sliding-window variants (a window of 1024 keys on the prefill and decode workloads).
     win = None

@@ -751,8 +751,11 @@ cudaError_t launch_bwd_d(const BwdArgs& a, cudaStream_t st, int num_sms) {
   // About two waves of blocks per chunk of heads.
   int ch = (2 * num_sms + nblk - 1) / nblk;
   ch = ch < 1 ? 1 : (ch > BH ? BH : ch);
-  const int BHkv = a.B * Hkv;
-  const int chkv = ch > BHkv ? BHkv : ch;
+  // A dK/dV CTA of a KV head streams the query tiles of its G query heads:
+  // chunks of ch / G KV heads keep the same query-tile footprint in L2.
+  const int BHkv = a.B * Hkv, G = a.H / Hkv;
+  int chkv = (ch + G - 1) / G;
+  chkv = chkv > BHkv ? BHkv : chkv;
   // PLX_FAULT_INJECT=bwd_stall makes one CTA's bounded waits run out (tests of
   // the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
