@@ -258,13 +258,13 @@ def run_gpu(args, rank, world, dist):
     kernel_ms = float(np.mean(per))
     value = sum_over_ranks(kv_bytes * args.steps, dist) / (total_ms * 1e-3) / 1e9
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
-    src_hash = kernel_hash("decode_mma.cu")
+    src_hash = kernel_hash("decode_gqa_tc.cu", "sm100.cuh")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 # The committed capture is of the default workload; other sizes report none.
                 "traffic": (traffic_from_profile("decode_bf16_B64_H16_L4096.json", src_hash)
                             if B == DECODE["B"] else None),
-                "peak_source": peak_src, "kernel": "decode_bf16_kernel<128>",
+                "peak_source": peak_src, "kernel": "decode_gqa_tc_kernel<1>",
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "frac_of_spec_8000": round(achieved / 8000.0, 4)}
 
@@ -555,7 +555,8 @@ def run_gpu(args, rank, world, dist):
                 "unit": "GB/s", "kernel_gbs": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9, 1),
                 "frac": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                 "algorithmic_bytes_per_launch": dbytes,
-                "traffic": (traffic_from_profile("decode_window_B64_H16_L4096_W1024.json", kernel_hash("decode_mma.cu"))
+                "traffic": (traffic_from_profile("decode_window_B64_H16_L4096_W1024.json",
+                                                kernel_hash("decode_gqa_tc.cu", "sm100.cuh"))
                             if dB == DECODE["B"] else None),
             },
         }
@@ -594,7 +595,8 @@ def run_gpu(args, rank, world, dist):
                        "l2": f"inputs larger than L2 ({g_kv / 1e9:.2f} GB KV); no flush"},
             "roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(g_ach / peaks["hbm_gbs"], 4), "traffic": None,
-                         "peak_source": peak_src, "kernel": f"decode_gqa_kernel<{gd}, {gH // gHkv}>",
+                         "peak_source": peak_src, "kernel": (f"decode_gqa_tc_kernel<{gH // gHkv}>" if gd == 128
+                                    else f"decode_gqa_kernel<{gd}, {gH // gHkv}>"),
                          "algorithmic_bytes_per_launch": g_alg},
             "gpu_launches": gsteps,
         }

@@ -48,7 +48,7 @@ struct Cfg {
   static constexpr int kHeadsPerWarp = G / kHeadSplits;
   static constexpr int kConsumerWarps = kSlices * kHeadSplits;
   static constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + the TMA producer warp
-  static constexpr int kMinCtas = G == 8 ? 1 : 2;  // = decode_gqa_ctas_per_sm(G)
+  static constexpr int kMinCtas = G == 8 ? 1 : 2;  // = decode_gqa_ctas_per_sm(G, 64)
   static constexpr int kStages = kMinCtas == 1 ? 6 : 3;
 };
 constexpr int kUnitRing = 4;
@@ -639,16 +639,13 @@ cudaError_t launch_gqa(const DecodeArgs& a, const CUtensorMap& mK, const CUtenso
 
 cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms) {
   if (a.Hkv < 1 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+  if (a.d == 128) return launch_decode_gqa_tc(a, st, num_sms);
   const long long rows = (long long)a.B * a.Hkv * a.L;
   if (rows + kBlk >= (1ll << 31)) return cudaErrorInvalidValue;
   CUtensorMap mK, mV;
   if (!make_cache_map(&mK, a.K, rows, a.d) || !make_cache_map(&mV, a.V, rows, a.d)) return cudaErrorInvalidValue;
   const int G = a.H / a.Hkv;
-  if (a.d == 128) {
-    if (G == 2) return launch_gqa<128, 2>(a, mK, mV, st, num_sms);
-    if (G == 4) return launch_gqa<128, 4>(a, mK, mV, st, num_sms);
-    if (G == 8) return launch_gqa<128, 8>(a, mK, mV, st, num_sms);
-  } else if (a.d == 64) {
+  if (a.d == 64) {
     if (G == 2) return launch_gqa<64, 2>(a, mK, mV, st, num_sms);
     if (G == 4) return launch_gqa<64, 4>(a, mK, mV, st, num_sms);
     if (G == 8) return launch_gqa<64, 8>(a, mK, mV, st, num_sms);

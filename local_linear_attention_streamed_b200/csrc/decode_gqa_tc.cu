@@ -1,0 +1,599 @@
+// Split-KV Parallax decode on the tensor cores (tcgen05 MMAs with TMEM
+// accumulators, TMA staging), bf16 caches, d = 128, one KV head per query
+// head (G = 1) or grouped KV heads (G = H / Hkv in {2, 4, 8}).
+//
+// G consecutive query heads read one KV head, so one pass over a KV head's
+// cache serves the whole group: the pages' decode packs the q and rho rows
+// into one tensor-core tile so that a single stream of K feeds both score
+// products (agihunt.info summary, decode paragraph), and grouping fills that
+// tile with the rows of every head of the group.
+//
+// Per staged block of 128 keys (one CTA per SM, persistent, units from a
+// global counter, unit = (b, KV head, key chunk)):
+//   * scores, keys as the MMA's M:  S^T [128 keys x 16] = K_blk [Q; R]^T
+//     (B rows 0..G-1 = q of the group's heads, rows 8..8+G-1 = rho);
+//   * one thread per key (TMEM lane) forms, per head, the weight
+//     w = 2^(s c - m) (lazy running max m, raised only when a block's max
+//     exceeds it by more than 2^8) and w t, each as a bf16 hi + lo pair, into
+//     a shared-memory tile W [128 keys x 4G];
+//   * value product, dims as the MMA's M:  O^T [128 dims x 4G] += V_blk^T W,
+//     with V read in place as an MN-major operand; the columns of head h are
+//     sum w_hi v, sum w_lo v, sum wt_hi v, sum wt_lo v, so O1 and O2 come out
+//     with about 16 bits of weight precision (the hi + lo split of the
+//     ungrouped decode).
+// omega = sum w and T = sum w t are kept per thread in fp32 and reduced at
+// the end of the unit.  Chunks of one (b, KV head) merge through fp32
+// partial records, by the last CTA to finish one (an arrival counter per
+// (b, KV head), left at zero).
+//
+// Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
+#include "plx_internal.cuh"
+#include "sm100.cuh"
+
+#include <math_constants.h>
+
+namespace plx {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;          // head dim (the MMA M of the value product)
+constexpr int kKeys = 128;       // keys per staged block (the MMA M of the score product)
+constexpr int kStages = 3;       // K/V staging ring (64 KB per stage)
+constexpr int kUnitRing = 4;
+constexpr int kThreads = 256;    // warp 0 TMA, warp 1 MMA, warps 4..7 one key / one dim per thread
+constexpr int kFirstEw = 4;
+constexpr float kLazyTau = 8.f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Value-product columns: (w_hi, w_lo, wt_hi, wt_lo) per head, at least the
+// MMA's minimum N of 16 (the spare rows of W stay zero).
+template <int G>
+constexpr int kCols = 4 * G < 16 ? 16 : 4 * G;
+
+// TMEM columns: two 16-column score stages, then two value accumulators.
+constexpr uint32_t kColS = 0, kColO = 32, kTmemCols = 128;
+
+// Instruction descriptor (kind::f16): D f32, A and B bf16, M = 128, N = n;
+// a_mn / b_mn = 1 for an MN-major A / B operand.
+__host__ __device__ constexpr uint32_t idesc(int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+// Byte offset of element column `col` (bf16) of row `row` in a 128B-swizzled
+// tile of 128-byte rows.
+__device__ __forceinline__ uint32_t sw128_elem(int row, int col) {
+  return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2);
+}
+
+template <int G>
+struct Smem {
+  static constexpr int NW = kCols<G>;
+  uint8_t k[kStages][2][kKeys * 128];  // [128 keys x 64 dims] per 64-dim half
+  uint8_t v[kStages][2][kKeys * 128];
+  uint8_t qr[2][2][16 * 128];          // per unit slot: [16 rows x 64 dims] per half
+  uint8_t w[2][2][NW * 128];           // per block slot: [NW rows x 64 keys] per 64-key half
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t qr_full[2], qr_empty[2];
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
+  uint64_t s_full[2], s_free[2], w_full[2], w_free[2];
+  uint64_t o_full[2], o_free[2];
+  uint64_t vote[2];  // block-max exchange among the four key warps
+  uint64_t rdv;      // rendezvous of the four key warps at the end of a unit
+  uint64_t drain;
+  long long unit_ring[kUnitRing];
+  int unit_n[kUnitRing];  // seqlens of the unit's batch row, read once by the producer
+  float red[2][4][G];   // per-warp block maxima of each head
+  float sums[4][2 * G]; // per-warp omega and T of each head
+  int last;
+  uint32_t tmem_base;
+  int abort;
+};
+
+static_assert(sizeof(Smem<8>) + 1024 <= 227 * 1024, "shared memory of one CTA");
+static_assert(kColO + 2 * kCols<8> <= kTmemCols, "TMEM columns");
+
+__device__ unsigned long long g_tc_unit_next;
+__device__ unsigned int g_tc_cta_done;
+
+// Bounded wait taken by a whole warp: every lane leaves with the same answer.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
+  if constexpr (N == 16) {
+    tmem_ld16(taddr, v);
+  } else {
+    static_assert(N == 32, "accumulator width");
+    tmem_ld32(taddr, v);
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[N]) {
+#pragma unroll
+  for (int c = 0; c < N / 16; ++c) {
+    uint32_t part[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) part[x] = v[16 * c + x];
+    tmem_st16(taddr + 16 * c, part);
+  }
+}
+
+// What every role derives from a unit index.
+struct Unit {
+  int b, kvh, bkv, c, n, kbeg, kend, nch, nblk;
+  bool bad;
+};
+__device__ __forceinline__ Unit unit_of(long long u, int n, const DecodeArgs& a) {
+  const int BKV = a.B * a.Hkv;
+  Unit x;
+  x.c = (int)(u / BKV);
+  x.bkv = (int)(u - (long long)x.c * BKV);
+  x.b = x.bkv / a.Hkv;
+  x.kvh = x.bkv - x.b * a.Hkv;
+  x.n = n;
+  x.bad = x.n < 1 || x.n > a.L;
+  // Keys lo..n-1 (lo > 0 only with a sliding window), cut into chunks.
+  const int lo = (!x.bad && a.window > 0 && x.n > a.window) ? x.n - a.window : 0;
+  x.kbeg = lo + x.c * a.chunk;
+  x.kend = x.bad ? x.kbeg : min(x.kbeg + a.chunk, x.n);
+  x.nblk = (!x.bad && x.kbeg < x.n) ? (x.kend - x.kbeg + kKeys - 1) / kKeys : 0;
+  x.nch = x.bad ? 0 : (x.n - lo + a.chunk - 1) / a.chunk;
+  return x;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
+                         DecodeArgs a) {
+  constexpr int NW = kCols<G>;
+  static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem<G>& sm = *reinterpret_cast<Smem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long units = (long long)a.B * a.Hkv * a.splits;
+  volatile int* abort = &sm.abort;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int s = 0; s < kUnitRing; ++s) {
+      mbar_init(&sm.unit_full[s], 1);
+      mbar_init(&sm.unit_empty[s], 5);  // the MMA thread and the four key warps
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.qr_full[s], 1);
+      mbar_init(&sm.qr_empty[s], 1);
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_free[s], 4);
+      mbar_init(&sm.w_full[s], 128);
+      mbar_init(&sm.w_free[s], 1);
+      mbar_init(&sm.o_full[s], 1);
+      mbar_init(&sm.o_free[s], 4);
+      mbar_init(&sm.vote[s], 4);
+    }
+    mbar_init(&sm.rdv, 4);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Operand rows that no copy and no thread writes stay zero: the q / rho
+  // tile's rows G..7 and 8+G..15, and the weight tile's rows past 4G.
+  for (int x = threadIdx.x; x < (int)(sizeof(sm.qr) / 16); x += kThreads)
+    reinterpret_cast<uint4*>(&sm.qr[0][0][0])[x] = make_uint4(0u, 0u, 0u, 0u);
+  for (int x = threadIdx.x; x < (int)(sizeof(sm.w) / 16); x += kThreads)
+    reinterpret_cast<uint4*>(&sm.w[0][0][0])[x] = make_uint4(0u, 0u, 0u, 0u);
+  fence_async_smem();
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&sm.tmem_base)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer: units, the group's q / rho rows, K and V blocks ----------------
+    if (lane == 0) {
+      long long u = blockIdx.x;  // first unit static, the rest from the counter
+      uint32_t pos = 0;          // K/V ring position
+      int last_kv[kStages], last_qr[2] = {-1, -1};
+      for (int s = 0; s < kStages; ++s) last_kv[s] = -1;
+      for (int ui = 0;; ++ui) {
+        const int slot = ui % kUnitRing;
+        if (!mbar_wait(&sm.unit_empty[slot], ((ui / kUnitRing) & 1) ^ 1, abort, a.status)) break;
+        const long long uu = u < units ? u : -1;
+        const int n = uu < 0 ? 0 : a.seqlens[(int)(uu % (a.B * a.Hkv)) / a.Hkv];
+        sm.unit_ring[slot] = uu;
+        sm.unit_n[slot] = n;
+        mbar_arrive(&sm.unit_full[slot]);
+        if (uu < 0) break;
+        const long long next = (long long)gridDim.x + (long long)atomicAdd(&g_tc_unit_next, 1ull);
+        const Unit x = unit_of(uu, n, a);
+        const int qs = ui & 1;
+        if (!mbar_wait(&sm.qr_empty[qs], ((ui >> 1) & 1) ^ 1, abort, a.status)) break;
+        mbar_expect_tx(&sm.qr_full[qs], 2 * 2 * G * 128);
+        last_qr[qs] = ui >> 1;
+        const int qrow = x.b * a.H + x.kvh * G;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tma_load_2d(sm.qr[qs][h], &tmQ, &sm.qr_full[qs], 64 * h, qrow);
+          tma_load_2d(sm.qr[qs][h] + 8 * 128, &tmR, &sm.qr_full[qs], 64 * h, qrow);
+        }
+        const int row0 = x.bkv * a.L + x.kbeg;  // < 2^31 (checked by the launcher)
+        bool ok = true;
+        for (int i = 0; i < x.nblk; ++i, ++pos) {
+          const int st = pos % kStages;
+          if (!(ok = mbar_wait(&sm.kv_empty[st], ((pos / kStages) & 1) ^ 1, abort, a.status))) break;
+          mbar_expect_tx(&sm.kv_full[st], 4 * kKeys * 128);
+          last_kv[st] = (int)(pos / kStages);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], 64 * h, row0 + kKeys * i);
+            tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], 64 * h, row0 + kKeys * i);
+          }
+        }
+        if (!ok) break;
+        u = next;
+      }
+      if (*abort) {  // let every copy issued here land before the CTA exits
+        for (int s = 0; s < kStages; ++s)
+          if (last_kv[s] >= 0) mbar_drain(&sm.kv_full[s], (uint32_t)(last_kv[s] & 1));
+        for (int s = 0; s < 2; ++s)
+          if (last_qr[s] >= 0) mbar_drain(&sm.qr_full[s], (uint32_t)(last_qr[s] & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      uint32_t pos = 0, blk = 0, ou = 0;
+      bool ok = true;
+      for (int ui = 0; ok; ++ui) {
+        const int slot = ui % kUnitRing;
+        if (!(ok = mbar_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
+        const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
+        const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
+        mbar_arrive(&sm.unit_empty[slot]);
+        if (uu < 0) break;
+        const Unit x = unit_of(uu, n, a);
+        const int qs = ui & 1;
+        if (!(ok = mbar_wait(&sm.qr_full[qs], (ui >> 1) & 1, abort, a.status))) break;
+        if (x.nblk == 0) {
+          mbar_arrive(&sm.qr_empty[qs]);
+          continue;
+        }
+        const int ob = ou & 1;
+        // The accumulator of two units back has been read out.
+        if (!(ok = mbar_wait(&sm.o_free[ob], ((ou >> 1) & 1) ^ 1, abort, a.status))) break;
+        const uint64_t bq = sdesc(smem_u32(sm.qr[qs][0]), 16, 1024);
+        // Scores of block bb (ring position p): S^T = K [Q; R]^T, both K-major.
+        auto issue_scores = [&](uint32_t p, uint32_t bb) -> bool {
+          const int st = p % kStages, sb = bb & 1;
+          if (!mbar_wait(&sm.kv_full[st], (p / kStages) & 1, abort, a.status)) return false;
+          if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
+          tc_fence_after();
+          const uint64_t ak = sdesc(smem_u32(sm.k[st][0]), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t oa = (ks >> 2) * (kKeys * 128) + (ks & 3) * 32;
+            const uint32_t ob2 = (ks >> 2) * (16 * 128) + (ks & 3) * 32;
+            mma_ss(tmem + kColS + 16 * sb, ak + (uint64_t)(oa >> 4), bq + (uint64_t)(ob2 >> 4), idesc(16, 0, 0),
+                   ks > 0 ? 1u : 0u);
+          }
+          mma_commit(&sm.s_full[sb]);
+          return true;
+        };
+        if (!(ok = issue_scores(pos, blk))) break;
+        for (int i = 0; i < x.nblk; ++i) {
+          const uint32_t p = pos + i, bb = blk + i;
+          // The next block's scores go ahead of this block's value product.
+          if (i + 1 < x.nblk) {
+            if (!(ok = issue_scores(p + 1, bb + 1))) break;
+          } else {
+            mma_commit(&sm.qr_empty[qs]);  // every score MMA of the unit is issued
+          }
+          const int st = p % kStages, sb = bb & 1;
+          if (!(ok = mbar_wait(&sm.w_full[sb], (bb >> 1) & 1, abort, a.status))) break;
+          tc_fence_after();
+          // V^T as an MN-major A operand: the two 64-dim halves LBO apart,
+          // 8-key groups 1024 bytes apart, 16 keys (one K step) 2048 bytes.
+          const uint64_t av = sdesc(smem_u32(sm.v[st][0]), kKeys * 128, 1024);
+          const uint64_t bw = sdesc(smem_u32(sm.w[sb][0]), 16, 1024);
+#pragma unroll
+          for (int ks = 0; ks < kKeys / 16; ++ks) {
+            const uint32_t ow = (ks >> 2) * (NW * 128) + (ks & 3) * 32;
+            mma_ss(tmem + kColO + NW * ob, av + (uint64_t)((ks * 2048) >> 4), bw + (uint64_t)(ow >> 4),
+                   idesc(NW, 1, 0), (i > 0 || ks > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm.kv_empty[st]);
+          mma_commit(&sm.w_free[sb]);
+        }
+        if (!ok) break;
+        mma_commit(&sm.o_full[ob]);
+        pos += x.nblk;
+        blk += x.nblk;
+        ++ou;
+      }
+      // Every MMA issued here completes before TMEM is freed.
+      mma_commit(&sm.drain);
+      mbar_drain(&sm.drain, 0);
+    }
+  } else if (warp >= kFirstEw) {
+    // ---------------- one key of every block (scores), one dim of the accumulator ----------------
+    const int q = warp - kFirstEw, r = 32 * q + lane;
+    const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
+    const float c_log2 = kLog2e / sqrtf((float)kD);
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+    uint32_t pos = 0, blk = 0, ou = 0, rv = 0;
+    // Rendezvous of the four key warps (bounded like every wait).
+    auto rendezvous = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.rdv);
+      const bool ok = warp_wait(&sm.rdv, rv & 1, abort, a.status);
+      ++rv;
+      return ok;
+    };
+    bool ok = true;
+    for (int ui = 0; ok; ++ui) {
+      const int slot = ui % kUnitRing;
+      if (!(ok = warp_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
+      const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
+      const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.unit_empty[slot]);
+      if (uu < 0) break;
+      const Unit x = unit_of(uu, n, a);
+      if (x.bad) {
+        if (x.c == 0) {
+          const long long bh0 = (long long)x.b * a.H + (long long)x.kvh * G;
+#pragma unroll
+          for (int h = 0; h < G; ++h) out[(bh0 + h) * kD + r] = __float2bfloat16(0.f);
+          if (r == 0) atomicOr(a.status, kStatusBadSeqlen);
+        }
+        continue;
+      }
+      if (x.nblk == 0) continue;
+      const int ob = ou & 1;
+      float hm[G], hom[G], hT[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        hm[h] = -CUDART_INF_F;
+        hom[h] = 0.f;
+        hT[h] = 0.f;
+      }
+      for (int i = 0; i < x.nblk; ++i) {
+        const uint32_t p = pos + i, bb = blk + i;
+        const int st = p % kStages, sb = bb & 1;
+        if (!(ok = warp_wait(&sm.s_full[sb], (bb >> 1) & 1, abort, a.status))) break;
+        tc_fence_after();
+        uint32_t sv[16];
+        tmem_ld16(lb + kColS + 16 * sb, sv);
+        tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+        const int key = x.kbeg + kKeys * i + r;
+        const bool valid = key < x.kend;
+        float xs[G], tv[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          xs[h] = valid ? __uint_as_float(sv[h]) * c_log2 : -CUDART_INF_F;
+          tv[h] = valid ? __uint_as_float(sv[8 + h]) : 0.f;
+        }
+        // Block max of every head over the four warps' keys.
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float mx = xs[h];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          if (lane == 0) sm.red[sb][q][h] = mx;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.vote[sb]);
+        if (!(ok = warp_wait(&sm.vote[sb], (bb >> 1) & 1, abort, a.status))) break;
+        bool raised = false;
+        float alpha[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float mblk = fmaxf(fmaxf(sm.red[sb][0][h], sm.red[sb][1][h]), fmaxf(sm.red[sb][2][h], sm.red[sb][3][h]));
+          const bool up = mblk > hm[h] + kLazyTau;  // always on the unit's first block (m = -inf)
+          alpha[h] = up ? exp2f(hm[h] - mblk) : 1.f;
+          hm[h] = up ? mblk : hm[h];
+          hom[h] *= alpha[h];
+          hT[h] *= alpha[h];
+          raised |= up;
+        }
+        if (raised && i > 0) {  // uniform over the four warps; rare after the first block
+          // Rescale the accumulator once the previous block's value MMAs are done.
+          const uint32_t pb = bb - 1;
+          if (!(ok = warp_wait(&sm.w_free[pb & 1], (pb >> 1) & 1, abort, a.status))) break;
+          tc_fence_after();
+          uint32_t ov[NW];
+          tmem_ld_cols<NW>(lb + kColO + NW * ob, ov);
+          tc_wait_ld();
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) ov[4 * h + k4] = __float_as_uint(__uint_as_float(ov[4 * h + k4]) * alpha[h]);
+          }
+          tmem_st_cols<NW>(lb + kColO + NW * ob, ov);
+          tc_wait_st();
+          tc_fence_before();
+        }
+        float wv[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          wv[h] = exp2f(xs[h] - hm[h]);
+          hom[h] += wv[h];
+          hT[h] += wv[h] * tv[h];
+        }
+        // The weight tile of two blocks back has been consumed.
+        if (!(ok = warp_wait(&sm.w_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
+        uint8_t* wt = sm.w[sb][r >> 6];
+        const int kk = r & 63;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float w = wv[h], wtv = wv[h] * tv[h];
+          const __nv_bfloat16 whi = __float2bfloat16_rn(w), thi = __float2bfloat16_rn(wtv);
+          const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
+          const __nv_bfloat16 tlo = __float2bfloat16_rn(wtv - __bfloat162float(thi));
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 0, kk)) = whi;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 1, kk)) = wlo;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 2, kk)) = thi;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 3, kk)) = tlo;
+        }
+        // Keys past the end of the sequence carry zero weight; their V rows
+        // (whatever the cache holds there, even NaN) are zeroed so that they
+        // cannot turn into NaN in the product.
+        if (key >= x.n) {
+          // (the stage's copy is long complete: the scores of this block read it)
+          if (!mbar_wait(&sm.kv_full[st], (p / kStages) & 1, abort, a.status)) ok = false;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4* row = reinterpret_cast<uint4*>(sm.v[st][h] + r * 128);
+#pragma unroll
+            for (int c16 = 0; c16 < 8; ++c16) row[c16] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_async_smem();
+        mbar_arrive(&sm.w_full[sb]);
+      }
+      if (!ok) break;
+      // ---- End of the unit: the accumulator (thread r holds dim r) and the sums.
+      if (!(ok = warp_wait(&sm.o_full[ob], (ou >> 1) & 1, abort, a.status))) break;
+      tc_fence_after();
+      uint32_t ov[NW];
+      tmem_ld_cols<NW>(lb + kColO + NW * ob, ov);
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free[ob]);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          hom[h] += __shfl_xor_sync(0xffffffffu, hom[h], o);
+          hT[h] += __shfl_xor_sync(0xffffffffu, hT[h], o);
+        }
+        if (lane == 0) {
+          sm.sums[q][2 * h] = hom[h];
+          sm.sums[q][2 * h + 1] = hT[h];
+        }
+      }
+      if (!(ok = rendezvous())) break;
+      const long long bh0 = (long long)x.b * a.H + (long long)x.kvh * G;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float om = (sm.sums[0][2 * h] + sm.sums[1][2 * h]) + (sm.sums[2][2 * h] + sm.sums[3][2 * h]);
+        const float TT =
+            (sm.sums[0][2 * h + 1] + sm.sums[1][2 * h + 1]) + (sm.sums[2][2 * h + 1] + sm.sums[3][2 * h + 1]);
+        const float o1 = __uint_as_float(ov[4 * h]) + __uint_as_float(ov[4 * h + 1]);
+        const float o2 = __uint_as_float(ov[4 * h + 2]) + __uint_as_float(ov[4 * h + 3]);
+        const long long bh = bh0 + h;
+        if (x.nch == 1) {
+          const float inv = 1.f / om;
+          out[bh * kD + r] = __float2bfloat16_rn(((1.f + TT * inv) * o1 - o2) * inv);
+        } else {
+          float* rec = a.partials + (bh * a.splits + x.c) * (2 * kD + 4);
+          if (r == 0) {
+            rec[0] = hm[h];
+            rec[1] = om;
+            rec[2] = TT;
+          }
+          rec[4 + r] = o1;
+          rec[4 + kD + r] = o2;
+        }
+      }
+      if (x.nch > 1) {
+        __threadfence();
+        if (!(ok = rendezvous())) break;
+        if (r == 0) sm.last = (atomicAdd(a.counters + x.bkv, 1) == x.nch - 1);
+        if (!(ok = rendezvous())) break;
+        if (sm.last) {
+          __threadfence();
+#pragma unroll 1
+          for (int h = 0; h < G; ++h) {
+            const long long bh = bh0 + h;
+            const float* base = a.partials + bh * a.splits * (2 * kD + 4);
+            float Mg = -CUDART_INF_F;
+            for (int cc = 0; cc < x.nch; ++cc) Mg = fmaxf(Mg, __ldcg(base + (long long)cc * (2 * kD + 4)));
+            float om = 0.f, TT = 0.f, p1 = 0.f, p2 = 0.f;
+            for (int cc = 0; cc < x.nch; ++cc) {
+              const float* rc = base + (long long)cc * (2 * kD + 4);
+              const float mc = __ldcg(rc);
+              const float sc = (mc == -CUDART_INF_F) ? 0.f : exp2f(mc - Mg);
+              om += sc * __ldcg(rc + 1);
+              TT += sc * __ldcg(rc + 2);
+              p1 += sc * __ldcg(rc + 4 + r);
+              p2 += sc * __ldcg(rc + 4 + kD + r);
+            }
+            const float inv = 1.f / om;
+            out[bh * kD + r] = __float2bfloat16_rn(((1.f + TT * inv) * p1 - p2) * inv);
+          }
+          if (r == 0) a.counters[x.bkv] = 0;
+        }
+      }
+      if (!(ok = rendezvous())) break;  // the sums and the flag are reused by the next unit
+      pos += x.nblk;
+      blk += x.nblk;
+      ++ou;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) {
+    // Every CTA fetched its last unit before this point; the last CTA to get
+    // here leaves the scheduler at zero for the next launch.
+    __threadfence();
+    if (atomicAdd(&g_tc_cta_done, 1u) == gridDim.x - 1) {
+      atomicExch(&g_tc_unit_next, 0ull);
+      atomicExch(&g_tc_cta_done, 0u);
+    }
+  }
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+  }
+}
+
+template <int G>
+cudaError_t launch_g(const DecodeArgs& a, cudaStream_t st, int num_sms) {
+  CUtensorMap mK, mV, mQ, mR;
+  const long long kv_rows = (long long)a.B * a.Hkv * a.L, q_rows = (long long)a.B * a.H;
+  if (!make_map(&mK, a.K, kv_rows, kKeys, kD) || !make_map(&mV, a.V, kv_rows, kKeys, kD) ||
+      !make_map(&mQ, a.q, q_rows, G, kD) || !make_map(&mR, a.r, q_rows, G, kD))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(Smem<G>) + 1024;
+  cudaError_t e =
+      cudaFuncSetAttribute(decode_gqa_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const long long units = (long long)a.B * a.Hkv * a.splits;
+  const long long grid = units < num_sms ? units : num_sms;
+  decode_gqa_tc_kernel<G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, mQ, mR, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_sms) {
+  if (a.d != kD || a.Hkv < 1 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+  if ((long long)a.B * a.Hkv * a.L + kKeys >= (1ll << 31)) return cudaErrorInvalidValue;
+  const int G = a.H / a.Hkv;
+  if (G == 1) return launch_g<1>(a, st, num_sms);
+  if (G == 2) return launch_g<2>(a, st, num_sms);
+  if (G == 4) return launch_g<4>(a, st, num_sms);
+  if (G == 8) return launch_g<8>(a, st, num_sms);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace plx

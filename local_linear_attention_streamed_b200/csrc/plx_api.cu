@@ -109,7 +109,7 @@ constexpr size_t kLtWorkspace = 32u << 20;  // cuBLASLt workspace of the fp8 GEM
 
 // Bytes of partial records a split decode needs (0 when keys are not split).
 size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk) {
-  decode_split_plan(B, H, L, num_sms, splits, chunk);
+  decode_split_plan(B, H, L, num_sms, splits, chunk, decode_bf16_ctas_per_sm(d));
   if (*splits <= 1) return 0;
   return sizeof(float) * (size_t)B * H * (size_t)(*splits) * (size_t)(2 * d + 4);
 }
@@ -365,7 +365,7 @@ int plx_decode_num_splits(int B, int H, int L, int d) {
   (void)d;
   if (B < 1 || H < 1 || L < 1) return 0;
   int splits = 1, chunk = 0;
-  decode_split_plan(B, H, L, num_sms_or_default(), &splits, &chunk);
+  decode_split_plan(B, H, L, num_sms_or_default(), &splits, &chunk, decode_bf16_ctas_per_sm(d));
   return splits;
 }
 
@@ -438,7 +438,7 @@ size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
   if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return 0;
   if (H == Hkv) return plx_decode_workspace_bytes(B, H, L, d);
   int splits = 1, chunk = 0;
-  decode_split_plan(B, Hkv, L, num_sms_or_default(), &splits, &chunk, decode_gqa_ctas_per_sm(H / Hkv));
+  decode_split_plan(B, Hkv, L, num_sms_or_default(), &splits, &chunk, decode_gqa_ctas_per_sm(H / Hkv, d));
   if (splits <= 1) return 0;
   return sizeof(float) * (size_t)B * H * (size_t)splits * (size_t)(2 * d + 4);
 }
@@ -478,7 +478,7 @@ static int decode_gqa_impl(const void* q, const void* r, const void* Kcache, con
   a.status = dc->status;
   a.window = window < L ? window : 0;
   decode_split_plan(B, Hkv, a.window > 0 ? a.window : L, dc->num_sms, &a.splits, &a.chunk,
-                    decode_gqa_ctas_per_sm(G));
+                    decode_gqa_ctas_per_sm(G, d));
   if (a.splits > 1) {
     const size_t need = sizeof(float) * (size_t)B * H * (size_t)a.splits * (size_t)(2 * d + 4);
     if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;

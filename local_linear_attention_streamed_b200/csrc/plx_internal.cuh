@@ -70,11 +70,17 @@ cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms
 // d in {64, 128}: K/V blocks staged by TMA, the q and rho rows of the heads of
 // a group in one MMA tile.
 cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms);
+// Decode on tcgen05 (d = 128; G = H / Hkv in {1, 2, 4, 8}); called by
+// launch_decode_gqa and, with Hkv = H, by launch_decode_bf16.
+cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_sms);
 // Split heuristic shared by the launcher and the workspace-size query;
 // ctas_per_sm is how many CTAs of the decode kernel an SM holds.
 void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk, int ctas_per_sm = 2);
-// CTAs per SM of the grouped-KV decode kernel for group size G.
-inline int decode_gqa_ctas_per_sm(int G) { return G == 8 ? 1 : 2; }
+// CTAs per SM of the grouped-KV decode kernels for group size G and head dim
+// d: the tensor-core kernel (d = 128) holds an SM alone.
+inline int decode_gqa_ctas_per_sm(int G, int d) { return (d == 128 || G == 8) ? 1 : 2; }
+// CTAs per SM of the ungrouped bf16 decode for head dim d (the split plan's input).
+inline int decode_bf16_ctas_per_sm(int d) { return d == 128 ? 1 : 2; }
 
 // bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
 bool prefill_tc_supported(int d);

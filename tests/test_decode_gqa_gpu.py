@@ -142,3 +142,24 @@ def test_gqa_full_size_sampled(plx, H, Hkv):
         got.append(out[b, h].double().cpu().numpy())
     assert rel_err_rms(np.stack(got), np.stack(want)) <= BF16_TOL
     assert torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("G", [2, 4, 8])
+def test_gqa_rising_scores_rescale(plx, G):
+    """Scores that grow along the sequence (K rows scaled by 1 + 20 j / L): the
+    running max rises block after block, so the accumulated products are
+    rescaled many times (in the d = 128 kernel, in TMEM) before the last one;
+    one (b, KV head) with a single chunk and one split into chunks."""
+    B, Hkv, L, d = 2, 2, 2048, 128
+    H = G * Hkv
+    specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
+    dev, ref = small_inputs(90 + G, specs, synth.BF16)
+    ramp = 1.0 + 20.0 * np.arange(L) / L
+    Kh = (ref["K"] * ramp[None, None, :, None])
+    dev["K"] = torch.from_numpy(Kh).to(torch.bfloat16).cuda()
+    ref["K"] = dev["K"].to(torch.float64).cpu().numpy()
+    sl_host = np.array([L, 1500], dtype=np.int32)
+    out = plx.decode_gqa(dev["q"], dev["r"], dev["K"], dev["V"], torch.from_numpy(sl_host).cuda())
+    assert plx.get_device_status() == 0
+    want = oracle.decode_gqa_ref(ref["q"], ref["r"], ref["K"], ref["V"], sl_host)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
