@@ -1,7 +1,7 @@
-// Split-KV Parallax decode for bf16 caches with d = 64 on warp-level MMAs
-// (d = 128 runs the tcgen05 decode of decode_gqa_tc.cu, which this file's
-// launcher calls with one KV head per query head), and the split plan both
-// use.
+// Split-KV Parallax decode for bf16 caches, d in {64, 128}, on warp-level
+// MMAs, and the split plan.  At d = 128 the launcher hands sizes whose units
+// carry enough keys (decode_bf16_tc) to the tcgen05 decode of
+// decode_gqa_tc.cu, with one KV head per query head.
 //
 // One decode query per (b, h) is HBM-bound: every cached key and value is read
 // once (8d flops per key against 4d bytes).  The kernel therefore optimises the
@@ -432,20 +432,29 @@ void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk
 }
 
 cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms) {
-  if (a.d == 128) {  // the tensor-core decode, one KV head per query head
+  const int keys = (a.window > 0 && a.window < a.L) ? a.window : a.L;
+  if (decode_bf16_tc((long long)a.B * a.H, keys, a.d)) {  // the tensor-core decode, Hkv = H
     DecodeArgs g = a;
     g.Hkv = a.H;
     return launch_decode_gqa_tc(g, st, num_sms);
   }
-  if (a.d != 64) return cudaErrorInvalidValue;
   long long units = (long long)a.B * a.H * a.splits;
   int per_sm = 0;
-  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_bf16_kernel<64>, kThreads, 0);
+  cudaError_t e;
+  if (a.d == 128) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_bf16_kernel<128>, kThreads, 0);
+  } else {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_bf16_kernel<64>, kThreads, 0);
+  }
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
   long long grid = (long long)num_sms * per_sm;
   if (grid > units) grid = units;
-  decode_bf16_kernel<64><<<(unsigned)grid, kThreads, 0, st>>>(a);
+  if (a.d == 128) {
+    decode_bf16_kernel<128><<<(unsigned)grid, kThreads, 0, st>>>(a);
+  } else {
+    decode_bf16_kernel<64><<<(unsigned)grid, kThreads, 0, st>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -79,8 +79,22 @@ void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk
 // CTAs per SM of the grouped-KV decode kernels for group size G and head dim
 // d: the tensor-core kernel (d = 128) holds an SM alone.
 inline int decode_gqa_ctas_per_sm(int G, int d) { return (d == 128 || G == 8) ? 1 : 2; }
-// CTAs per SM of the ungrouped bf16 decode for head dim d (the split plan's input).
-inline int decode_bf16_ctas_per_sm(int d) { return d == 128 ? 1 : 2; }
+// Which kernel serves the ungrouped bf16 decode of bh (b, h) pairs with
+// `keys` visible keys per query (L, or the window) and head dim d: the
+// tensor-core kernel (one CTA per SM) once units carry enough keys to hide its
+// per-unit start-up and merge, else the warp-MMA kernel (two CTAs per SM),
+// which wins on short sequences and on few of them (the decode sweep, H = 16,
+// lengths uniform on [L/2, L]).  A pure function of the sizes, so that the
+// split plan, the workspace size and the launch agree.
+inline bool decode_bf16_tc(long long bh, int keys, int d) {
+  if (d != 128) return false;
+  if (keys >= 16384) return true;
+  if (keys >= 2048) return bh >= 256;
+  if (keys >= 1024) return bh >= 512 && bh <= 2048;
+  return false;
+}
+// CTAs per SM of that kernel (the split plan's input).
+inline int decode_bf16_ctas_per_sm(long long bh, int keys, int d) { return decode_bf16_tc(bh, keys, d) ? 1 : 2; }
 
 // bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
 bool prefill_tc_supported(int d);

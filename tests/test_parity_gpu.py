@@ -192,6 +192,30 @@ def test_bf16_decode_repeatable_and_user_workspace(plx):
     assert rel_err_rms(a, want) <= BF16_TOL
 
 
+def test_bf16_decode_tensor_core_sizes_every_output(plx):
+    """Sizes the tensor-core decode serves (256 (b, h) pairs, 2048 keys):
+    every output, lengths at the 128-key block edges (1, 127, 128, 129, 2047,
+    2048, ...) and NaN in the cache past every length, which must not leak."""
+    B, H, L, d = 16, 16, 2048, 128
+    specs = synth.decode_specs(B, H, L, d)
+    dev, ref = small_inputs(25, specs, synth.BF16)
+    seqlens = np.array([1, 2, 127, 128, 129, 255, 256, 257, 1000, 1023, 1024, 1025, 2046, 2047, 2048, 640],
+                       dtype=np.int32)
+    for b in range(B):
+        dev["K"][b, :, seqlens[b]:] = float("nan")
+        dev["V"][b, :, seqlens[b]:] = float("nan")
+    out = plx.decode(dev["q"], dev["r"], dev["K"], dev["V"], torch.from_numpy(seqlens).cuda())
+    assert plx.get_device_status() == 0
+    assert torch.isfinite(out).all()
+    want = oracle.decode_ref(ref["q"], ref["r"], ref["K"], ref["V"], seqlens)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+    # The sliding-window form over the same cache (the last 1500 keys).
+    outw = plx.decode_window(dev["q"], dev["r"], dev["K"], dev["V"], torch.from_numpy(seqlens).cuda(), 1500)
+    assert plx.get_device_status() == 0
+    wantw = oracle.decode_ref(ref["q"], ref["r"], ref["K"], ref["V"], seqlens, window=1500)
+    assert rel_err_rms(to_f64(outw), wantw) <= BF16_TOL
+
+
 def test_fp32_decode(plx):
     B, H, L, d = 3, 2, 300, 64
     got, want, status = _decode_small(plx, 23, B, H, L, d, [300, 1, 157], dtype=synth.F32)

@@ -51,18 +51,15 @@ def test_noalloc_matches_regular_decode_on_two_calls():
             assert free == free_after_first
 
 
-def test_noalloc_scratch_holds_every_split_plan():
-    """The fixed scratch (8 MiB: 128 KiB of counters, the rest partial records)
-    holds the records of every split plan on this device: the split plan only
-    cuts keys into chunks when the (b, h) pairs alone leave the last wave of
-    CTAs underfilled, which bounds B H S.  The size check that returns
-    PLX_ERR_WORKSPACE guards devices with other SM counts."""
+def test_noalloc_rejects_sizes_beyond_its_scratch():
     from local_linear_attention_streamed_b200 import plx
-    cap = (8 << 20) - (128 << 10)
-    for d in (64, 128):
-        for L in (256, 1024, 4096, 65536):
-            for bh in list(range(1, 600)) + list(range(600, 32769, 37)):
-                S = plx.lib.plx_decode_num_splits(bh, 1, L, d)
-                assert S >= 1
-                if S > 1:
-                    assert bh * S * (2 * d + 4) * 4 <= cap and bh * 4 <= (128 << 10), (d, L, bh, S)
+    B, H, L, d = 250, 16, 1024, 128  # 4000 (b, h) x 3 splits of fp32 records > 8 MiB
+    S = plx.lib.plx_decode_num_splits(B, H, L, d)
+    assert S > 1 and B * H * S * (2 * d + 4) * 4 > (8 << 20) - (128 << 10)
+    small = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    sl = torch.ones(B, dtype=torch.int32, device="cuda")
+    rc = plx.lib.plx_decode_noalloc(small.data_ptr(), small.data_ptr(), small.data_ptr(),
+                                    small.data_ptr(), sl.data_ptr(), small.data_ptr(), B, H, L, d,
+                                    None)
+    assert rc == -5
+    assert plx.get_device_status() == 0
