@@ -23,6 +23,8 @@
 // TMEM (512 columns): one S stage (S1 at 0, S2 at 64: 64 fp32 columns each),
 // two P buffers at 128 and 192 (bf16 pairs: bf16(w) in columns 0..31 and
 // bf16(w (t - c)) in 32..63), O1 at 256 and O2 at 384 (128 fp32 columns each).
+// At D = 64, O1 and O2 take 256..383 and a second S stage sits at 384 (one
+// stage per softmax warpgroup).
 // The scores of block g+1 are computed as soon as the softmax has loaded those
 // of block g into registers, and the value MMAs of block g read P buffer g % 2,
 // so the tensor pipe runs ahead of the softmax by a block instead of waiting
@@ -108,8 +110,9 @@ struct Smem {
   // together, and the stage frees once that block's value MMAs completed.
   uint64_t kv_full[kStages], kv_empty[kStages];
   // Block g's scores complete on s_full[g % 2] (the barrier of the softmax
-  // warpgroup that owns the block); its P on p_full[g % 2].
-  uint64_t s_full[2], s_free, p_full[2];
+  // warpgroup that owns the block); its P on p_full[g % 2].  The S stage goes
+  // back to the score issuer on s_free[0] (one stage) or s_free[g % 2] (two).
+  uint64_t s_full[2], s_free[2], p_full[2];
   uint64_t o_full, o_empty, drain;
   // Row state handed from the owner of block g to the owner of block g + 1:
   // (running max, centre, the poster's own sum w, its own sum w (t - c)) in
@@ -191,6 +194,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   constexpr bool kWin = kMode == 1, kSparse = kMode == 2;
+  // At D = 64, O1 and O2 end at column 384, so a second S stage fits in TMEM
+  // (columns 384..511): each softmax warpgroup then has its own, and the
+  // scores of block g + 1 need not wait until the owner of block g has read
+  // its scores.  At D = 128 the 512 columns hold one stage.
+  constexpr bool kTwoS = D == 64;
+  static_assert(!kTwoS || kColO1 + 2 * D <= 384, "second S stage above O1, O2");
   // Rows that may see no key in a block (window or block sparsity) need the
   // guards for an empty running max.
   constexpr bool kRobust = kMode != 0;
@@ -221,7 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);  // the owning warpgroup's threads
     }
-    mbar_init(&sm.s_free, 4);  // one lane of each warp of the owning warpgroup
+    mbar_init(&sm.s_free[0], 4);  // one lane of each warp of the owning warpgroup
+    mbar_init(&sm.s_free[1], 4);
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(&sm.tile_full[s], 1);
       mbar_init(&sm.tile_empty[s], 10);  // both MMA threads and one lane of each softmax warp
@@ -321,8 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           // wait on the critical path comes last, right before the issue.
           const uint32_t st = g % kStages;
           if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
-          if (g > 0 && !(ok = mbar_wait(&sm.s_free, (g - 1) & 1, abort, p.status))) break;
+          if constexpr (kTwoS) {
+            if (g > 1 && !(ok = mbar_wait(&sm.s_free[g & 1], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
+          } else {
+            if (g > 0 && !(ok = mbar_wait(&sm.s_free[0], (g - 1) & 1, abort, p.status))) break;
+          }
           tc_fence_after();
+          const uint32_t sst = kTwoS ? (g & 1) * 384u : 0u;  // the S stage of block g
           const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
           // S1 and S2 k-steps interleaved (one B tile feeds both GEMMs); every
           // MMA comes from the descriptors built once plus a compile-time
@@ -332,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int ks = 0; ks < D / 16; ++ks) {
             const uint64_t off = (uint64_t)((((ks >> 2) * kHalfQ) + (ks & 3) * 32) >> 4);
             const uint64_t koff = (uint64_t)((((ks >> 2) * kHalfKV) + (ks & 3) * 32) >> 4);
-            mma_ss(tmem + kColS1, dQ + off, dk + koff, kIdescS, ks > 0);
-            mma_ss(tmem + kColS2, dR + off, dk + koff, kIdescS, ks > 0);
+            mma_ss(tmem + kColS1 + sst, dQ + off, dk + koff, kIdescS, ks > 0);
+            mma_ss(tmem + kColS2 + sst, dR + off, dk + koff, kIdescS, ks > 0);
           }
           mma_commit(&sm.s_full[g & 1]);
           if (j + 1 == ti.nblk) mma_commit(&sm.q_empty);
@@ -509,14 +524,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int kb = kblock(ti, j) * kBN;
         uint32_t x[64], y[64];
-        tmem_ld32(sb + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tmem_ld32(sb + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tmem_ld32(sb + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
-        tmem_ld32(sb + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
+        const uint32_t ss = sb + (kTwoS ? (uint32_t)wg * 384u : 0u);  // this block's S stage
+        tmem_ld32(ss + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
+        tmem_ld32(ss + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
+        tmem_ld32(ss + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
+        tmem_ld32(ss + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free);  // the S stage goes back to the MMA
+        if (lane == 0) mbar_arrive(&sm.s_free[kTwoS ? wg : 0]);  // the S stage goes back to the MMA
         if ((p.causal && kb + kBN - 1 > ti.m * kBM) || kb + kBN > p.N ||
             (kWin && kb < ti.m * kBM + kBM - window)) {
           // Block-uniform: only blocks that cross the diagonal, the end or the
