@@ -520,24 +520,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = rendezvous())) break;
         if (sm.last) {
           __threadfence();
-#pragma unroll 1
+          // One pass over the chunks with a running max, every head's record
+          // of a chunk loaded at once: one L2 round trip per chunk, not one
+          // per value.
+          float Mg[G], om[G], TT[G], p1[G], p2[G];
+#pragma unroll
           for (int h = 0; h < G; ++h) {
-            const long long bh = bh0 + h;
-            const float* base = a.partials + bh * a.splits * (2 * kD + 4);
-            float Mg = -CUDART_INF_F;
-            for (int cc = 0; cc < x.nch; ++cc) Mg = fmaxf(Mg, __ldcg(base + (long long)cc * (2 * kD + 4)));
-            float om = 0.f, TT = 0.f, p1 = 0.f, p2 = 0.f;
-            for (int cc = 0; cc < x.nch; ++cc) {
-              const float* rc = base + (long long)cc * (2 * kD + 4);
-              const float mc = __ldcg(rc);
-              const float sc = (mc == -CUDART_INF_F) ? 0.f : exp2f(mc - Mg);
-              om += sc * __ldcg(rc + 1);
-              TT += sc * __ldcg(rc + 2);
-              p1 += sc * __ldcg(rc + 4 + r);
-              p2 += sc * __ldcg(rc + 4 + kD + r);
+            Mg[h] = -CUDART_INF_F;
+            om[h] = TT[h] = p1[h] = p2[h] = 0.f;
+          }
+          for (int cc = 0; cc < x.nch; ++cc) {
+            float mc[G], oc[G], tcv[G], q1[G], q2[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float* rc = a.partials + ((bh0 + h) * a.splits + cc) * (2 * kD + 4);
+              mc[h] = __ldcg(rc);
+              oc[h] = __ldcg(rc + 1);
+              tcv[h] = __ldcg(rc + 2);
+              q1[h] = __ldcg(rc + 4 + r);
+              q2[h] = __ldcg(rc + 4 + kD + r);
             }
-            const float inv = 1.f / om;
-            out[bh * kD + r] = __float2bfloat16_rn(((1.f + TT * inv) * p1 - p2) * inv);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const float Mn = fmaxf(Mg[h], mc[h]);  // finite: every chunk holds a key
+              const float so = exp2f(Mg[h] - Mn), sc = exp2f(mc[h] - Mn);  // 2^-inf = 0 on the first
+              om[h] = so * om[h] + sc * oc[h];
+              TT[h] = so * TT[h] + sc * tcv[h];
+              p1[h] = so * p1[h] + sc * q1[h];
+              p2[h] = so * p2[h] + sc * q2[h];
+              Mg[h] = Mn;
+            }
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float inv = 1.f / om[h];
+            out[(bh0 + h) * kD + r] = __float2bfloat16_rn(((1.f + TT[h] * inv) * p1[h] - p2[h]) * inv);
           }
           if (r == 0) a.counters[x.bkv] = 0;
         }
