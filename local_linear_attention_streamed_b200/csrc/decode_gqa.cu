@@ -554,8 +554,11 @@ __global__ void __launch_bounds__(Cfg<D, G>::kThreads, Cfg<D, G>::kMinCtas)
             const long long bh = (long long)b * a.H + (long long)kvh * G + hh;
             const float* base = a.partials + bh * a.splits * (2 * D + 4);
             float Mg = -CUDART_INF_F;
+            // Several chunks' loads in flight per round trip.
+#pragma unroll 4
             for (int cc = 0; cc < nch; ++cc) Mg = fmaxf(Mg, __ldcg(base + (long long)cc * (2 * D + 4)));
             float om = 0.f, TT = 0.f, p1 = 0.f, p2 = 0.f;
+#pragma unroll 4
             for (int cc = 0; cc < nch; ++cc) {
               const float* r = base + (long long)cc * (2 * D + 4);
               const float mc = __ldcg(r);

@@ -368,8 +368,11 @@ __global__ void __launch_bounds__(kThreads) decode_bf16_kernel(DecodeArgs a) {
       __threadfence();
       const float* base = a.partials + (long long)bh * a.splits * (2 * D + 4);
       float Mg = -CUDART_INF_F;
+      // Several chunks' loads in flight per round trip.
+#pragma unroll 4
       for (int cc = 0; cc < nch; ++cc) Mg = fmaxf(Mg, __ldcg(base + (long long)cc * (2 * D + 4)));
       float om = 0.f, TT = 0.f, p1 = 0.f, p2 = 0.f;
+#pragma unroll 4
       for (int cc = 0; cc < nch; ++cc) {
         const float* r = base + (long long)cc * (2 * D + 4);
         float mc = __ldcg(r);
