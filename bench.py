@@ -594,7 +594,10 @@ def run_gpu(args, rank, world, dist):
                                    f"L={gL} d={gd} bf16, all seqlens {gL}",
                        "l2": f"inputs larger than L2 ({g_kv / 1e9:.2f} GB KV); no flush"},
             "roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(g_ach / peaks["hbm_gbs"], 4), "traffic": None,
+                         "unit": "GB/s", "frac": round(g_ach / peaks["hbm_gbs"], 4),
+                         "traffic": (traffic_from_profile("decode_gqa_B64_H32_Hkv8_L4096.json",
+                                                          kernel_hash("decode_gqa_tc.cu", "sm100.cuh"))
+                                     if (gB, gH, gHkv, gL, gd) == (64, 32, 8, 4096, 128) else None),
                          "peak_source": peak_src, "kernel": (f"decode_gqa_tc_kernel<{gH // gHkv}>" if gd == 128
                                     else f"decode_gqa_kernel<{gd}, {gH // gHkv}>"),
                          "algorithmic_bytes_per_launch": g_alg},
