@@ -77,7 +77,10 @@ def test_decode_gqa_rejects_bad_arguments(lib):
     assert lib.plx_decode_gqa(*ok, 1, 8, 2, 64, 96, None, 0, None) == -2
     assert lib.plx_decode_gqa(A, A, A, A + 8, A, A, 1, 8, 2, 64, 128, None, 0, None) == -3
     assert lib.plx_decode_gqa_workspace_bytes(1, 8, 3, 64, 128) == 0
-    S = lib.plx_decode_num_splits(1, 2, 8192, 128)  # groups of 4 and 2 keep two CTAs per SM
+    # Two (b, KV head) pairs over 8192 keys: the split plan takes the most
+    # chunks it allows (L / 256) for one or two CTAs per SM alike, so the
+    # ungrouped plan of the same pairs gives the grouped decode's count.
+    S = lib.plx_decode_num_splits(1, 2, 8192, 128)
     assert S > 1
     assert lib.plx_decode_gqa_workspace_bytes(1, 8, 2, 8192, 128) == 8 * S * (2 * 128 + 4) * 4
     assert lib.plx_decode_gqa_workspace_bytes(1, 16, 2, 8192, 128) > 0
