@@ -104,6 +104,12 @@ int plx_prefill_window(const void* Q, const void* K, const void* V, const void* 
 int plx_prefill_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
                     int Hkv, int N, int d, int causal, void* stream);
 
+/* plx_prefill_gqa with a sliding window of `window` keys (query i sees keys
+ * i - window + 1 .. i, as plx_prefill_window).  window >= 1, else
+ * PLX_ERR_INVALID_ARG. */
+int plx_prefill_gqa_window(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                           int Hkv, int N, int d, int window, void* stream);
+
 /*
  * Block-sparse causal prefill, bf16, d in {64, 128}: query i sees key j when
  * j <= i and block_mask[i / 128][j / 64] is non-zero (the pages list
@@ -167,6 +173,16 @@ int plx_prefill_train_gqa(const void* Q, const void* K, const void* V, const voi
                           float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal,
                           void* stream);
 
+/* The training forward in its general form: Hkv KV heads (as
+ * plx_prefill_train_gqa; Hkv = H for one KV head per query head) and a
+ * sliding window of `window` keys (0: none; a window implies the causal
+ * mask, and `causal` is then ignored).  Hkv >= 1 dividing H and window >= 0,
+ * else PLX_ERR_INVALID_ARG.  Every other plx_prefill_train* call is this one
+ * with some arguments fixed. */
+int plx_prefill_train_ex(const void* Q, const void* K, const void* V, const void* R, void* out, void* vbar,
+                         float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal, int window,
+                         void* stream);
+
 /* Bytes of the statistics workspace plx_prefill_bwd needs:
  * 16 * B * H * (N rounded up to a multiple of 128); 0 for invalid sizes. */
 size_t plx_prefill_bwd_workspace_bytes(int B, int H, int N, int d);
@@ -211,6 +227,15 @@ int plx_prefill_bwd_gqa(const void* Q, const void* K, const void* V, const void*
                         const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ, void* dK,
                         void* dV, void* dR, int B, int H, int Hkv, int N, int d, int causal, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/* The backward pass in its general form, for the tensors plx_prefill_train_ex
+ * saved with the same Hkv, causal and window (dK, dV [B, Hkv, N, d]).
+ * Hkv >= 1 dividing H and window >= 0, else PLX_ERR_INVALID_ARG; workspace
+ * as plx_prefill_bwd. */
+int plx_prefill_bwd_ex(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                       const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ, void* dK,
+                       void* dV, void* dR, int B, int H, int Hkv, int N, int d, int causal, int window,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * One decode step with split-KV: every (b, h) streams its cache rows

@@ -191,8 +191,8 @@ int plx_prefill_window(const void* Q, const void* K, const void* V, const void* 
   return prefill_impl(Q, K, V, R, out, B, H, N, d, 1, window, dtype, stream);
 }
 
-int plx_prefill_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
-                    int Hkv, int N, int d, int causal, void* stream) {
+static int prefill_gqa_impl(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                            int Hkv, int N, int d, int causal, int window, void* stream) {
   if (!Q || !K || !V || !R || !out) return PLX_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || Hkv < 1 || N < 1 || d < 1 || H % Hkv != 0) return PLX_ERR_INVALID_ARG;
   if (!prefill_tc_supported(d)) return PLX_ERR_UNSUPPORTED;
@@ -204,7 +204,19 @@ int plx_prefill_gqa(const void* Q, const void* K, const void* V, const void* R, 
   if ((rc = current_device(&dc)) != PLX_OK) return rc;
   PrefillArgs a{Q, K, V, R, out, B, H, N, d, causal ? 1 : 0, dc->status};
   a.Hkv = Hkv;
+  a.window = window < N ? window : 0;
   return cuda_rc(launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream), dc->num_sms));
+}
+
+int plx_prefill_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                    int Hkv, int N, int d, int causal, void* stream) {
+  return prefill_gqa_impl(Q, K, V, R, out, B, H, Hkv, N, d, causal, 0, stream);
+}
+
+int plx_prefill_gqa_window(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                           int Hkv, int N, int d, int window, void* stream) {
+  if (window < 1) return PLX_ERR_INVALID_ARG;
+  return prefill_gqa_impl(Q, K, V, R, out, B, H, Hkv, N, d, 1, window, stream);
 }
 
 int plx_prefill_block_sparse(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
@@ -288,6 +300,14 @@ int plx_prefill_train_window(const void* Q, const void* K, const void* V, const 
   return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, 1, window, stream);
 }
 
+int plx_prefill_train_ex(const void* Q, const void* K, const void* V, const void* R, void* out, void* vbar,
+                         float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal, int window,
+                         void* stream) {
+  if (Hkv < 1 || window < 0) return PLX_ERR_INVALID_ARG;
+  return prefill_train_impl(Q, K, V, R, out, vbar, lse, tbar, B, H, N, d, window > 0 ? 1 : causal, window, stream,
+                            Hkv);
+}
+
 int plx_prefill_train_gqa(const void* Q, const void* K, const void* V, const void* R, void* out, void* vbar,
                           float* lse, float* tbar, int B, int H, int Hkv, int N, int d, int causal,
                           void* stream) {
@@ -350,6 +370,15 @@ int plx_prefill_bwd_window(const void* Q, const void* K, const void* V, const vo
   if (window < 1) return PLX_ERR_INVALID_ARG;
   return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, 1, window, workspace,
                           workspace_bytes, stream);
+}
+
+int plx_prefill_bwd_ex(const void* Q, const void* K, const void* V, const void* R, const void* out,
+                       const void* vbar, const float* lse, const float* tbar, const void* dO, void* dQ, void* dK,
+                       void* dV, void* dR, int B, int H, int Hkv, int N, int d, int causal, int window,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (Hkv < 1 || window < 0) return PLX_ERR_INVALID_ARG;
+  return prefill_bwd_impl(Q, K, V, R, out, vbar, lse, tbar, dO, dQ, dK, dV, dR, B, H, N, d, window > 0 ? 1 : causal,
+                          window, workspace, workspace_bytes, stream, Hkv);
 }
 
 int plx_prefill_bwd_gqa(const void* Q, const void* K, const void* V, const void* R, const void* out,

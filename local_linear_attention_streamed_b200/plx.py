@@ -47,6 +47,9 @@ SIGNATURES = {
     "plx_prefill_train_window": (_i, [_vp] * 8 + [_i] * 5 + [_vp]),
     "plx_prefill_bwd_window": (_i, [_vp] * 13 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_prefill_train_gqa": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
+    "plx_prefill_train_ex": (_i, [_vp] * 8 + [_i] * 7 + [_vp]),
+    "plx_prefill_bwd_ex": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
+    "plx_prefill_gqa_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_prefill_bwd_gqa": (_i, [_vp] * 13 + [_i] * 6 + [_vp, _sz, _vp]),
     "plx_get_device_status": (_i, [_vp]),
     "plx_status_string": (ctypes.c_char_p, [_i]),
@@ -138,17 +141,23 @@ def prefill_window(Q, K, V, R, window: int, out=None, stream=None):
     return out
 
 
-def prefill_gqa(Q, K, V, R, causal: bool = True, out=None, stream=None):
-    """bf16 prefill with grouped KV heads: Q, R [B, H, N, d]; K, V [B, Hkv, N, d]."""
+def prefill_gqa(Q, K, V, R, causal: bool = True, out=None, stream=None, window=None):
+    """bf16 prefill with grouped KV heads: Q, R [B, H, N, d]; K, V [B, Hkv, N, d]
+    (``window``: the last W keys of each query, as prefill_window)."""
     B, H, N, d = Q.shape
     Hkv = K.shape[1]
     if K.shape != (B, Hkv, N, d) or V.shape != K.shape or R.shape != Q.shape:
         raise ValueError("K, V must be [B, Hkv, N, d] and R like Q")
     if out is None:
         out = torch.empty_like(Q)
-    rc = lib.plx_prefill_gqa(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
-                             B, H, Hkv, N, d, int(bool(causal)), _stream_ptr(stream))
-    _check(rc, "plx_prefill_gqa")
+    if window is None:
+        rc = lib.plx_prefill_gqa(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                 B, H, Hkv, N, d, int(bool(causal)), _stream_ptr(stream))
+        _check(rc, "plx_prefill_gqa")
+    else:
+        rc = lib.plx_prefill_gqa_window(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                        B, H, Hkv, N, d, int(window), _stream_ptr(stream))
+        _check(rc, "plx_prefill_gqa_window")
     return out
 
 
@@ -189,15 +198,12 @@ def decode_window(q, r, Kcache, Vcache, seqlens, window: int, out=None, workspac
     return out
 
 
-def _kv_heads(Q, K, V, window):
-    """KV heads of K and V ([B, Hkv, N, d], H a multiple of Hkv); grouping and
-    a window are not combined."""
+def _kv_heads(Q, K, V):
+    """KV heads of K and V ([B, Hkv, N, d], H a multiple of Hkv)."""
     B, H, N, d = Q.shape
     Hkv = K.shape[1]
     if K.shape != (B, Hkv, N, d) or V.shape != K.shape or Hkv < 1 or H % Hkv:
         raise ValueError("K, V must be [B, Hkv, N, d] with H a multiple of Hkv")
-    if Hkv != H and window is not None:
-        raise ValueError("grouped KV heads take no window")
     return Hkv
 
 
@@ -211,7 +217,7 @@ def prefill_train(Q, K, V, R, causal: bool = True, stream=None, window=None):
     include/plx.h).
     """
     B, H, N, d = Q.shape
-    Hkv = _kv_heads(Q, K, V, window)
+    Hkv = _kv_heads(Q, K, V)
     for n, t in (("K", K), ("V", V), ("R", R)):
         if t.dtype != Q.dtype:
             raise ValueError(f"{n} must match Q's dtype")
@@ -224,10 +230,10 @@ def prefill_train(Q, K, V, R, causal: bool = True, stream=None, window=None):
     lse = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     tbar = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
     if Hkv != H:
-        rc = lib.plx_prefill_train_gqa(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
-                                       _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, Hkv, N, d,
-                                       int(bool(causal)), _stream_ptr(stream))
-        _check(rc, "plx_prefill_train_gqa")
+        rc = lib.plx_prefill_train_ex(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                      _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, Hkv, N, d,
+                                      int(bool(causal)), 0 if window is None else int(window), _stream_ptr(stream))
+        _check(rc, "plx_prefill_train_ex")
     elif window is None:
         rc = lib.plx_prefill_train(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
                                    _dev(vbar, "vbar"), _dev(lse, "lse"), _dev(tbar, "tbar"), B, H, N, d,
@@ -255,7 +261,7 @@ def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, 
     its group's query heads.
     """
     B, H, N, d = Q.shape
-    Hkv = _kv_heads(Q, K, V, window)
+    Hkv = _kv_heads(Q, K, V)
     for n, t in (("K", K), ("V", V)):
         if t.dtype != torch.bfloat16:
             raise ValueError(f"{n} must be bf16")
@@ -276,8 +282,9 @@ def prefill_backward(Q, K, V, R, out, vbar, lse, tbar, dO, causal: bool = True, 
             _dev(lse, "lse"), _dev(tbar, "tbar"), _dev(dO, "dO"), _dev(dQ, "dQ"), _dev(dK, "dK"),
             _dev(dV, "dV"), _dev(dR, "dR"), B, H, N, d)
     if Hkv != H:
-        rc = lib.plx_prefill_bwd_gqa(*args[:14], H, Hkv, N, d, int(bool(causal)), ws, wsb, _stream_ptr(stream))
-        _check(rc, "plx_prefill_bwd_gqa")
+        rc = lib.plx_prefill_bwd_ex(*args[:14], H, Hkv, N, d, int(bool(causal)), 0 if window is None else int(window),
+                                    ws, wsb, _stream_ptr(stream))
+        _check(rc, "plx_prefill_bwd_ex")
     elif window is None:
         rc = lib.plx_prefill_bwd(*args, int(bool(causal)), ws, wsb, _stream_ptr(stream))
         _check(rc, "plx_prefill_bwd")
@@ -310,7 +317,7 @@ class ParallaxAttention(torch.autograd.Function):
 def parallax_attention(Q, K, V, R, causal: bool = True, window=None):
     """Differentiable bf16 Parallax attention over [B, H, N, d] (d in {64, 128});
     ``window`` (None or W >= 1) makes it the sliding-window prefill; K and V
-    may have fewer heads (grouped KV heads, no window)."""
+    may have fewer heads (grouped KV heads, with or without a window)."""
     return ParallaxAttention.apply(Q, K, V, R, causal, window)
 
 

@@ -248,8 +248,8 @@ def test_gqa_backward_rejects_bad_groups(plx):
     kv = torch.zeros((B, 4, N, d), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(ValueError):
         plx.prefill_train(q, kv, kv, q, True)
-    with pytest.raises(ValueError):
-        plx.prefill_train(q, kv[:, :3], kv[:, :3], q, True, window=16)
+    with pytest.raises(ValueError):  # K and V of different head counts
+        plx.prefill_train(q, kv, kv[:, :2].contiguous(), q, True)
 
 
 def test_gqa_backward_full_size_group(plx):
@@ -276,3 +276,27 @@ def test_gqa_backward_full_size_group(plx):
     got = [grads[0][b, hk * G:(hk + 1) * G], grads[1][b, hk:hk + 1], grads[2][b, hk:hk + 1],
            grads[3][b, hk * G:(hk + 1) * G]]
     _check_grads(got, [w[0] for w in want], where=(b, hk))
+
+
+@pytest.mark.parametrize("G,N,d,W", [(2, 300, 128, 37), (4, 320, 128, 128), (4, 260, 64, 64), (8, 200, 128, 150)])
+def test_gqa_window_prefill_and_backward(plx, G, N, d, W):
+    """Grouped KV heads with a sliding window: the inference prefill against
+    the oracle on the KV heads repeated over each group, the training forward
+    equal to it bit for bit, and every gradient element (dK, dV per KV head,
+    summed over the group) against the oracle's."""
+    B, Hkv = 1, 2
+    H = G * Hkv
+    dev, ref = small_inputs(1500 + 10 * G + W, _gqa_specs(B, H, Hkv, N, d), synth.BF16)
+    out = plx.prefill_gqa(dev["Q"], dev["K"], dev["V"], dev["R"], window=W)
+    assert plx.get_device_status() == 0
+    Kr, Vr = (np.repeat(ref[n], G, axis=1) for n in ("K", "V"))
+    want = oracle.prefill_ref(ref["Q"], Kr, Vr, ref["R"], window=W)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+    saved = plx.prefill_train(dev["Q"], dev["K"], dev["V"], dev["R"], True, window=W)
+    assert torch.equal(saved[0], out)
+    grads = plx.prefill_backward(dev["Q"], dev["K"], dev["V"], dev["R"], *saved, dev["dO"], True, window=W)
+    torch.cuda.synchronize()
+    assert plx.get_device_status() == 0
+    assert grads[1].shape == dev["K"].shape
+    wgrads = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], True, window=W)
+    _check_grads(grads, wgrads, where=(G, W))

@@ -239,3 +239,25 @@ def test_grouped_kv_gradients_match_finite_differences():
             xs[a][idx] = old
             g[idx] = (fp - fm) / (2 * h)
         assert np.max(np.abs(got[a] - g)) < 1e-7 * max(1.0, np.max(np.abs(g)))
+
+
+def test_grouped_window_gradients_are_the_repeated_heads_summed():
+    """Grouped KV heads under a sliding window: the gradients equal those of
+    the same problem with K and V repeated over each group (one KV head per
+    query head), dK and dV summed over the group's query heads."""
+    rng = np.random.default_rng(102)
+    B, H, Hkv, N, d, W = 1, 6, 2, 9, 3, 4
+    G = H // Hkv
+    Q, R, dO = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    K, V = rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hkv, N, d))
+    got = oracle.parallax_backward_ref(Q, K, V, R, dO, True, window=W)
+    Kr, Vr = np.repeat(K, G, axis=1), np.repeat(V, G, axis=1)
+    full = oracle.parallax_backward_ref(Q, Kr, Vr, R, dO, True, window=W)
+    np.testing.assert_allclose(got[0], full[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[3], full[3], rtol=0, atol=1e-12)
+    for a in (1, 2):
+        summed = full[a].reshape(B, Hkv, G, N, d).sum(axis=2)
+        np.testing.assert_allclose(got[a], summed, rtol=0, atol=1e-12)
+    # The window matters here: the causal gradients differ.
+    causal = oracle.parallax_backward_ref(Q, K, V, R, dO, True)
+    assert np.max(np.abs(causal[1] - got[1])) > 1e-3
