@@ -25,7 +25,8 @@
  *   - Scores are scaled by 1/sqrt(d); the probe term t = rho . k is not scaled.
  *   - causal != 0: query row i sees keys 0..i (diagonal included).  causal == 0:
  *     every row sees all N keys.
- *   - Every head has its own K and V (no grouping).
+ *   - Every head has its own K and V, except in the entry points that take Hkv
+ *     (grouped KV heads: query head h reads KV head h / (H / Hkv)).
  *   - out has the dtype of the inputs; arithmetic is fp32.
  *
  * Memory and ownership: every tensor pointer is a DEVICE pointer owned by the
@@ -369,6 +370,8 @@ int plx_layer_forward_fp8(const void* x, const void* WQ, const void* WK, const v
  * Waits for `stream`, then reads and clears this device's kernel status word.
  * Returns PLX_OK, or the first device-reported error since the last read
  * (PLX_ERR_BAD_SEQLEN, PLX_ERR_TIMEOUT), or PLX_ERR_CUDA if the wait failed.
+ * On PLX_ERR_TIMEOUT it also zeroes the library's decode arrival counters,
+ * which a decode whose waits ran out may have left above zero.
  */
 int plx_get_device_status(void* stream);
 

@@ -32,6 +32,9 @@
 
 #include <math_constants.h>
 
+#include <cstdlib>
+#include <cstring>
+
 namespace plx {
 namespace {
 
@@ -234,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < x.nblk; ++i, ++pos) {
           const int st = pos % kStages;
           if (!(ok = mbar_wait(&sm.kv_empty[st], ((pos / kStages) & 1) ^ 1, abort, a.status))) break;
+          // The failure-detection test withholds CTA 0's K/V: the MMA thread's
+          // bounded wait runs out and every role unwinds through the abort path.
+          if (a.inject_stall && blockIdx.x == 0) continue;
           mbar_expect_tx(&sm.kv_full[st], 4 * kKeys * 128);
           last_kv[st] = (int)(pos / kStages);
 #pragma unroll
@@ -584,7 +590,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int G>
-cudaError_t launch_g(const DecodeArgs& a, cudaStream_t st, int num_sms) {
+cudaError_t launch_g(const DecodeArgs& args, cudaStream_t st, int num_sms) {
+  // PLX_FAULT_INJECT=decode_stall makes one CTA's bounded waits run out (tests
+  // of the timeout status only).
+  DecodeArgs a = args;
+  const char* fi = getenv("PLX_FAULT_INJECT");
+  a.inject_stall = (fi != nullptr && strcmp(fi, "decode_stall") == 0) ? 1 : 0;
   CUtensorMap mK, mV, mQ, mR;
   const long long kv_rows = (long long)a.B * a.Hkv * a.L, q_rows = (long long)a.B * a.H;
   if (!make_map(&mK, a.K, kv_rows, kKeys, kD) || !make_map(&mV, a.V, kv_rows, kKeys, kD) ||

@@ -740,6 +740,12 @@ int plx_get_device_status(void* stream) {
     if (cudaMemcpy(dc->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return PLX_ERR_CUDA;
   }
+  if (word & kStatusTimeout) {
+    // A decode whose waits ran out may have left arrival counters of
+    // unfinished (b, KV head) pairs above zero: clear them for the next call.
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dc->counters && cudaMemset(dc->counters, 0, dc->counters_bytes) != cudaSuccess) return PLX_ERR_CUDA;
+  }
   if (word & kStatusBadSeqlen) return PLX_ERR_BAD_SEQLEN;
   if (word & kStatusTimeout) return PLX_ERR_TIMEOUT;
   return PLX_OK;

@@ -58,6 +58,7 @@ struct DecodeArgs {
   int* status;
   int Hkv;          // KV heads (grouped-KV decode only; H is a multiple of it)
   int window;       // sliding window: the last `window` keys of each sequence (0: all)
+  int inject_stall = 0;  // failure-detection test (tensor-core decode): CTA 0 never loads its K/V
 };
 
 // SIMT kernels: any d that is a multiple of 32 up to 128, f32 or bf16 storage.

@@ -1,6 +1,7 @@
 """Failure detection on the GPU without a fault.
 
-Every wait in the tcgen05 prefill kernel is bounded in time.  With
+Every wait in the tcgen05 prefill, backward and decode kernels is bounded in
+time.  With
 PLX_FAULT_INJECT=prefill_stall the TMA producer withholds the first Q/R tile,
 so a barrier that nothing will complete is waited on: the kernel must give up
 after its limit, report PLX_ERR_TIMEOUT through plx_get_device_status, free
@@ -50,3 +51,29 @@ def test_backward_timeout_is_reported_and_context_survives(monkeypatch):
     want = oracle.parallax_backward_ref(ref["Q"], ref["K"], ref["V"], ref["R"], ref["dO"], True)
     for g, w in zip(grads, want):
         assert rel_err_fro(to_f64(g), w) <= GRAD_TOL
+
+
+def test_decode_timeout_is_reported_and_context_survives(monkeypatch):
+    """PLX_FAULT_INJECT=decode_stall: CTA 0 of the tensor-core decode never
+    receives its K/V blocks; its bounded waits run out, the status word
+    reports the timeout, the library clears the arrival counters that the
+    unfinished (b, KV head) pairs left behind, and the next decode on the same
+    context (keys split into chunks, so the counters matter) is correct."""
+    import torch
+    from local_linear_attention_streamed_b200 import plx
+    B, Hkv, G, L, d = 1, 2, 4, 8192, 128
+    H = G * Hkv
+    specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
+    dev, ref = small_inputs(33, specs, synth.BF16)
+    sl_host = np.array([L - 5], dtype=np.int32)
+    sl = torch.from_numpy(sl_host).cuda()
+    assert plx.get_device_status() == 0
+    monkeypatch.setenv("PLX_FAULT_INJECT", "decode_stall")
+    plx.decode_gqa(dev["q"], dev["r"], dev["K"], dev["V"], sl)
+    assert plx.get_device_status() == -7  # PLX_ERR_TIMEOUT
+    monkeypatch.delenv("PLX_FAULT_INJECT")
+    want = oracle.decode_gqa_ref(ref["q"], ref["r"], ref["K"], ref["V"], sl_host)
+    for _ in range(2):
+        out = plx.decode_gqa(dev["q"], dev["r"], dev["K"], dev["V"], sl)
+        assert plx.get_device_status() == 0
+        assert rel_err_rms(to_f64(out), want) <= BF16_TOL
