@@ -63,8 +63,9 @@ typedef enum { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
 #define PLX_ERR_CUDA (-4)         /* a CUDA runtime/driver call or launch failed   */
 #define PLX_ERR_WORKSPACE (-5)    /* caller workspace smaller than required        */
 #define PLX_ERR_BAD_SEQLEN (-6)   /* device-reported: a seqlens[b] outside 1..L    */
-#define PLX_ERR_TIMEOUT (-7)      /* device-reported: a bounded wait gave up (tests force
-                                     it with the environment PLX_FAULT_INJECT=prefill_stall) */
+#define PLX_ERR_TIMEOUT (-7)      /* device-reported: a bounded wait gave up (tests force it
+                                     with the environment PLX_FAULT_INJECT=prefill_stall,
+                                     bwd_stall or decode_stall) */
 
 /* Name of the CUDA error behind this thread's last PLX_ERR_CUDA from a kernel
  * launch ("no error" if there was none).  Static string. */
