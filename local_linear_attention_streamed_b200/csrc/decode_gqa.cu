@@ -1,4 +1,6 @@
-// Split-KV Parallax decode with grouped KV heads, bf16 caches, d in {64, 128}.
+// Split-KV Parallax decode with grouped KV heads on warp-level MMAs, bf16
+// caches, d = 64 (the launcher hands d = 128 to the tcgen05 decode of
+// decode_gqa_tc.cu; the kernel template still takes D in {64, 128}).
 //
 // G = H / Hkv consecutive query heads read one KV head.  The pages' decode
 // packs the q and rho rows into one tensor-core tile so that one stream of K
