@@ -96,8 +96,11 @@ def test_layer_and_norm_rope_reject_bad_arguments(lib):
 
 
 def test_decode_split_plan(lib):
+    # Sizes on both sides of the kernel choice (tensor-core decode: one CTA
+    # per SM; warp-MMA decode: two), whose split plans differ.
     for (B, H, L) in [(64, 16, 4096), (1, 16, 32768), (2048, 16, 4096), (1, 1, 1), (3, 5, 1000),
-                      (1, 16, 128), (8, 16, 16384)]:
+                      (1, 16, 128), (8, 16, 16384), (64, 16, 1024), (256, 16, 1024), (16, 16, 2048),
+                      (8, 16, 2048), (1, 16, 16384), (3, 7, 20000)]:
         S = lib.plx_decode_num_splits(B, H, L, 128)
         assert 1 <= S <= max(1, L // 256) + 1
         ws = lib.plx_decode_workspace_bytes(B, H, L, 128)

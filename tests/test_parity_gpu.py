@@ -1,6 +1,6 @@
 """GPU parity: libplx.so against the float64 oracle on the same seeded inputs.
 
-Bars (stated with the method's spec workloads): fp32 inputs
+Bars: fp32 inputs
 max_e |g - o| / max(|o_e|, RMS(o)) <= 1e-5; bf16 inputs max |g - o| / RMS(o)
 <= 2e-2.  Small cases are compared element by element over every output;
 full-size workloads on sampled outputs that the oracle recomputes from the
