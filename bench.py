@@ -264,7 +264,7 @@ def run_gpu(args, rank, world, dist):
                 # The committed capture is of the default workload; other sizes report none.
                 "traffic": (traffic_from_profile("decode_bf16_B64_H16_L4096.json", src_hash)
                             if B == DECODE["B"] else None),
-                "peak_source": peak_src, "kernel": "decode_gqa_tc_kernel<1>",
+                "peak_source": peak_src, "kernel": "decode_gqa_tc_kernel<128, 1>",
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "frac_of_spec_8000": round(achieved / 8000.0, 4)}
 
@@ -598,7 +598,7 @@ def run_gpu(args, rank, world, dist):
                          "traffic": (traffic_from_profile("decode_gqa_B64_H32_Hkv8_L4096.json",
                                                           kernel_hash("decode_gqa_tc.cu", "sm100.cuh"))
                                      if (gB, gH, gHkv, gL, gd) == (64, 32, 8, 4096, 128) else None),
-                         "peak_source": peak_src, "kernel": (f"decode_gqa_tc_kernel<{gH // gHkv}>" if gd == 128
+                         "peak_source": peak_src, "kernel": (f"decode_gqa_tc_kernel<{gd}, {gH // gHkv}>" if gd == 128 or gHkv % 2 == 0
                                     else f"decode_gqa_kernel<{gd}, {gH // gHkv}>"),
                          "algorithmic_bytes_per_launch": g_alg},
             "gpu_launches": gsteps,

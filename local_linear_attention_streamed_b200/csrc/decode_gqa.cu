@@ -1,6 +1,7 @@
 // Split-KV Parallax decode with grouped KV heads on warp-level MMAs, bf16
-// caches, d = 64 (the launcher hands d = 128 to the tcgen05 decode of
-// decode_gqa_tc.cu; the kernel template still takes D in {64, 128}).
+// caches, d = 64 with an odd number of KV heads (the launcher hands d = 128,
+// and d = 64 with Hkv even, to the tcgen05 decode of decode_gqa_tc.cu; the
+// kernel template still takes D in {64, 128}).
 //
 // G = H / Hkv consecutive query heads read one KV head.  The pages' decode
 // packs the q and rho rows into one tensor-core tile so that one stream of K
@@ -644,7 +645,7 @@ cudaError_t launch_gqa(const DecodeArgs& a, const CUtensorMap& mK, const CUtenso
 
 cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms) {
   if (a.Hkv < 1 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
-  if (a.d == 128) return launch_decode_gqa_tc(a, st, num_sms);
+  if (decode_gqa_tc(a.Hkv, a.d)) return launch_decode_gqa_tc(a, st, num_sms);
   const long long rows = (long long)a.B * a.Hkv * a.L;
   if (rows + kBlk >= (1ll << 31)) return cudaErrorInvalidValue;
   CUtensorMap mK, mV;

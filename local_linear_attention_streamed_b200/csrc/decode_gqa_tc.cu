@@ -1,6 +1,7 @@
 // Split-KV Parallax decode on the tensor cores (tcgen05 MMAs with TMEM
-// accumulators, TMA staging), bf16 caches, d = 128, one KV head per query
-// head (G = 1) or grouped KV heads (G = H / Hkv in {2, 4, 8}).
+// accumulators, TMA staging), bf16 caches, d = 128 with one KV head per query
+// head (G = 1) or grouped KV heads (G = H / Hkv in {2, 4, 8}), and d = 64
+// with grouped KV heads taken two KV heads at a time (see "d = 64" below).
 //
 // G consecutive query heads read one KV head, so one pass over a KV head's
 // cache serves the whole group: the pages' decode packs the q and rho rows
@@ -26,6 +27,14 @@
 // partial records, by the last CTA to finish one (an arrival counter per
 // (b, KV head), left at zero).
 //
+// d = 64.  The value product needs 128 dims as its M, so a unit takes a pair
+// of KV heads (Hkv even): their 64-dim K (and V) blocks sit side by side as
+// the two 64-dim halves of one 128-dim tile, the q / rho operand is
+// block-diagonal (member p's rows 16p.. carry its heads' q and rho in half p
+// and zeros in the other half), so one score MMA (N = 32) gives both members'
+// scores, and the value product's lanes 0..63 / 64..127 are the two members'
+// dims, each reading its own member's weight columns.
+//
 // Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
 #include "plx_internal.cuh"
 #include "sm100.cuh"
@@ -40,22 +49,31 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kD = 128;          // head dim (the MMA M of the value product)
 constexpr int kKeys = 128;       // keys per staged block (the MMA M of the score product)
-constexpr int kStages = 3;       // K/V staging ring (64 KB per stage)
 constexpr int kUnitRing = 4;
 constexpr int kThreads = 256;    // warp 0 TMA, warp 1 MMA, warps 4..7 one key / one dim per thread
 constexpr int kFirstEw = 4;
 constexpr float kLazyTau = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Value-product columns: (w_hi, w_lo, wt_hi, wt_lo) per head, at least the
-// MMA's minimum N of 16 (the spare rows of W stay zero).
-template <int G>
-constexpr int kCols = 4 * G < 16 ? 16 : 4 * G;
-
-// TMEM columns: two 16-column score stages, then two value accumulators.
-constexpr uint32_t kColS = 0, kColO = 32, kTmemCols = 128;
+// Geometry per head dim D (the staged tiles are 128 dims wide either way):
+// KV heads per unit, rows of the q / rho operand (the score MMA's N), query
+// heads per unit, value-product columns ((w_hi, w_lo, wt_hi, wt_lo) per query
+// head, at least the MMA's minimum N of 16; spare rows of W stay zero), K/V
+// stages (64 KB each; two where the weight tiles are largest), and TMEM:
+// two score stages, then two value accumulators.
+template <int D, int G>
+struct Geo {
+  static constexpr int kPair = D == 64 ? 2 : 1;
+  static constexpr int kRows = 16 * kPair;
+  static constexpr int kHeads = G * kPair;
+  static constexpr int NW = 4 * kHeads < 16 ? 16 : 4 * kHeads;
+  static constexpr int kStages = (D == 64 && G == 8) ? 2 : 3;
+  static constexpr uint32_t kColS = 0, kColO = 2 * kRows;
+  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 128;
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(kColO + 2 * NW <= kTmemCols, "TMEM columns");
+};
 
 // Instruction descriptor (kind::f16): D f32, A and B bf16, M = 128, N = n;
 // a_mn / b_mn = 1 for an MN-major A / B operand.
@@ -70,12 +88,13 @@ __device__ __forceinline__ uint32_t sw128_elem(int row, int col) {
   return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2);
 }
 
-template <int G>
+template <int D, int G>
 struct Smem {
-  static constexpr int NW = kCols<G>;
-  uint8_t k[kStages][2][kKeys * 128];  // [128 keys x 64 dims] per 64-dim half
+  using Gm = Geo<D, G>;
+  static constexpr int NW = Gm::NW, kStages = Gm::kStages;
+  uint8_t k[kStages][2][kKeys * 128];  // [128 keys x 64 dims] per 64-dim half (d = 64: per member)
   uint8_t v[kStages][2][kKeys * 128];
-  uint8_t qr[2][2][16 * 128];          // per unit slot: [16 rows x 64 dims] per half
+  uint8_t qr[2][2][Gm::kRows * 128];   // per unit slot: [rows x 64 dims] per half
   uint8_t w[2][2][NW * 128];           // per block slot: [NW rows x 64 keys] per 64-key half
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t qr_full[2], qr_empty[2];
@@ -87,15 +106,16 @@ struct Smem {
   uint64_t drain;
   long long unit_ring[kUnitRing];
   int unit_n[kUnitRing];  // seqlens of the unit's batch row, read once by the producer
-  float red[2][4][G];   // per-warp block maxima of each head
-  float sums[4][2 * G]; // per-warp omega and T of each head
+  float red[2][4][Gm::kHeads];    // per-warp block maxima of each head
+  float sums[4][2 * Gm::kHeads];  // per-warp omega and T of each head
   int last;
   uint32_t tmem_base;
   int abort;
 };
 
-static_assert(sizeof(Smem<8>) + 1024 <= 227 * 1024, "shared memory of one CTA");
-static_assert(kColO + 2 * kCols<8> <= kTmemCols, "TMEM columns");
+static_assert(sizeof(Smem<128, 8>) + 1024 <= 227 * 1024 && sizeof(Smem<64, 8>) + 1024 <= 227 * 1024 &&
+                  sizeof(Smem<64, 4>) + 1024 <= 227 * 1024 && sizeof(Smem<64, 2>) + 1024 <= 227 * 1024,
+              "shared memory of one CTA");
 
 __device__ unsigned long long g_tc_unit_next;
 __device__ unsigned int g_tc_cta_done;
@@ -107,11 +127,12 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
+  static_assert(N % 16 == 0 && N <= 64, "accumulator width");
   if constexpr (N == 16) {
     tmem_ld16(taddr, v);
   } else {
-    static_assert(N == 32, "accumulator width");
-    tmem_ld32(taddr, v);
+#pragma unroll
+    for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
   }
 }
 template <int N>
@@ -125,18 +146,25 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)
   }
 }
 
-// What every role derives from a unit index.
+// What every role derives from a unit index: unit u covers KV heads
+// kvh .. kvh + kPair - 1 of batch row b (bkv = b Hkv + kvh) over key chunk c.
 struct Unit {
   int b, kvh, bkv, c, n, kbeg, kend, nch, nblk;
   bool bad;
 };
-__device__ __forceinline__ Unit unit_of(long long u, int n, const DecodeArgs& a) {
-  const int BKV = a.B * a.Hkv;
+// Batch row of unit u (units are chunk-major over the (b, KV-head group) pairs).
+__device__ __forceinline__ int unit_row(long long u, int kPair, const DecodeArgs& a) {
+  const int per_b = a.Hkv / kPair;
+  return (int)(u % ((long long)a.B * per_b)) / per_b;
+}
+__device__ __forceinline__ Unit unit_of(long long u, int n, int kPair, const DecodeArgs& a) {
+  const int per_b = a.Hkv / kPair, BU = a.B * per_b;
   Unit x;
-  x.c = (int)(u / BKV);
-  x.bkv = (int)(u - (long long)x.c * BKV);
-  x.b = x.bkv / a.Hkv;
-  x.kvh = x.bkv - x.b * a.Hkv;
+  x.c = (int)(u / BU);
+  const int bu = (int)(u - (long long)x.c * BU);
+  x.b = bu / per_b;
+  x.kvh = (bu - x.b * per_b) * kPair;
+  x.bkv = x.b * a.Hkv + x.kvh;
   x.n = n;
   x.bad = x.n < 1 || x.n > a.L;
   // Keys lo..n-1 (lo > 0 only with a sliding window), cut into chunks.
@@ -148,17 +176,21 @@ __device__ __forceinline__ Unit unit_of(long long u, int n, const DecodeArgs& a)
   return x;
 }
 
-template <int G>
+template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                          DecodeArgs a) {
-  constexpr int NW = kCols<G>;
+  using Gm = Geo<D, G>;
+  constexpr int NW = Gm::NW, kStages = Gm::kStages, kPair = Gm::kPair, kRows = Gm::kRows;
+  constexpr int kHeads = Gm::kHeads;
+  constexpr uint32_t kColS = Gm::kColS, kColO = Gm::kColO, kTmemCols = Gm::kTmemCols;
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem<G>& sm = *reinterpret_cast<Smem<G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<D, G>& sm =
+      *reinterpret_cast<Smem<D, G>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long units = (long long)a.B * a.Hkv * a.splits;
+  const long long units = (long long)a.B * (a.Hkv / kPair) * a.splits;
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
@@ -215,24 +247,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = ui % kUnitRing;
         if (!mbar_wait(&sm.unit_empty[slot], ((ui / kUnitRing) & 1) ^ 1, abort, a.status)) break;
         const long long uu = u < units ? u : -1;
-        const int n = uu < 0 ? 0 : a.seqlens[(int)(uu % (a.B * a.Hkv)) / a.Hkv];
+        const int n = uu < 0 ? 0 : a.seqlens[unit_row(uu, kPair, a)];
         sm.unit_ring[slot] = uu;
         sm.unit_n[slot] = n;
         mbar_arrive(&sm.unit_full[slot]);
         if (uu < 0) break;
         const long long next = (long long)gridDim.x + (long long)atomicAdd(&g_tc_unit_next, 1ull);
-        const Unit x = unit_of(uu, n, a);
+        const Unit x = unit_of(uu, n, kPair, a);
         const int qs = ui & 1;
         if (!mbar_wait(&sm.qr_empty[qs], ((ui >> 1) & 1) ^ 1, abort, a.status)) break;
         mbar_expect_tx(&sm.qr_full[qs], 2 * 2 * G * 128);
         last_qr[qs] = ui >> 1;
-        const int qrow = x.b * a.H + x.kvh * G;
+        // Two boxes of G rows x 64 dims each for q and for rho: the two
+        // 64-dim halves of one KV head's group (d = 128), or one box per
+        // member of the pair into its own half, at rows 16p (d = 64).
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_2d(sm.qr[qs][h], &tmQ, &sm.qr_full[qs], 64 * h, qrow);
-          tma_load_2d(sm.qr[qs][h] + 8 * 128, &tmR, &sm.qr_full[qs], 64 * h, qrow);
+          const int mem = kPair == 2 ? h : 0;
+          const int qrow = x.b * a.H + (x.kvh + mem) * G;
+          uint8_t* dst = sm.qr[qs][h] + 16 * mem * 128;
+          tma_load_2d(dst, &tmQ, &sm.qr_full[qs], kPair == 2 ? 0 : 64 * h, qrow);
+          tma_load_2d(dst + 8 * 128, &tmR, &sm.qr_full[qs], kPair == 2 ? 0 : 64 * h, qrow);
         }
-        const int row0 = x.bkv * a.L + x.kbeg;  // < 2^31 (checked by the launcher)
         bool ok = true;
         for (int i = 0; i < x.nblk; ++i, ++pos) {
           const int st = pos % kStages;
@@ -242,10 +278,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (a.inject_stall && blockIdx.x == 0) continue;
           mbar_expect_tx(&sm.kv_full[st], 4 * kKeys * 128);
           last_kv[st] = (int)(pos / kStages);
+          // The two 64-dim halves of the block: of one KV head (d = 128), or
+          // one per member of the pair (d = 64).  Rows < 2^31 (launcher check).
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], 64 * h, row0 + kKeys * i);
-            tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], 64 * h, row0 + kKeys * i);
+            const int row = (x.bkv + (kPair == 2 ? h : 0)) * a.L + x.kbeg + kKeys * i;
+            const int xc = kPair == 2 ? 0 : 64 * h;
+            tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], xc, row);
+            tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], xc, row);
           }
         }
         if (!ok) break;
@@ -270,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
         mbar_arrive(&sm.unit_empty[slot]);
         if (uu < 0) break;
-        const Unit x = unit_of(uu, n, a);
+        const Unit x = unit_of(uu, n, kPair, a);
         const int qs = ui & 1;
         if (!(ok = mbar_wait(&sm.qr_full[qs], (ui >> 1) & 1, abort, a.status))) break;
         if (x.nblk == 0) {
@@ -289,10 +329,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint64_t ak = sdesc(smem_u32(sm.k[st][0]), 16, 1024);
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
+          for (int ks = 0; ks < 128 / 16; ++ks) {  // the staged tiles are 128 dims wide
             const uint32_t oa = (ks >> 2) * (kKeys * 128) + (ks & 3) * 32;
-            const uint32_t ob2 = (ks >> 2) * (16 * 128) + (ks & 3) * 32;
-            mma_ss(tmem + kColS + 16 * sb, ak + (uint64_t)(oa >> 4), bq + (uint64_t)(ob2 >> 4), idesc(16, 0, 0),
+            const uint32_t ob2 = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
+            mma_ss(tmem + kColS + kRows * sb, ak + (uint64_t)(oa >> 4), bq + (uint64_t)(ob2 >> 4), idesc(kRows, 0, 0),
                    ks > 0 ? 1u : 0u);
           }
           mma_commit(&sm.s_full[sb]);
@@ -337,7 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- one key of every block (scores), one dim of the accumulator ----------------
     const int q = warp - kFirstEw, r = 32 * q + lane;
     const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
-    const float c_log2 = kLog2e / sqrtf((float)kD);
+    const float c_log2 = kLog2e / sqrtf((float)D);
+    // Thread r is key r of every block and, at the end of a unit, dim
+    // r % D of member r / D of the pair (d = 64) or dim r (d = 128).
+    const int mem = r / D, dim = r % D;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
     uint32_t pos = 0, blk = 0, ou = 0, rv = 0;
     // Rendezvous of the four key warps (bounded like every wait).
@@ -357,21 +400,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.unit_empty[slot]);
       if (uu < 0) break;
-      const Unit x = unit_of(uu, n, a);
+      const Unit x = unit_of(uu, n, kPair, a);
       if (x.bad) {
         if (x.c == 0) {
-          const long long bh0 = (long long)x.b * a.H + (long long)x.kvh * G;
+          const long long bh0 = (long long)x.b * a.H + (long long)(x.kvh + mem) * G;
 #pragma unroll
-          for (int h = 0; h < G; ++h) out[(bh0 + h) * kD + r] = __float2bfloat16(0.f);
+          for (int h = 0; h < G; ++h) out[(bh0 + h) * D + dim] = __float2bfloat16(0.f);
           if (r == 0) atomicOr(a.status, kStatusBadSeqlen);
         }
         continue;
       }
       if (x.nblk == 0) continue;
       const int ob = ou & 1;
-      float hm[G], hom[G], hT[G];
+      // Per query head of the unit (head hh: member hh / G, its head hh % G).
+      float hm[kHeads], hom[kHeads], hT[kHeads];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < kHeads; ++h) {
         hm[h] = -CUDART_INF_F;
         hom[h] = 0.f;
         hT[h] = 0.f;
@@ -381,23 +425,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = p % kStages, sb = bb & 1;
         if (!(ok = warp_wait(&sm.s_full[sb], (bb >> 1) & 1, abort, a.status))) break;
         tc_fence_after();
-        uint32_t sv[16];
-        tmem_ld16(lb + kColS + 16 * sb, sv);
+        uint32_t sv[kRows];
+        tmem_ld_cols<kRows>(lb + kColS + kRows * sb, sv);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[sb]);
         const int key = x.kbeg + kKeys * i + r;
         const bool valid = key < x.kend;
-        float xs[G], tv[G];
+        float xs[kHeads], tv[kHeads];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-          xs[h] = valid ? __uint_as_float(sv[h]) * c_log2 : -CUDART_INF_F;
-          tv[h] = valid ? __uint_as_float(sv[8 + h]) : 0.f;
+        for (int h = 0; h < kHeads; ++h) {  // q of head hh in column 16 (hh / G) + hh % G, rho 8 further
+          const int col = 16 * (h / G) + h % G;
+          xs[h] = valid ? __uint_as_float(sv[col]) * c_log2 : -CUDART_INF_F;
+          tv[h] = valid ? __uint_as_float(sv[col + 8]) : 0.f;
         }
         // Block max of every head over the four warps' keys.
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < kHeads; ++h) {
           float mx = xs[h];
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -407,9 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm.vote[sb]);
         if (!(ok = warp_wait(&sm.vote[sb], (bb >> 1) & 1, abort, a.status))) break;
         bool raised = false;
-        float alpha[G];
+        float alpha[kHeads];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < kHeads; ++h) {
           const float mblk = fmaxf(fmaxf(sm.red[sb][0][h], sm.red[sb][1][h]), fmaxf(sm.red[sb][2][h], sm.red[sb][3][h]));
           const bool up = mblk > hm[h] + kLazyTau;  // always on the unit's first block (m = -inf)
           alpha[h] = up ? exp2f(hm[h] - mblk) : 1.f;
@@ -427,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_cols<NW>(lb + kColO + NW * ob, ov);
           tc_wait_ld();
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
+          for (int h = 0; h < kHeads; ++h) {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) ov[4 * h + k4] = __float_as_uint(__uint_as_float(ov[4 * h + k4]) * alpha[h]);
           }
@@ -435,9 +480,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_wait_st();
           tc_fence_before();
         }
-        float wv[G];
+        float wv[kHeads];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < kHeads; ++h) {
           wv[h] = exp2f(xs[h] - hm[h]);
           hom[h] += wv[h];
           hT[h] += wv[h] * tv[h];
@@ -447,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* wt = sm.w[sb][r >> 6];
         const int kk = r & 63;
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+        for (int h = 0; h < kHeads; ++h) {
           const float w = wv[h], wtv = wv[h] * tv[h];
           const __nv_bfloat16 whi = __float2bfloat16_rn(w), thi = __float2bfloat16_rn(wtv);
           const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
@@ -474,7 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.w_full[sb]);
       }
       if (!ok) break;
-      // ---- End of the unit: the accumulator (thread r holds dim r) and the sums.
+      // ---- End of the unit: the accumulator (thread r holds dim `dim` of
+      // member `mem`) and the sums.
       if (!(ok = warp_wait(&sm.o_full[ob], (ou >> 1) & 1, abort, a.status))) break;
       tc_fence_after();
       uint32_t ov[NW];
@@ -484,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[ob]);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < kHeads; ++h) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
           hom[h] += __shfl_xor_sync(0xffffffffu, hom[h], o);
@@ -496,9 +542,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!(ok = rendezvous())) break;
+      // The unit's query heads are consecutive from bh0: head hh of the unit
+      // is query head bh0 + hh (member hh / G).
       const long long bh0 = (long long)x.b * a.H + (long long)x.kvh * G;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
+      for (int h = 0; h < kHeads; ++h) {
+        if (h / G != mem) continue;  // this thread's member (warp-uniform)
         const float om = (sm.sums[0][2 * h] + sm.sums[1][2 * h]) + (sm.sums[2][2 * h] + sm.sums[3][2 * h]);
         const float TT =
             (sm.sums[0][2 * h + 1] + sm.sums[1][2 * h + 1]) + (sm.sums[2][2 * h + 1] + sm.sums[3][2 * h + 1]);
@@ -507,16 +556,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long bh = bh0 + h;
         if (x.nch == 1) {
           const float inv = 1.f / om;
-          out[bh * kD + r] = __float2bfloat16_rn(((1.f + TT * inv) * o1 - o2) * inv);
+          out[bh * D + dim] = __float2bfloat16_rn(((1.f + TT * inv) * o1 - o2) * inv);
         } else {
-          float* rec = a.partials + (bh * a.splits + x.c) * (2 * kD + 4);
-          if (r == 0) {
+          float* rec = a.partials + (bh * a.splits + x.c) * (2 * D + 4);
+          if (dim == 0) {
             rec[0] = hm[h];
             rec[1] = om;
             rec[2] = TT;
           }
-          rec[4 + r] = o1;
-          rec[4 + kD + r] = o2;
+          rec[4 + dim] = o1;
+          rec[4 + D + dim] = o2;
         }
       }
       if (x.nch > 1) {
@@ -538,13 +587,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < x.nch; ++cc) {
             float mc[G], oc[G], tcv[G], q1[G], q2[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              const float* rc = a.partials + ((bh0 + h) * a.splits + cc) * (2 * kD + 4);
+            for (int h = 0; h < G; ++h) {  // this thread's member's heads
+              const float* rc = a.partials + ((bh0 + mem * G + h) * a.splits + cc) * (2 * D + 4);
               mc[h] = __ldcg(rc);
               oc[h] = __ldcg(rc + 1);
               tcv[h] = __ldcg(rc + 2);
-              q1[h] = __ldcg(rc + 4 + r);
-              q2[h] = __ldcg(rc + 4 + kD + r);
+              q1[h] = __ldcg(rc + 4 + dim);
+              q2[h] = __ldcg(rc + 4 + D + dim);
             }
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -560,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h = 0; h < G; ++h) {
             const float inv = 1.f / om[h];
-            out[(bh0 + h) * kD + r] = __float2bfloat16_rn(((1.f + TT[h] * inv) * p1[h] - p2[h]) * inv);
+            out[(bh0 + mem * G + h) * D + dim] = __float2bfloat16_rn(((1.f + TT[h] * inv) * p1[h] - p2[h]) * inv);
           }
           if (r == 0) a.counters[x.bkv] = 0;
         }
@@ -589,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int G>
+template <int D, int G>
 cudaError_t launch_g(const DecodeArgs& args, cudaStream_t st, int num_sms) {
   // PLX_FAULT_INJECT=decode_stall makes one CTA's bounded waits run out (tests
   // of the timeout status only).
@@ -598,29 +647,36 @@ cudaError_t launch_g(const DecodeArgs& args, cudaStream_t st, int num_sms) {
   a.inject_stall = (fi != nullptr && strcmp(fi, "decode_stall") == 0) ? 1 : 0;
   CUtensorMap mK, mV, mQ, mR;
   const long long kv_rows = (long long)a.B * a.Hkv * a.L, q_rows = (long long)a.B * a.H;
-  if (!make_map(&mK, a.K, kv_rows, kKeys, kD) || !make_map(&mV, a.V, kv_rows, kKeys, kD) ||
-      !make_map(&mQ, a.q, q_rows, G, kD) || !make_map(&mR, a.r, q_rows, G, kD))
+  if (!make_map(&mK, a.K, kv_rows, kKeys, D) || !make_map(&mV, a.V, kv_rows, kKeys, D) ||
+      !make_map(&mQ, a.q, q_rows, G, D) || !make_map(&mR, a.r, q_rows, G, D))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(Smem<G>) + 1024;
+  const size_t smem = sizeof(Smem<D, G>) + 1024;
+  static_assert(sizeof(Smem<D, G>) + 1024 <= 227 * 1024, "shared memory of one CTA");
   cudaError_t e =
-      cudaFuncSetAttribute(decode_gqa_tc_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaFuncSetAttribute(decode_gqa_tc_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long units = (long long)a.B * a.Hkv * a.splits;
+  const long long units = (long long)a.B * (a.Hkv / Geo<D, G>::kPair) * a.splits;
   const long long grid = units < num_sms ? units : num_sms;
-  decode_gqa_tc_kernel<G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, mQ, mR, a);
+  decode_gqa_tc_kernel<D, G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, mQ, mR, a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_sms) {
-  if (a.d != kD || a.Hkv < 1 || a.H % a.Hkv != 0) return cudaErrorInvalidValue;
+  if (a.Hkv < 1 || a.H % a.Hkv != 0 || !decode_gqa_tc(a.Hkv, a.d)) return cudaErrorInvalidValue;
   if ((long long)a.B * a.Hkv * a.L + kKeys >= (1ll << 31)) return cudaErrorInvalidValue;
   const int G = a.H / a.Hkv;
-  if (G == 1) return launch_g<1>(a, st, num_sms);
-  if (G == 2) return launch_g<2>(a, st, num_sms);
-  if (G == 4) return launch_g<4>(a, st, num_sms);
-  if (G == 8) return launch_g<8>(a, st, num_sms);
+  if (a.d == 128) {
+    if (G == 1) return launch_g<128, 1>(a, st, num_sms);
+    if (G == 2) return launch_g<128, 2>(a, st, num_sms);
+    if (G == 4) return launch_g<128, 4>(a, st, num_sms);
+    if (G == 8) return launch_g<128, 8>(a, st, num_sms);
+  } else {
+    if (G == 2) return launch_g<64, 2>(a, st, num_sms);
+    if (G == 4) return launch_g<64, 4>(a, st, num_sms);
+    if (G == 8) return launch_g<64, 8>(a, st, num_sms);
+  }
   return cudaErrorInvalidValue;
 }
 

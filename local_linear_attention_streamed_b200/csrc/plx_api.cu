@@ -467,7 +467,8 @@ size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d) {
   if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return 0;
   if (H == Hkv) return plx_decode_workspace_bytes(B, H, L, d);
   int splits = 1, chunk = 0;
-  decode_split_plan(B, Hkv, L, num_sms_or_default(), &splits, &chunk, decode_gqa_ctas_per_sm(H / Hkv, d));
+  decode_split_plan(B, Hkv / decode_gqa_kv_per_unit(Hkv, d), L, num_sms_or_default(), &splits, &chunk,
+                    decode_gqa_ctas_per_sm(H / Hkv, Hkv, d));
   if (splits <= 1) return 0;
   return sizeof(float) * (size_t)B * H * (size_t)splits * (size_t)(2 * d + 4);
 }
@@ -506,8 +507,8 @@ static int decode_gqa_impl(const void* q, const void* r, const void* Kcache, con
   a.d = d;
   a.status = dc->status;
   a.window = window < L ? window : 0;
-  decode_split_plan(B, Hkv, a.window > 0 ? a.window : L, dc->num_sms, &a.splits, &a.chunk,
-                    decode_gqa_ctas_per_sm(G, d));
+  decode_split_plan(B, Hkv / decode_gqa_kv_per_unit(Hkv, d), a.window > 0 ? a.window : L, dc->num_sms, &a.splits,
+                    &a.chunk, decode_gqa_ctas_per_sm(G, Hkv, d));
   if (a.splits > 1) {
     const size_t need = sizeof(float) * (size_t)B * H * (size_t)a.splits * (size_t)(2 * d + 4);
     if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;

@@ -77,9 +77,13 @@ cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_s
 // Split heuristic shared by the launcher and the workspace-size query;
 // ctas_per_sm is how many CTAs of the decode kernel an SM holds.
 void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk, int ctas_per_sm = 2);
-// CTAs per SM of the grouped-KV decode kernels for group size G and head dim
-// d: the tensor-core kernel (d = 128) holds an SM alone.
-inline int decode_gqa_ctas_per_sm(int G, int d) { return (d == 128 || G == 8) ? 1 : 2; }
+// The grouped-KV decode runs on the tensor-core kernel at d = 128, and at
+// d = 64 with groups of 2, 4 or 8 when Hkv is even (two KV heads per unit);
+// otherwise on the warp-MMA kernel.  KV heads per unit and CTAs per SM of the
+// kernel that runs (the split plan's inputs).
+inline bool decode_gqa_tc(int Hkv, int d) { return d == 128 || (d == 64 && Hkv % 2 == 0); }
+inline int decode_gqa_kv_per_unit(int Hkv, int d) { return (d == 64 && Hkv % 2 == 0) ? 2 : 1; }
+inline int decode_gqa_ctas_per_sm(int G, int Hkv, int d) { return (decode_gqa_tc(Hkv, d) || G == 8) ? 1 : 2; }
 // Which kernel serves the ungrouped bf16 decode of bh (b, h) pairs with
 // `keys` visible keys per query (L, or the window) and head dim d: the
 // tensor-core kernel (one CTA per SM) once units carry enough keys to hide its

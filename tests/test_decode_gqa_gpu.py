@@ -38,14 +38,16 @@ def test_gqa_small_ragged(plx, d, G, Hkv):
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("G", [2, 4, 8])
-def test_gqa_split_keys(plx, G):
-    """Few (b, KV head) pairs and long contexts: keys split into chunks merged in-kernel."""
-    B, Hkv, L, d = 1, 2, 8192, 128
+def test_gqa_split_keys(plx, G, d):
+    """Few (b, KV head) pairs and long contexts: keys split into chunks merged
+    in-kernel (at d = 64 the two KV heads form one unit of the tensor-core kernel)."""
+    B, Hkv, L = 1, 2, 8192
     H = G * Hkv
     assert plx.lib.plx_decode_num_splits(B, Hkv, L, d) > 1
     specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
-    dev, ref = small_inputs(60 + G, specs, synth.BF16)
+    dev, ref = small_inputs(60 + G + d, specs, synth.BF16)
     sl_host = np.array([L - 37], dtype=np.int32)
     out = plx.decode_gqa(dev["q"], dev["r"], dev["K"], dev["V"], torch.from_numpy(sl_host).cuda())
     assert plx.get_device_status() == 0
@@ -83,9 +85,10 @@ def test_gqa_group_of_one_is_the_ungrouped_decode(plx):
     assert torch.equal(a, b)
 
 
-def test_gqa_cache_past_seqlen_never_leaks(plx):
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa_cache_past_seqlen_never_leaks(plx, d):
     """NaN in the cache past each sequence's length must not reach the outputs."""
-    B, Hkv, G, L, d = 3, 2, 8, 320, 128
+    B, Hkv, G, L = 3, 2, 8, 320
     H = G * Hkv
     specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
     dev, ref = small_inputs(73, specs, synth.BF16)
@@ -100,8 +103,9 @@ def test_gqa_cache_past_seqlen_never_leaks(plx):
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
 
 
-def test_gqa_bad_seqlen_reports_and_zeroes(plx):
-    B, Hkv, G, L, d = 3, 2, 4, 256, 128
+@pytest.mark.parametrize("d", [64, 128])
+def test_gqa_bad_seqlen_reports_and_zeroes(plx, d):
+    B, Hkv, G, L = 3, 2, 4, 256
     H = G * Hkv
     specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
     dev, ref = small_inputs(74, specs, synth.BF16)
@@ -144,16 +148,17 @@ def test_gqa_full_size_sampled(plx, H, Hkv):
     assert torch.isfinite(out).all()
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("G", [2, 4, 8])
-def test_gqa_rising_scores_rescale(plx, G):
+def test_gqa_rising_scores_rescale(plx, G, d):
     """Scores that grow along the sequence (K rows scaled by 1 + 20 j / L): the
     running max rises block after block, so the accumulated products are
     rescaled many times (in the d = 128 kernel, in TMEM) before the last one;
     one (b, KV head) with a single chunk and one split into chunks."""
-    B, Hkv, L, d = 2, 2, 2048, 128
+    B, Hkv, L = 2, 2, 2048
     H = G * Hkv
     specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
-    dev, ref = small_inputs(90 + G, specs, synth.BF16)
+    dev, ref = small_inputs(90 + G + d, specs, synth.BF16)
     ramp = 1.0 + 20.0 * np.arange(L) / L
     Kh = (ref["K"] * ramp[None, None, :, None])
     dev["K"] = torch.from_numpy(Kh).to(torch.bfloat16).cuda()
