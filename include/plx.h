@@ -313,11 +313,16 @@ size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d);
  * GPU that loads the library holds until the process exits.  Limits: when the
  * keys are split, B*H <= 32768 and B*H*splits*(2d+4)*4 bytes <= 8 MiB - 128 KiB
  * (splits = plx_decode_num_splits); larger sizes return PLX_ERR_WORKSPACE before
- * anything is launched.  No cudaMalloc, cudaFree or allocating library routine is
- * called.  The first call on a device looks up the array's device address (make
- * that first call before any stream capture); every call clears the counters with
- * an asynchronous memset on `stream`.  All calls share the one array, so calls
- * that overlap on the GPU (other streams, other threads) race: order them.
+ * anything is launched; sizes plx_decode_ex rejects (B*H > 2^24, B*H*L + 128 >=
+ * 2^31) return PLX_ERR_UNSUPPORTED here too.  No cudaMalloc, cudaFree or
+ * allocating library routine is called.  The first call on a device looks up the
+ * array's device address; under CUDA's lazy module loading (the default) that
+ * lookup is also what makes the driver load the array's module and reserve its
+ * 8 MiB on that device.  So make the first call on each device before the caller
+ * reserves the rest of device memory, and before any stream capture; later calls
+ * reserve nothing.  Every call clears the counters with an asynchronous memset on
+ * `stream`.  All calls share the one array, so calls that overlap on the GPU
+ * (other streams, other threads) race: order them.
  */
 int plx_decode_noalloc(const void* q, const void* r, const void* Kcache, const void* Vcache,
                        const int32_t* seqlens, void* out, int B, int H, int L, int d,
@@ -343,7 +348,11 @@ size_t plx_layer_workspace_bytes(int B, int N, int H, int d);
  *   o         = causal Parallax prefill over [B, H, N, d]
  *   y         = o W_O                          (o merged back to [B, N, H*d])
  * x, y: bf16 [B, N, H*d].  workspace: device memory of plx_layer_workspace_bytes()
- * bytes, or NULL for a library-owned one.
+ * bytes, 256-byte aligned, or NULL for a library-owned one.  A caller workspace
+ * is nine slots of round_up(B*N*H*d*2, 256) bytes; on return slots 4..7 hold the
+ * attention inputs q, k, v, rho and slot 8 the attention output, all bf16
+ * [B, H, N, d] (slots 0..3 hold the projections, slot 0 then the merged
+ * attention output), so a caller can inspect exactly what the prefill consumed.
  */
 int plx_layer_forward(const void* x, const void* WQ, const void* WK, const void* WV,
                       const void* WR, const void* WO, void* y, int B, int N, int H, int d,

@@ -47,6 +47,7 @@ extern "C" int plx_decode_noalloc(const void* q, const void* r, const void* Kcac
   if (!a16(q) || !a16(r) || !a16(Kcache) || !a16(Vcache) || !a16(out) ||
       (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_MISALIGNED;
+  if (!decode_sizes_supported(B, H, H, L)) return PLX_ERR_UNSUPPORTED;  // as plx_decode_ex
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

@@ -415,7 +415,7 @@ static int decode_impl(const void* q, const void* r, const void* Kcache, const v
   if (!aligned16(q) || !aligned16(r) || !aligned16(Kcache) || !aligned16(Vcache) ||
       !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_MISALIGNED;
-  if ((long long)B * H > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  if (!decode_sizes_supported(B, H, H, L)) return PLX_ERR_UNSUPPORTED;
   DeviceCache* dc = nullptr;
   if ((rc = current_device(&dc)) != PLX_OK) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -487,8 +487,7 @@ static int decode_gqa_impl(const void* q, const void* r, const void* Kcache, con
   if (!aligned16(q) || !aligned16(r) || !aligned16(Kcache) || !aligned16(Vcache) ||
       !aligned16(out) || (reinterpret_cast<uintptr_t>(seqlens) & 3u))
     return PLX_ERR_MISALIGNED;
-  if ((long long)B * H > (1ll << 24) || (long long)B * Hkv * L + 64 >= (1ll << 31))
-    return PLX_ERR_UNSUPPORTED;
+  if (!decode_sizes_supported(B, H, Hkv, L)) return PLX_ERR_UNSUPPORTED;
   int rc;
   DeviceCache* dc = nullptr;
   if ((rc = current_device(&dc)) != PLX_OK) return rc;

@@ -101,6 +101,14 @@ inline bool decode_bf16_tc(long long bh, int keys, int d) {
 // CTAs per SM of that kernel (the split plan's input).
 inline int decode_bf16_ctas_per_sm(long long bh, int keys, int d) { return decode_bf16_tc(bh, keys, d) ? 1 : 2; }
 
+// Sizes every decode entry point accepts: at most 2^24 query (b, h) pairs, and
+// cache rows (B * KV heads * L) that stay below 2^31 even after the largest
+// staged key block (128 keys) is added to the last row a unit can start at, so
+// that whichever decode kernel the sizes select can address them.
+inline bool decode_sizes_supported(int B, int H, int Hkv, int L) {
+  return (long long)B * H <= (1ll << 24) && (long long)B * Hkv * L + 128 < (1ll << 31);
+}
+
 // bf16 causal/full prefill on tcgen05 + TMA + TMEM, d == 128.
 bool prefill_tc_supported(int d);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st, int num_sms);

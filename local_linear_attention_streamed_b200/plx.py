@@ -410,6 +410,21 @@ def layer_forward(x, WQ, WK, WV, WR, WO, H: int, out=None, workspace=None, strea
     return out
 
 
+def layer_workspace_bytes(B: int, N: int, H: int, d: int) -> int:
+    return int(lib.plx_layer_workspace_bytes(B, N, H, d))
+
+
+def layer_workspace_views(workspace, B: int, N: int, H: int, d: int) -> dict:
+    """Views of a caller workspace after plx_layer_forward returned: the layer's
+    own bf16 attention inputs q, k, v, rho and its attention output, each
+    [B, H, N, d] (the slots the header lists)."""
+    slot = -(-(B * N * H * d * 2) // 256) * 256
+    assert workspace.dtype == torch.uint8 and workspace.numel() >= 9 * slot
+    def view(i):
+        return workspace[i * slot:i * slot + B * N * H * d * 2].view(torch.bfloat16).view(B, H, N, d)
+    return {"q": view(4), "k": view(5), "v": view(6), "rho": view(7), "attn": view(8)}
+
+
 def layer_forward_fp8(x, WQ, WK, WV, WR, WO, H: int, out=None, workspace=None, stream=None):
     """The layer of layer_forward with its five linears in dynamic per-tensor fp8 (e4m3)."""
     B, N, D = x.shape

@@ -68,6 +68,21 @@ def test_decode_rejects_bad_arguments(lib):
     assert lib.plx_decode_ex(A, A, A, A, A + 2, A, 1, 1, 8, 128, 1, None, 0, None) == -3
 
 
+def test_decode_size_bounds_are_shared(lib):
+    """Every decode entry point rejects the same oversized problems on the host:
+    more than 2^24 query (b, h) pairs, or cache rows (B * KV heads * L) that
+    reach 2^31 once a 128-key block is added."""
+    ok = [A] * 6
+    big_bh = (1 << 24) // 16 + 1
+    assert lib.plx_decode_ex(*ok, big_bh, 16, 8, 128, 1, None, 0, None) == -2
+    assert lib.plx_decode_noalloc(*ok, big_bh, 16, 8, 128, None) == -2
+    rows_L = ((1 << 31) - 128) // 64       # B * Hkv = 64: B*Hkv*L + 128 just reaches 2^31
+    assert lib.plx_decode_ex(*ok, 4, 16, rows_L, 128, 1, None, 0, None) == -2
+    assert lib.plx_decode_noalloc(*ok, 4, 16, rows_L, 128, None) == -2
+    assert lib.plx_decode_gqa(*ok, 4, 64, 16, rows_L, 128, None, 0, None) == -2
+    assert lib.plx_decode_window(*ok, 4, 64, 16, rows_L, 128, 1024, 1, None, 0, None) == -2
+
+
 def test_decode_gqa_rejects_bad_arguments(lib):
     ok = [A] * 6
     assert lib.plx_decode_gqa(A, A, A, A, None, A, 1, 8, 2, 64, 128, None, 0, None) == -1

@@ -366,6 +366,43 @@ def test_config_layer_full_size_sampled(plx):
     assert torch.isfinite(y).all()
 
 
+def test_config_layer_attention_stage_full_size(plx):
+    """The attention stage of the layer workload (B=4, N=8192, 16 heads of 128)
+    held to the attention bar: the bf16 q, k, v, rho the layer itself produced
+    (read back from a caller workspace) go to the oracle, whose rows must match
+    the layer's own attention output within BF16_TOL.  Then plx_prefill on the
+    same tensors must reproduce that output bit for bit."""
+    B, N, D, H = 4, 8192, 2048, 16
+    d = D // H
+    seed = 1005
+    specs = synth.layer_specs(B, N, D)
+    dev = device_inputs(seed, specs, synth.BF16)
+    ws = torch.empty(plx.layer_workspace_bytes(B, N, H, d), dtype=torch.uint8, device="cuda")
+    y = plx.layer_forward(dev["x"], dev["WQ"], dev["WK"], dev["WV"], dev["WR"], dev["WO"], H,
+                          workspace=ws)
+    assert plx.get_device_status() == 0
+    assert torch.isfinite(y).all()
+    v = plx.layer_workspace_views(ws, B, N, H, d)
+    attn = v["attn"].clone()
+    again = plx.prefill(v["q"], v["k"], v["v"], v["rho"], causal=True)
+    assert plx.get_device_status() == 0
+    assert torch.equal(again, attn)
+    rows = [0, 1, 2, 63, 64, 127, 128, 129, 4095, 4096, 8064, 8190, 8191]
+    rng = np.random.default_rng(55)
+    got, want = [], []
+    for (b, h) in [(0, 0), (1, 7), (3, 15)]:
+        extra = [int(i) for i in rng.integers(0, N, size=6)]
+        Kh, Vh = to_f64(v["k"][b, h]), to_f64(v["v"][b, h])
+        qh, rh = to_f64(v["q"][b, h]), to_f64(v["rho"][b, h])
+        ah = to_f64(attn[b, h])
+        for i in rows + extra:
+            want.append(oracle.parallax_row(qh[i], rh[i], Kh[:i + 1], Vh[:i + 1]))
+            got.append(ah[i])
+    assert rel_err_rms(np.stack(got), np.stack(want)) <= BF16_TOL
+    del dev, ws, attn, again
+    torch.cuda.empty_cache()
+
+
 # ---------------------------------------------------------------------------
 # Prefill with grouped KV heads.
 # ---------------------------------------------------------------------------
