@@ -300,6 +300,38 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
 size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d);
 
 /*
+ * Writes an fp8 (e4m3) KV cache: every row of X (bf16 [rows, d], d in {64, 128})
+ * gets its own fp32 scale s = max|x| / 448 (scales[row]) and d codes
+ * e4m3(x / s) (codes [rows, d], one byte each; round to nearest even, both
+ * divisions in IEEE fp32); an all-zero row gets s = 0 and zero codes.  The row
+ * then stands for code * s.  This is the reading of the pages' dynamic fp8
+ * (rainbus.top summary, reproduction notes: dynamic fp8 precision) for a cache
+ * that grows a token at a time: each appended key or value row is quantised on
+ * its own, so rows = B*Hkv*L for a whole cache or the new rows of one step.
+ * X and codes 16-byte aligned, scales 4-byte aligned; device memory, caller-owned.
+ */
+int plx_kv_quantize_fp8(const void* X, void* codes, float* scales, long long rows, int d, void* stream);
+
+/* Workspace plx_decode_fp8kv needs for its partial records (0 if keys are not split). */
+size_t plx_decode_fp8kv_workspace_bytes(int B, int H, int Hkv, int L, int d);
+
+/*
+ * One decode step over an e4m3 KV cache written by plx_kv_quantize_fp8: the
+ * result of plx_decode_gqa over the cache values code * scale (rainbus.top
+ * summary, 方法步骤详情: the streamed S1/S2, O1/O2 form; out = ((1 + T/omega) O1
+ * - O2) / omega).  q, r, out: bf16 [B, H, d]; Kcodes, Vcodes: e4m3 [B, Hkv, L, d];
+ * Kscales, Vscales: fp32 [B, Hkv, L]; seqlens: int32 [B] in 1..L (others write
+ * zeros and report PLX_ERR_BAD_SEQLEN).  Query head h reads KV head h / (H/Hkv),
+ * groups of 1, 2, 4 or 8; d = 128, else PLX_ERR_UNSUPPORTED.  It reads
+ * 2 * (d + 4) bytes per cached row instead of the bf16 decode's 4 d.
+ * workspace: plx_decode_fp8kv_workspace_bytes() bytes, 256-byte aligned, or NULL
+ * for a library-owned one.  Pointers 16-byte aligned (scales and seqlens 4).
+ */
+int plx_decode_fp8kv(const void* q, const void* r, const void* Kcodes, const float* Kscales,
+                     const void* Vcodes, const float* Vscales, const int32_t* seqlens, void* out, int B,
+                     int H, int Hkv, int L, int d, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * plx_decode_noalloc — one bf16 decode step that allocates nothing.
  * (The paper has no counterpart: this is a deployment variant of plx_decode_ex.)
  *

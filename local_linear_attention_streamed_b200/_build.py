@@ -24,8 +24,8 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompi
 LIBS = {
     "libplx.so": {
         "srcs": ["plx_api.cu", "simt.cu", "decode_mma.cu", "prefill_tc.cu", "norm_rope.cu",
-                 "decode_noalloc.cu", "decode_gqa.cu", "decode_gqa_tc.cu", "backward_tc.cu", "fp8_linear.cu"],
-        "deps": ["plx_internal.cuh", "sm100.cuh"],
+                 "decode_noalloc.cu", "decode_gqa.cu", "decode_gqa_tc.cu", "backward_tc.cu", "fp8_linear.cu", "decode_fp8kv.cu"],
+        "deps": ["plx_internal.cuh", "sm100.cuh", "decode_tc_common.cuh"],
         "link": ["-lcublas", "-lcublasLt", f"-Xlinker", f"-rpath={os.path.join(CUDA_HOME, 'lib64')}"],
     },
     "libplx_synth.so": {

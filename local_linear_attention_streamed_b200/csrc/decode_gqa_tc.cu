@@ -38,6 +38,7 @@
 // Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
 #include "plx_internal.cuh"
 #include "sm100.cuh"
+#include "decode_tc_common.cuh"
 
 #include <math_constants.h>
 
@@ -48,8 +49,8 @@ namespace plx {
 namespace {
 
 using namespace sm100;
+using namespace dtc;
 
-constexpr int kKeys = 128;       // keys per staged block (the MMA M of the score product)
 constexpr int kUnitRing = 4;
 constexpr int kThreads = 256;    // warp 0 TMA, warp 1 MMA, warps 4..7 one key / one dim per thread
 constexpr int kFirstEw = 4;
@@ -74,19 +75,6 @@ struct Geo {
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(kColO + 2 * NW <= kTmemCols, "TMEM columns");
 };
-
-// Instruction descriptor (kind::f16): D f32, A and B bf16, M = 128, N = n;
-// a_mn / b_mn = 1 for an MN-major A / B operand.
-__host__ __device__ constexpr uint32_t idesc(int n, int a_mn, int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
-         ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
-}
-
-// Byte offset of element column `col` (bf16) of row `row` in a 128B-swizzled
-// tile of 128-byte rows.
-__device__ __forceinline__ uint32_t sw128_elem(int row, int col) {
-  return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7))) << 4) + (col & 7) * 2);
-}
 
 template <int D, int G>
 struct Smem {
@@ -119,62 +107,6 @@ static_assert(sizeof(Smem<128, 8>) + 1024 <= 227 * 1024 && sizeof(Smem<64, 8>) +
 
 __device__ unsigned long long g_tc_unit_next;
 __device__ unsigned int g_tc_cta_done;
-
-// Bounded wait taken by a whole warp: every lane leaves with the same answer.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, status));
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
-  static_assert(N % 16 == 0 && N <= 64, "accumulator width");
-  if constexpr (N == 16) {
-    tmem_ld16(taddr, v);
-  } else {
-#pragma unroll
-    for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
-  }
-}
-template <int N>
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[N]) {
-#pragma unroll
-  for (int c = 0; c < N / 16; ++c) {
-    uint32_t part[16];
-#pragma unroll
-    for (int x = 0; x < 16; ++x) part[x] = v[16 * c + x];
-    tmem_st16(taddr + 16 * c, part);
-  }
-}
-
-// What every role derives from a unit index: unit u covers KV heads
-// kvh .. kvh + kPair - 1 of batch row b (bkv = b Hkv + kvh) over key chunk c.
-struct Unit {
-  int b, kvh, bkv, c, n, kbeg, kend, nch, nblk;
-  bool bad;
-};
-// Batch row of unit u (units are chunk-major over the (b, KV-head group) pairs).
-__device__ __forceinline__ int unit_row(long long u, int kPair, const DecodeArgs& a) {
-  const int per_b = a.Hkv / kPair;
-  return (int)(u % ((long long)a.B * per_b)) / per_b;
-}
-__device__ __forceinline__ Unit unit_of(long long u, int n, int kPair, const DecodeArgs& a) {
-  const int per_b = a.Hkv / kPair, BU = a.B * per_b;
-  Unit x;
-  x.c = (int)(u / BU);
-  const int bu = (int)(u - (long long)x.c * BU);
-  x.b = bu / per_b;
-  x.kvh = (bu - x.b * per_b) * kPair;
-  x.bkv = x.b * a.Hkv + x.kvh;
-  x.n = n;
-  x.bad = x.n < 1 || x.n > a.L;
-  // Keys lo..n-1 (lo > 0 only with a sliding window), cut into chunks.
-  const int lo = (!x.bad && a.window > 0 && x.n > a.window) ? x.n - a.window : 0;
-  x.kbeg = lo + x.c * a.chunk;
-  x.kend = x.bad ? x.kbeg : min(x.kbeg + a.chunk, x.n);
-  x.nblk = (!x.bad && x.kbeg < x.n) ? (x.kend - x.kbeg + kKeys - 1) / kKeys : 0;
-  x.nch = x.bad ? 0 : (x.n - lo + a.chunk - 1) / a.chunk;
-  return x;
-}
 
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1)

@@ -535,6 +535,74 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
                          stream);
 }
 
+int plx_kv_quantize_fp8(const void* X, void* codes, float* scales, long long rows, int d, void* stream) {
+  if (!X || !codes || !scales || rows < 1) return PLX_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u)) return PLX_ERR_MISALIGNED;
+  DeviceCache* dc = nullptr;
+  int rc = current_device(&dc);
+  if (rc != PLX_OK) return rc;
+  return cuda_rc(launch_kv_quantize_fp8(X, codes, scales, rows, d, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t plx_decode_fp8kv_workspace_bytes(int B, int H, int Hkv, int L, int d) {
+  if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return 0;
+  int splits = 1, chunk = 0;
+  decode_split_plan(B, Hkv, L, num_sms_or_default(), &splits, &chunk, 1);
+  if (splits <= 1) return 0;
+  return sizeof(float) * (size_t)B * H * (size_t)splits * (size_t)(2 * d + 4);
+}
+
+int plx_decode_fp8kv(const void* q, const void* r, const void* Kcodes, const float* Kscales, const void* Vcodes,
+                     const float* Vscales, const int32_t* seqlens, void* out, int B, int H, int Hkv, int L, int d,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !r || !Kcodes || !Kscales || !Vcodes || !Vscales || !seqlens || !out) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || L < 1 || d < 1 || H % Hkv != 0) return PLX_ERR_INVALID_ARG;
+  const int G = H / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return PLX_ERR_UNSUPPORTED;
+  if (d != 128) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(r) || !aligned16(Kcodes) || !aligned16(Vcodes) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(Kscales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(Vscales) & 3u))
+    return PLX_ERR_MISALIGNED;
+  if (!decode_sizes_supported(B, H, Hkv, L)) return PLX_ERR_UNSUPPORTED;
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  DecodeArgs a{};
+  a.q = q;
+  a.r = r;
+  a.K = Kcodes;
+  a.V = Vcodes;
+  a.Kscale = Kscales;
+  a.Vscale = Vscales;
+  a.seqlens = seqlens;
+  a.out = out;
+  a.B = B;
+  a.H = H;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.d = d;
+  a.status = dc->status;
+  decode_split_plan(B, Hkv, L, dc->num_sms, &a.splits, &a.chunk, 1);
+  if (a.splits > 1) {
+    const size_t need = sizeof(float) * (size_t)B * H * (size_t)a.splits * (size_t)(2 * d + 4);
+    if (workspace && workspace_bytes < need) return PLX_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLX_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((rc = grow(&dc->counters, &dc->counters_bytes, sizeof(int) * (size_t)B * Hkv, st)) != PLX_OK) return rc;
+    a.counters = static_cast<int*>(dc->counters);
+    if (workspace) {
+      a.partials = static_cast<float*>(workspace);
+    } else {
+      if ((rc = grow(&dc->decode_ws, &dc->decode_ws_bytes, need, st)) != PLX_OK) return rc;
+      a.partials = static_cast<float*>(dc->decode_ws);
+    }
+  }
+  return cuda_rc(launch_decode_fp8kv(a, st, dc->num_sms));
+}
+
 size_t plx_decode_window_workspace_bytes(int B, int H, int Hkv, int L, int d, int window) {
   if (window < 1) return 0;
   const int Leff = window < L ? window : L;

@@ -59,6 +59,10 @@ struct DecodeArgs {
   int Hkv;          // KV heads (grouped-KV decode only; H is a multiple of it)
   int window;       // sliding window: the last `window` keys of each sequence (0: all)
   int inject_stall = 0;  // failure-detection test (tensor-core decode): CTA 0 never loads its K/V
+  // e4m3 caches (decode_fp8kv): K and V hold one byte per element, and these
+  // fp32 [B*Hkv*L] arrays the scale of every cached row.
+  const float* Kscale = nullptr;
+  const float* Vscale = nullptr;
 };
 
 // SIMT kernels: any d that is a multiple of 32 up to 128, f32 or bf16 storage.
@@ -74,6 +78,11 @@ cudaError_t launch_decode_gqa(const DecodeArgs& a, cudaStream_t st, int num_sms)
 // Decode on tcgen05 (d = 128; G = H / Hkv in {1, 2, 4, 8}); called by
 // launch_decode_gqa and, with Hkv = H, by launch_decode_bf16.
 cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_sms);
+// Decode over an e4m3 cache with per-row scales (d = 128, G = H / Hkv in {1, 2, 4, 8}).
+cudaError_t launch_decode_fp8kv(const DecodeArgs& a, cudaStream_t st, int num_sms);
+// Per-row dynamic e4m3 quantisation of bf16 cache rows [rows, d] (d in {64, 128}).
+cudaError_t launch_kv_quantize_fp8(const void* X, void* codes, float* scales, long long rows, int d,
+                                   cudaStream_t st);
 // Split heuristic shared by the launcher and the workspace-size query;
 // ctas_per_sm is how many CTAs of the decode kernel an SM holds.
 void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk, int ctas_per_sm = 2);

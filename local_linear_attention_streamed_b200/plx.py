@@ -51,6 +51,9 @@ SIGNATURES = {
     "plx_prefill_bwd_ex": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
     "plx_prefill_gqa_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_prefill_bwd_gqa": (_i, [_vp] * 13 + [_i] * 6 + [_vp, _sz, _vp]),
+    "plx_kv_quantize_fp8": (_i, [_vp, _vp, _vp, ctypes.c_longlong, _i, _vp]),
+    "plx_decode_fp8kv_workspace_bytes": (_sz, [_i] * 5),
+    "plx_decode_fp8kv": (_i, [_vp] * 8 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_get_device_status": (_i, [_vp]),
     "plx_status_string": (ctypes.c_char_p, [_i]),
     "plx_last_cuda_error": (ctypes.c_char_p, []),
@@ -379,6 +382,42 @@ def decode_gqa(q, r, Kcache, Vcache, seqlens, out=None, workspace=None, stream=N
                             _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, Hkv, L, d,
                             ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(rc, "plx_decode_gqa")
+    return out
+
+
+def kv_quantize_fp8(X, codes=None, scales=None, stream=None):
+    """Per-row dynamic e4m3 quantisation of bf16 cache rows X[..., d]:
+    returns (codes uint8 [..., d], scales float32 [...])."""
+    d = X.shape[-1]
+    rows = X.numel() // d
+    if codes is None:
+        codes = torch.empty(X.shape, dtype=torch.uint8, device=X.device)
+    if scales is None:
+        scales = torch.empty(X.shape[:-1], dtype=torch.float32, device=X.device)
+    rc = lib.plx_kv_quantize_fp8(_dev(X, "X"), _dev(codes, "codes"), _dev(scales, "scales"), rows, d,
+                                 _stream_ptr(stream))
+    _check(rc, "plx_kv_quantize_fp8")
+    return codes, scales
+
+
+def decode_fp8kv_workspace_bytes(B: int, H: int, Hkv: int, L: int, d: int) -> int:
+    return int(lib.plx_decode_fp8kv_workspace_bytes(B, H, Hkv, L, d))
+
+
+def decode_fp8kv(q, r, Kcodes, Kscales, Vcodes, Vscales, seqlens, out=None, workspace=None, stream=None):
+    """Decode over an e4m3 cache: q, r bf16 [B, H, d]; codes uint8 [B, Hkv, L, d];
+    scales float32 [B, Hkv, L]; seqlens int32 [B]."""
+    B, H, d = q.shape
+    Hkv, L = Kcodes.shape[1], Kcodes.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        ws_ptr, ws_bytes = _dev(workspace, "workspace"), workspace.numel() * workspace.element_size()
+    rc = lib.plx_decode_fp8kv(_dev(q, "q"), _dev(r, "r"), _dev(Kcodes, "Kcodes"), _dev(Kscales, "Kscales"),
+                              _dev(Vcodes, "Vcodes"), _dev(Vscales, "Vscales"), _dev(seqlens, "seqlens"),
+                              _dev(out, "out"), B, H, Hkv, L, d, ws_ptr, ws_bytes, _stream_ptr(stream))
+    _check(rc, "plx_decode_fp8kv")
     return out
 
 
