@@ -11,7 +11,9 @@ under "prefill", a layer step (projections, RMSNorm+RoPE, attention) under
 "layer", and the grouped-KV decode B=64, H=32, Hkv=8, L=4096, d=128 in GB/s
 under "decode_gqa", the training forward plus backward pass of the
 prefill workload under "prefill.backward", and sliding windows of 1024 keys on
-the prefill and decode workloads under "window".  For N > 1 GPUs (launched by torchrun) every rank runs the
+the prefill and decode workloads under "window", the decode over an e4m3 KV
+cache (the decode workload's shape and groups of 4) under "decode_fp8kv", and
+five cells of the decode sweep under "decode_sweep".  For N > 1 GPUs (launched by torchrun) every rank runs the
 same per-GPU workload on its own seeded inputs with no data-path collective
 (weak scaling); time is the max over ranks.
 
@@ -50,6 +52,8 @@ LAYER = dict(B=4, N=8192, D=2048, H=16)
 SWEEP_B = [1, 8, 64, 256, 1024, 2048]
 SWEEP_L = [128, 1024, 4096, 16384, 32768]
 SWEEP_MAX_BYTES = 150e9
+# Sweep cells in the default line: few long sequences, mid-size and large batches, short contexts.
+SWEEP_SUBSET = [(1, 32768), (8, 4096), (64, 1024), (256, 16384), (2048, 128)]
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -606,6 +610,59 @@ def run_gpu(args, rank, world, dist):
         del gt
         torch.cuda.empty_cache()
 
+    # ---- Decode over an e4m3 KV cache: the decode workload's shape, and groups of 4.
+    fp8kv = None
+    if not args.no_fp8kv:
+        fp8kv = {}
+        for (fB, fH, fHkv, fL, fd) in [(DECODE["B"], DECODE["H"], DECODE["H"], DECODE["L"], DECODE["d"]),
+                                       tuple(DECODE_GQA[k] for k in ("B", "H", "Hkv", "L", "d"))]:
+            fspecs = synth.decode_gqa_specs(fB, fH, fHkv, fL, fd)
+            ft = {}
+            for name, spec in fspecs.items():
+                ft[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+                synth.device_fill(ft[name].data_ptr(), synth.BF16, seed + 6, spec)
+            Kc, Ks = plx.kv_quantize_fp8(ft["K"])
+            Vc, Vs = plx.kv_quantize_fp8(ft["V"])
+            del ft["K"], ft["V"]
+            fsl = torch.full((fB,), fL, dtype=torch.int32, device=dev)
+            fout = torch.empty_like(ft["q"])
+
+            def fdec():
+                plx.decode_fp8kv(ft["q"], ft["r"], Kc, Ks, Vc, Vs, fsl, out=fout)
+
+            fsteps = max(1, args.steps // 2)
+            f_total, f_per = timed(fdec, fsteps, max(3, args.warmup // 2), stream, dist)
+            if plx.get_device_status() != 0:
+                raise RuntimeError("fp8-cache decode reported a device error")
+            f_total = max_over_ranks(f_total, dist)
+            f_kv = fB * fHkv * fL * (fd + 4) * 2          # codes and scales of K and V
+            f_alg = f_kv + 3 * fB * fH * fd * 2           # + q, r, out
+            f_ms = float(np.mean(f_per))
+            f_ach = f_alg / (f_ms * 1e-3) / 1e9
+            keys = fB * fHkv * fL
+            entry = {
+                "metric": "fp8-cache decode KV GB/s", "unit": "GB/s",
+                "value": round(sum_over_ranks(f_kv * fsteps, dist) / (f_total * 1e-3) / 1e9, 2),
+                "ms_per_step": round(f_total / fsteps, 4), "steps": fsteps,
+                "cached_rows_per_s": round(sum_over_ranks(keys * fsteps, dist) / (f_total * 1e-3), 1),
+                "config": {"workload": f"decode B={fB} H={fH} Hkv={fHkv} L={fL} d={fd}, e4m3 cache with "
+                                       f"per-row fp32 scales ({f_kv / 1e9:.2f} GB), bf16 q, rho, out",
+                           "l2": "inputs larger than L2; no flush"},
+                "roofline": {"bound": "hbm", "achieved": round(f_ach, 1), "peak": peaks["hbm_gbs"],
+                             "unit": "GB/s", "frac": round(f_ach / peaks["hbm_gbs"], 4), "traffic": None,
+                             "peak_source": peak_src, "kernel": f"decode_fp8kv_kernel<{fH // fHkv}>",
+                             "algorithmic_bytes_per_launch": f_alg},
+                "gpu_launches": fsteps,
+            }
+            fp8kv["groups_of_%d" % (fH // fHkv)] = entry
+            del ft, Kc, Vc, Ks, Vs
+            torch.cuda.empty_cache()
+
+    # ---- A fixed subset of the decode sweep (batch x context, ragged lengths).
+    sweep = None
+    if not args.no_sweep and dist is None:
+        sweep = [sweep_cell(sB, sL, max(5, args.steps // 5), 3, peaks) for (sB, sL) in SWEEP_SUBSET]
+
     # ---- Full layer (x [4, 8192, 2048], 16 heads of 128).
     layer = None
     if not args.no_layer:
@@ -675,7 +732,7 @@ def run_gpu(args, rank, world, dist):
     return {
         "value": round(value, 2), "ms_per_step": round(ms_step, 4), "roofline": roofline,
         "e2e": e2e, "clocks": clk.summary(), "prefill": prefill, "layer": layer, "decode_gqa": gqa,
-        "window": win,
+        "window": win, "decode_fp8kv": fp8kv, "decode_sweep": sweep,
         "gpu_launches": args.steps,
         "kernel_ms": kernel_ms,
     }
@@ -773,47 +830,59 @@ def oracle_prefill_sample(budget_s):
 # Sweep.
 # ---------------------------------------------------------------------------
 
-def run_sweep(args):
+def sweep_cell(B, L, steps, warmup, peaks, dist=None, seed=1003):
+    """One decode sweep cell (H=16, d=128 bf16, lengths uniform on [L/2, L]):
+    GB/s of algorithmic bytes per launch, CUDA events on the launching stream."""
     import torch
     from local_linear_attention_streamed_b200 import plx, synth
-    peaks, peak_src = load_peaks()
     H, d = 16, 128
     stream = torch.cuda.current_stream()
+    alloc = B * H * L * d * 2 * 2
+    specs = synth.decode_specs(B, H, L, d)
+    t = {}
+    for name, spec in specs.items():
+        t[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device="cuda")
+        synth.device_fill(t[name].data_ptr(), synth.BF16, seed, spec)
+    sl_host = synth.seqlens(seed, B, L, ragged=True)
+    sl = torch.from_numpy(sl_host).cuda()
+    out = torch.empty_like(t["q"])
+    kv, alg = decode_bytes(sl_host, H, d)
+    # Cells that fit in L2 rotate through enough copies to defeat it.
+    copies = 1 if alloc > 4 * L2_BYTES else int(math.ceil(4 * L2_BYTES / alloc))
+    extra = [{n: v.clone() for n, v in t.items()} for _ in range(copies - 1)]
+    sets = [t] + extra
+    idx = [0]
+
+    def fn():
+        s = sets[idx[0] % len(sets)]
+        idx[0] += 1
+        plx.decode(s["q"], s["r"], s["K"], s["V"], sl, out=out)
+
+    total, per = timed(fn, steps, warmup, stream, dist)
+    if plx.get_device_status() != 0:
+        raise RuntimeError(f"decode sweep cell {(B, L)} reported a device error")
+    ms = float(np.mean(per))
+    cell = {"cell": [B, L], "kv_gb": round(kv / 1e9, 4), "us_per_launch": round(ms * 1e3, 2),
+            "GBps": round(alg / (ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "splits": plx.lib.plx_decode_num_splits(B, H, L, d),
+            "kernel": "tensor-core" if plx.lib.plx_decode_uses_tc(B, H, L, d) else "warp-mma",
+            "l2_copies": copies}
+    del t, extra, sets
+    torch.cuda.empty_cache()
+    return cell
+
+
+def run_sweep(args):
+    peaks, peak_src = load_peaks()
+    H, d = 16, 128
     for B in SWEEP_B:
         for L in SWEEP_L:
             alloc = B * H * L * d * 2 * 2
             if alloc > SWEEP_MAX_BYTES:
                 print(json.dumps({"cell": [B, L], "skipped": f"KV cache {alloc / 1e9:.1f} GB > 150 GB"}))
                 continue
-            specs = synth.decode_specs(B, H, L, d)
-            t = {}
-            for name, spec in specs.items():
-                t[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device="cuda")
-                synth.device_fill(t[name].data_ptr(), synth.BF16, 1003, spec)
-            sl_host = synth.seqlens(1003, B, L, ragged=True)
-            sl = torch.from_numpy(sl_host).cuda()
-            out = torch.empty_like(t["q"])
-            kv, alg = decode_bytes(sl_host, H, d)
-            # Cells that fit in L2 rotate through enough copies to defeat it.
-            copies = 1 if alloc > 4 * 126e6 else int(math.ceil(4 * 126e6 / alloc))
-            extra = [{n: v.clone() for n, v in t.items()} for _ in range(copies - 1)]
-            sets = [t] + extra
-            idx = [0]
-
-            def fn():
-                s = sets[idx[0] % len(sets)]
-                idx[0] += 1
-                plx.decode(s["q"], s["r"], s["K"], s["V"], sl, out=out)
-
-            total, per = timed(fn, args.steps, args.warmup, stream)
-            ms = float(np.mean(per))
-            print(json.dumps({"cell": [B, L], "kv_gb": round(kv / 1e9, 4), "us_per_launch": round(ms * 1e3, 2),
-                              "GBps": round(alg / (ms * 1e-3) / 1e9, 1),
-                              "frac_hbm": round(alg / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-                              "splits": plx.lib.plx_decode_num_splits(B, H, L, d),
-                              "l2_copies": copies}), flush=True)
-            del t, extra, sets
-            torch.cuda.empty_cache()
+            print(json.dumps(sweep_cell(B, L, args.steps, args.warmup, peaks)), flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -831,6 +900,8 @@ def main():
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-window", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
+    ap.add_argument("--no-fp8kv", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
                     help="decode batch (smaller values for profiler captures only)")
@@ -914,7 +985,7 @@ def main():
             "data": "synthetic", "config": cfg, "roofline": res["roofline"], "cpu_baseline": cpu,
             "e2e": res["e2e"], "gpu_launches": res["gpu_launches"], "clocks": res["clocks"],
             "prefill": res["prefill"], "layer": res["layer"], "decode_gqa": res["decode_gqa"],
-            "window": res["window"]}
+            "window": res["window"], "decode_fp8kv": res["decode_fp8kv"], "decode_sweep": res["decode_sweep"]}
     print(json.dumps(line))
 
 

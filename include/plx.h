@@ -273,6 +273,14 @@ size_t plx_decode_workspace_bytes(int B, int H, int L, int d);
 int plx_decode_num_splits(int B, int H, int L, int d);
 
 /*
+ * 1 if plx_decode_ex (bf16) runs these sizes on the tcgen05 decode kernel, 0 if
+ * on the warp-MMA kernel (the choice is a pure function of the sizes, made so
+ * that the split plan, the workspace size and the launch agree); negative for
+ * invalid sizes.  For tests and diagnostics.
+ */
+int plx_decode_uses_tc(int B, int H, int L, int d);
+
+/*
  * One bf16 decode step with grouped KV heads: H query heads share Hkv KV heads,
  * query head h reading KV head h / (H / Hkv) (consecutive query heads form a
  * group).  The pages' decode packs the q and rho rows into one tensor-core tile

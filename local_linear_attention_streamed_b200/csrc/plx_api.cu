@@ -398,6 +398,11 @@ int plx_decode_num_splits(int B, int H, int L, int d) {
   return splits;
 }
 
+int plx_decode_uses_tc(int B, int H, int L, int d) {
+  if (B < 1 || H < 1 || L < 1 || (d != 64 && d != 128)) return PLX_ERR_INVALID_ARG;
+  return decode_bf16_tc((long long)B * H, L, d) ? 1 : 0;
+}
+
 size_t plx_decode_workspace_bytes(int B, int H, int L, int d) {
   if (B < 1 || H < 1 || L < 1 || d < 1) return 0;
   int splits = 1, chunk = 0;

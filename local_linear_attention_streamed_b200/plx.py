@@ -28,6 +28,7 @@ SIGNATURES = {
     "plx_decode_ex": (_i, [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_decode_workspace_bytes": (_sz, [_i] * 4),
     "plx_decode_num_splits": (_i, [_i] * 4),
+    "plx_decode_uses_tc": (_i, [_i] * 4),
     "plx_decode_noalloc": (_i, [_vp] * 6 + [_i] * 4 + [_vp]),
     "plx_decode_gqa": (_i, [_vp] * 6 + [_i] * 5 + [_vp, _sz, _vp]),
     "plx_decode_gqa_workspace_bytes": (_sz, [_i] * 5),
