@@ -20,7 +20,8 @@
 //     [2^14, 2^15) before the (then exact) conversion to f16, and the
 //     softmax threads undo 2^e and apply the key's scale in fp32.
 //   * values, dims as the MMA's M:  O^T [128 dims x 4G] += V_blk^T W in bf16:
-//     e4m3 codes convert exactly to bf16 (through f16), and the value row's
+//     e4m3 codes convert exactly to bf16 (integer bit moves and one
+//     multiply by a power of two), and the value row's
 //     scale is folded into that key's weights (w s_v and w t s_v, each a bf16
 //     hi + lo pair), so omega and T stay plain sums of w and w t.
 // Roles (one persistent CTA per SM, units = (b, KV head, key chunk) from a
@@ -103,12 +104,25 @@ __device__ __forceinline__ void e4m3x16_to_f16(const uint4 c, uint32_t (&h)[8]) 
     h[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
   }
 }
-// An f16x2 word whose values are exact in bf16 (all e4m3 values are) -> bf16x2.
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
-  unsigned short lo, hi;
-  asm("cvt.rn.bf16.f16 %0, %1;" : "=h"(lo) : "h"((unsigned short)(h & 0xffffu)));
-  asm("cvt.rn.bf16.f16 %0, %1;" : "=h"(hi) : "h"((unsigned short)(h >> 16)));
-  return (uint32_t)lo | ((uint32_t)hi << 16);
+// 4 e4m3 codes (code 0 in the low byte) -> 2 bf16x2 words, exactly, on the
+// integer and FMA pipes (the conversion instructions share the XU pipe with
+// the exponentials and would bound the stream).  With a code in the high byte
+// of a 16-bit lane, its sign bit is bf16's sign bit, and its 4 exponent and 3
+// mantissa bits shifted right by 4 land in bf16's exponent and top mantissa
+// bits: the lane then holds the code's value times 2^-120 (exponent bias 7
+// against 127), subnormal codes included.  One bf16x2 multiply by 2^120
+// restores the value exactly.
+__device__ __forceinline__ uint32_t bf16x2_times_2p120(uint32_t v) {
+  __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162*>(&v);
+  const uint32_t k = 0x7B807B80u;  // 2^120 in both lanes (exponent field 247)
+  const __nv_bfloat162 r = __hmul2(a, *reinterpret_cast<const __nv_bfloat162*>(&k));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+__device__ __forceinline__ void e4m3x4_to_bf16(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  const uint32_t w0 = __byte_perm(x, 0u, 0x1404);  // [code1, 0, code0, 0]
+  const uint32_t w1 = __byte_perm(x, 0u, 0x3424);  // [code3, 0, code2, 0]
+  lo = bf16x2_times_2p120((w0 & 0x80008000u) | ((w0 & 0x7F007F00u) >> 4));
+  hi = bf16x2_times_2p120((w1 & 0x80008000u) | ((w1 & 0x7F007F00u) >> 4));
 }
 
 template <int G>
@@ -623,9 +637,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < 8; ++c) {
           uint32_t h8[8];
           if (inside) {
-            e4m3x16_to_f16(*reinterpret_cast<const uint4*>(vr + sw128_chunk(r, c)), h8);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) h8[k] = f16x2_to_bf16x2(h8[k]);
+            const uint4 cv = *reinterpret_cast<const uint4*>(vr + sw128_chunk(r, c));
+            e4m3x4_to_bf16(cv.x, h8[0], h8[1]);
+            e4m3x4_to_bf16(cv.y, h8[2], h8[3]);
+            e4m3x4_to_bf16(cv.z, h8[4], h8[5]);
+            e4m3x4_to_bf16(cv.w, h8[6], h8[7]);
           } else {
 #pragma unroll
             for (int k = 0; k < 8; ++k) h8[k] = 0u;

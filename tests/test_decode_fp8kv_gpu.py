@@ -112,6 +112,29 @@ def test_fp8kv_garbage_past_the_lengths_does_not_leak(plx):
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
 
 
+def test_fp8kv_subnormal_codes(plx):
+    """Rows with one element 10^4 times the rest: most codes of those rows are
+    e4m3 subnormals (below 2^-6 after scaling), in K and in V."""
+    B, H, Hkv, L, d = 2, 4, 2, 400, 128
+    rng = np.random.default_rng(96)
+    K = rng.standard_normal((B, Hkv, L, d))
+    V = rng.standard_normal((B, Hkv, L, d))
+    for X in (K, V):
+        X[..., 0] = 1e4 * np.where(rng.random((B, Hkv, L)) < 0.5, 1.0, -1.0)
+    K /= 1e3
+    q = rng.standard_normal((B, H, d))
+    r = 0.25 * rng.standard_normal((B, H, d))
+    (Kd, Kr), (Vd, Vr), (qd, qr), (rd, rr) = _bf16(K), _bf16(V), _bf16(q), _bf16(r)
+    gpu, orc = _fp8_case(plx, Kd, Vd, Kr, Vr)
+    codes = orc[2]
+    assert np.mean((codes & 0x78) == 0) > 0.5  # exponent field 0: subnormal (or zero) codes
+    sl = np.array([400, 257], dtype=np.int32)
+    out = plx.decode_fp8kv(qd, rd, *gpu, torch.from_numpy(sl).cuda())
+    assert plx.get_device_status() == 0
+    want = oracle.decode_fp8kv_ref(qr, rr, *orc, sl)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
 @pytest.mark.parametrize("key_scale", [1.0, 3.0])
 def test_fp8kv_true_normal(plx, key_scale):
     """Unbounded normal draws (q, k RMS rows, keys optionally x 3; v ~ N(0, 1); rho ~ N(0, 0.25^2))."""
