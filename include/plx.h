@@ -333,7 +333,7 @@ size_t plx_decode_fp8kv_workspace_bytes(int B, int H, int Hkv, int L, int d);
  * groups of 1, 2, 4 or 8; d = 128, else PLX_ERR_UNSUPPORTED.  It reads
  * 2 * (d + 4) bytes per cached row instead of the bf16 decode's 4 d.
  * workspace: plx_decode_fp8kv_workspace_bytes() bytes, 256-byte aligned, or NULL
- * for a library-owned one.  Pointers 16-byte aligned (scales and seqlens 4).
+ * for a library-owned one.  Pointers 16-byte aligned (seqlens 4).
  */
 int plx_decode_fp8kv(const void* q, const void* r, const void* Kcodes, const float* Kscales,
                      const void* Vcodes, const float* Vscales, const int32_t* seqlens, void* out, int B,

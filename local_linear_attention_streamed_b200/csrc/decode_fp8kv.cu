@@ -55,6 +55,8 @@ constexpr int kThreads = 384;
 constexpr int kQrWarp = 2, kFirstEw = 4, kFirstCv = 8;
 constexpr int kUnitRing = 4;
 constexpr int kStages = 4;       // raw e4m3 K + V blocks, 32 KB each
+constexpr int kScaleBox = kKeys + 4;   // scales per staged box (128 keys + up to 3 before them)
+constexpr int kScaleBoxPad = 160;      // box rounded up to 128 bytes
 constexpr int kRows = 16;        // q rows 0..G-1, rho rows 8..8+G-1 of the score operand
 constexpr float kLazyTau = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -69,6 +71,9 @@ struct SmemF {
   uint8_t vc[2][2][kKeys * 128];         // bf16 V block per buffer: [128 keys x 64 dims] per half
   uint8_t qr[2][2][kRows * 128];         // f16 q / rho operand per unit slot: [16 rows x 64 dims] per half
   uint8_t w[2][2][NW * 128];             // bf16 weights per block slot: [NW rows x 64 keys] per half
+  // Per raw stage, the K and V scales of the block's keys: a box of kScaleBox
+  // floats starting at the block's first key rounded down to a 16-byte boundary.
+  alignas(128) float sc[kStages][2][kScaleBoxPad];
   uint64_t raw_full[kStages], raw_empty[kStages];
   uint64_t kc_full[2], kc_free[2], vc_full[2], vc_free[2];
   uint64_t qr_full[2], qr_empty[2];
@@ -128,6 +133,7 @@ __device__ __forceinline__ void e4m3x4_to_bf16(uint32_t x, uint32_t& lo, uint32_
 template <int G>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_fp8kv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
                         DecodeArgs a) {
   using Sm = SmemF<G>;
   constexpr int NW = Sm::NW;
@@ -141,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], 4);  // the four converter warps
+      mbar_init(&sm.raw_empty[s], 8);  // the four converter warps and the four key warps
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
@@ -219,11 +225,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = pos % kStages;
           if (!(ok = mbar_wait(&sm.raw_empty[st], ((pos / kStages) & 1) ^ 1, abort, a.status))) break;
           if (a.inject_stall && blockIdx.x == 0) continue;
-          mbar_expect_tx(&sm.raw_full[st], 2 * kKeys * 128);
+          mbar_expect_tx(&sm.raw_full[st], 2 * kKeys * 128 + 2 * kScaleBox * 4);
           last_kv[st] = (int)(pos / kStages);
           const int row = x.bkv * a.L + x.kbeg + kKeys * i;  // < 2^31 (launcher check)
           tma_load_2d(sm.raw[st][0], &tmK, &sm.raw_full[st], 0, row);
           tma_load_2d(sm.raw[st][1], &tmV, &sm.raw_full[st], 0, row);
+          // Scales: the 1-D box must start on a 16-byte boundary (a multiple of
+          // 4 floats); the key threads index from the remainder.
+          tma_load_1d(sm.sc[st][0], &tmKs, &sm.raw_full[st], row & ~3);
+          tma_load_1d(sm.sc[st][1], &tmVs, &sm.raw_full[st], row & ~3);
         }
         if (!ok) break;
         u = next;
@@ -415,12 +425,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; i < x.nblk; ++i) {
         const uint32_t bb = blk + i;
-        const int sb = bb & 1;
+        const int sb = bb & 1, st = bb % kStages;
         const int key = x.kbeg + kKeys * i + r;
         const bool valid = key < x.kend, inside = key < x.n;
-        // The key's scales (no row past the sequence is read: its weight is 0).
-        const float sk = inside ? __ldg(a.Kscale + srow + key) : 0.f;
-        const float sv = inside ? __ldg(a.Vscale + srow + key) : 0.f;
+        // The key's scales from the raw stage (staged with the block's codes;
+        // rows past the sequence get weight 0 whatever they hold).
+        if (!(ok = warp_wait(&sm.raw_full[st], (bb / kStages) & 1, abort, a.status))) break;
+        const int off = (int)((srow + x.kbeg + kKeys * i) & 3);
+        const float sk = inside ? sm.sc[st][0][off + r] : 0.f;
+        const float sv = inside ? sm.sc[st][1][off + r] : 0.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
         if (!(ok = warp_wait(&sm.s_full[sb], (bb >> 1) & 1, abort, a.status))) break;
         tc_fence_after();
         uint32_t sv16[kRows];
@@ -693,20 +708,37 @@ bool make_map_e4m3(CUtensorMap* m, const void* base, long long rows) {
   return r == CUDA_SUCCESS;
 }
 
+// 1-D view of a scale array of `rows` floats, boxes of kScaleBox floats
+// (elements past the end read as zero).
+bool make_map_scales(CUtensorMap* m, const float* base, long long rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[1] = {(cuuint64_t)rows};
+  cuuint64_t strides[1] = {0};
+  cuuint32_t box[1] = {(cuuint32_t)kScaleBox};
+  cuuint32_t estr[1] = {1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<float*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int G>
 cudaError_t launch_f8(const DecodeArgs& args, cudaStream_t st, int num_sms) {
   DecodeArgs a = args;
   const char* fi = getenv("PLX_FAULT_INJECT");
   a.inject_stall = (fi != nullptr && strcmp(fi, "decode_stall") == 0) ? 1 : 0;
-  CUtensorMap mK, mV;
+  CUtensorMap mK, mV, mKs, mVs;
   const long long kv_rows = (long long)a.B * a.Hkv * a.L;
-  if (!make_map_e4m3(&mK, a.K, kv_rows) || !make_map_e4m3(&mV, a.V, kv_rows)) return cudaErrorInvalidValue;
+  if (!make_map_e4m3(&mK, a.K, kv_rows) || !make_map_e4m3(&mV, a.V, kv_rows) ||
+      !make_map_scales(&mKs, a.Kscale, kv_rows) || !make_map_scales(&mVs, a.Vscale, kv_rows))
+    return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemF<G>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(decode_fp8kv_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long units = (long long)a.B * a.Hkv * a.splits;
   const long long grid = units < num_sms ? units : num_sms;
-  decode_fp8kv_kernel<G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, a);
+  decode_fp8kv_kernel<G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, mKs, mVs, a);
   return cudaGetLastError();
 }
 

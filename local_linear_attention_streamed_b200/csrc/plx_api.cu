@@ -567,8 +567,7 @@ int plx_decode_fp8kv(const void* q, const void* r, const void* Kcodes, const flo
   if (G != 1 && G != 2 && G != 4 && G != 8) return PLX_ERR_UNSUPPORTED;
   if (d != 128) return PLX_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(r) || !aligned16(Kcodes) || !aligned16(Vcodes) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || (reinterpret_cast<uintptr_t>(Kscales) & 3u) ||
-      (reinterpret_cast<uintptr_t>(Vscales) & 3u))
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) || !aligned16(Kscales) || !aligned16(Vscales))
     return PLX_ERR_MISALIGNED;
   if (!decode_sizes_supported(B, H, Hkv, L)) return PLX_ERR_UNSUPPORTED;
   int rc;
