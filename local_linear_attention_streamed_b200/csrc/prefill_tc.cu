@@ -10,27 +10,29 @@
 //                 (rainbus.top summary, "方法步骤详情": S1 and S2 per KV block
 //                 from one shared instruction stream);
 //   warp 2      value MMA issuer (one elected thread): O1 += P V and
-//                 O2 += (w t) V with P and w t (as a bf16 hi + lo pair) read
-//                 from TMEM and V from shared memory ("accumulate O1 and O2 in
-//                 parallel").  Two issuing threads keep the tensor pipe fed
-//                 while either one waits on a barrier (an MMA issue stalls
-//                 until the pipe takes it).
+//                 O2 += (w t) V with P and w t read from TMEM (w t also as a
+//                 bf16 remainder from shared memory) and V from shared memory
+//                 ("accumulate O1 and O2 in parallel").  Two issuing threads
+//                 keep the tensor pipe fed while either one waits on a barrier
+//                 (an MMA issue stalls until the pipe takes it).
 //   warps 2..9  two softmax warpgroups, each thread = one half (32 keys of every
 //               block, 64 output dims) of one query row (= TMEM lane): one running
 //               max and one rescale factor shared by both branches (agihunt.info
 //               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
-//               P = bf16(w), bf16(w (t - c)) and the bf16 remainder of w (t - c),
-//               and the epilogue out = ((1 + T/omega) O1 - O2) / omega.
-// TMEM (512 columns): two S stages at 0 and 128 (S1 at +0, S2 at +64: 64 fp32
-// columns each), O1 at 256 and O2 after it (D fp32 columns each).  Block g
-// uses stage g % 2, which is also the softmax warpgroup that owns it.  Once
-// that warpgroup has loaded its scores it writes its value operands over them
-// in place (bf16 pairs: P at +0, the hi part of w (t - c) at +32, its lo part
-// at +64), and the value MMAs read them there.  So the scores of block g + 1
-// never wait for the softmax of block g: they need only the value MMAs of
-// block g - 1 to have finished with the other stage.  Each thread reads the
-// whole row of S1 to take the block's row max without an exchange; the row
-// sums are exchanged once per block.
+//               P = bf16(w) and bf16(w (t - c)) into a P buffer, and the
+//               epilogue out = ((1 + T/omega) O1 - O2) / omega.
+// TMEM (512 columns): one S stage (S1 at 0, S2 at 64: 64 fp32 columns each),
+// two P buffers at 128 and 192 (bf16 pairs: bf16(w) in columns 0..31 and
+// bf16(w (t - c)) in 32..63), O1 at 256 and O2 at 384 (128 fp32 columns each).
+// At D = 64, O1 and O2 take 256..383 and a second S stage sits at 384 (one
+// stage per softmax warpgroup).
+// The scores of block g+1 are computed as soon as the softmax has loaded those
+// of block g into registers, and the value MMAs of block g read P buffer g % 2,
+// so the tensor pipe runs ahead of the softmax by a block instead of waiting
+// for it: the two overlap without either one's latency entering the other's
+// period.  Each softmax thread reads the whole row of S1 (its partner's half
+// too) to take the block's row max without an exchange; the row sums are
+// exchanged once per block.
 //
 // Centring.  The output is unchanged when every t_ij of a query is shifted by
 // the same c_i (the pages' key-query difference z_ij = k_j - q_i is one such
@@ -39,7 +41,8 @@
 // stay well conditioned when one key dominates a row and |t| is large; with
 // c = 0 a single bf16 rounding of w t there is amplified by |t| (tens, in
 // trained models and in the rescale test).  w (t - c) also enters the value
-// product as a bf16 hi + lo pair (one more MMA per block): with one bf16 term
+// product with its bf16 remainder, bf16(w (t - c) - bf16(w (t - c))), as the
+// shared-memory A operand of one more MMA per block: with the one bf16 term,
 // its rounding alone moved early rows of true-normal inputs by up to 3.3 % of
 // their RMS, against 1.9 % with the pair.  c is set from the first block and
 // moved (O2 -= delta O1 in TMEM) only when the running mean drifts by more than
@@ -62,7 +65,6 @@ namespace {
 
 constexpr int kBM = 128;                 // queries per tile
 constexpr int kBN = 64;                  // keys per block
-constexpr int kStages = 4;               // K/V ring depth
 constexpr int kTileRing = 4;             // tile indices in flight from producer to consumers
 // 12 warps in three warpgroups: {TMA, S MMA, PV MMA, idle} and two softmax
 // warpgroups.  The first gives registers to the other two (setmaxnreg):
@@ -75,10 +77,9 @@ constexpr uint32_t kHalfQ = kBM * 128;       // one 64-dim half of a Q tile (128
 constexpr uint32_t kHalfKV = kBN * 128;      // one 64-dim half of a K/V block
 constexpr float kLazyTau = 8.f;
 
-// TMEM column map: S stage s at 128 s (S1 at +0, S2 at +64; after the softmax
-// the same stage holds P at +0 and w (t - c) as hi at +32 and lo at +64, bf16
-// pairs), O1 (D columns from 256) and O2 (after O1).
-constexpr uint32_t kColStage = 128, kColS1 = 0, kColS2 = 64, kColPT = 32, kColPTlo = 64, kColO1 = 256;
+// TMEM column map: the S stage, two P buffers (bf16(w) then bf16(w (t - c))
+// in each), O1 (D columns from 256) and O2 (after O1).
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColO1 = 256;
 
 // Instruction descriptors (kind::f16): D f32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), A K-major, B K-major (S) or MN-major (bit 16, PV),
@@ -91,6 +92,8 @@ struct Dims {
   static constexpr uint32_t kQBytes = kBM * D * 2;      // Q tile (also R tile)
   static constexpr uint32_t kKVBytes = kBN * D * 2;     // one K or V block
   static constexpr uint32_t kColO2 = kColO1 + D;
+  // K/V ring depth: at D = 128 the two remainder buffers leave room for 3.
+  static constexpr int kStages = D == 128 ? 3 : 4;
   // Re-centre t once its running mean drifts this far (section "Centring"
   // above).  2 at D = 128: 1.7 % on the rescale test, and 8 % faster than 1
   // (fewer O passes).  At D = 64 the rescale test gives 2.7 % (causal) with
@@ -103,20 +106,23 @@ struct Dims {
 template <int D>
 struct Smem {
   static constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
+  static constexpr int kStages = Dims<D>::kStages;
   // Tiles first (1024-byte aligned for the 128B swizzle).
   uint8_t q[kQBytes];
   uint8_t r[kQBytes];
   uint8_t k[kStages][kKVBytes];
   uint8_t v[kStages][kKVBytes];
+  // Per P buffer, the bf16 remainder of w (t - c): [128 rows x 64 keys], one
+  // 128-byte swizzled row per query (the A operand of the third value MMA).
+  uint8_t plo[2][kBM * 128];
   uint64_t q_full, q_empty;
   // One full and one empty barrier per K/V stage: K and V of a block land
   // together, and the stage frees once that block's value MMAs completed.
   uint64_t kv_full[kStages], kv_empty[kStages];
   // Block g's scores complete on s_full[g % 2] (the barrier of the softmax
-  // warpgroup that owns the block and of its S stage); its value operands on
-  // p_full[g % 2]; the stage is free for block g + 2 once block g's value
-  // MMAs completed (stage_free[g % 2]).
-  uint64_t s_full[2], p_full[2], stage_free[2];
+  // warpgroup that owns the block); its P on p_full[g % 2].  The S stage goes
+  // back to the score issuer on s_free[0] (one stage) or s_free[g % 2] (two).
+  uint64_t s_full[2], s_free[2], p_full[2];
   uint64_t o_full, o_empty, drain;
   // Row state handed from the owner of block g to the owner of block g + 1:
   // (running max, centre, the poster's own sum w, its own sum w (t - c)) in
@@ -125,10 +131,14 @@ struct Smem {
   uint32_t post_flag[2][kBM];
   // Tile indices handed from the producer to the MMA and softmax roles.
   int tile_ring[kTileRing];
+  uint32_t s_issued;  // blocks whose scores were issued (all ones: no more)
   uint64_t tile_full[kTileRing], tile_empty[kTileRing];
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(Smem<128>) + 1024 <= 227 * 1024 && sizeof(Smem<64>) + 1024 <= 227 * 1024,
+              "shared memory of one CTA");
 
 using namespace sm100;
 
@@ -197,7 +207,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                       Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   constexpr bool kWin = kMode == 1, kSparse = kMode == 2;
-  static_assert(2 * kColStage <= kColO1 && kColO1 + 2 * D <= 512, "TMEM columns");
+  // At D = 64, O1 and O2 end at column 384, so a second S stage fits in TMEM
+  // (columns 384..511): each softmax warpgroup then has its own, and the
+  // scores of block g + 1 need not wait until the owner of block g has read
+  // its scores.  At D = 128 the 512 columns hold one stage.
+  constexpr bool kTwoS = D == 64;
+  static_assert(!kTwoS || kColO1 + 2 * D <= 384, "second S stage above O1, O2");
   // Rows that may see no key in a block (window or block sparsity) need the
   // guards for an empty running max.
   constexpr bool kRobust = kMode != 0;
@@ -207,6 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto kblock = [&](const TileInfo& ti, int j) { return kSparse ? p.blk_idx[ti.j0 + j] : ti.j0 + j; };
   constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
   constexpr uint32_t kColO2 = Dims<D>::kColO2, kIdescPV = Dims<D>::kIdescPV;
+  constexpr int kStages = Dims<D>::kStages;
   constexpr int kHalves = Dims<D>::kHalves;
   Smem<D>& sm =
       *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -227,8 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 128);  // the owning warpgroup's threads
-      mbar_init(&sm.stage_free[s], 1);
     }
+    mbar_init(&sm.s_free[0], 4);  // one lane of each warp of the owning warpgroup
+    mbar_init(&sm.s_free[1], 4);
     for (int s = 0; s < kTileRing; ++s) {
       mbar_init(&sm.tile_full[s], 1);
       mbar_init(&sm.tile_empty[s], 10);  // both MMA threads and one lane of each softmax warp
@@ -236,6 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sm.o_full, 1);
     mbar_init(&sm.o_empty, 256);
     mbar_init(&sm.drain, 2);  // one commit from each MMA thread
+    sm.s_issued = 0;
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -322,14 +340,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         if (!(ok = mbar_wait(&sm.q_full, tc & 1, abort, p.status))) break;
         for (int j = 0; j < ti.nblk; ++j, ++g) {
-          // K of this block (long resident: checked first), then S stage
-          // g % 2, free once the value MMAs of block g - 2 have read the
-          // operands the softmax wrote over that block's scores.
+          // K of this block (long resident: checked first), then the S stage,
+          // free once the softmax has read the previous block's scores: the
+          // wait on the critical path comes last, right before the issue.
           const uint32_t st = g % kStages;
           if (!(ok = mbar_wait(&sm.kv_full[st], (g / kStages) & 1, abort, p.status))) break;
-          if (!(ok = mbar_wait(&sm.stage_free[g & 1], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
+          if constexpr (kTwoS) {
+            if (g > 1 && !(ok = mbar_wait(&sm.s_free[g & 1], ((g >> 1) & 1) ^ 1, abort, p.status))) break;
+          } else {
+            if (g > 0 && !(ok = mbar_wait(&sm.s_free[0], (g - 1) & 1, abort, p.status))) break;
+          }
           tc_fence_after();
-          const uint32_t sst = (g & 1) * kColStage;  // the S stage of block g
+          const uint32_t sst = kTwoS ? (g & 1) * 384u : 0u;  // the S stage of block g
           const uint64_t dk = dK0 + (uint64_t)(st * (kKVBytes >> 4));
           // S1 and S2 k-steps interleaved (one B tile feeds both GEMMs); every
           // MMA comes from the descriptors built once plus a compile-time
@@ -344,19 +366,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           mma_commit(&sm.s_full[g & 1]);
           if (j + 1 == ti.nblk) mma_commit(&sm.q_empty);
+          *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) = g + 1;
         }
       }
+      // No more scores: the value issuer stops waiting for them.
+      *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) = 0xFFFFFFFFu;
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
   } else if (warp == kPVWarp) {
     // ---------------- value MMA issuer ----------------
-    // Block g's value MMAs go as soon as its operands are in TMEM: the scores
-    // of block g + 2 wait for them to free S stage g % 2.
+    // The scores of the next blocks are the critical path (the single S stage
+    // frees only when the softmax has loaded the previous block), so the
+    // value MMAs of block k go into the tensor pipe only behind the scores of
+    // block k + 2: issuing stalls while the pipe is full, so issue order is
+    // the order the pipe works in.  (The scores never wait on these values:
+    // the softmax waits for block k's before it overwrites P buffer k % 2.)
     if (lane == 0) {
       uint32_t g = 0;
       int tc = 0;
       const uint64_t dV0 = sdesc(smem_u32(sm.v[0]), kHalfKV, 1024);
+      const uint64_t dL0 = sdesc(smem_u32(sm.plo[0]), 16, 1024);
       const uint32_t oa1 = tmem + kColO1, oa2 = tmem + kColO2;
       bool ok = true;
       for (; ok; ++tc) {
@@ -371,10 +401,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < ti.nblk; ++j, ++g) {
           const uint32_t b = g & 1;
           if (!(ok = mbar_wait(&sm.p_full[b], (g >> 1) & 1, abort, p.status))) break;
+          // Behind the scores of block g + 2 (bounded in time like every wait).
+          if ((int)(*reinterpret_cast<volatile uint32_t*>(&sm.s_issued) - (g + 3)) < 0) {
+            const unsigned long long t0 = now_ns();
+            while ((int)(*reinterpret_cast<volatile uint32_t*>(&sm.s_issued) - (g + 3)) < 0 &&
+                   *reinterpret_cast<volatile uint32_t*>(&sm.s_issued) != 0xFFFFFFFFu) {
+              if (*abort) {
+                ok = false;
+                break;
+              }
+              if (now_ns() - t0 > kWaitNs) {
+                *abort = 1;
+                atomicOr(p.status, kStatusTimeout);
+                ok = false;
+                break;
+              }
+              __nanosleep(32);
+            }
+            if (!ok) break;
+          }
           tc_fence_after();
           const uint32_t st = g % kStages;
           const uint64_t dv = dV0 + (uint64_t)(st * (kKVBytes >> 4));
-          const uint32_t pbase = tmem + b * kColStage;
+          const uint32_t pbase = tmem + kColP + b * kColPBuf;
           const uint32_t first = (j == 0) ? 0u : 1u;
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
@@ -383,12 +432,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_ts(oa1, pbase + ks * 8, bv, kIdescPV, acc);
             mma_ts(oa2, pbase + kColPT + ks * 8, bv, kIdescPV, acc);
           }
+          // O2 += (remainder of w (t - c)) V: A K-major from shared memory.
+          const uint64_t dl = dL0 + (uint64_t)((b * (kBM * 128)) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks)  // the lo part of w (t - c): O2 accumulates already
-            mma_ts(oa2, pbase + kColPTlo + ks * 8, dv + (uint64_t)((ks * 2048) >> 4), kIdescPV, 1u);
-          // Frees the K/V stage and S stage b.
+          for (int ks = 0; ks < kBN / 16; ++ks)
+            mma_ss(oa2, dl + (uint64_t)((ks * 32) >> 4), dv + (uint64_t)((ks * 2048) >> 4), kIdescPV, 1u);
+          // Frees the K/V stage and P buffer b.
           mma_commit(&sm.kv_empty[st]);
-          mma_commit(&sm.stage_free[b]);
         }
         if (!ok) break;
         mma_commit(&sm.o_full);
@@ -494,12 +544,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int kb = kblock(ti, j) * kBN;
         uint32_t x[64], y[64];
-        const uint32_t ss = sb + (uint32_t)wg * kColStage;  // this block's S stage (g % 2 == wg)
+        const uint32_t ss = sb + (kTwoS ? (uint32_t)wg * 384u : 0u);  // this block's S stage
         tmem_ld32(ss + kColS1, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
         tmem_ld32(ss + kColS1 + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
         tmem_ld32(ss + kColS2, *reinterpret_cast<uint32_t(*)[32]>(&y[0]));
         tmem_ld32(ss + kColS2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&y[32]));
         tc_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[kTwoS ? wg : 0]);  // the S stage goes back to the MMA
         if ((p.causal && kb + kBN - 1 > ti.m * kBM) || kb + kBN > p.N ||
             (kWin && kb < ti.m * kBM + kBM - window)) {
           // Block-uniform: only blocks that cross the diagonal, the end or the
@@ -648,12 +701,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_wait_st();
           }
         }
-        // The value operands go over this block's scores (S stage wg, already
-        // in registers).  w (t - c) is a - delta w with the centre settled
-        // above, and is written as bf16 hi + lo.
-        const uint32_t pb = ss;
+        // P buffer wg (= g % 2) is free once the value MMAs of block g - 2, its
+        // last reader, completed (the MMA issuer runs them after the scores).
+        if (g >= 2) {
+          const uint32_t gq = g - 2;
+          if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
+          tc_fence_after();
+        }
+        const uint32_t pb = sb + kColP + (uint32_t)wg * kColPBuf;
+        // bf16(w (t - c)) is a - delta w with the centre settled above; its
+        // bf16 remainder goes to this row of the shared-memory buffer.
         const bool moved = __any_sync(0xffffffffu, delta != 0.f);
         const uint64_t nd2 = f2(-delta, -delta);
+        uint8_t* lrow = sm.plo[wg] + row * 128;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint32_t P[16], PT[16], PL[16];
@@ -669,8 +729,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(pb + 16 * h, P);
           tmem_st16(pb + kColPT + 16 * h, PT);
-          tmem_st16(pb + kColPTlo + 16 * h, PL);
+          // keys 32h .. 32h + 31: 16-byte chunks 4h .. 4h + 3 of the row (128B swizzle)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(lrow + (((4 * h + c) ^ (row & 7)) << 4)) =
+                make_uint4(PL[4 * c], PL[4 * c + 1], PL[4 * c + 2], PL[4 * c + 3]);
         }
+        fence_async_smem();
         tc_wait_st();
         tc_fence_before();
         mbar_arrive(&sm.p_full[wg]);
