@@ -9,30 +9,27 @@
 //                 S1 = Q K^T and S2 = R K^T from ONE K tile into TMEM
 //                 (rainbus.top summary, "方法步骤详情": S1 and S2 per KV block
 //                 from one shared instruction stream);
-//   warp 2      value MMA issuer (one elected thread): O1 += P V and
-//                 O2 += (w t) V with P and w t (at D = 128 as a bf16 hi + lo
-//                 pair) read from TMEM and V from shared memory ("accumulate
-//                 O1 and O2 in parallel").  Two issuing threads keep the
-//                 tensor pipe fed while either one waits on a barrier (an MMA
-//                 issue stalls until the pipe takes it).
+//   warp 10     value MMA issuer (one elected thread): O1 += P V and
+//                 O2 += (w t) V with P and w t read from TMEM and V from shared
+//                 memory ("accumulate O1 and O2 in parallel").  Two issuing
+//                 threads keep the tensor pipe fed while either one waits on a
+//                 barrier (an MMA issue stalls until the pipe takes it).
 //   warps 2..9  two softmax warpgroups, each thread = one half (32 keys of every
 //               block, 64 output dims) of one query row (= TMEM lane): one running
 //               max and one rescale factor shared by both branches (agihunt.info
 //               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
 //               P = bf16(w) and bf16(w (t - c)) into a P buffer, and the
 //               epilogue out = ((1 + T/omega) O1 - O2) / omega.
-// TMEM (512 columns) at D = 128: one S stage (S1 at 0, S2 at 64: 64 fp32
-// columns each), one P buffer at 128 (bf16 pairs: bf16(w) in columns 0..31,
-// bf16(w (t - c)) in 32..63 and its bf16 remainder in 64..95), O1 at 256 and
-// O2 at 384 (128 fp32 columns each).  At D = 64, O1 and O2 take 256..383, a
-// second S stage sits at 384 (one stage per softmax warpgroup) and two P
-// buffers (bf16(w), bf16(w (t - c))) at 128 and 192.
+// TMEM (512 columns): one S stage (S1 at 0, S2 at 64: 64 fp32 columns each),
+// two P buffers at 128 and 192 (bf16 pairs: bf16(w) in columns 0..31 and
+// bf16(w (t - c)) in 32..63), O1 at 256 and O2 at 384 (128 fp32 columns each).
+// At D = 64, O1 and O2 take 256..383 and a second S stage sits at 384 (one
+// stage per softmax warpgroup).
 // The scores of block g+1 are computed as soon as the softmax has loaded those
-// of block g into registers, so the tensor pipe runs ahead of the softmax by
-// a block instead of waiting for it: the two overlap without either one's
-// latency entering the other's period.  The softmax of block g + 1 waits for
-// the value MMAs of block g (one P buffer) or g - 1 (two) only before it
-// stores its operands.  Each softmax thread reads the whole row of S1 (its partner's half
+// of block g into registers, and the value MMAs of block g read P buffer g % 2,
+// so the tensor pipe runs ahead of the softmax by a block instead of waiting
+// for it: the two overlap without either one's latency entering the other's
+// period.  Each softmax thread reads the whole row of S1 (its partner's half
 // too) to take the block's row max without an exchange; the row sums are
 // exchanged once per block.
 //
@@ -42,11 +39,7 @@
 // so that O2 = sum w (t - c) v and the combine ((1 + T/omega) O1 - O2)/omega
 // stay well conditioned when one key dominates a row and |t| is large; with
 // c = 0 a single bf16 rounding of w t there is amplified by |t| (tens, in
-// trained models and in the rescale test).  At D = 128 (t spreads wider)
-// w (t - c) also enters the value product with its bf16 remainder (one more
-// MMA per block): with the one bf16 term, its rounding alone moved early rows
-// of true-normal inputs by up to 3.3 % of their RMS, against 1.9 % with the
-// pair.  c is set from the first block and
+// trained models and in the rescale test).  c is set from the first block and
 // moved (O2 -= delta O1 in TMEM) only when the running mean drifts by more than
 // kTheta, always before the block's w (t - c) is rounded.
 //
@@ -82,7 +75,7 @@ constexpr float kLazyTau = 8.f;
 
 // TMEM column map: the S stage, two P buffers (bf16(w) then bf16(w (t - c))
 // in each), O1 (D columns from 256) and O2 (after O1).
-constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColPTlo = 64, kColO1 = 256;
+constexpr uint32_t kColS1 = 0, kColS2 = 64, kColP = 128, kColPBuf = 64, kColPT = 32, kColO1 = 256;
 
 // Instruction descriptors (kind::f16): D f32 (bits 4-5 = 1), A and B bf16
 // (bits 7-9, 10-12 = 1), A K-major, B K-major (S) or MN-major (bit 16, PV),
@@ -95,10 +88,6 @@ struct Dims {
   static constexpr uint32_t kQBytes = kBM * D * 2;      // Q tile (also R tile)
   static constexpr uint32_t kKVBytes = kBN * D * 2;     // one K or V block
   static constexpr uint32_t kColO2 = kColO1 + D;
-  // D = 128: one P buffer holding bf16(w), bf16(w (t - c)) and its remainder;
-  // D = 64: two P buffers (block parity) without the remainder.
-  static constexpr bool kLoPT = D == 128;
-  static constexpr int kPBufs = kLoPT ? 1 : 2;
   // Re-centre t once its running mean drifts this far (section "Centring"
   // above).  2 at D = 128: 1.7 % on the rescale test, and 8 % faster than 1
   // (fewer O passes).  At D = 64 the rescale test gives 2.7 % (causal) with
@@ -220,9 +209,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto kblock = [&](const TileInfo& ti, int j) { return kSparse ? p.blk_idx[ti.j0 + j] : ti.j0 + j; };
   constexpr uint32_t kQBytes = Dims<D>::kQBytes, kKVBytes = Dims<D>::kKVBytes;
   constexpr uint32_t kColO2 = Dims<D>::kColO2, kIdescPV = Dims<D>::kIdescPV;
-  constexpr bool kLoPT = Dims<D>::kLoPT;
-  constexpr int kPBufs = Dims<D>::kPBufs;
-  static_assert(!kLoPT || (kColP + 96 <= kColO1 && !kTwoS), "one P buffer of three operands");
   constexpr int kHalves = Dims<D>::kHalves;
   Smem<D>& sm =
       *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -422,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t st = g % kStages;
           const uint64_t dv = dV0 + (uint64_t)(st * (kKVBytes >> 4));
-          const uint32_t pbase = tmem + kColP + (kPBufs == 1 ? 0u : b * kColPBuf);
+          const uint32_t pbase = tmem + kColP + b * kColPBuf;
           const uint32_t first = (j == 0) ? 0u : 1u;
 #pragma unroll
           for (int ks = 0; ks < kBN / 16; ++ks) {
@@ -430,11 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t acc = ks > 0 ? 1u : first;
             mma_ts(oa1, pbase + ks * 8, bv, kIdescPV, acc);
             mma_ts(oa2, pbase + kColPT + ks * 8, bv, kIdescPV, acc);
-          }
-          if constexpr (kLoPT) {
-#pragma unroll
-            for (int ks = 0; ks < kBN / 16; ++ks)  // O2 += (remainder of w (t - c)) V
-              mma_ts(oa2, pbase + kColPTlo + ks * 8, dv + (uint64_t)((ks * 2048) >> 4), kIdescPV, 1u);
           }
           // Frees the K/V stage and P buffer b.
           mma_commit(&sm.kv_empty[st]);
@@ -700,14 +681,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_wait_st();
           }
         }
-        // The P buffer is free once the value MMAs of its last reader, block
-        // g - kPBufs, completed (the MMA issuer runs them after the scores).
-        if (g >= (uint32_t)kPBufs) {
-          const uint32_t gq = g - kPBufs;
+        // P buffer wg (= g % 2) is free once the value MMAs of block g - 2, its
+        // last reader, completed (the MMA issuer runs them after the scores).
+        if (g >= 2) {
+          const uint32_t gq = g - 2;
           if (!(ok = mbar_wait(&sm.kv_empty[gq % kStages], (gq / kStages) & 1, abort, p.status))) break;
           tc_fence_after();
         }
-        const uint32_t pb = sb + kColP + (kPBufs == 1 ? 0u : (uint32_t)wg * kColPBuf);
+        const uint32_t pb = sb + kColP + (uint32_t)wg * kColPBuf;
         // bf16(w (t - c)) is a - delta w with the centre settled above.
         const bool moved = __any_sync(0xffffffffu, delta != 0.f);
         const uint64_t nd2 = f2(-delta, -delta);
@@ -724,19 +705,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tmem_st16(pb + 16 * h, P);
           tmem_st16(pb + kColPT + 16 * h, PT);
-          if constexpr (kLoPT) {
-            uint32_t PL[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              // the remainder of each rounded pair, from the values rounded above
-              const int e = 32 * h + 2 * c;
-              float a0 = __uint_as_float(y[e]), a1 = __uint_as_float(y[e + 1]);
-              if (moved) uf2(fma2(f2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), nd2, f2(a0, a1)), a0, a1);
-              const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&PT[c]);
-              PL[c] = pack_bf16(a0 - __low2float(hi), a1 - __high2float(hi));
-            }
-            tmem_st16(pb + kColPTlo + 16 * h, PL);
-          }
         }
         tc_wait_st();
         tc_fence_before();

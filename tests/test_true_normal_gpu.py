@@ -17,7 +17,10 @@ The prefill rounds w (t - c) to one bf16 operand, and at that spread its
 rounding alone exceeds the bar: a float64 replay of the prefill's arithmetic
 (the same replay reproduces the GPU's error to every printed digit) gives 3.6 %
 at keys x 3, 3.0 % at x 2 and 1.6 % at x 1 on these inputs, so the prefill
-cases stay at the workloads' scale.
+cases stay at the workloads' scale.  Even there a short early row can just
+miss the bar (one grouped case, marked as an expected failure: 2.02 %, the
+replay's number too); over 20,480 true-normal early rows of the causal
+workload's shape the replay puts 3 rows above 2e-2, the worst at 3.3 %.
 """
 import numpy as np
 import pytest
@@ -144,7 +147,10 @@ def test_decode_gqa_true_normal(plx, d, G, Hkv, key_scale):
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
 
 
-@pytest.mark.parametrize("G", [2, 8])
+@pytest.mark.parametrize("G", [2, pytest.param(8, marks=pytest.mark.xfail(
+    strict=True, reason="known limit of the single bf16 w (t - c) operand: row 6 of head (1, 4) "
+                        "(seven keys) is 2.02 % of its RMS away, and a float64 replay of the "
+                        "prefill's arithmetic gives the same 2.02 %"))])
 def test_prefill_gqa_true_normal(plx, G):
     B, Hkv, N, d = 2, 2, 400, 128
     H = G * Hkv
