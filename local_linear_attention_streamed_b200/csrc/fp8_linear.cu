@@ -14,6 +14,8 @@
 // device-side scale pointers, so no host synchronisation).
 #include "plx_internal.cuh"
 
+#include <mutex>
+
 #include <cublasLt.h>
 #include <cuda_fp8.h>
 
@@ -165,43 +167,97 @@ cudaError_t launch_quant_t(const void* const* W, int count, int rows, int cols, 
 // Y[M, Dout] (bf16, row-major) = (X8[M, Din] Wt8[Dout, Din]^T) * sX * sW, both
 // operands e4m3 row-major.  Column-major view for cuBLASLt: Y^T = Wt8 X8^T with
 // A = Wt8 stored Din x Dout (transposed), B = X8 stored Din x M.
-int fp8_gemm(void* lt_handle, const void* Wt8, const void* X8, void* Y, int Dout, int Din, long long M,
-             const float* sW, const float* sX, void* ws, size_t ws_bytes, cudaStream_t st) {
-  cublasLtHandle_t lt = static_cast<cublasLtHandle_t>(lt_handle);
+//
+// The matmul descriptor, the three layouts and the algorithm the heuristic
+// picks depend only on the handle and the sizes, so they are built once per
+// shape and kept (a layer step runs five GEMMs of two shapes); only the scale
+// pointers, which may move with the caller's workspace, are set per call.
+namespace {
+
+struct Fp8Plan {
+  void* lt = nullptr;
+  int Dout = 0, Din = 0;
+  long long M = 0;
+  size_t ws_bytes = 0;
   cublasLtMatmulDesc_t op = nullptr;
   cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
+  cublasLtMatmulAlgo_t algo{};
+};
+
+constexpr int kPlans = 16;
+std::mutex g_plan_mu;
+Fp8Plan g_plans[kPlans];
+int g_plan_next = 0;
+
+void destroy_plan(Fp8Plan& p) {
+  if (p.lc) cublasLtMatrixLayoutDestroy(p.lc);
+  if (p.lb) cublasLtMatrixLayoutDestroy(p.lb);
+  if (p.la) cublasLtMatrixLayoutDestroy(p.la);
+  if (p.op) cublasLtMatmulDescDestroy(p.op);
+  p = Fp8Plan{};
+}
+
+// The cached plan for these sizes, built on first use (nullptr on failure).
+Fp8Plan* plan_for(void* lt_handle, int Dout, int Din, long long M, size_t ws_bytes) {
+  for (Fp8Plan& p : g_plans)
+    if (p.op && p.lt == lt_handle && p.Dout == Dout && p.Din == Din && p.M == M && p.ws_bytes == ws_bytes)
+      return &p;
+  Fp8Plan& p = g_plans[g_plan_next];
+  g_plan_next = (g_plan_next + 1) % kPlans;
+  destroy_plan(p);
+  cublasLtHandle_t lt = static_cast<cublasLtHandle_t>(lt_handle);
   cublasLtMatmulPreference_t pref = nullptr;
-  int rc = -1;
+  bool ok = false;
   do {
-    if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
+    if (cublasLtMatmulDescCreate(&p.op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS) break;
     const cublasOperation_t tA = CUBLAS_OP_T, tB = CUBLAS_OP_N;
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &tA, sizeof(tA));
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tB, sizeof(tB));
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_A_SCALE_POINTER, &sW, sizeof(sW));
-    cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_B_SCALE_POINTER, &sX, sizeof(sX));
-    if (cublasLtMatrixLayoutCreate(&la, CUDA_R_8F_E4M3, Din, Dout, Din) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatrixLayoutCreate(&lb, CUDA_R_8F_E4M3, Din, (uint64_t)M, Din) != CUBLAS_STATUS_SUCCESS) break;
-    if (cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, Dout, (uint64_t)M, Dout) != CUBLAS_STATUS_SUCCESS) break;
+    cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSA, &tA, sizeof(tA));
+    cublasLtMatmulDescSetAttribute(p.op, CUBLASLT_MATMUL_DESC_TRANSB, &tB, sizeof(tB));
+    if (cublasLtMatrixLayoutCreate(&p.la, CUDA_R_8F_E4M3, Din, Dout, Din) != CUBLAS_STATUS_SUCCESS) break;
+    if (cublasLtMatrixLayoutCreate(&p.lb, CUDA_R_8F_E4M3, Din, (uint64_t)M, Din) != CUBLAS_STATUS_SUCCESS) break;
+    if (cublasLtMatrixLayoutCreate(&p.lc, CUDA_R_16BF, Dout, (uint64_t)M, Dout) != CUBLAS_STATUS_SUCCESS) break;
     if (cublasLtMatmulPreferenceCreate(&pref) != CUBLAS_STATUS_SUCCESS) break;
     cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES, &ws_bytes,
                                          sizeof(ws_bytes));
     cublasLtMatmulHeuristicResult_t heur;
     int found = 0;
-    if (cublasLtMatmulAlgoGetHeuristic(lt, op, la, lb, lc, lc, pref, 1, &heur, &found) != CUBLAS_STATUS_SUCCESS ||
+    if (cublasLtMatmulAlgoGetHeuristic(lt, p.op, p.la, p.lb, p.lc, p.lc, pref, 1, &heur, &found) !=
+            CUBLAS_STATUS_SUCCESS ||
         found < 1)
       break;
-    const float one = 1.f, zero = 0.f;
-    if (cublasLtMatmul(lt, op, &one, Wt8, la, X8, lb, &zero, Y, lc, Y, lc, &heur.algo, ws, ws_bytes, st) !=
-        CUBLAS_STATUS_SUCCESS)
-      break;
-    rc = 0;
+    p.algo = heur.algo;
+    ok = true;
   } while (false);
   if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return rc;
+  if (!ok) {
+    destroy_plan(p);
+    return nullptr;
+  }
+  p.lt = lt_handle;
+  p.Dout = Dout;
+  p.Din = Din;
+  p.M = M;
+  p.ws_bytes = ws_bytes;
+  return &p;
+}
+
+}  // namespace
+
+int fp8_gemm(void* lt_handle, const void* Wt8, const void* X8, void* Y, int Dout, int Din, long long M,
+             const float* sW, const float* sX, void* ws, size_t ws_bytes, cudaStream_t st) {
+  std::lock_guard<std::mutex> lk(g_plan_mu);
+  Fp8Plan* p = plan_for(lt_handle, Dout, Din, M, ws_bytes);
+  if (!p) return -1;
+  if (cublasLtMatmulDescSetAttribute(p->op, CUBLASLT_MATMUL_DESC_A_SCALE_POINTER, &sW, sizeof(sW)) !=
+          CUBLAS_STATUS_SUCCESS ||
+      cublasLtMatmulDescSetAttribute(p->op, CUBLASLT_MATMUL_DESC_B_SCALE_POINTER, &sX, sizeof(sX)) !=
+          CUBLAS_STATUS_SUCCESS)
+    return -1;
+  const float one = 1.f, zero = 0.f;
+  if (cublasLtMatmul(static_cast<cublasLtHandle_t>(lt_handle), p->op, &one, Wt8, p->la, X8, p->lb, &zero, Y, p->lc,
+                     Y, p->lc, &p->algo, ws, ws_bytes, st) != CUBLAS_STATUS_SUCCESS)
+    return -1;
+  return 0;
 }
 
 }  // namespace plx
