@@ -17,7 +17,8 @@ five cells of the decode sweep under "decode_sweep".  For N > 1 GPUs (launched b
 same per-GPU workload on its own seeded inputs with no data-path collective
 (weak scaling); time is the max over ranks.
 
-`--impl reference` times the float64 CPU oracle (the only reference this
+`--only NAME` runs one workload four times and exits (what the profiler
+captures under profiles/ run).  `--impl reference` times the float64 CPU oracle (the only reference this
 method has) on bounded samples of the same workload.  `--sweep` prints one
 line per decode sweep cell instead.
 """
@@ -886,6 +887,71 @@ def run_sweep(args):
 
 
 # ---------------------------------------------------------------------------
+# One workload, a few launches (what profiler captures run: one kernel, a few
+# launches, a few GB on the device).
+# ---------------------------------------------------------------------------
+
+ONLY = ("decode", "decode_gqa", "decode_window", "decode_fp8kv", "prefill", "prefill_window", "backward")
+
+
+def run_only(name, launches=4):
+    import torch
+    from local_linear_attention_streamed_b200 import plx, synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    def fill(specs, seed):
+        t = {}
+        for n, spec in specs.items():
+            t[n] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(t[n].data_ptr(), synth.BF16, seed, spec)
+        return t
+
+    if name in ("decode", "decode_window"):
+        B, H, L, d = (DECODE[k] for k in ("B", "H", "L", "d"))
+        t = fill(synth.decode_specs(B, H, L, d), 1002)
+        sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+        if name == "decode":
+            def f():
+                plx.decode(t["q"], t["r"], t["K"], t["V"], sl)
+        else:
+            def f():
+                plx.decode_window(t["q"], t["r"], t["K"], t["V"], sl, WINDOW)
+    elif name in ("decode_gqa", "decode_fp8kv"):
+        B, H, Hkv, L, d = ((DECODE_GQA[k] for k in ("B", "H", "Hkv", "L", "d")) if name == "decode_gqa"
+                           else (DECODE["B"], DECODE["H"], DECODE["H"], DECODE["L"], DECODE["d"]))
+        t = fill(synth.decode_gqa_specs(B, H, Hkv, L, d), 1007)
+        sl = torch.full((B,), L, dtype=torch.int32, device=dev)
+        if name == "decode_gqa":
+            def f():
+                plx.decode_gqa(t["q"], t["r"], t["K"], t["V"], sl)
+        else:
+            Kc, Ks = plx.kv_quantize_fp8(t.pop("K"))
+            Vc, Vs = plx.kv_quantize_fp8(t.pop("V"))
+
+            def f():
+                plx.decode_fp8kv(t["q"], t["r"], Kc, Ks, Vc, Vs, sl)
+    else:
+        B, H, N, d = (PREFILL[k] for k in ("B", "H", "N", "d"))
+        t = fill(synth.backward_specs(B, H, N, d), 1004)
+        if name == "prefill":
+            def f():
+                plx.prefill(t["Q"], t["K"], t["V"], t["R"], causal=True)
+        elif name == "prefill_window":
+            def f():
+                plx.prefill_window(t["Q"], t["K"], t["V"], t["R"], WINDOW)
+        else:
+            saved = plx.prefill_train(t["Q"], t["K"], t["V"], t["R"], True)
+
+            def f():
+                plx.prefill_backward(t["Q"], t["K"], t["V"], t["R"], *saved, t["dO"], True)
+    for _ in range(launches):
+        f()
+    torch.cuda.synchronize()
+    status = plx.get_device_status()
+    if status != 0:
+        raise RuntimeError(f"{name} reported {plx.status_string(status)}")
+    print(json.dumps({"only": name, "launches": launches, "status": "ok"}))
+
 
 def main():
     ap = argparse.ArgumentParser()
@@ -902,6 +968,8 @@ def main():
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-fp8kv", action="store_true")
     ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--only", choices=ONLY, default=None,
+                    help="run one workload a few times and exit (for profiler captures)")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work per leg")
     ap.add_argument("--decode-batch", type=int, default=DECODE["B"],
                     help="decode batch (smaller values for profiler captures only)")
@@ -953,6 +1021,13 @@ def main():
         dist = tdist
     else:
         torch.cuda.set_device(0)
+
+    if args.only is not None:
+        if rank == 0:
+            run_only(args.only)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
 
     if args.sweep:
         if rank == 0:

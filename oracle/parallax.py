@@ -130,6 +130,36 @@ def prefill_ref(Q, K, V, R, causal: bool = True, rows=None, window=None) -> np.n
     return np.stack(res) if res else np.zeros((0, d))
 
 
+def dilated_visible_keys(i: int, dilation: int, window=None) -> np.ndarray:
+    """Indices of the keys query i sees under a dilated window: i, i - r,
+    i - 2r, ... (r = dilation), the last ``window`` of them (all when None)."""
+    keys = np.arange(i, -1, -int(dilation), dtype=np.int64)[::-1]
+    if window is not None:
+        keys = keys[-int(window):]
+    return keys
+
+
+def prefill_dilated_ref(Q, K, V, R, dilation: int, window=None, rows=None) -> np.ndarray:
+    """Oracle for a dilated causal prefill (the pages list dilated sparsity
+    with sliding-window and block-sparse patterns as future work, rainbus.top
+    "未来方向", and fix no rule).  Reading: the dilated sliding window, query i
+    sees its own key and every r-th key before it, i - k r for k = 0 ..
+    window - 1 (all k when window is None).  Q, R [B, H, N, d]; K, V
+    [B, Hkv, N, d] (query head h reads KV head h // (H // Hkv)).  ``rows`` as
+    prefill_ref."""
+    B, H, N, d = Q.shape
+    G = H // K.shape[1]
+    rows_iter = ([(b, h, i) for b in range(B) for h in range(H) for i in range(N)] if rows is None
+                 else list(rows))
+    res = []
+    for (b, h, i) in rows_iter:
+        ks = dilated_visible_keys(i, dilation, window)
+        res.append(parallax_row(Q[b, h, i], R[b, h, i], K[b, h // G, ks], V[b, h // G, ks]))
+    if rows is None:
+        return np.stack(res).reshape(B, H, N, d)
+    return np.stack(res) if res else np.zeros((0, d))
+
+
 def prefill_gqa_ref(Q, K, V, R, causal: bool = True) -> np.ndarray:
     """Oracle for a prefill with grouped KV heads: Q, R [B, H, N, d]; K, V
     [B, Hkv, N, d]; query head h reads KV head h // (H // Hkv)."""
