@@ -531,6 +531,18 @@ def run_gpu(args, rank, world, dist):
             spairs += int(np.sum(bmask[t, :full])) * 64 + (i % 64 + 1)
         sflops = 8.0 * wd * spairs * wB * wH
         s_ach = sflops / (float(np.mean(s_per)) * 1e-3) / 1e12
+
+        # Dilated prefill (dilation 4, the whole residue class: query i sees
+        # keys i, i - 4, i - 8, ...) on the same inputs.
+        DIL = 4
+
+        def dpre():
+            plx.prefill_dilated(wt2["Q"], wt2["K"], wt2["V"], wt2["R"], DIL, 0, out=sout)
+
+        g_total, g_per = timed(dpre, wsteps, max(3, args.warmup // 2), stream, dist)
+        n_cls = wN // DIL
+        gflops = 8.0 * wd * DIL * n_cls * (n_cls + 1) / 2 * wB * wH
+        g_ach = gflops / (float(np.mean(g_per)) * 1e-3) / 1e12
         del wt2, sout
         d_total, d_per = timed(wdec, args.steps, args.warmup, stream, dist)
         dbytes = dB * dH * min(W, dL) * dd * 2 * 2 + 3 * dB * dH * dd * 2
@@ -553,6 +565,13 @@ def run_gpu(args, rank, world, dist):
                 "value": round(sum_over_ranks(sflops * wsteps, dist) / (max_over_ranks(s_total, dist) * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "kernel_tflops": round(s_ach, 1), "frac": round(s_ach / peaks["bf16_tflops"], 4),
                 "algorithmic_flops_per_launch": sflops,
+            },
+            "dilated_prefill": {
+                "workload": f"dilated prefill B={wB} H={wH} N={wN} d={wd} bf16, dilation {DIL} (query i sees keys "
+                            f"i, i - {DIL}, i - {2 * DIL}, ...)",
+                "value": round(sum_over_ranks(gflops * wsteps, dist) / (max_over_ranks(g_total, dist) * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "kernel_tflops": round(g_ach, 1), "frac": round(g_ach / peaks["bf16_tflops"], 4),
+                "algorithmic_flops_per_launch": gflops,
             },
             "decode": {
                 "workload": f"sliding-window decode W={W} B={dB} H={dH} L={dL} d={dd} bf16 (all lengths {dL})",

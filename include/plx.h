@@ -308,6 +308,22 @@ int plx_decode_gqa(const void* q, const void* r, const void* Kcache, const void*
 size_t plx_decode_gqa_workspace_bytes(int B, int H, int Hkv, int L, int d);
 
 /*
+ * Dilated causal prefill: query i sees keys i, i - r, i - 2r, ... (r =
+ * dilation), the last `window` of them, or every one back to the start when
+ * window is 0.  The pages list kernels that combine Parallax with dilated
+ * sparsity next to sliding-window and block-sparse ones as future work
+ * (rainbus.top summary, 未来方向) and fix no rule; this is the dilated sliding
+ * window.  Every key a query sees lies in its residue class mod r, so each
+ * class runs as the causal (windowed) prefill of its own subsequence, read and
+ * written through strided views: no masked MMA work.  bf16, d in {64, 128};
+ * Q, R, out [B, H, N, d]; K, V [B, Hkv, N, d] (query head h reads KV head
+ * h / (H/Hkv)); N must be a multiple of r (else PLX_ERR_UNSUPPORTED).  r = 1
+ * is plx_prefill_gqa (window 0) or plx_prefill_gqa_window.
+ */
+int plx_prefill_dilated(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                        int Hkv, int N, int d, int dilation, int window, void* stream);
+
+/*
  * Writes an fp8 (e4m3) KV cache: every row of X (bf16 [rows, d], d in {64, 128})
  * gets its own fp32 scale s = max|x| / 448 (scales[row]) and d codes
  * e4m3(x / s) (codes [rows, d], one byte each; round to nearest even, both

@@ -219,6 +219,27 @@ int plx_prefill_gqa_window(const void* Q, const void* K, const void* V, const vo
   return prefill_gqa_impl(Q, K, V, R, out, B, H, Hkv, N, d, 1, window, stream);
 }
 
+int plx_prefill_dilated(const void* Q, const void* K, const void* V, const void* R, void* out, int B, int H,
+                        int Hkv, int N, int d, int dilation, int window, void* stream) {
+  if (!Q || !K || !V || !R || !out) return PLX_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || Hkv < 1 || N < 1 || d < 1 || H % Hkv != 0 || dilation < 1 || window < 0)
+    return PLX_ERR_INVALID_ARG;
+  if (!prefill_tc_supported(d) || N % dilation != 0) return PLX_ERR_UNSUPPORTED;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(R) || !aligned16(out))
+    return PLX_ERR_MISALIGNED;
+  if ((long long)B * H * dilation > (1ll << 24)) return PLX_ERR_UNSUPPORTED;
+  int rc;
+  DeviceCache* dc = nullptr;
+  if ((rc = current_device(&dc)) != PLX_OK) return rc;
+  PrefillArgs a{Q, K, V, R, out, B, H, N, d, 1, dc->status};
+  a.Hkv = Hkv;
+  a.dilation = dilation;
+  // The window counts keys of the query's residue class; one covering the
+  // whole class (N / dilation keys) is the causal mask within the class.
+  a.window = window < N / dilation ? window : 0;
+  return cuda_rc(launch_prefill_tc(a, reinterpret_cast<cudaStream_t>(stream), dc->num_sms));
+}
+
 int plx_prefill_block_sparse(const void* Q, const void* K, const void* V, const void* R, void* out, int B,
                              int H, int N, int d, const uint8_t* block_mask, void* stream) {
   if (!Q || !K || !V || !R || !out || !block_mask) return PLX_ERR_INVALID_ARG;

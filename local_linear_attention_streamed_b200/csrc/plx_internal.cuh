@@ -41,6 +41,10 @@ struct PrefillArgs {
   // Grouped KV heads (tensor-core path): K and V are [B, Hkv, N, d] and query
   // head h reads KV head h / (H / Hkv); 0 means Hkv = H.
   int Hkv = 0;
+  // Dilation r (tensor-core path; 1 or 0: none): query i sees keys i, i - r,
+  // i - 2r, ... (the causal and window masks within its residue class mod r).
+  // N must be a multiple of r.
+  int dilation = 1;
 };
 
 struct DecodeArgs {

@@ -183,6 +183,12 @@ struct Params {
   float* vbar;
   float* lse;
   float* tbar;
+  // Dilation r (1: none).  With r > 1 the kernel runs B*H*r sequences of N/r
+  // rows (p.N is N/r): sequence (bh, rho) holds rows rho, rho + r, rho + 2r, ...
+  // of head bh, read through 3-D tensor maps [rows/r, r, d] and written back
+  // to those rows, so the causal (and window) masks act within a residue
+  // class: query i sees keys i, i - r, i - 2r, ...
+  int dil;
 };
 
 // kMode: 0 causal or full, 1 sliding window, 2 block-sparse.  The causal and
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem<D>& sm =
       *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.B * p.H;
+  const int BH = p.B * p.H * p.dil;  // sequences (dilation: one per residue class of each head)
   const int ntile = (p.N + kBM - 1) / kBM;
   const int tiles = ntile * BH;
   volatile int* abort = &sm.abort;
@@ -273,9 +279,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sm.tile_full[slot]);
         if (t < 0) break;
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
-        const int row0 = ti.bh * p.N;
+        // Sequence ti.bh is residue class rho of head hb (rho = 0 without dilation).
+        const int hb = ti.bh / p.dil, rho = ti.bh - hb * p.dil;
+        const int row0 = hb * p.N;
         // Grouped KV heads: consecutive query heads share one K/V head.
-        const int kvrow0 = ((ti.bh / p.H) * p.Hkv + (ti.bh % p.H) / (p.H / p.Hkv)) * p.N;
+        const int kvrow0 = ((hb / p.H) * p.Hkv + (hb % p.H) / (p.H / p.Hkv)) * p.N;
+        // Rows of a 2-D map, or (residue class, row within it) of a 3-D one.
+        auto load = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int x, int row) {
+          if (p.dil == 1) {
+            tma_load_2d(dst, map, bar, x, row);
+          } else {
+            tma_load_3d(dst, map, bar, x, rho, row);
+          }
+        };
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
         mbar_expect_tx(&sm.q_full, 2 * kQBytes);
         q_issued = tc;
@@ -284,8 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // unwinds through the abort path.
         if (!(p.inject_stall && tc == 0)) {
           for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
-            tma_load_2d(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+            load(sm.q + h * kHalfQ, &tmQ, &sm.q_full, 64 * h, row0 + ti.m * kBM);
+            load(sm.r + h * kHalfQ, &tmR, &sm.q_full, 64 * h, row0 + ti.m * kBM);
           }
         }
         for (int j = 0; j < ti.nblk; ++j, ++kv) {
@@ -295,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&sm.kv_full[st], 2 * kKVBytes);
           kv_issued[st] = kv / kStages;
           for (int h = 0; h < kHalves; ++h) {
-            tma_load_2d(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
-            tma_load_2d(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
+            load(sm.k[st] + h * kHalfKV, &tmK, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
+            load(sm.v[st] + h * kHalfKV, &tmV, &sm.kv_full[st], 64 * h, kvrow0 + kblock(ti, j) * kBN);
           }
         }
       }
@@ -736,7 +752,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       gb += ti.nblk;
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
-      const long long grow = (long long)ti.bh * p.N + i;
+      // The output row: row i of the sequence, or of its residue class.
+      const int ohb = ti.bh / p.dil, orho = ti.bh - ohb * p.dil;
+      const long long grow = (long long)ohb * p.N * p.dil + orho + (long long)p.dil * i;
       __nv_bfloat16* orow = i < p.N ? p.out + grow * D : nullptr;
       float* vrow = (i < p.N && p.vbar != nullptr) ? p.vbar + grow * D : nullptr;
       if (vrow != nullptr && wg == 0) {
@@ -784,26 +802,36 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
   const long long rows = (long long)a.B * a.H * a.N;
   const long long kv_rows = (long long)a.B * (a.Hkv > 0 ? a.Hkv : a.H) * a.N;
   if (rows >= (1ll << 31)) return cudaErrorInvalidValue;
+  const int dil = a.dilation > 1 ? a.dilation : 1;
+  if (a.N % dil != 0 || (dil > 1 && (a.blk_ptr != nullptr || a.vbar != nullptr))) return cudaErrorInvalidValue;
+  const int n = a.N / dil;  // rows per sequence the kernel runs
   CUtensorMap mQ, mR, mK, mV;
-  if (!make_map(&mQ, a.Q, rows, kBM, D) || !make_map(&mR, a.R, rows, kBM, D) ||
-      !make_map(&mK, a.K, kv_rows, kBN, D) || !make_map(&mV, a.V, kv_rows, kBN, D))
-    return cudaErrorInvalidValue;
-  const int ntile = (a.N + kBM - 1) / kBM;
+  if (dil == 1) {
+    if (!make_map(&mQ, a.Q, rows, kBM, D) || !make_map(&mR, a.R, rows, kBM, D) ||
+        !make_map(&mK, a.K, kv_rows, kBN, D) || !make_map(&mV, a.V, kv_rows, kBN, D))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map_strided(&mQ, a.Q, rows, dil, kBM, D) || !make_map_strided(&mR, a.R, rows, dil, kBM, D) ||
+        !make_map_strided(&mK, a.K, kv_rows, dil, kBN, D) || !make_map_strided(&mV, a.V, kv_rows, dil, kBN, D))
+      return cudaErrorInvalidValue;
+  }
+  const int ntile = (n + kBM - 1) / kBM;
+  const int seqs = a.B * a.H * dil;
   int ch = (2 * num_sms + ntile - 1) / ntile;  // about two waves of tiles per chunk
-  ch = ch < 1 ? 1 : (ch > a.B * a.H ? a.B * a.H : ch);
+  ch = ch < 1 ? 1 : (ch > seqs ? seqs : ch);
   // PLX_FAULT_INJECT=prefill_stall makes the kernel's bounded waits run out
   // (tests of the timeout status only).
   const char* fi = getenv("PLX_FAULT_INJECT");
   const int inject = (fi != nullptr && strcmp(fi, "prefill_stall") == 0) ? 1 : 0;
-  Params p{a.B,      a.H,    a.N, a.causal, a.Hkv > 0 ? a.Hkv : a.H, a.window, a.blk_ptr, a.blk_idx, ch, inject,
+  Params p{a.B,      a.H,    n, a.causal, a.Hkv > 0 ? a.Hkv : a.H, a.window, a.blk_ptr, a.blk_idx, ch, inject,
            reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
-           reinterpret_cast<float*>(a.vbar), a.lse, a.tbar};
+           reinterpret_cast<float*>(a.vbar), a.lse, a.tbar, dil};
   const size_t smem = sizeof(Smem<D>) + 1024;
   auto kernel = a.blk_ptr != nullptr ? prefill_tc_kernel<D, 2>
                 : (a.window > 0 ? prefill_tc_kernel<D, 1> : prefill_tc_kernel<D, 0>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long long tiles = (long long)((a.N + kBM - 1) / kBM) * a.B * a.H;
+  const long long tiles = (long long)ntile * seqs;
   const int grid = (int)(tiles < num_sms ? tiles : num_sms);
   kernel<<<grid, kThreads, smem, st>>>(mQ, mR, mK, mV, p);
   return cudaGetLastError();

@@ -134,6 +134,15 @@ __device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, 128B swizzle, sm100 version bits.
 __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
   uint64_t d = 0;
@@ -287,6 +296,23 @@ inline bool make_map(CUtensorMap* m, const void* base, long long rows, int box_r
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// 3-D view [rows / r, r, d] of a row-major bf16 tensor whose row count is a
+// multiple of r: coordinate (x, y, z) is element x of row z r + y.  Boxes of
+// 64 dims x 1 x box_rows load box_rows rows of one residue class mod r, in the
+// same 128B-swizzled shared layout as make_map's boxes.
+inline bool make_map_strided(CUtensorMap* m, const void* base, long long rows, int r, int box_rows, int d) {
+  auto enc = get_encode();
+  if (!enc || r < 1 || rows % r != 0) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)r, (cuuint64_t)(rows / r)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * r};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult res = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return res == CUDA_SUCCESS;
 }
 
 }  // namespace sm100

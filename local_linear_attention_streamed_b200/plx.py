@@ -52,6 +52,7 @@ SIGNATURES = {
     "plx_prefill_bwd_ex": (_i, [_vp] * 13 + [_i] * 7 + [_vp, _sz, _vp]),
     "plx_prefill_gqa_window": (_i, [_vp] * 5 + [_i] * 6 + [_vp]),
     "plx_prefill_bwd_gqa": (_i, [_vp] * 13 + [_i] * 6 + [_vp, _sz, _vp]),
+    "plx_prefill_dilated": (_i, [_vp] * 5 + [_i] * 7 + [_vp]),
     "plx_kv_quantize_fp8": (_i, [_vp, _vp, _vp, ctypes.c_longlong, _i, _vp]),
     "plx_decode_fp8kv_workspace_bytes": (_sz, [_i] * 5),
     "plx_decode_fp8kv": (_i, [_vp] * 8 + [_i] * 5 + [_vp, _sz, _vp]),
@@ -383,6 +384,19 @@ def decode_gqa(q, r, Kcache, Vcache, seqlens, out=None, workspace=None, stream=N
                             _dev(seqlens, "seqlens"), _dev(out, "out"), B, H, Hkv, L, d,
                             ws_ptr, ws_bytes, _stream_ptr(stream))
     _check(rc, "plx_decode_gqa")
+    return out
+
+
+def prefill_dilated(Q, K, V, R, dilation: int, window: int = 0, out=None, stream=None):
+    """Dilated causal prefill: query i sees keys i, i - r, i - 2r, ... (the last
+    ``window`` of them; all when 0).  Q, R [B, H, N, d]; K, V [B, Hkv, N, d]."""
+    B, H, N, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    rc = lib.plx_prefill_dilated(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(R, "R"), _dev(out, "out"),
+                                 B, H, Hkv, N, d, dilation, window, _stream_ptr(stream))
+    _check(rc, "plx_prefill_dilated")
     return out
 
 
