@@ -109,8 +109,9 @@ def kernel_hash(*names):
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(name, src_hash, units_scale=1.0):
-    """dram read+write bytes per launch from a committed ncu summary, if still current."""
+def profile_field(name, src_hash, key):
+    """A field of a committed ncu summary under profiles/, if the summary is
+    still current (its kernel sources hash to src_hash), else None."""
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
         return None
@@ -118,7 +119,13 @@ def traffic_from_profile(name, src_hash, units_scale=1.0):
         p = json.load(f)
     if p.get("kernel_source_hash") != src_hash:
         return None
-    return float(p["dram_bytes_per_launch"]) * units_scale
+    return p.get(key)
+
+
+def traffic_from_profile(name, src_hash, units_scale=1.0):
+    """dram read+write bytes per launch from a committed ncu summary, if still current."""
+    v = profile_field(name, src_hash, "dram_bytes_per_launch")
+    return None if v is None else float(v) * units_scale
 
 
 # ---------------------------------------------------------------------------
@@ -263,7 +270,7 @@ def run_gpu(args, rank, world, dist):
     kernel_ms = float(np.mean(per))
     value = sum_over_ranks(kv_bytes * args.steps, dist) / (total_ms * 1e-3) / 1e9
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
-    src_hash = kernel_hash("decode_gqa_tc.cu", "sm100.cuh")
+    src_hash = kernel_hash("decode_gqa_tc.cu", "decode_tc_common.cuh", "sm100.cuh")
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 # The committed capture is of the default workload; other sizes report none.
@@ -339,6 +346,11 @@ def run_gpu(args, rank, world, dist):
                          "traffic": (traffic_from_profile("prefill_B8_H16_N4096.json",
                                                           kernel_hash("prefill_tc.cu", "sm100.cuh"))
                                      if pB == PREFILL["B"] else None),
+                         # ncu: sm__pipe_tensor_cycles_active (% of peak, elapsed) of one full-size launch
+                         "tensor_pipe_active_pct": (profile_field("prefill_B8_H16_N4096.json",
+                                                                  kernel_hash("prefill_tc.cu", "sm100.cuh"),
+                                                                  "tensor_pipe_active_pct")
+                                                    if pB == PREFILL["B"] else None),
                          "peak_source": peak_src, "algorithmic_flops_per_launch": flops},
             "gpu_launches": psteps,
         }
@@ -580,7 +592,7 @@ def run_gpu(args, rank, world, dist):
                 "frac": round(dbytes / (float(np.mean(d_per)) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
                 "algorithmic_bytes_per_launch": dbytes,
                 "traffic": (traffic_from_profile("decode_window_B64_H16_L4096_W1024.json",
-                                                kernel_hash("decode_gqa_tc.cu", "sm100.cuh"))
+                                                kernel_hash("decode_gqa_tc.cu", "decode_tc_common.cuh", "sm100.cuh"))
                             if dB == DECODE["B"] else None),
             },
         }
@@ -620,7 +632,7 @@ def run_gpu(args, rank, world, dist):
             "roofline": {"bound": "hbm", "achieved": round(g_ach, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(g_ach / peaks["hbm_gbs"], 4),
                          "traffic": (traffic_from_profile("decode_gqa_B64_H32_Hkv8_L4096.json",
-                                                          kernel_hash("decode_gqa_tc.cu", "sm100.cuh"))
+                                                          kernel_hash("decode_gqa_tc.cu", "decode_tc_common.cuh", "sm100.cuh"))
                                      if (gB, gH, gHkv, gL, gd) == (64, 32, 8, 4096, 128) else None),
                          "peak_source": peak_src, "kernel": (f"decode_gqa_tc_kernel<{gd}, {gH // gHkv}>" if gd == 128 or gHkv % 2 == 0
                                     else f"decode_gqa_kernel<{gd}, {gH // gHkv}>"),
@@ -669,7 +681,11 @@ def run_gpu(args, rank, world, dist):
                                        f"per-row fp32 scales ({f_kv / 1e9:.2f} GB), bf16 q, rho, out",
                            "l2": "inputs larger than L2; no flush"},
                 "roofline": {"bound": "hbm", "achieved": round(f_ach, 1), "peak": peaks["hbm_gbs"],
-                             "unit": "GB/s", "frac": round(f_ach / peaks["hbm_gbs"], 4), "traffic": None,
+                             "unit": "GB/s", "frac": round(f_ach / peaks["hbm_gbs"], 4),
+                             "traffic": (traffic_from_profile("decode_fp8kv_B64_H16_L4096.json",
+                                                              kernel_hash("decode_fp8kv.cu", "decode_tc_common.cuh",
+                                                                          "sm100.cuh"))
+                                         if (fB, fH, fHkv) == (DECODE["B"], DECODE["H"], DECODE["H"]) else None),
                              "peak_source": peak_src, "kernel": f"decode_fp8kv_kernel<{fH // fHkv}>",
                              "algorithmic_bytes_per_launch": f_alg},
                 "gpu_launches": fsteps,
