@@ -191,9 +191,11 @@ struct Params {
   int dil;
 };
 
-// kMode: 0 causal or full, 1 sliding window, 2 block-sparse.  The causal and
-// full prefills compile without any of the other variants' per-row logic.
-template <int D, int kMode>
+// kMode: 0 causal or full, 1 sliding window, 2 block-sparse; kDil: dilated
+// (strided 3-D loads and row mapping; modes 0 and 1).  The causal and full
+// prefills compile without any of the other variants' per-row logic (a
+// run-time dilation branch alone cost the causal kernel 11 %).
+template <int D, int kMode, bool kDil>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -219,7 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem<D>& sm =
       *reinterpret_cast<Smem<D>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.B * p.H * p.dil;  // sequences (dilation: one per residue class of each head)
+  static_assert(!kDil || kMode != 2, "dilation with the causal or window masks");
+  const int dil = kDil ? p.dil : 1;
+  const int BH = p.B * p.H * dil;  // sequences (dilation: one per residue class of each head)
   const int ntile = (p.N + kBM - 1) / kBM;
   const int tiles = ntile * BH;
   volatile int* abort = &sm.abort;
@@ -280,16 +284,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (t < 0) break;
         const TileInfo ti = tile_info(t, BH, p.N, p.causal, p.chunk_heads, window, blk_ptr);
         // Sequence ti.bh is residue class rho of head hb (rho = 0 without dilation).
-        const int hb = ti.bh / p.dil, rho = ti.bh - hb * p.dil;
+        const int hb = kDil ? ti.bh / dil : ti.bh, rho = kDil ? ti.bh - hb * dil : 0;
         const int row0 = hb * p.N;
         // Grouped KV heads: consecutive query heads share one K/V head.
         const int kvrow0 = ((hb / p.H) * p.Hkv + (hb % p.H) / (p.H / p.Hkv)) * p.N;
         // Rows of a 2-D map, or (residue class, row within it) of a 3-D one.
         auto load = [&](void* dst, const CUtensorMap* map, uint64_t* bar, int x, int row) {
-          if (p.dil == 1) {
-            tma_load_2d(dst, map, bar, x, row);
-          } else {
+          if constexpr (kDil) {
             tma_load_3d(dst, map, bar, x, rho, row);
+          } else {
+            tma_load_2d(dst, map, bar, x, row);
           }
         };
         if (tc > 0 && !mbar_wait(&sm.q_empty, (tc - 1) & 1, abort, p.status)) break;
@@ -753,8 +757,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = 1.f / omega;
       const float c1 = (1.f + T * inv) * inv;
       // The output row: row i of the sequence, or of its residue class.
-      const int ohb = ti.bh / p.dil, orho = ti.bh - ohb * p.dil;
-      const long long grow = (long long)ohb * p.N * p.dil + orho + (long long)p.dil * i;
+      long long grow = (long long)ti.bh * p.N + i;
+      if constexpr (kDil) {
+        const int ohb = ti.bh / dil, orho = ti.bh - ohb * dil;
+        grow = (long long)ohb * p.N * dil + orho + (long long)dil * i;
+      }
       __nv_bfloat16* orow = i < p.N ? p.out + grow * D : nullptr;
       float* vrow = (i < p.N && p.vbar != nullptr) ? p.vbar + grow * D : nullptr;
       if (vrow != nullptr && wg == 0) {
@@ -827,8 +834,9 @@ cudaError_t launch_d(const PrefillArgs& a, cudaStream_t st, int num_sms) {
            reinterpret_cast<__nv_bfloat16*>(a.out), a.status,
            reinterpret_cast<float*>(a.vbar), a.lse, a.tbar, dil};
   const size_t smem = sizeof(Smem<D>) + 1024;
-  auto kernel = a.blk_ptr != nullptr ? prefill_tc_kernel<D, 2>
-                : (a.window > 0 ? prefill_tc_kernel<D, 1> : prefill_tc_kernel<D, 0>);
+  auto kernel = a.blk_ptr != nullptr ? prefill_tc_kernel<D, 2, false>
+                : dil > 1 ? (a.window > 0 ? prefill_tc_kernel<D, 1, true> : prefill_tc_kernel<D, 0, true>)
+                          : (a.window > 0 ? prefill_tc_kernel<D, 1, false> : prefill_tc_kernel<D, 0, false>);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const long long tiles = (long long)ntile * seqs;
