@@ -641,6 +641,36 @@ def run_gpu(args, rank, world, dist):
         }
         del gt
         torch.cuda.empty_cache()
+        # Head dim halved at the same width (64 x 32 heads): the tensor-core
+        # decode takes two heads a unit.
+        hB, hH, hL, hd = DECODE["B"], 32, DECODE["L"], 64
+        hspecs = synth.decode_specs(hB, hH, hL, hd)
+        ht = {}
+        for name, spec in hspecs.items():
+            ht[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+            synth.device_fill(ht[name].data_ptr(), synth.BF16, seed + 8, spec)
+        hsl = torch.full((hB,), hL, dtype=torch.int32, device=dev)
+        hout = torch.empty_like(ht["q"])
+
+        def hdec():
+            plx.decode(ht["q"], ht["r"], ht["K"], ht["V"], hsl, out=hout)
+
+        h_total, h_per = timed(hdec, gsteps, max(3, args.warmup // 2), stream, dist)
+        if plx.get_device_status() != 0:
+            raise RuntimeError("d = 64 decode reported a device error")
+        h_kv = hB * hH * hL * hd * 2 * 2
+        h_alg = h_kv + 3 * hB * hH * hd * 2
+        h_ach = h_alg / (float(np.mean(h_per)) * 1e-3) / 1e9
+        gqa["d64"] = {
+            "workload": f"decode B={hB} H={hH} L={hL} d={hd} bf16, all lengths {hL} (head dim halved, same width)",
+            "value": round(sum_over_ranks(h_kv * gsteps, dist) / (max_over_ranks(h_total, dist) * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "kernel_gbs": round(h_ach, 1), "frac": round(h_ach / peaks["hbm_gbs"], 4),
+            "kernel": ("decode_gqa_tc_kernel<64, 1> (two heads a unit)" if plx.lib.plx_decode_uses_tc(hB, hH, hL, hd)
+                       else "decode_bf16_kernel<64>"),
+            "algorithmic_bytes_per_launch": h_alg,
+        }
+        del ht
+        torch.cuda.empty_cache()
 
     # ---- Decode over an e4m3 KV cache: the decode workload's shape, and groups of 4.
     fp8kv = None

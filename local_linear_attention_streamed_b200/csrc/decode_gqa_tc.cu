@@ -605,6 +605,7 @@ cudaError_t launch_decode_gqa_tc(const DecodeArgs& a, cudaStream_t st, int num_s
     if (G == 4) return launch_g<128, 4>(a, st, num_sms);
     if (G == 8) return launch_g<128, 8>(a, st, num_sms);
   } else {
+    if (G == 1) return launch_g<64, 1>(a, st, num_sms);  // two heads a unit, one query head each
     if (G == 2) return launch_g<64, 2>(a, st, num_sms);
     if (G == 4) return launch_g<64, 4>(a, st, num_sms);
     if (G == 8) return launch_g<64, 8>(a, st, num_sms);

@@ -436,7 +436,7 @@ void decode_split_plan(int B, int H, int L, int num_sms, int* splits, int* chunk
 
 cudaError_t launch_decode_bf16(const DecodeArgs& a, cudaStream_t st, int num_sms) {
   const int keys = (a.window > 0 && a.window < a.L) ? a.window : a.L;
-  if (decode_bf16_tc((long long)a.B * a.H, keys, a.d)) {  // the tensor-core decode, Hkv = H
+  if (decode_bf16_tc_h(a.B, a.H, keys, a.d)) {  // the tensor-core decode, Hkv = H
     DecodeArgs g = a;
     g.Hkv = a.H;
     return launch_decode_gqa_tc(g, st, num_sms);

@@ -54,7 +54,7 @@ extern "C" int plx_decode_noalloc(const void* q, const void* r, const void* Kcac
     return PLX_ERR_CUDA;
 
   DecodeArgs a{};
-  decode_split_plan(B, H, L, sms, &a.splits, &a.chunk, decode_bf16_ctas_per_sm((long long)B * H, L, d));
+  decode_bf16_plan(B, H, L, d, sms, &a.splits, &a.chunk);
   const size_t bh = (size_t)B * H;
   const size_t partial_bytes = a.splits > 1 ? sizeof(float) * bh * a.splits * (2 * d + 4) : 0;
   if (a.splits > 1 && (bh * sizeof(int) > kCounterBytes || partial_bytes > kPartialBytes))

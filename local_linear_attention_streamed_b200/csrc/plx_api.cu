@@ -109,7 +109,7 @@ constexpr size_t kLtWorkspace = 32u << 20;  // cuBLASLt workspace of the fp8 GEM
 
 // Bytes of partial records a split decode needs (0 when keys are not split).
 size_t decode_ws_layout(int B, int H, int L, int d, int num_sms, int* splits, int* chunk) {
-  decode_split_plan(B, H, L, num_sms, splits, chunk, decode_bf16_ctas_per_sm((long long)B * H, L, d));
+  decode_bf16_plan(B, H, L, d, num_sms, splits, chunk);
   if (*splits <= 1) return 0;
   return sizeof(float) * (size_t)B * H * (size_t)(*splits) * (size_t)(2 * d + 4);
 }
@@ -415,13 +415,13 @@ int plx_decode_num_splits(int B, int H, int L, int d) {
   (void)d;
   if (B < 1 || H < 1 || L < 1) return 0;
   int splits = 1, chunk = 0;
-  decode_split_plan(B, H, L, num_sms_or_default(), &splits, &chunk, decode_bf16_ctas_per_sm((long long)B * H, L, d));
+  decode_bf16_plan(B, H, L, d, num_sms_or_default(), &splits, &chunk);
   return splits;
 }
 
 int plx_decode_uses_tc(int B, int H, int L, int d) {
   if (B < 1 || H < 1 || L < 1 || (d != 64 && d != 128)) return PLX_ERR_INVALID_ARG;
-  return decode_bf16_tc((long long)B * H, L, d) ? 1 : 0;
+  return decode_bf16_tc_h(B, H, L, d) ? 1 : 0;
 }
 
 size_t plx_decode_workspace_bytes(int B, int H, int L, int d) {

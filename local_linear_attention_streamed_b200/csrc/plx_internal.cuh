@@ -113,6 +113,23 @@ inline bool decode_bf16_tc(long long bh, int keys, int d) {
 }
 // CTAs per SM of that kernel (the split plan's input).
 inline int decode_bf16_ctas_per_sm(long long bh, int keys, int d) { return decode_bf16_tc(bh, keys, d) ? 1 : 2; }
+// The ungrouped bf16 decode's kernel: at d = 128 the size rule above; at d = 64
+// with H even the tcgen05 kernel takes two heads a unit (their 64-dim halves
+// side by side, as for grouped KV heads) for long contexts over few heads
+// (>= 16384 keys, B*H < 128: 1.16x at B=1, H=32, L=32768), else the warp-MMA
+// kernel, which measured equal or faster elsewhere (0.95 of the copy peak at
+// B=64, H=32, L=4096; 1.5x at L=128).
+inline bool decode_bf16_tc_h(int B, int H, int keys, int d) {
+  if (d == 64) return H % 2 == 0 && keys >= 16384 && (long long)B * H < 128;
+  return decode_bf16_tc((long long)B * H, keys, d);
+}
+// The split plan of the ungrouped bf16 decode (units (b, h), or (b, head pair)
+// on the d = 64 tensor-core kernel), shared by the launch, the workspace size
+// and the diagnostics so that they agree.
+inline void decode_bf16_plan(int B, int H, int keys, int d, int num_sms, int* splits, int* chunk) {
+  const bool tc = decode_bf16_tc_h(B, H, keys, d);
+  decode_split_plan(B, (tc && d == 64) ? H / 2 : H, keys, num_sms, splits, chunk, tc ? 1 : 2);
+}
 
 // Sizes every decode entry point accepts: at most 2^24 query (b, h) pairs, and
 // cache rows (B * KV heads * L) that stay below 2^31 even after the largest

@@ -216,6 +216,41 @@ def test_bf16_decode_tensor_core_sizes_every_output(plx):
     assert rel_err_rms(to_f64(outw), wantw) <= BF16_TOL
 
 
+@pytest.mark.parametrize("window", [None, 17000])
+def test_bf16_decode_d64_head_pairs_every_output(plx, window):
+    """d = 64 with H even at sizes the tensor-core decode serves (long caches,
+    few heads): two heads a unit (side-by-side 64-dim halves).  Every output,
+    lengths at 128-key block edges, NaN in the cache past every length."""
+    B, H, L, d = 4, 8, 20480, 64
+    assert plx.lib.plx_decode_uses_tc(B, H, L, d) == 1
+    specs = synth.decode_specs(B, H, L, d)
+    dev, ref = small_inputs(26, specs, synth.BF16)
+    seqlens = np.array([1, 129, 17025, 20480], dtype=np.int32)
+    for b in range(B):
+        dev["K"][b, :, seqlens[b]:] = float("nan")
+        dev["V"][b, :, seqlens[b]:] = float("nan")
+    sl = torch.from_numpy(seqlens).cuda()
+    if window is None:
+        out = plx.decode(dev["q"], dev["r"], dev["K"], dev["V"], sl)
+    else:
+        out = plx.decode_window(dev["q"], dev["r"], dev["K"], dev["V"], sl, window)
+    assert plx.get_device_status() == 0
+    assert torch.isfinite(out).all()
+    want = oracle.decode_ref(ref["q"], ref["r"], ref["K"], ref["V"], seqlens, window=window)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
+def test_bf16_decode_d64_head_pairs_split_keys(plx):
+    """Few head pairs over long caches: chunks merged in-kernel, repeatable."""
+    B, H, L, d = 1, 4, 16384, 64
+    assert plx.lib.plx_decode_uses_tc(B, H, L, d) == 1 and plx.lib.plx_decode_num_splits(B, H, L, d) > 1
+    got, want, status = _decode_small(plx, 27, B, H, L, d, [L - 77])
+    assert status == 0
+    assert rel_err_rms(got, want) <= BF16_TOL
+    again, _, _ = _decode_small(plx, 27, B, H, L, d, [L - 77])
+    assert np.array_equal(got, again)
+
+
 def test_fp32_decode(plx):
     B, H, L, d = 3, 2, 300, 64
     got, want, status = _decode_small(plx, 23, B, H, L, d, [300, 1, 157], dtype=synth.F32)
