@@ -29,8 +29,9 @@
 // blocks by TMA; warp 1 issues the MMAs; warps 2-3 build the q / rho operand
 // of each unit; warps 4-7 own one key each (scores, weights) and at the end
 // of a unit one dim each (output or partial record, merged by the last CTA of
-// a (b, KV head)); warps 8-11 own one key each and convert its K row into
-// TMEM and its V row into the bf16 value tile.
+// a (b, KV head)); warps 8-15, two per TMEM lane quarter, own one key each
+// and convert half of its K row into TMEM and half of its V row into the bf16
+// value tile.
 //
 // Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
 #include "plx_internal.cuh"
@@ -51,8 +52,13 @@ using namespace sm100;
 using namespace dtc;
 
 constexpr int D = 128;
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;
 constexpr int kQrWarp = 2, kFirstEw = 4, kFirstCv = 8;
+constexpr int kCvWarps = 8;  // two per TMEM lane quarter, each converting half of every row
+// Register split (setmaxnreg, per warpgroup): the launch gives 512 x 128; the
+// control warpgroup and the two converter warpgroups hand registers to the
+// key warpgroup: 128 x 96 + 128 x 208 + 256 x 88 = 61,440 <= 65,536.
+constexpr int kRegsControl = 96, kRegsKey = 208, kRegsConv = 88;
 constexpr int kUnitRing = 4;
 constexpr int kStages = 4;       // raw e4m3 K + V blocks, 32 KB each
 constexpr int kScaleBox = kKeys + 4;   // scales per staged box (128 keys + up to 3 before them)
@@ -147,16 +153,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], 8);  // the four converter warps and the four key warps
+      mbar_init(&sm.raw_empty[s], kCvWarps + 4);  // the converter warps and the four key warps
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
-      mbar_init(&sm.unit_empty[s], 11);  // MMA thread, 2 q / rho warps, 4 key warps, 4 converter warps
+      mbar_init(&sm.unit_empty[s], 7 + kCvWarps);  // MMA thread, 2 q / rho warps, 4 key warps, the converters
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.kc_full[s], 4);
+      mbar_init(&sm.kc_full[s], kCvWarps);
       mbar_init(&sm.kc_free[s], 1);
-      mbar_init(&sm.vc_full[s], 4);
+      mbar_init(&sm.vc_full[s], kCvWarps);
       mbar_init(&sm.vc_free[s], 1);
       mbar_init(&sm.qr_full[s], 2);
       mbar_init(&sm.qr_empty[s], 5);  // the MMA thread's commit and the four key warps
@@ -202,6 +208,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
+  if (warp < kFirstEw) {
+  // Each warpgroup sets its share once, at the head of its branch.
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
   if (warp == 0) {
     // ---------------- TMA producer: units and raw e4m3 K / V blocks ----------------
     if (lane == 0) {
@@ -314,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&sm.drain);
       mbar_drain(&sm.drain, 0);
     }
-  } else if (warp < kFirstEw) {
+  } else {
     // ---------------- q / rho operand of each unit (f16, one power-of-two scale per row) ----------------
     const int t = threadIdx.x - 32 * kQrWarp;  // 0..63
     const int row = t >> 2, quarter = t & 3;    // 16 rows x 4 quarters of 32 dims
@@ -371,7 +380,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.qr_full[qs]);
     }
+  }
   } else if (warp < kFirstCv) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsKey));
     // ---------------- one key of every block (scores, weights), one dim of the accumulator ----------------
     const int q = warp - kFirstEw, r = 32 * q + lane;
     const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
@@ -607,8 +618,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++ou;
     }
   } else {
-    // ---------------- converters: key r's K row to TMEM (f16), its V row to the bf16 tile ----------------
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsConv));
+    // ---------------- converters: half of key r's K row to TMEM (f16), of its V row to the bf16 tile ----------------
     const int cq = warp & 3, r = 32 * cq + lane;  // warp w reaches TMEM lanes 32 (w % 4) ..
+    const int half = (warp - kFirstCv) >> 2;       // dims 64 half .. 64 half + 63
     const uint32_t lk = tmem + ((uint32_t)(32 * cq) << 16) + kColK;
     uint32_t pos = 0, blk = 0;
     bool ok = true;
@@ -628,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint8_t* kr = sm.raw[st][0];
 #pragma unroll
-        for (int c2 = 0; c2 < 4; ++c2) {
+        for (int c2 = 2 * half; c2 < 2 * half + 2; ++c2) {
           uint32_t cols[16];
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
@@ -649,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool inside = x.kbeg + kKeys * i + r < x.n;
         const uint8_t* vr = sm.raw[st][1];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
           uint32_t h8[8];
           if (inside) {
             const uint4 cv = *reinterpret_cast<const uint4*>(vr + sw128_chunk(r, c));
