@@ -77,3 +77,32 @@ def test_decode_timeout_is_reported_and_context_survives(monkeypatch):
         out = plx.decode_gqa(dev["q"], dev["r"], dev["K"], dev["V"], sl)
         assert plx.get_device_status() == 0
         assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
+def test_fp8kv_decode_timeout_is_reported_and_context_survives(monkeypatch):
+    """The e4m3-cache decode under PLX_FAULT_INJECT=decode_stall: CTA 0 never
+    receives its code blocks, the converter and key warps' bounded waits run
+    out, the timeout is reported (and the arrival counters cleared), and the
+    next two decodes on the same context are correct."""
+    import torch
+    from local_linear_attention_streamed_b200 import plx
+    B, Hkv, G, L, d = 1, 2, 4, 8192, 128
+    H = G * Hkv
+    specs = synth.decode_gqa_specs(B, H, Hkv, L, d)
+    dev, ref = small_inputs(34, specs, synth.BF16)
+    Kc, Ks = plx.kv_quantize_fp8(dev["K"])
+    Vc, Vs = plx.kv_quantize_fp8(dev["V"])
+    oKc, oKs = oracle.kv_quantize_fp8_ref(ref["K"])
+    oVc, oVs = oracle.kv_quantize_fp8_ref(ref["V"])
+    sl_host = np.array([L - 5], dtype=np.int32)
+    sl = torch.from_numpy(sl_host).cuda()
+    assert plx.get_device_status() == 0
+    monkeypatch.setenv("PLX_FAULT_INJECT", "decode_stall")
+    plx.decode_fp8kv(dev["q"], dev["r"], Kc, Ks, Vc, Vs, sl)
+    assert plx.get_device_status() == -7  # PLX_ERR_TIMEOUT
+    monkeypatch.delenv("PLX_FAULT_INJECT")
+    want = oracle.decode_fp8kv_ref(ref["q"], ref["r"], oKc, oKs, oVc, oVs, sl_host)
+    for _ in range(2):
+        out = plx.decode_fp8kv(dev["q"], dev["r"], Kc, Ks, Vc, Vs, sl)
+        assert plx.get_device_status() == 0
+        assert rel_err_rms(to_f64(out), want) <= BF16_TOL
