@@ -10,15 +10,17 @@
 //
 // The decode streams half the bytes of the bf16 decode (128 + 4 bytes per
 // cached row instead of 256), so the same HBM stream carries twice the keys.
-// The tensor cores take no mixed operands, and the score and value products
-// keep their bf16-decode precision:
-//   * scores, keys as the MMA's M:  S^T [128 keys x 16] = K_blk [Q; R]^T in
-//     f16: e4m3 converts exactly to f16 (one instruction per pair), and the
-//     converted K block goes to TMEM as the MMA's A operand, so it costs no
-//     shared-memory bandwidth.  q and rho are bf16 inputs; each row is scaled
-//     by a power of two 2^-e that brings its largest element into
-//     [2^14, 2^15) before the (then exact) conversion to f16, and the
-//     softmax threads undo 2^e and apply the key's scale in fp32.
+// The score and value products keep the bf16 decode's precision:
+//   * scores, keys as the MMA's M:  S^T [128 keys x N] = K_blk B^T as e4m3
+//     MMAs (kind::f8f6f4, K = 32) straight from the staged codes, with no
+//     conversion.  B holds each q and rho row as three e4m3 terms
+//     (hi + mid + lo, each the rounding of what the previous ones left):
+//     after the row is scaled by the power of two 2^-e that brings its
+//     largest element into [2^7, 2^8), three terms represent every bf16
+//     element exactly down to 2^-17 of the row's largest, so the three
+//     score columns of a row add up to the f32 score of the unrounded
+//     operand.  The softmax threads add them, undo 2^e and apply the key's
+//     scale in fp32.  N = 6G rounded up to 16.
 //   * values, dims as the MMA's M:  O^T [128 dims x 4G] += V_blk^T W in bf16:
 //     e4m3 codes convert exactly to bf16 (integer bit moves and one
 //     multiply by a power of two), and the value row's
@@ -29,9 +31,8 @@
 // blocks by TMA; warp 1 issues the MMAs; warps 2-3 build the q / rho operand
 // of each unit; warps 4-7 own one key each (scores, weights) and at the end
 // of a unit one dim each (output or partial record, merged by the last CTA of
-// a (b, KV head)); warps 8-15, two per TMEM lane quarter, own one key each
-// and convert half of its K row into TMEM and half of its V row into the bf16
-// value tile.
+// a (b, KV head)); warps 8-15, two per key (one per 64-dim half of its V
+// row), convert the value rows into the bf16 value tile.
 //
 // Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
 #include "plx_internal.cuh"
@@ -54,7 +55,7 @@ using namespace dtc;
 constexpr int D = 128;
 constexpr int kThreads = 512;
 constexpr int kQrWarp = 2, kFirstEw = 4, kFirstCv = 8;
-constexpr int kCvWarps = 8;  // two per TMEM lane quarter, each converting half of every row
+constexpr int kCvWarps = 8;  // two per 32 keys, each converting half of every value row
 // Register split (setmaxnreg, per warpgroup): the launch gives 512 x 128; the
 // control warpgroup and the two converter warpgroups hand registers to the
 // key warpgroup: 128 x 96 + 128 x 208 + 256 x 88 = 61,440 <= 65,536.
@@ -63,25 +64,32 @@ constexpr int kUnitRing = 4;
 constexpr int kStages = 4;       // raw e4m3 K + V blocks, 32 KB each
 constexpr int kScaleBox = kKeys + 4;   // scales per staged box (128 keys + up to 3 before them)
 constexpr int kScaleBoxPad = 160;      // box rounded up to 128 bytes
-constexpr int kRows = 16;        // q rows 0..G-1, rho rows 8..8+G-1 of the score operand
 constexpr float kLazyTau = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;
-// TMEM columns: two score stages, two value accumulators, two f16 K operands
-// (64 columns = 128 f16 dims each).
-constexpr uint32_t kColS = 0, kColO = 32, kColK = 128, kTmemCols = 256;
+// TMEM columns: two score stages (N columns each) from 0, two value
+// accumulators (NW columns each) from 128.
+constexpr uint32_t kColS = 0, kColO = 128, kTmemCols = 256;
+
+// Row of the score operand B holding term `term` (0 hi, 1 mid, 2 lo) of the
+// q (kind 0) or rho (kind 1) row of head h of the group.
+template <int G>
+__host__ __device__ constexpr int brow(int term, int kind, int h) {
+  return term * 2 * G + kind * G + h;
+}
 
 template <int G>
 struct SmemF {
   static constexpr int NW = 4 * G < 16 ? 16 : 4 * G;
+  static constexpr int NB = (6 * G + 15) / 16 * 16;  // score operand rows (the MMA's N)
   uint8_t raw[kStages][2][kKeys * 128];  // e4m3 [128 keys x 128 dims]: K, V
   uint8_t vc[2][2][kKeys * 128];         // bf16 V block per buffer: [128 keys x 64 dims] per half
-  uint8_t qr[2][2][kRows * 128];         // f16 q / rho operand per unit slot: [16 rows x 64 dims] per half
+  uint8_t qr[2][NB * 128];               // e4m3 q / rho terms per unit slot: [NB rows x 128 dims]
   uint8_t w[2][2][NW * 128];             // bf16 weights per block slot: [NW rows x 64 keys] per half
   // Per raw stage, the K and V scales of the block's keys: a box of kScaleBox
   // floats starting at the block's first key rounded down to a 16-byte boundary.
   alignas(128) float sc[kStages][2][kScaleBoxPad];
   uint64_t raw_full[kStages], raw_empty[kStages];
-  uint64_t kc_full[2], kc_free[2], vc_full[2], vc_free[2];
+  uint64_t vc_full[2], vc_free[2];
   uint64_t qr_full[2], qr_empty[2];
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t s_full[2], s_free[2], w_full[2], w_free[2];
@@ -91,7 +99,7 @@ struct SmemF {
   uint64_t drain;
   long long unit_ring[kUnitRing];
   int unit_n[kUnitRing];
-  int qexp[2][kRows];  // per unit slot: e of each q / rho row (the row was scaled by 2^-e)
+  int qexp[2][16];  // per unit slot: e of the q row of head h (h) and of its rho row (8 + h)
   float red[2][4][G];
   float sums[4][2 * G];
   int last;
@@ -104,17 +112,6 @@ static_assert(sizeof(SmemF<8>) + 1024 <= 227 * 1024, "shared memory of one CTA")
 __device__ unsigned long long g_f8_unit_next;
 __device__ unsigned int g_f8_cta_done;
 
-// 16 e4m3 codes -> 8 f16x2 words (element 2k in the low half of word k).
-__device__ __forceinline__ void e4m3x16_to_f16(const uint4 c, uint32_t (&h)[8]) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] & 0xffffu), __NV_E4M3);
-    const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[i] >> 16), __NV_E4M3);
-    h[2 * i] = (uint32_t)lo.x | ((uint32_t)lo.y << 16);
-    h[2 * i + 1] = (uint32_t)hi.x | ((uint32_t)hi.y << 16);
-  }
-}
 // 4 e4m3 codes (code 0 in the low byte) -> 2 bf16x2 words, exactly, on the
 // integer and FMA pipes (the conversion instructions share the XU pipe with
 // the exponentials and would bound the stream).  With a code in the high byte
@@ -153,15 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.raw_full[s], 1);
-      mbar_init(&sm.raw_empty[s], kCvWarps + 4);  // the converter warps and the four key warps
+      mbar_init(&sm.raw_empty[s], kCvWarps + 5);  // the converters, the key warps, the score MMAs' commit
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
       mbar_init(&sm.unit_empty[s], 7 + kCvWarps);  // MMA thread, 2 q / rho warps, 4 key warps, the converters
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.kc_full[s], kCvWarps);
-      mbar_init(&sm.kc_free[s], 1);
       mbar_init(&sm.vc_full[s], kCvWarps);
       mbar_init(&sm.vc_free[s], 1);
       mbar_init(&sm.qr_full[s], 2);
@@ -179,10 +174,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  // Operand rows no thread writes stay zero: the q / rho tile's rows G..7 and
-  // 8+G..15, and the weight tile's rows past 4G.
+  // Operand rows no thread writes stay zero: the q / rho tile's rows past 6G
+  // and the weight tile's rows past 4G.
   for (int x = threadIdx.x; x < (int)(sizeof(sm.qr) / 16); x += kThreads)
-    reinterpret_cast<uint4*>(&sm.qr[0][0][0])[x] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(&sm.qr[0][0])[x] = make_uint4(0u, 0u, 0u, 0u);
   for (int x = threadIdx.x; x < (int)(sizeof(sm.w) / 16); x += kThreads)
     reinterpret_cast<uint4*>(&sm.w[0][0][0])[x] = make_uint4(0u, 0u, 0u, 0u);
   fence_async_smem();
@@ -273,21 +268,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int ob = ou & 1;
         if (!(ok = mbar_wait(&sm.o_free[ob], ((ou >> 1) & 1) ^ 1, abort, a.status))) break;
-        const uint64_t bq = sdesc(smem_u32(sm.qr[qs][0]), 16, 1024);
-        // Scores of block bb: S^T = K [Q; R]^T with K (f16) from TMEM buffer bb & 1.
+        const uint64_t bq = sdesc(smem_u32(sm.qr[qs]), 16, 1024);
+        // Scores of block bb: S^T = K B^T, e4m3 x e4m3, K straight from its raw
+        // stage (K-major, 128-byte rows, 128B swizzle; 32 codes per K step).
         auto issue_scores = [&](uint32_t bb) -> bool {
-          const int kb = bb & 1, sb = bb & 1;
-          if (!mbar_wait(&sm.kc_full[kb], (bb >> 1) & 1, abort, a.status)) return false;
+          const int st = bb % kStages, sb = bb & 1;
+          if (!mbar_wait(&sm.raw_full[st], (bb / kStages) & 1, abort, a.status)) return false;
           if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
           tc_fence_after();
+          const uint64_t ak = sdesc(smem_u32(sm.raw[st][0]), 16, 1024);
 #pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks) {
-            const uint32_t ob2 = (ks >> 2) * (kRows * 128) + (ks & 3) * 32;
-            mma_ts(tmem + kColS + kRows * sb, tmem + kColK + 64 * kb + 8 * ks, bq + (uint64_t)(ob2 >> 4),
-                   idesc_f16kind(kRows, 0, 0, false), ks > 0 ? 1u : 0u);
-          }
+          for (int ks = 0; ks < D / 32; ++ks)
+            mma_ss_f8(tmem + kColS + Sm::NB * sb, ak + (uint64_t)((ks * 32) >> 4), bq + (uint64_t)((ks * 32) >> 4),
+                      idesc_e4m3(Sm::NB), ks > 0 ? 1u : 0u);
           mma_commit(&sm.s_full[sb]);
-          mma_commit(&sm.kc_free[kb]);
+          mma_commit(&sm.raw_empty[st]);  // the K codes are read
           return true;
         };
         if (!(ok = issue_scores(blk))) break;
@@ -324,10 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(&sm.drain, 0);
     }
   } else {
-    // ---------------- q / rho operand of each unit (f16, one power-of-two scale per row) ----------------
+    // ---------------- q / rho operand of each unit (three e4m3 terms, one power-of-two scale per row) ----------------
     const int t = threadIdx.x - 32 * kQrWarp;  // 0..63
-    const int row = t >> 2, quarter = t & 3;    // 16 rows x 4 quarters of 32 dims
-    const int head = row & 7;
+    const int row = t >> 2, quarter = t & 3;    // q rows 0..7, rho rows 8..15 (head = row & 7) x 4 quarters of 32 dims
+    const int kind = row >> 3, head = row & 7;
     const bool live = head < G;
     bool ok = true;
     for (int ui = 0; ok; ++ui) {
@@ -341,7 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4 v[4];
       float m = 0.f;
       if (live) {
-        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(row < 8 ? a.q : a.r) +
+        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(kind == 0 ? a.q : a.r) +
                                    ((long long)x.b * a.H + (long long)x.kvh * G + head) * D + 32 * quarter;
 #pragma unroll
         for (int c = 0; c < 4; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
@@ -357,22 +352,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      // 2^-e brings the largest element into [2^14, 2^15): the f16 conversion
-      // is then exact for every element not far below it.
-      const int e = (m > 0.f && m <= 3.4e38f) ? ilogbf(m) - 14 : 0;
+      // 2^-e brings the largest element into [2^7, 2^8) (below e4m3's 448).
+      const int e = (m > 0.f && m <= 3.4e38f) ? ilogbf(m) - 7 : 0;
       if (live) {
-        uint8_t* dst = sm.qr[qs][quarter >> 1];
+        // Per term, 32 codes (8 words of 4) of this quarter of the row.
+        uint32_t tw[3][8];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t wd[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          uint32_t hw[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const __half2 hh = __floats2half2_rn(ldexpf(__uint_as_float(wd[k] << 16), -e),
-                                                 ldexpf(__uint_as_float(wd[k] & 0xffff0000u), -e));
-            hw[k] = *reinterpret_cast<const uint32_t*>(&hh);
+            float2 y = make_float2(ldexpf(__uint_as_float(wd[k] << 16), -e),
+                                   ldexpf(__uint_as_float(wd[k] & 0xffff0000u), -e));
+#pragma unroll
+            for (int term = 0; term < 3; ++term) {
+              // Round what is left to e4m3 and keep the (exact) remainder.
+              const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
+              y.x -= __half2float(__ushort_as_half(hr.x));
+              y.y -= __half2float(__ushort_as_half(hr.y));
+              const int wi = 2 * c + (k >> 1);
+              if ((k & 1) == 0) {
+                tw[term][wi] = (uint32_t)p;
+              } else {
+                tw[term][wi] |= (uint32_t)p << 16;
+              }
+            }
           }
-          *reinterpret_cast<uint4*>(dst + sw128_chunk(row, 4 * (quarter & 1) + c)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+          uint8_t* dst = sm.qr[qs];
+          const int rr = brow<G>(term, kind, head);
+          *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * quarter)) =
+              make_uint4(tw[term][0], tw[term][1], tw[term][2], tw[term][3]);
+          *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * quarter + 1)) =
+              make_uint4(tw[term][4], tw[term][5], tw[term][6], tw[term][7]);
         }
         if (quarter == 0) sm.qexp[qs][row] = e;
       }
@@ -449,8 +464,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm.raw_empty[st]);
         if (!(ok = warp_wait(&sm.s_full[sb], (bb >> 1) & 1, abort, a.status))) break;
         tc_fence_after();
-        uint32_t sv16[kRows];
-        tmem_ld16(lb + kColS + kRows * sb, sv16);
+        uint32_t sc[Sm::NB];
+        tmem_ld_cols<Sm::NB>(lb + kColS + Sm::NB * sb, sc);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -458,8 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         float xs[G], tv[G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          xs[h] = valid ? __uint_as_float(sv16[h]) * (sk * fq[h]) : -CUDART_INF_F;
-          tv[h] = valid ? __uint_as_float(sv16[8 + h]) * (sk * fr[h]) : 0.f;
+          // hi + (mid + lo): the three terms' dot products with the key.
+          const float sq = __uint_as_float(sc[brow<G>(0, 0, h)]) +
+                           (__uint_as_float(sc[brow<G>(1, 0, h)]) + __uint_as_float(sc[brow<G>(2, 0, h)]));
+          const float sr = __uint_as_float(sc[brow<G>(0, 1, h)]) +
+                           (__uint_as_float(sc[brow<G>(1, 1, h)]) + __uint_as_float(sc[brow<G>(2, 1, h)]));
+          xs[h] = valid ? sq * (sk * fq[h]) : -CUDART_INF_F;
+          tv[h] = valid ? sr * (sk * fr[h]) : 0.f;
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -619,10 +639,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsConv));
-    // ---------------- converters: half of key r's K row to TMEM (f16), of its V row to the bf16 tile ----------------
-    const int cq = warp & 3, r = 32 * cq + lane;  // warp w reaches TMEM lanes 32 (w % 4) ..
-    const int half = (warp - kFirstCv) >> 2;       // dims 64 half .. 64 half + 63
-    const uint32_t lk = tmem + ((uint32_t)(32 * cq) << 16) + kColK;
+    // ---------------- converters: half of key r's V row to the bf16 value tile ----------------
+    const int cq = warp & 3, r = 32 * cq + lane;
+    const int half = (warp - kFirstCv) >> 2;  // dims 64 half .. 64 half + 63
     uint32_t pos = 0, blk = 0;
     bool ok = true;
     for (int ui = 0; ok; ++ui) {
@@ -634,28 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x.nblk == 0) continue;
       for (int i = 0; i < x.nblk; ++i) {
         const uint32_t p = pos + i, bb = blk + i;
-        const int st = p % kStages, kb = bb & 1, vb = bb & 1;
+        const int st = p % kStages, vb = bb & 1;
         if (!(ok = warp_wait(&sm.raw_full[st], (p / kStages) & 1, abort, a.status))) break;
-        // K: 128 codes -> 64 f16x2 columns of this thread's TMEM lane.
-        if (!(ok = warp_wait(&sm.kc_free[kb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
-        tc_fence_after();
-        const uint8_t* kr = sm.raw[st][0];
-#pragma unroll
-        for (int c2 = 2 * half; c2 < 2 * half + 2; ++c2) {
-          uint32_t cols[16];
-#pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            uint32_t h8[8];
-            e4m3x16_to_f16(*reinterpret_cast<const uint4*>(kr + sw128_chunk(r, 2 * c2 + hc)), h8);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) cols[8 * hc + k] = h8[k];
-          }
-          tmem_st16(lk + 64 * kb + 16 * c2, cols);
-        }
-        tc_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.kc_full[kb]);
         // V: 128 codes -> 128 bf16 in key row r of the value tile (rows past
         // the sequence are zeroed: the cache there may hold anything).
         if (!(ok = warp_wait(&sm.vc_free[vb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
@@ -683,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(&sm.vc_full[vb]);
-          mbar_arrive(&sm.raw_empty[st]);  // both rows of the stage are read
+          mbar_arrive(&sm.raw_empty[st]);  // the value codes are read
         }
       }
       if (!ok) break;

@@ -21,6 +21,11 @@ __host__ __device__ constexpr uint32_t idesc_f16kind(int n, int a_mn, int b_mn, 
          ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
 }
 __host__ __device__ constexpr uint32_t idesc(int n, int a_mn, int b_mn) { return idesc_f16kind(n, a_mn, b_mn, true); }
+// Instruction descriptor (kind::f8f6f4): D f32, M = 128, N = n, A and B e4m3
+// (type code 0), both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
 
 // Byte offset of element column `col` (2-byte elements) of row `row` in a
 // 128B-swizzled tile of 128-byte rows.
@@ -40,12 +45,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 template <int N>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[N]) {
   static_assert(N % 16 == 0 && N <= 64, "accumulator width");
-  if constexpr (N == 16) {
-    tmem_ld16(taddr, v);
-  } else {
 #pragma unroll
-    for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
-  }
+  for (int c = 0; c < N / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&v[32 * c]));
+  if constexpr (N % 32 == 16) tmem_ld16(taddr + (N - 16), *reinterpret_cast<uint32_t(*)[16]>(&v[N - 16]));
 }
 template <int N>
 __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[N]) {

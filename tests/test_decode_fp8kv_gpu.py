@@ -163,6 +163,34 @@ def test_fp8kv_true_normal(plx, key_scale):
     assert rel_err_rms(to_f64(out), want) <= BF16_TOL
 
 
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_fp8kv_wide_range_queries(plx, G):
+    """q and rho rows whose elements span many binades (|x| ~ 2^U(-12, 0)), and
+    rows with one element 2^10 times the rest: the score operand must keep the
+    small elements too.  Keys x 3 make the softmax sharp, so score errors show."""
+    B, Hkv, L, d = 3, 2, 700, 128
+    H = G * Hkv
+    rng = np.random.default_rng(140 + G)
+    def rms(x):
+        return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True))
+    def wide(shape):
+        return rng.standard_normal(shape) * 2.0 ** rng.uniform(-12, 0, shape)
+    qh = rms(wide((B, H, d)))
+    rh = 0.25 * rms(wide((B, H, d)))
+    qh[0, :, 5] *= 2.0 ** 10
+    rh[1, :, 77] *= 2.0 ** 10
+    q, qr = _bf16(qh)
+    r, rr = _bf16(rh)
+    K, Kr = _bf16(3.0 * rms(rng.standard_normal((B, Hkv, L, d))))
+    V, Vr = _bf16(rng.standard_normal((B, Hkv, L, d)))
+    gpu, orc = _fp8_case(plx, K, V, Kr, Vr)
+    sl = np.array([700, 129, 512], dtype=np.int32)
+    out = plx.decode_fp8kv(q, r, *gpu, torch.from_numpy(sl).cuda())
+    assert plx.get_device_status() == 0
+    want = oracle.decode_fp8kv_ref(qr, rr, *orc, sl)
+    assert rel_err_rms(to_f64(out), want) <= BF16_TOL
+
+
 @pytest.mark.parametrize("Hkv", [16, 4])
 def test_fp8kv_decode_workload_sampled(plx, Hkv):
     """The decode workload's shape (B=64, H=16, L=4096, d=128, all lengths 4096)
