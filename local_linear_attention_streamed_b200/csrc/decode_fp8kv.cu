@@ -28,11 +28,15 @@
 //     hi + lo pair), so omega and T stay plain sums of w and w t.
 // Roles (one persistent CTA per SM, units = (b, KV head, key chunk) from a
 // global counter, as in the bf16 decode): warp 0 stages raw e4m3 K and V
-// blocks by TMA; warp 1 issues the MMAs; warps 2-3 build the q / rho operand
-// of each unit; warps 4-7 own one key each (scores, weights) and at the end
-// of a unit one dim each (output or partial record, merged by the last CTA of
-// a (b, KV head)); warps 8-15, two per key (one per 64-dim half of its V
-// row), convert the value rows into the bf16 value tile.
+// blocks by TMA; for groups of 1 and 2 warp 1 issues the score MMAs and warp 3
+// the value MMAs (one issuing thread each: an issue waits for the tensor pipe
+// to take the MMA, and either thread's barrier waits then overlap the other's
+// issues), for larger groups warp 1 issues both; warp 2 builds the q / rho
+// operand of each unit; warps 4-7 own one key each
+// (scores, weights) and at the end of a unit one dim each (output or partial
+// record, merged by the last CTA of a (b, KV head)); warps 8-15, two per key
+// (one per 64-dim half of its V row), convert the value rows into the bf16
+// value tile.
 //
 // Formulas: rainbus.top summary "方法步骤详情"; out = ((1 + T/omega) O1 - O2) / omega.
 #include "plx_internal.cuh"
@@ -54,16 +58,15 @@ using namespace dtc;
 
 constexpr int D = 128;
 constexpr int kThreads = 512;
-constexpr int kQrWarp = 2, kFirstEw = 4, kFirstCv = 8;
+constexpr int kQrWarp = 2, kPVWarp = 3, kFirstEw = 4, kFirstCv = 8;
 constexpr int kCvWarps = 8;  // two per 32 keys, each converting half of every value row
 // Register split (setmaxnreg, per warpgroup): the launch gives 512 x 128; the
 // control warpgroup and the two converter warpgroups hand registers to the
 // key warpgroup: 128 x 96 + 128 x 208 + 256 x 88 = 61,440 <= 65,536.
 constexpr int kRegsControl = 96, kRegsKey = 208, kRegsConv = 88;
 constexpr int kUnitRing = 4;
-constexpr int kStages = 4;       // raw e4m3 K + V blocks, 32 KB each
 constexpr int kScaleBox = kKeys + 4;   // scales per staged box (128 keys + up to 3 before them)
-constexpr int kScaleBoxPad = 160;      // box rounded up to 128 bytes
+constexpr int kScaleBoxPad = 160;      // box rounded up to 128 bytes (a tensor copy's destination alignment)
 constexpr float kLazyTau = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;
 // TMEM columns: two score stages (N columns each) from 0, two value
@@ -81,6 +84,7 @@ template <int G>
 struct SmemF {
   static constexpr int NW = 4 * G < 16 ? 16 : 4 * G;
   static constexpr int NB = (6 * G + 15) / 16 * 16;  // score operand rows (the MMA's N)
+  static constexpr int kStages = 4;      // raw stages in flight (as many as shared memory holds)
   uint8_t raw[kStages][2][kKeys * 128];  // e4m3 [128 keys x 128 dims]: K, V
   uint8_t vc[2][2][kKeys * 128];         // bf16 V block per buffer: [128 keys x 64 dims] per half
   uint8_t qr[2][NB * 128];               // e4m3 q / rho terms per unit slot: [NB rows x 128 dims]
@@ -107,7 +111,8 @@ struct SmemF {
   int abort;
 };
 
-static_assert(sizeof(SmemF<8>) + 1024 <= 227 * 1024, "shared memory of one CTA");
+static_assert(sizeof(SmemF<8>) + 1024 <= 227 * 1024 && sizeof(SmemF<4>) + 1024 <= 227 * 1024,
+              "shared memory of one CTA");
 
 __device__ unsigned long long g_f8_unit_next;
 __device__ unsigned int g_f8_cta_done;
@@ -140,6 +145,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         DecodeArgs a) {
   using Sm = SmemF<G>;
   constexpr int NW = Sm::NW;
+  constexpr int kStages = Sm::kStages;
+  // Small groups issue scores and values from two threads; from 4 heads a
+  // group, where the key warps bound the block period, one thread issues
+  // both in the order the key warps consume them (measured faster there).
+  constexpr bool kSplit = G <= 2;
+  // The q / rho operand is built by warp 2, and by warp 3 as well when that
+  // warp issues no MMAs: kQrParts threads per operand row.
+  constexpr int kQrWarps = kSplit ? 1 : 2, kQrParts = 2 * kQrWarps, kQPT = 4 / kQrParts;
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Sm& sm = *reinterpret_cast<Sm*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -154,23 +167,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
-      mbar_init(&sm.unit_empty[s], 7 + kCvWarps);  // MMA thread, 2 q / rho warps, 4 key warps, the converters
+      // The MMA thread(s), the q / rho warp(s), 4 key warps, the converters.
+      mbar_init(&sm.unit_empty[s], 7 + kCvWarps);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.vc_full[s], kCvWarps);
       mbar_init(&sm.vc_free[s], 1);
-      mbar_init(&sm.qr_full[s], 2);
+      mbar_init(&sm.qr_full[s], kQrWarps);
       mbar_init(&sm.qr_empty[s], 5);  // the MMA thread's commit and the four key warps
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.s_free[s], 4);
-      mbar_init(&sm.w_full[s], 128);
+      mbar_init(&sm.w_full[s], 4);  // one arrival per key warp
       mbar_init(&sm.w_free[s], 1);
       mbar_init(&sm.o_full[s], 1);
       mbar_init(&sm.o_free[s], 4);
       mbar_init(&sm.vote[s], 4);
     }
     mbar_init(&sm.rdv, 4);
-    mbar_init(&sm.drain, 1);
+    mbar_init(&sm.drain, kSplit ? 2 : 1);  // one commit from each MMA issuer
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -209,20 +223,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------- TMA producer: units and raw e4m3 K / V blocks ----------------
     if (lane == 0) {
-      long long u = blockIdx.x;
       uint32_t pos = 0;
       int last_kv[kStages];
       for (int s = 0; s < kStages; ++s) last_kv[s] = -1;
-      for (int ui = 0;; ++ui) {
+      // Units are published one ahead of their loads, so the roles that
+      // prepare a unit (the q / rho operand, read from global memory behind
+      // the cache stream) have the whole previous unit to do it.
+      auto publish = [&](int ui, long long uu, int& n) -> bool {
         const int slot = ui % kUnitRing;
-        if (!mbar_wait(&sm.unit_empty[slot], ((ui / kUnitRing) & 1) ^ 1, abort, a.status)) break;
-        const long long uu = u < units ? u : -1;
-        const int n = uu < 0 ? 0 : a.seqlens[unit_row(uu, 1, a)];
+        if (!mbar_wait(&sm.unit_empty[slot], ((ui / kUnitRing) & 1) ^ 1, abort, a.status)) return false;
+        n = uu < 0 ? 0 : a.seqlens[unit_row(uu, 1, a)];
         sm.unit_ring[slot] = uu;
         sm.unit_n[slot] = n;
         mbar_arrive(&sm.unit_full[slot]);
-        if (uu < 0) break;
-        const long long next = (long long)gridDim.x + (long long)atomicAdd(&g_f8_unit_next, 1ull);
+        return true;
+      };
+      long long uu = blockIdx.x;  // the grid never exceeds the unit count
+      int n = 0;
+      bool live = publish(0, uu, n);
+      for (int ui = 1; live; ++ui) {
+        long long nx = (long long)gridDim.x + (long long)atomicAdd(&g_f8_unit_next, 1ull);
+        if (nx >= units) nx = -1;
+        int nn = 0;
+        if (!publish(ui, nx, nn)) break;
         const Unit x = unit_of(uu, n, 1, a);
         bool ok = true;
         for (int i = 0; i < x.nblk; ++i, ++pos) {
@@ -240,7 +263,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_1d(sm.sc[st][1], &tmVs, &sm.raw_full[st], row & ~3);
         }
         if (!ok) break;
-        u = next;
+        uu = nx;
+        n = nn;
+        live = uu >= 0;
       }
       if (*abort) {
         for (int s = 0; s < kStages; ++s)
@@ -248,80 +273,172 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      uint32_t blk = 0, ou = 0;
-      bool ok = true;
-      for (int ui = 0; ok; ++ui) {
-        const int slot = ui % kUnitRing;
-        if (!(ok = mbar_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
-        const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
-        const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
-        mbar_arrive(&sm.unit_empty[slot]);
-        if (uu < 0) break;
-        const Unit x = unit_of(uu, n, 1, a);
-        const int qs = ui & 1;
-        if (!(ok = mbar_wait(&sm.qr_full[qs], (ui >> 1) & 1, abort, a.status))) break;
-        if (x.nblk == 0) {
-          mbar_arrive(&sm.qr_empty[qs]);
-          continue;
-        }
-        const int ob = ou & 1;
-        if (!(ok = mbar_wait(&sm.o_free[ob], ((ou >> 1) & 1) ^ 1, abort, a.status))) break;
-        const uint64_t bq = sdesc(smem_u32(sm.qr[qs]), 16, 1024);
-        // Scores of block bb: S^T = K B^T, e4m3 x e4m3, K straight from its raw
-        // stage (K-major, 128-byte rows, 128B swizzle; 32 codes per K step).
-        auto issue_scores = [&](uint32_t bb) -> bool {
-          const int st = bb % kStages, sb = bb & 1;
-          if (!mbar_wait(&sm.raw_full[st], (bb / kStages) & 1, abort, a.status)) return false;
-          if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
-          tc_fence_after();
-          const uint64_t ak = sdesc(smem_u32(sm.raw[st][0]), 16, 1024);
-#pragma unroll
-          for (int ks = 0; ks < D / 32; ++ks)
-            mma_ss_f8(tmem + kColS + Sm::NB * sb, ak + (uint64_t)((ks * 32) >> 4), bq + (uint64_t)((ks * 32) >> 4),
-                      idesc_e4m3(Sm::NB), ks > 0 ? 1u : 0u);
-          mma_commit(&sm.s_full[sb]);
-          mma_commit(&sm.raw_empty[st]);  // the K codes are read
-          return true;
-        };
-        if (!(ok = issue_scores(blk))) break;
-        for (int i = 0; i < x.nblk; ++i) {
-          const uint32_t bb = blk + i;
-          if (i + 1 < x.nblk) {
-            if (!(ok = issue_scores(bb + 1))) break;
-          } else {
-            mma_commit(&sm.qr_empty[qs]);  // every score MMA of the unit is issued
+    if constexpr (kSplit) {
+      // ---------------- score MMA issuer ----------------
+      if (lane == 0) {
+        uint32_t blk = 0;
+        bool ok = true;
+        for (int ui = 0; ok; ++ui) {
+          const int slot = ui % kUnitRing;
+          if (!(ok = mbar_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
+          const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
+          const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
+          mbar_arrive(&sm.unit_empty[slot]);
+          if (uu < 0) break;
+          const Unit x = unit_of(uu, n, 1, a);
+          const int qs = ui & 1;
+          if (!(ok = mbar_wait(&sm.qr_full[qs], (ui >> 1) & 1, abort, a.status))) break;
+          if (x.nblk == 0) {
+            mbar_arrive(&sm.qr_empty[qs]);
+            continue;
           }
-          const int sb = bb & 1, vb = bb & 1;
-          if (!(ok = mbar_wait(&sm.w_full[sb], (bb >> 1) & 1, abort, a.status))) break;
-          if (!(ok = mbar_wait(&sm.vc_full[vb], (bb >> 1) & 1, abort, a.status))) break;
-          tc_fence_after();
-          // V^T as an MN-major A operand: the two 64-dim halves LBO apart,
-          // 8-key groups 1024 bytes apart, 16 keys (one K step) 2048 bytes.
-          const uint64_t av = sdesc(smem_u32(sm.vc[vb][0]), kKeys * 128, 1024);
-          const uint64_t bw = sdesc(smem_u32(sm.w[sb][0]), 16, 1024);
-#pragma unroll
-          for (int ks = 0; ks < kKeys / 16; ++ks) {
-            const uint32_t ow = (ks >> 2) * (NW * 128) + (ks & 3) * 32;
-            mma_ss(tmem + kColO + NW * ob, av + (uint64_t)((ks * 2048) >> 4), bw + (uint64_t)(ow >> 4),
-                   idesc(NW, 1, 0), (i > 0 || ks > 0) ? 1u : 0u);
+          const uint64_t bq = sdesc(smem_u32(sm.qr[qs]), 16, 1024);
+          // Scores of block bb: S^T = K B^T, e4m3 x e4m3, K straight from its raw
+          // stage (K-major, 128-byte rows, 128B swizzle; 32 codes per K step).
+          for (int i = 0; i < x.nblk; ++i) {
+            const uint32_t bb = blk + i;
+            const int st = bb % kStages, sb = bb & 1;
+            if (!(ok = mbar_wait(&sm.raw_full[st], (bb / kStages) & 1, abort, a.status))) break;
+            if (!(ok = mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
+            tc_fence_after();
+            const uint64_t ak = sdesc(smem_u32(sm.raw[st][0]), 16, 1024);
+  #pragma unroll
+            for (int ks = 0; ks < D / 32; ++ks)
+              mma_ss_f8(tmem + kColS + Sm::NB * sb, ak + (uint64_t)((ks * 32) >> 4), bq + (uint64_t)((ks * 32) >> 4),
+                        idesc_e4m3(Sm::NB), ks > 0 ? 1u : 0u);
+            mma_commit(&sm.s_full[sb]);
+            mma_commit(&sm.raw_empty[st]);  // the K codes are read
           }
-          mma_commit(&sm.w_free[sb]);
-          mma_commit(&sm.vc_free[vb]);
+          if (!ok) break;
+          mma_commit(&sm.qr_empty[qs]);  // every score MMA of the unit is issued
+          blk += x.nblk;
         }
-        if (!ok) break;
-        mma_commit(&sm.o_full[ob]);
-        blk += x.nblk;
-        ++ou;
+        mma_commit(&sm.drain);
+        mbar_drain(&sm.drain, 0);
       }
-      mma_commit(&sm.drain);
-      mbar_drain(&sm.drain, 0);
+    } else {
+      // ---------------- MMA issuer: the scores of block i + 1, then the values of block i ----------------
+      if (lane == 0) {
+        uint32_t blk = 0, ou = 0;
+        bool ok = true;
+        for (int ui = 0; ok; ++ui) {
+          const int slot = ui % kUnitRing;
+          if (!(ok = mbar_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
+          const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
+          const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
+          mbar_arrive(&sm.unit_empty[slot]);
+          if (uu < 0) break;
+          const Unit x = unit_of(uu, n, 1, a);
+          const int qs = ui & 1;
+          if (!(ok = mbar_wait(&sm.qr_full[qs], (ui >> 1) & 1, abort, a.status))) break;
+          if (x.nblk == 0) {
+            mbar_arrive(&sm.qr_empty[qs]);
+            continue;
+          }
+          const int ob = ou & 1;
+          if (!(ok = mbar_wait(&sm.o_free[ob], ((ou >> 1) & 1) ^ 1, abort, a.status))) break;
+          const uint64_t bq = sdesc(smem_u32(sm.qr[qs]), 16, 1024);
+          // Scores of block bb: S^T = K B^T, e4m3 x e4m3, K straight from its raw
+          // stage (K-major, 128-byte rows, 128B swizzle; 32 codes per K step).
+          auto issue_scores = [&](uint32_t bb) -> bool {
+            const int st = bb % kStages, sb = bb & 1;
+            if (!mbar_wait(&sm.raw_full[st], (bb / kStages) & 1, abort, a.status)) return false;
+            if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
+            tc_fence_after();
+            const uint64_t ak = sdesc(smem_u32(sm.raw[st][0]), 16, 1024);
+  #pragma unroll
+            for (int ks = 0; ks < D / 32; ++ks)
+              mma_ss_f8(tmem + kColS + Sm::NB * sb, ak + (uint64_t)((ks * 32) >> 4), bq + (uint64_t)((ks * 32) >> 4),
+                        idesc_e4m3(Sm::NB), ks > 0 ? 1u : 0u);
+            mma_commit(&sm.s_full[sb]);
+            mma_commit(&sm.raw_empty[st]);  // the K codes are read
+            return true;
+          };
+          if (!(ok = issue_scores(blk))) break;
+          for (int i = 0; i < x.nblk; ++i) {
+            const uint32_t bb = blk + i;
+            if (i + 1 < x.nblk) {
+              if (!(ok = issue_scores(bb + 1))) break;
+            } else {
+              mma_commit(&sm.qr_empty[qs]);  // every score MMA of the unit is issued
+            }
+            const int sb = bb & 1, vb = bb & 1;
+            if (!(ok = mbar_wait(&sm.w_full[sb], (bb >> 1) & 1, abort, a.status))) break;
+            if (!(ok = mbar_wait(&sm.vc_full[vb], (bb >> 1) & 1, abort, a.status))) break;
+            tc_fence_after();
+            // V^T as an MN-major A operand: the two 64-dim halves LBO apart,
+            // 8-key groups 1024 bytes apart, 16 keys (one K step) 2048 bytes.
+            const uint64_t av = sdesc(smem_u32(sm.vc[vb][0]), kKeys * 128, 1024);
+            const uint64_t bw = sdesc(smem_u32(sm.w[sb][0]), 16, 1024);
+  #pragma unroll
+            for (int ks = 0; ks < kKeys / 16; ++ks) {
+              const uint32_t ow = (ks >> 2) * (NW * 128) + (ks & 3) * 32;
+              mma_ss(tmem + kColO + NW * ob, av + (uint64_t)((ks * 2048) >> 4), bw + (uint64_t)(ow >> 4),
+                     idesc(NW, 1, 0), (i > 0 || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.w_free[sb]);
+            mma_commit(&sm.vc_free[vb]);
+          }
+          if (!ok) break;
+          mma_commit(&sm.o_full[ob]);
+          blk += x.nblk;
+          ++ou;
+        }
+        mma_commit(&sm.drain);
+        mbar_drain(&sm.drain, 0);
+      }
+    }
+  } else if (kSplit && warp == kPVWarp) {
+    {
+      // ---------------- value MMA issuer ----------------
+      if (lane == 0) {
+        uint32_t blk = 0, ou = 0;
+        bool ok = true;
+        for (int ui = 0; ok; ++ui) {
+          const int slot = ui % kUnitRing;
+          if (!(ok = mbar_wait(&sm.unit_full[slot], (ui / kUnitRing) & 1, abort, a.status))) break;
+          const long long uu = *reinterpret_cast<volatile long long*>(&sm.unit_ring[slot]);
+          const int n = *reinterpret_cast<volatile int*>(&sm.unit_n[slot]);
+          mbar_arrive(&sm.unit_empty[slot]);
+          if (uu < 0) break;
+          const Unit x = unit_of(uu, n, 1, a);
+          if (x.nblk == 0) continue;
+          const int ob = ou & 1;
+          if (!(ok = mbar_wait(&sm.o_free[ob], ((ou >> 1) & 1) ^ 1, abort, a.status))) break;
+          for (int i = 0; i < x.nblk; ++i) {
+            const uint32_t bb = blk + i;
+            const int sb = bb & 1, vb = bb & 1;
+            if (!(ok = mbar_wait(&sm.w_full[sb], (bb >> 1) & 1, abort, a.status))) break;
+            if (!(ok = mbar_wait(&sm.vc_full[vb], (bb >> 1) & 1, abort, a.status))) break;
+            tc_fence_after();
+            // V^T as an MN-major A operand: the two 64-dim halves LBO apart,
+            // 8-key groups 1024 bytes apart, 16 keys (one K step) 2048 bytes.
+            const uint64_t av = sdesc(smem_u32(sm.vc[vb][0]), kKeys * 128, 1024);
+            const uint64_t bw = sdesc(smem_u32(sm.w[sb][0]), 16, 1024);
+  #pragma unroll
+            for (int ks = 0; ks < kKeys / 16; ++ks) {
+              const uint32_t ow = (ks >> 2) * (NW * 128) + (ks & 3) * 32;
+              mma_ss(tmem + kColO + NW * ob, av + (uint64_t)((ks * 2048) >> 4), bw + (uint64_t)(ow >> 4),
+                     idesc(NW, 1, 0), (i > 0 || ks > 0) ? 1u : 0u);
+            }
+            mma_commit(&sm.w_free[sb]);
+            mma_commit(&sm.vc_free[vb]);
+          }
+          if (!ok) break;
+          mma_commit(&sm.o_full[ob]);
+          blk += x.nblk;
+          ++ou;
+        }
+        mma_commit(&sm.drain);
+        mbar_drain(&sm.drain, 0);
+      }
     }
   } else {
     // ---------------- q / rho operand of each unit (three e4m3 terms, one power-of-two scale per row) ----------------
-    const int t = threadIdx.x - 32 * kQrWarp;  // 0..63
-    const int row = t >> 2, quarter = t & 3;    // q rows 0..7, rho rows 8..15 (head = row & 7) x 4 quarters of 32 dims
+    // q rows 0..7, rho rows 8..15 (head = row & 7), kQrParts threads a row
+    // (kQPT quarters of 32 dims each).
+    const int t = threadIdx.x - 32 * kQrWarp;
+    const int row = t / kQrParts, hf = t % kQrParts;
     const int kind = row >> 3, head = row & 7;
     const bool live = head < G;
     bool ok = true;
@@ -333,16 +450,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Unit x = unit_of(uu, n, 1, a);
       const int qs = ui & 1;
       if (!(ok = warp_wait(&sm.qr_empty[qs], ((ui >> 1) & 1) ^ 1, abort, a.status))) break;
-      uint4 v[4];
+      // The row's largest magnitude first; the conversion reads the row again
+      // (from L1) a quarter at a time, which keeps this warpgroup's registers low.
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(kind == 0 ? a.q : a.r) +
+          ((long long)x.b * a.H + (long long)x.kvh * G + head) * D + 32 * kQPT * hf);
       float m = 0.f;
       if (live) {
-        const __nv_bfloat16* src = reinterpret_cast<const __nv_bfloat16*>(kind == 0 ? a.q : a.r) +
-                                   ((long long)x.b * a.H + (long long)x.kvh * G + head) * D + 32 * quarter;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) v[c] = __ldg(reinterpret_cast<const uint4*>(src) + c);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wd[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        for (int c = 0; c < 4 * kQPT; ++c) {
+          const uint4 vc = __ldg(src + c);
+          const uint32_t wd[4] = {vc.x, vc.y, vc.z, vc.w};
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             m = fmaxf(m, fabsf(__uint_as_float(wd[k] << 16)));
@@ -350,46 +468,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+#pragma unroll
+      for (int o = 1; o < kQrParts; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       // 2^-e brings the largest element into [2^7, 2^8) (below e4m3's 448).
       const int e = (m > 0.f && m <= 3.4e38f) ? ilogbf(m) - 7 : 0;
       if (live) {
-        // Per term, 32 codes (8 words of 4) of this quarter of the row.
-        uint32_t tw[3][8];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wd[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        for (int qq = 0; qq < kQPT; ++qq) {
+          // Per term, the 32 codes (8 words of 4) of dims 32 (kQPT hf + qq) ..
+          uint32_t tw[3][8];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float2 y = make_float2(ldexpf(__uint_as_float(wd[k] << 16), -e),
-                                   ldexpf(__uint_as_float(wd[k] & 0xffff0000u), -e));
+          for (int c = 0; c < 4; ++c) {
+            const uint4 vc = __ldg(src + 4 * qq + c);
+            const uint32_t wd[4] = {vc.x, vc.y, vc.z, vc.w};
 #pragma unroll
-            for (int term = 0; term < 3; ++term) {
-              // Round what is left to e4m3 and keep the (exact) remainder.
-              const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
-              const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
-              y.x -= __half2float(__ushort_as_half(hr.x));
-              y.y -= __half2float(__ushort_as_half(hr.y));
-              const int wi = 2 * c + (k >> 1);
-              if ((k & 1) == 0) {
-                tw[term][wi] = (uint32_t)p;
-              } else {
-                tw[term][wi] |= (uint32_t)p << 16;
+            for (int k = 0; k < 4; ++k) {
+              float2 y = make_float2(ldexpf(__uint_as_float(wd[k] << 16), -e),
+                                     ldexpf(__uint_as_float(wd[k] & 0xffff0000u), -e));
+#pragma unroll
+              for (int term = 0; term < 3; ++term) {
+                // Round what is left to e4m3 and keep the (exact) remainder.
+                const __nv_fp8x2_storage_t p = __nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3);
+                const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(p, __NV_E4M3);
+                y.x -= __half2float(__ushort_as_half(hr.x));
+                y.y -= __half2float(__ushort_as_half(hr.y));
+                const int wi = 2 * c + (k >> 1);
+                if ((k & 1) == 0) {
+                  tw[term][wi] = (uint32_t)p;
+                } else {
+                  tw[term][wi] |= (uint32_t)p << 16;
+                }
               }
             }
           }
-        }
+          const int q4 = kQPT * hf + qq;  // 32-dim quarter: 16-byte chunks 2 q4, 2 q4 + 1
 #pragma unroll
-        for (int term = 0; term < 3; ++term) {
-          uint8_t* dst = sm.qr[qs];
-          const int rr = brow<G>(term, kind, head);
-          *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * quarter)) =
-              make_uint4(tw[term][0], tw[term][1], tw[term][2], tw[term][3]);
-          *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * quarter + 1)) =
-              make_uint4(tw[term][4], tw[term][5], tw[term][6], tw[term][7]);
+          for (int term = 0; term < 3; ++term) {
+            uint8_t* dst = sm.qr[qs];
+            const int rr = brow<G>(term, kind, head);
+            *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * q4)) =
+                make_uint4(tw[term][0], tw[term][1], tw[term][2], tw[term][3]);
+            *reinterpret_cast<uint4*>(dst + sw128_chunk(rr, 2 * q4 + 1)) =
+                make_uint4(tw[term][4], tw[term][5], tw[term][6], tw[term][7]);
+          }
         }
-        if (quarter == 0) sm.qexp[qs][row] = e;
+        if (hf == 0) sm.qexp[qs][row] = e;
       }
       fence_async_smem();
       __syncwarp();
@@ -542,7 +665,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 3, kk)) = tlo;
         }
         fence_async_smem();
-        mbar_arrive(&sm.w_full[sb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.w_full[sb]);
       }
       if (!ok) break;
       // ---- End of the unit: thread r holds dim r of the accumulator.
