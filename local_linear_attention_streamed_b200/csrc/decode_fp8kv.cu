@@ -104,7 +104,7 @@ struct SmemF {
   long long unit_ring[kUnitRing];
   int unit_n[kUnitRing];
   int qexp[2][16];  // per unit slot: e of the q row of head h (h) and of its rho row (8 + h)
-  float red[2][4][G];
+  alignas(16) float red[2][4][G];  // per-warp block maxima of each head
   float sums[4][2 * G];
   int last;
   uint32_t tmem_base;
@@ -604,21 +604,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           xs[h] = valid ? sq * (sk * fq[h]) : -CUDART_INF_F;
           tv[h] = valid ? sr * (sk * fr[h]) : 0.f;
         }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          float mx = xs[h];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          if (lane == 0) sm.red[sb][q][h] = mx;
+        {
+          const float mx = warp_max_scatter<G>(xs, lane);  // head lane / (32 / G)
+          if ((lane & (32 / G - 1)) == 0) sm.red[sb][q][lane / (32 / G)] = mx;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.vote[sb]);
         if (!(ok = warp_wait(&sm.vote[sb], (bb >> 1) & 1, abort, a.status))) break;
         bool raised = false;
-        float alpha[G];
+        float alpha[G], mb[G];
+        block_max4<G>(sm.red[sb], mb);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
-          const float mblk = fmaxf(fmaxf(sm.red[sb][0][h], sm.red[sb][1][h]), fmaxf(sm.red[sb][2][h], sm.red[sb][3][h]));
+          const float mblk = mb[h];
           const bool up = mblk > hm[h] + kLazyTau;
           alpha[h] = up ? exp2f(hm[h] - mblk) : 1.f;
           hm[h] = up ? mblk : hm[h];

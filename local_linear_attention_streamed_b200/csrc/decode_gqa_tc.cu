@@ -94,7 +94,7 @@ struct Smem {
   uint64_t drain;
   long long unit_ring[kUnitRing];
   int unit_n[kUnitRing];  // seqlens of the unit's batch row, read once by the producer
-  float red[2][4][Gm::kHeads];    // per-warp block maxima of each head
+  alignas(16) float red[2][4][Gm::kHeads];  // per-warp block maxima of each head
   float sums[4][2 * Gm::kHeads];  // per-warp omega and T of each head
   int last;
   uint32_t tmem_base;
@@ -373,21 +373,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tv[h] = valid ? __uint_as_float(sv[col + 8]) : 0.f;
         }
         // Block max of every head over the four warps' keys.
-#pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          float mx = xs[h];
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          if (lane == 0) sm.red[sb][q][h] = mx;
+        {
+          const float mx = warp_max_scatter<kHeads>(xs, lane);  // head lane / (32 / kHeads)
+          if ((lane & (32 / kHeads - 1)) == 0) sm.red[sb][q][lane / (32 / kHeads)] = mx;
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.vote[sb]);
         if (!(ok = warp_wait(&sm.vote[sb], (bb >> 1) & 1, abort, a.status))) break;
         bool raised = false;
-        float alpha[kHeads];
+        float alpha[kHeads], mb[kHeads];
+        block_max4<kHeads>(sm.red[sb], mb);
 #pragma unroll
         for (int h = 0; h < kHeads; ++h) {
-          const float mblk = fmaxf(fmaxf(sm.red[sb][0][h], sm.red[sb][1][h]), fmaxf(sm.red[sb][2][h], sm.red[sb][3][h]));
+          const float mblk = mb[h];
           const bool up = mblk > hm[h] + kLazyTau;  // always on the unit's first block (m = -inf)
           alpha[h] = up ? exp2f(hm[h] - mblk) : 1.f;
           hm[h] = up ? mblk : hm[h];

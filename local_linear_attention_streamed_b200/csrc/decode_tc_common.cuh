@@ -60,6 +60,62 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)
   }
 }
 
+// Warp maxima of H values per lane (H a power of two <= 32) in H - 1 + 5 -
+// log2 H shuffles instead of 5 H: a reduce-scatter (at each step a lane keeps
+// half of its values and takes the partner's maxima of that half), then a
+// butterfly over the remaining lanes.  Afterwards lane l holds the maximum
+// over the warp of value number l / (32 / H).
+template <int N, int O>
+struct MaxScatter {
+  template <int H>
+  static __device__ __forceinline__ void run(float (&v)[H], int lane) {
+    const bool upper = (lane & O) != 0;
+#pragma unroll
+    for (int j = 0; j < N / 2; ++j) {
+      const float keep = upper ? v[j + N / 2] : v[j];
+      const float give = upper ? v[j] : v[j + N / 2];
+      v[j] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, give, O));
+    }
+    MaxScatter<N / 2, O / 2>::run(v, lane);
+  }
+};
+template <int O>
+struct MaxScatter<1, O> {
+  template <int H>
+  static __device__ __forceinline__ void run(float (&v)[H], int) {
+#pragma unroll
+    for (int o = O; o > 0; o >>= 1) v[0] = fmaxf(v[0], __shfl_xor_sync(0xffffffffu, v[0], o));
+  }
+};
+template <int H>
+__device__ __forceinline__ float warp_max_scatter(const float (&x)[H], int lane) {
+  static_assert(H >= 1 && H <= 32 && (H & (H - 1)) == 0, "a power of two");
+  float v[H];
+#pragma unroll
+  for (int j = 0; j < H; ++j) v[j] = x[j];
+  MaxScatter<H, 16>::run(v, lane);
+  return v[0];
+}
+// The block maxima of H values: each of 4 warps wrote its row red[w][0..H)
+// (16-byte aligned rows when H % 4 == 0).
+template <int H>
+__device__ __forceinline__ void block_max4(const float (&red)[4][H], float (&m)[H]) {
+  if constexpr (H % 4 == 0) {
+#pragma unroll
+    for (int c = 0; c < H / 4; ++c) {
+      const float4 a = reinterpret_cast<const float4*>(red[0])[c], b = reinterpret_cast<const float4*>(red[1])[c];
+      const float4 e = reinterpret_cast<const float4*>(red[2])[c], f = reinterpret_cast<const float4*>(red[3])[c];
+      m[4 * c + 0] = fmaxf(fmaxf(a.x, b.x), fmaxf(e.x, f.x));
+      m[4 * c + 1] = fmaxf(fmaxf(a.y, b.y), fmaxf(e.y, f.y));
+      m[4 * c + 2] = fmaxf(fmaxf(a.z, b.z), fmaxf(e.z, f.z));
+      m[4 * c + 3] = fmaxf(fmaxf(a.w, b.w), fmaxf(e.w, f.w));
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < H; ++h) m[h] = fmaxf(fmaxf(red[0][h], red[1][h]), fmaxf(red[2][h], red[3][h]));
+  }
+}
+
 // What every role derives from a unit index: unit u covers KV heads
 // kvh .. kvh + kPair - 1 of batch row b (bkv = b Hkv + kvh) over key chunk c.
 struct Unit {
