@@ -52,8 +52,7 @@ using namespace sm100;
 using namespace dtc;
 
 constexpr int kUnitRing = 4;
-constexpr int kThreads = 256;    // warp 0 TMA, warp 1 MMA, warps 4..7 one key / one dim per thread
-constexpr int kFirstEw = 4;
+constexpr int kFirstEw = 4;  // warp 0 TMA, warp 1 MMA, warps 4.. the key warpgroup(s)
 constexpr float kLazyTau = 8.f;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -72,6 +71,15 @@ struct Geo {
   static constexpr int kStages = (D == 64 && G == 8) ? 2 : 3;
   static constexpr uint32_t kColS = 0, kColO = 2 * kRows;
   static constexpr uint32_t kTmemCols = D == 64 ? 256 : 128;
+  // Key warpgroups: with 8 or more query heads a unit, two warpgroups split
+  // the heads (each thread still owns one key, and one dim at the end), so
+  // the per-key work of a block is done by twice the threads.  Warpgroup kg
+  // takes kHW heads; its weight rows and accumulator columns are the block
+  // 4 kHW kg .. 4 kHW (kg + 1) - 1.
+  static constexpr int kKW = kHeads >= 8 ? 2 : 1;
+  static constexpr int kHW = kHeads / kKW;
+  static constexpr int kWCols = kKW == 1 ? NW : 4 * kHW;
+  static constexpr int kThreads = 128 * (1 + kKW);
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(kColO + 2 * NW <= kTmemCols, "TMEM columns");
 };
@@ -89,13 +97,13 @@ struct Smem {
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t s_full[2], s_free[2], w_full[2], w_free[2];
   uint64_t o_full[2], o_free[2];
-  uint64_t vote[2];  // block-max exchange among the four key warps
-  uint64_t rdv;      // rendezvous of the four key warps at the end of a unit
+  uint64_t vote[Gm::kKW][2];  // block-max exchange among a warpgroup's four key warps
+  uint64_t rdv;               // rendezvous of the key warps at the end of a unit
   uint64_t drain;
   long long unit_ring[kUnitRing];
   int unit_n[kUnitRing];  // seqlens of the unit's batch row, read once by the producer
-  alignas(16) float red[2][4][Gm::kHeads];  // per-warp block maxima of each head
-  float sums[4][2 * Gm::kHeads];  // per-warp omega and T of each head
+  alignas(16) float red[Gm::kKW][2][4][Gm::kHW];  // per-warp block maxima of each head
+  float sums[Gm::kKW][4][2 * Gm::kHW];             // per-warp omega and T of each head
   int last;
   uint32_t tmem_base;
   int abort;
@@ -109,13 +117,14 @@ __device__ unsigned long long g_tc_unit_next;
 __device__ unsigned int g_tc_cta_done;
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
     decode_gqa_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                          DecodeArgs a) {
   using Gm = Geo<D, G>;
   constexpr int NW = Gm::NW, kStages = Gm::kStages, kPair = Gm::kPair, kRows = Gm::kRows;
-  constexpr int kHeads = Gm::kHeads;
+  constexpr int kKW = Gm::kKW, kHW = Gm::kHW, kWCols = Gm::kWCols;
+  constexpr int kThreads = Gm::kThreads;
   constexpr uint32_t kColS = Gm::kColS, kColO = Gm::kColO, kTmemCols = Gm::kTmemCols;
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -132,20 +141,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
-      mbar_init(&sm.unit_empty[s], 5);  // the MMA thread and the four key warps
+      mbar_init(&sm.unit_empty[s], 1 + 4 * kKW);  // the MMA thread and the key warps
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.qr_full[s], 1);
       mbar_init(&sm.qr_empty[s], 1);
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], 4);
-      mbar_init(&sm.w_full[s], 128);
+      mbar_init(&sm.s_free[s], 4 * kKW);
+      mbar_init(&sm.w_full[s], 4 * kKW);  // one arrival per key warp
       mbar_init(&sm.w_free[s], 1);
       mbar_init(&sm.o_full[s], 1);
-      mbar_init(&sm.o_free[s], 4);
-      mbar_init(&sm.vote[s], 4);
+      mbar_init(&sm.o_free[s], 4 * kKW);
+      for (int g = 0; g < kKW; ++g) mbar_init(&sm.vote[g][s], 4);
     }
-    mbar_init(&sm.rdv, 4);
+    mbar_init(&sm.rdv, 4 * kKW);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -307,15 +316,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kFirstEw) {
     // ---------------- one key of every block (scores), one dim of the accumulator ----------------
-    const int q = warp - kFirstEw, r = 32 * q + lane;
+    // Key warpgroup kg (warps 4 + 4 kg ..) takes kHW of the unit's heads: its
+    // local head j is head hh(j) = member * G + kg * hpm + j % hpm of the unit
+    // (member j / hpm), with hpm = G / kKW heads of each member.
+    const int kg = (warp - kFirstEw) >> 2, q = warp & 3, r = 32 * q + lane;
+    constexpr int hpm = G / kKW;
+    auto hh_of = [&](int j) { return (j / hpm) * G + kg * hpm + j % hpm; };
     const uint32_t lb = tmem + ((uint32_t)(32 * q) << 16);
+    const uint32_t wcol = kColO + (uint32_t)(kWCols * kg);  // this warpgroup's accumulator columns (plus NW ob)
     const float c_log2 = kLog2e / sqrtf((float)D);
     // Thread r is key r of every block and, at the end of a unit, dim
     // r % D of member r / D of the pair (d = 64) or dim r (d = 128).
     const int mem = r / D, dim = r % D;
     __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
     uint32_t pos = 0, blk = 0, ou = 0, rv = 0;
-    // Rendezvous of the four key warps (bounded like every wait).
+    // Rendezvous of all key warps (bounded like every wait).
     auto rendezvous = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.rdv);
@@ -334,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (uu < 0) break;
       const Unit x = unit_of(uu, n, kPair, a);
       if (x.bad) {
-        if (x.c == 0) {
+        if (x.c == 0 && kg == 0) {
           const long long bh0 = (long long)x.b * a.H + (long long)(x.kvh + mem) * G;
 #pragma unroll
           for (int h = 0; h < G; ++h) out[(bh0 + h) * D + dim] = __float2bfloat16(0.f);
@@ -344,13 +359,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (x.nblk == 0) continue;
       const int ob = ou & 1;
-      // Per query head of the unit (head hh: member hh / G, its head hh % G).
-      float hm[kHeads], hom[kHeads], hT[kHeads];
+      // Per local head j: running max, omega and T of this thread's keys.
+      float hm[kHW], hom[kHW], hT[kHW];
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
-        hm[h] = -CUDART_INF_F;
-        hom[h] = 0.f;
-        hT[h] = 0.f;
+      for (int j = 0; j < kHW; ++j) {
+        hm[j] = -CUDART_INF_F;
+        hom[j] = 0.f;
+        hT[j] = 0.f;
       }
       for (int i = 0; i < x.nblk; ++i) {
         const uint32_t p = pos + i, bb = blk + i;
@@ -365,77 +380,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sm.s_free[sb]);
         const int key = x.kbeg + kKeys * i + r;
         const bool valid = key < x.kend;
-        float xs[kHeads], tv[kHeads];
+        float xs[kHW], tv[kHW];
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {  // q of head hh in column 16 (hh / G) + hh % G, rho 8 further
-          const int col = 16 * (h / G) + h % G;
-          xs[h] = valid ? __uint_as_float(sv[col]) * c_log2 : -CUDART_INF_F;
-          tv[h] = valid ? __uint_as_float(sv[col + 8]) : 0.f;
+        for (int j = 0; j < kHW; ++j) {  // q of head hh in column 16 (hh / G) + hh % G, rho 8 further
+          // Warpgroup 1's heads sit hpm columns after warpgroup 0's (selected,
+          // so that every register index stays a constant).
+          const int c0 = 16 * (j / hpm) + j % hpm;
+          const uint32_t sq = kg == 0 ? sv[c0] : sv[(c0 + hpm) % kRows];
+          const uint32_t sr = kg == 0 ? sv[c0 + 8] : sv[(c0 + hpm + 8) % kRows];
+          xs[j] = valid ? __uint_as_float(sq) * c_log2 : -CUDART_INF_F;
+          tv[j] = valid ? __uint_as_float(sr) : 0.f;
         }
-        // Block max of every head over the four warps' keys.
+        // Block max of every head over the warpgroup's four warps' keys.
         {
-          const float mx = warp_max_scatter<kHeads>(xs, lane);  // head lane / (32 / kHeads)
-          if ((lane & (32 / kHeads - 1)) == 0) sm.red[sb][q][lane / (32 / kHeads)] = mx;
+          const float mx = warp_max_scatter<kHW>(xs, lane);  // local head lane / (32 / kHW)
+          if ((lane & (32 / kHW - 1)) == 0) sm.red[kg][sb][q][lane / (32 / kHW)] = mx;
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.vote[sb]);
-        if (!(ok = warp_wait(&sm.vote[sb], (bb >> 1) & 1, abort, a.status))) break;
+        if (lane == 0) mbar_arrive(&sm.vote[kg][sb]);
+        if (!(ok = warp_wait(&sm.vote[kg][sb], (bb >> 1) & 1, abort, a.status))) break;
         bool raised = false;
-        float alpha[kHeads], mb[kHeads];
-        block_max4<kHeads>(sm.red[sb], mb);
+        float alpha[kHW], mb[kHW];
+        block_max4<kHW>(sm.red[kg][sb], mb);
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          const float mblk = mb[h];
-          const bool up = mblk > hm[h] + kLazyTau;  // always on the unit's first block (m = -inf)
-          alpha[h] = up ? exp2f(hm[h] - mblk) : 1.f;
-          hm[h] = up ? mblk : hm[h];
-          hom[h] *= alpha[h];
-          hT[h] *= alpha[h];
+        for (int j = 0; j < kHW; ++j) {
+          const bool up = mb[j] > hm[j] + kLazyTau;  // always on the unit's first block (m = -inf)
+          alpha[j] = up ? exp2f(hm[j] - mb[j]) : 1.f;
+          hm[j] = up ? mb[j] : hm[j];
+          hom[j] *= alpha[j];
+          hT[j] *= alpha[j];
           raised |= up;
         }
-        if (raised && i > 0) {  // uniform over the four warps; rare after the first block
-          // Rescale the accumulator once the previous block's value MMAs are done.
+        if (raised && i > 0) {  // uniform over the warpgroup; rare after the first block
+          // Rescale this warpgroup's accumulator columns once the previous
+          // block's value MMAs are done.
           const uint32_t pb = bb - 1;
           if (!(ok = warp_wait(&sm.w_free[pb & 1], (pb >> 1) & 1, abort, a.status))) break;
           tc_fence_after();
-          uint32_t ov[NW];
-          tmem_ld_cols<NW>(lb + kColO + NW * ob, ov);
+          uint32_t ov[kWCols];
+          tmem_ld_cols<kWCols>(lb + wcol + NW * ob, ov);
           tc_wait_ld();
 #pragma unroll
-          for (int h = 0; h < kHeads; ++h) {
+          for (int j = 0; j < kHW; ++j) {
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) ov[4 * h + k4] = __float_as_uint(__uint_as_float(ov[4 * h + k4]) * alpha[h]);
+            for (int k4 = 0; k4 < 4; ++k4) ov[4 * j + k4] = __float_as_uint(__uint_as_float(ov[4 * j + k4]) * alpha[j]);
           }
-          tmem_st_cols<NW>(lb + kColO + NW * ob, ov);
+          tmem_st_cols<kWCols>(lb + wcol + NW * ob, ov);
           tc_wait_st();
           tc_fence_before();
         }
-        float wv[kHeads];
+        float wv[kHW];
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          wv[h] = exp2f(xs[h] - hm[h]);
-          hom[h] += wv[h];
-          hT[h] += wv[h] * tv[h];
+        for (int j = 0; j < kHW; ++j) {
+          wv[j] = exp2f(xs[j] - hm[j]);
+          hom[j] += wv[j];
+          hT[j] += wv[j] * tv[j];
         }
         // The weight tile of two blocks back has been consumed.
         if (!(ok = warp_wait(&sm.w_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
         uint8_t* wt = sm.w[sb][r >> 6];
         const int kk = r & 63;
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          const float w = wv[h], wtv = wv[h] * tv[h];
+        for (int j = 0; j < kHW; ++j) {
+          const int row = 4 * (kHW * kg + j);
+          const float w = wv[j], wtv = wv[j] * tv[j];
           const __nv_bfloat16 whi = __float2bfloat16_rn(w), thi = __float2bfloat16_rn(wtv);
           const __nv_bfloat16 wlo = __float2bfloat16_rn(w - __bfloat162float(whi));
           const __nv_bfloat16 tlo = __float2bfloat16_rn(wtv - __bfloat162float(thi));
-          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 0, kk)) = whi;
-          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 1, kk)) = wlo;
-          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 2, kk)) = thi;
-          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(4 * h + 3, kk)) = tlo;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(row + 0, kk)) = whi;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(row + 1, kk)) = wlo;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(row + 2, kk)) = thi;
+          *reinterpret_cast<__nv_bfloat16*>(wt + sw128_elem(row + 3, kk)) = tlo;
         }
         // Keys past the end of the sequence carry zero weight; their V rows
         // (whatever the cache holds there, even NaN) are zeroed so that they
         // cannot turn into NaN in the product.
-        if (key >= x.n) {
+        if (kg == 0 && key >= x.n) {
           // (the stage's copy is long complete: the scores of this block read it)
           if (!mbar_wait(&sm.kv_full[st], (p / kStages) & 1, abort, a.status)) ok = false;
 #pragma unroll
@@ -446,29 +466,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_async_smem();
-        mbar_arrive(&sm.w_full[sb]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.w_full[sb]);
       }
       if (!ok) break;
       // ---- End of the unit: the accumulator (thread r holds dim `dim` of
       // member `mem`) and the sums.
       if (!(ok = warp_wait(&sm.o_full[ob], (ou >> 1) & 1, abort, a.status))) break;
       tc_fence_after();
-      uint32_t ov[NW];
-      tmem_ld_cols<NW>(lb + kColO + NW * ob, ov);
+      uint32_t ov[kWCols];
+      tmem_ld_cols<kWCols>(lb + wcol + NW * ob, ov);
       tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[ob]);
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
+      for (int j = 0; j < kHW; ++j) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-          hom[h] += __shfl_xor_sync(0xffffffffu, hom[h], o);
-          hT[h] += __shfl_xor_sync(0xffffffffu, hT[h], o);
+          hom[j] += __shfl_xor_sync(0xffffffffu, hom[j], o);
+          hT[j] += __shfl_xor_sync(0xffffffffu, hT[j], o);
         }
         if (lane == 0) {
-          sm.sums[q][2 * h] = hom[h];
-          sm.sums[q][2 * h + 1] = hT[h];
+          sm.sums[kg][q][2 * j] = hom[j];
+          sm.sums[kg][q][2 * j + 1] = hT[j];
         }
       }
       if (!(ok = rendezvous())) break;
@@ -476,21 +497,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       // is query head bh0 + hh (member hh / G).
       const long long bh0 = (long long)x.b * a.H + (long long)x.kvh * G;
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
-        if (h / G != mem) continue;  // this thread's member (warp-uniform)
-        const float om = (sm.sums[0][2 * h] + sm.sums[1][2 * h]) + (sm.sums[2][2 * h] + sm.sums[3][2 * h]);
-        const float TT =
-            (sm.sums[0][2 * h + 1] + sm.sums[1][2 * h + 1]) + (sm.sums[2][2 * h + 1] + sm.sums[3][2 * h + 1]);
-        const float o1 = __uint_as_float(ov[4 * h]) + __uint_as_float(ov[4 * h + 1]);
-        const float o2 = __uint_as_float(ov[4 * h + 2]) + __uint_as_float(ov[4 * h + 3]);
-        const long long bh = bh0 + h;
+      for (int j = 0; j < kHW; ++j) {
+        if (j / hpm != mem) continue;  // this thread's member (warp-uniform)
+        const float om = (sm.sums[kg][0][2 * j] + sm.sums[kg][1][2 * j]) + (sm.sums[kg][2][2 * j] + sm.sums[kg][3][2 * j]);
+        const float TT = (sm.sums[kg][0][2 * j + 1] + sm.sums[kg][1][2 * j + 1]) +
+                         (sm.sums[kg][2][2 * j + 1] + sm.sums[kg][3][2 * j + 1]);
+        const float o1 = __uint_as_float(ov[4 * j]) + __uint_as_float(ov[4 * j + 1]);
+        const float o2 = __uint_as_float(ov[4 * j + 2]) + __uint_as_float(ov[4 * j + 3]);
+        const long long bh = bh0 + hh_of(j);
         if (x.nch == 1) {
           const float inv = 1.f / om;
           out[bh * D + dim] = __float2bfloat16_rn(((1.f + TT * inv) * o1 - o2) * inv);
         } else {
           float* rec = a.partials + (bh * a.splits + x.c) * (2 * D + 4);
           if (dim == 0) {
-            rec[0] = hm[h];
+            rec[0] = hm[j];
             rec[1] = om;
             rec[2] = TT;
           }
@@ -501,24 +522,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (x.nch > 1) {
         __threadfence();
         if (!(ok = rendezvous())) break;
-        if (r == 0) sm.last = (atomicAdd(a.counters + x.bkv, 1) == x.nch - 1);
+        if (kg == 0 && r == 0) sm.last = (atomicAdd(a.counters + x.bkv, 1) == x.nch - 1);
         if (!(ok = rendezvous())) break;
         if (sm.last) {
           __threadfence();
           // One pass over the chunks with a running max, every head's record
           // of a chunk loaded at once: one L2 round trip per chunk, not one
-          // per value.
-          float Mg[G], om[G], TT[G], p1[G], p2[G];
+          // per value.  This thread merges its warpgroup's heads of its member.
+          float Mg[hpm], om[hpm], TT[hpm], p1[hpm], p2[hpm];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
+          for (int h = 0; h < hpm; ++h) {
             Mg[h] = -CUDART_INF_F;
             om[h] = TT[h] = p1[h] = p2[h] = 0.f;
           }
           for (int cc = 0; cc < x.nch; ++cc) {
-            float mc[G], oc[G], tcv[G], q1[G], q2[G];
+            float mc[hpm], oc[hpm], tcv[hpm], q1[hpm], q2[hpm];
 #pragma unroll
-            for (int h = 0; h < G; ++h) {  // this thread's member's heads
-              const float* rc = a.partials + ((bh0 + mem * G + h) * a.splits + cc) * (2 * D + 4);
+            for (int h = 0; h < hpm; ++h) {
+              const float* rc = a.partials + ((bh0 + mem * G + kg * hpm + h) * a.splits + cc) * (2 * D + 4);
               mc[h] = __ldcg(rc);
               oc[h] = __ldcg(rc + 1);
               tcv[h] = __ldcg(rc + 2);
@@ -526,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               q2[h] = __ldcg(rc + 4 + D + dim);
             }
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
+            for (int h = 0; h < hpm; ++h) {
               const float Mn = fmaxf(Mg[h], mc[h]);  // finite: every chunk holds a key
               const float so = exp2f(Mg[h] - Mn), sc = exp2f(mc[h] - Mn);  // 2^-inf = 0 on the first
               om[h] = so * om[h] + sc * oc[h];
@@ -537,11 +558,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
+          for (int h = 0; h < hpm; ++h) {
             const float inv = 1.f / om[h];
-            out[(bh0 + mem * G + h) * D + dim] = __float2bfloat16_rn(((1.f + TT[h] * inv) * p1[h] - p2[h]) * inv);
+            out[(bh0 + mem * G + kg * hpm + h) * D + dim] =
+                __float2bfloat16_rn(((1.f + TT[h] * inv) * p1[h] - p2[h]) * inv);
           }
-          if (r == 0) a.counters[x.bkv] = 0;
+          if (kg == 0 && r == 0) a.counters[x.bkv] = 0;
         }
       }
       if (!(ok = rendezvous())) break;  // the sums and the flag are reused by the next unit
@@ -587,7 +609,7 @@ cudaError_t launch_g(const DecodeArgs& args, cudaStream_t st, int num_sms) {
   if (e != cudaSuccess) return e;
   const long long units = (long long)a.B * (a.Hkv / Geo<D, G>::kPair) * a.splits;
   const long long grid = units < num_sms ? units : num_sms;
-  decode_gqa_tc_kernel<D, G><<<(unsigned)grid, kThreads, smem, st>>>(mK, mV, mQ, mR, a);
+  decode_gqa_tc_kernel<D, G><<<(unsigned)grid, Geo<D, G>::kThreads, smem, st>>>(mK, mV, mQ, mR, a);
   return cudaGetLastError();
 }
 
