@@ -68,7 +68,10 @@ struct Geo {
   static constexpr int kRows = 16 * kPair;
   static constexpr int kHeads = G * kPair;
   static constexpr int NW = 4 * kHeads < 16 ? 16 : 4 * kHeads;
-  static constexpr int kStages = (D == 64 && G == 8) ? 2 : 3;
+  // K and V blocks travel in separate rings: a K stage is free once the
+  // block's scores are computed, a V stage only after its value product, so
+  // V gets the deeper ring where shared memory is short.
+  static constexpr int kKS = (D == 64 && G == 8) ? 2 : 3, kVS = 3;
   static constexpr uint32_t kColS = 0, kColO = 2 * kRows;
   static constexpr uint32_t kTmemCols = D == 64 ? 256 : 128;
   // Key warpgroups: with 8 or more query heads a unit, two warpgroups split
@@ -87,12 +90,12 @@ struct Geo {
 template <int D, int G>
 struct Smem {
   using Gm = Geo<D, G>;
-  static constexpr int NW = Gm::NW, kStages = Gm::kStages;
-  uint8_t k[kStages][2][kKeys * 128];  // [128 keys x 64 dims] per 64-dim half (d = 64: per member)
-  uint8_t v[kStages][2][kKeys * 128];
+  static constexpr int NW = Gm::NW, kKS = Gm::kKS, kVS = Gm::kVS;
+  uint8_t k[kKS][2][kKeys * 128];  // [128 keys x 64 dims] per 64-dim half (d = 64: per member)
+  uint8_t v[kVS][2][kKeys * 128];
   uint8_t qr[2][2][Gm::kRows * 128];   // per unit slot: [rows x 64 dims] per half
   uint8_t w[2][2][NW * 128];           // per block slot: [NW rows x 64 keys] per 64-key half
-  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kKS], k_empty[kKS], v_full[kVS], v_empty[kVS];
   uint64_t qr_full[2], qr_empty[2];
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];
   uint64_t s_full[2], s_free[2], w_full[2], w_free[2];
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
                          const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmR,
                          DecodeArgs a) {
   using Gm = Geo<D, G>;
-  constexpr int NW = Gm::NW, kStages = Gm::kStages, kPair = Gm::kPair, kRows = Gm::kRows;
+  constexpr int NW = Gm::NW, kKS = Gm::kKS, kVS = Gm::kVS, kPair = Gm::kPair, kRows = Gm::kRows;
   constexpr int kKW = Gm::kKW, kHW = Gm::kHW, kWCols = Gm::kWCols;
   constexpr int kThreads = Gm::kThreads;
   constexpr uint32_t kColS = Gm::kColS, kColO = Gm::kColO, kTmemCols = Gm::kTmemCols;
@@ -135,9 +138,13 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
   volatile int* abort = &sm.abort;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.kv_full[s], 1);
-      mbar_init(&sm.kv_empty[s], 1);
+    for (int s = 0; s < kKS; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      mbar_init(&sm.v_full[s], 1);
+      mbar_init(&sm.v_empty[s], 1);
     }
     for (int s = 0; s < kUnitRing; ++s) {
       mbar_init(&sm.unit_full[s], 1);
@@ -181,9 +188,10 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
     // ---------------- TMA producer: units, the group's q / rho rows, K and V blocks ----------------
     if (lane == 0) {
       long long u = blockIdx.x;  // first unit static, the rest from the counter
-      uint32_t pos = 0;          // K/V ring position
-      int last_kv[kStages], last_qr[2] = {-1, -1};
-      for (int s = 0; s < kStages; ++s) last_kv[s] = -1;
+      uint32_t pos = 0;          // block count: position in both rings
+      int last_k[kKS], last_v[kVS], last_qr[2] = {-1, -1};
+      for (int s = 0; s < kKS; ++s) last_k[s] = -1;
+      for (int s = 0; s < kVS; ++s) last_v[s] = -1;
       for (int ui = 0;; ++ui) {
         const int slot = ui % kUnitRing;
         if (!mbar_wait(&sm.unit_empty[slot], ((ui / kUnitRing) & 1) ^ 1, abort, a.status)) break;
@@ -212,29 +220,37 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
         }
         bool ok = true;
         for (int i = 0; i < x.nblk; ++i, ++pos) {
-          const int st = pos % kStages;
-          if (!(ok = mbar_wait(&sm.kv_empty[st], ((pos / kStages) & 1) ^ 1, abort, a.status))) break;
+          const int ks = pos % kKS, vs = pos % kVS;
+          if (!(ok = mbar_wait(&sm.k_empty[ks], ((pos / kKS) & 1) ^ 1, abort, a.status))) break;
           // The failure-detection test withholds CTA 0's K/V: the MMA thread's
           // bounded wait runs out and every role unwinds through the abort path.
           if (a.inject_stall && blockIdx.x == 0) continue;
-          mbar_expect_tx(&sm.kv_full[st], 4 * kKeys * 128);
-          last_kv[st] = (int)(pos / kStages);
+          mbar_expect_tx(&sm.k_full[ks], 2 * kKeys * 128);
+          last_k[ks] = (int)(pos / kKS);
           // The two 64-dim halves of the block: of one KV head (d = 128), or
           // one per member of the pair (d = 64).  Rows < 2^31 (launcher check).
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const int row = (x.bkv + (kPair == 2 ? h : 0)) * a.L + x.kbeg + kKeys * i;
-            const int xc = kPair == 2 ? 0 : 64 * h;
-            tma_load_2d(sm.k[st][h], &tmK, &sm.kv_full[st], xc, row);
-            tma_load_2d(sm.v[st][h], &tmV, &sm.kv_full[st], xc, row);
+            tma_load_2d(sm.k[ks][h], &tmK, &sm.k_full[ks], kPair == 2 ? 0 : 64 * h, row);
+          }
+          if (!(ok = mbar_wait(&sm.v_empty[vs], ((pos / kVS) & 1) ^ 1, abort, a.status))) break;
+          mbar_expect_tx(&sm.v_full[vs], 2 * kKeys * 128);
+          last_v[vs] = (int)(pos / kVS);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int row = (x.bkv + (kPair == 2 ? h : 0)) * a.L + x.kbeg + kKeys * i;
+            tma_load_2d(sm.v[vs][h], &tmV, &sm.v_full[vs], kPair == 2 ? 0 : 64 * h, row);
           }
         }
         if (!ok) break;
         u = next;
       }
       if (*abort) {  // let every copy issued here land before the CTA exits
-        for (int s = 0; s < kStages; ++s)
-          if (last_kv[s] >= 0) mbar_drain(&sm.kv_full[s], (uint32_t)(last_kv[s] & 1));
+        for (int s = 0; s < kKS; ++s)
+          if (last_k[s] >= 0) mbar_drain(&sm.k_full[s], (uint32_t)(last_k[s] & 1));
+        for (int s = 0; s < kVS; ++s)
+          if (last_v[s] >= 0) mbar_drain(&sm.v_full[s], (uint32_t)(last_v[s] & 1));
         for (int s = 0; s < 2; ++s)
           if (last_qr[s] >= 0) mbar_drain(&sm.qr_full[s], (uint32_t)(last_qr[s] & 1));
       }
@@ -264,8 +280,8 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
         const uint64_t bq = sdesc(smem_u32(sm.qr[qs][0]), 16, 1024);
         // Scores of block bb (ring position p): S^T = K [Q; R]^T, both K-major.
         auto issue_scores = [&](uint32_t p, uint32_t bb) -> bool {
-          const int st = p % kStages, sb = bb & 1;
-          if (!mbar_wait(&sm.kv_full[st], (p / kStages) & 1, abort, a.status)) return false;
+          const int st = p % kKS, sb = bb & 1;
+          if (!mbar_wait(&sm.k_full[st], (p / kKS) & 1, abort, a.status)) return false;
           if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
           tc_fence_after();
           const uint64_t ak = sdesc(smem_u32(sm.k[st][0]), 16, 1024);
@@ -277,6 +293,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
                    ks > 0 ? 1u : 0u);
           }
           mma_commit(&sm.s_full[sb]);
+          mma_commit(&sm.k_empty[st]);  // the K block is read
           return true;
         };
         if (!(ok = issue_scores(pos, blk))) break;
@@ -288,7 +305,8 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
           } else {
             mma_commit(&sm.qr_empty[qs]);  // every score MMA of the unit is issued
           }
-          const int st = p % kStages, sb = bb & 1;
+          const int st = p % kVS, sb = bb & 1;
+          if (!(ok = mbar_wait(&sm.v_full[st], (p / kVS) & 1, abort, a.status))) break;
           if (!(ok = mbar_wait(&sm.w_full[sb], (bb >> 1) & 1, abort, a.status))) break;
           tc_fence_after();
           // V^T as an MN-major A operand: the two 64-dim halves LBO apart,
@@ -301,7 +319,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
             mma_ss(tmem + kColO + NW * ob, av + (uint64_t)((ks * 2048) >> 4), bw + (uint64_t)(ow >> 4),
                    idesc(NW, 1, 0), (i > 0 || ks > 0) ? 1u : 0u);
           }
-          mma_commit(&sm.kv_empty[st]);
+          mma_commit(&sm.v_empty[st]);
           mma_commit(&sm.w_free[sb]);
         }
         if (!ok) break;
@@ -369,7 +387,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
       }
       for (int i = 0; i < x.nblk; ++i) {
         const uint32_t p = pos + i, bb = blk + i;
-        const int st = p % kStages, sb = bb & 1;
+        const int st = p % kVS, sb = bb & 1;
         if (!(ok = warp_wait(&sm.s_full[sb], (bb >> 1) & 1, abort, a.status))) break;
         tc_fence_after();
         uint32_t sv[kRows];
@@ -456,8 +474,8 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
         // (whatever the cache holds there, even NaN) are zeroed so that they
         // cannot turn into NaN in the product.
         if (kg == 0 && key >= x.n) {
-          // (the stage's copy is long complete: the scores of this block read it)
-          if (!mbar_wait(&sm.kv_full[st], (p / kStages) & 1, abort, a.status)) ok = false;
+          // (the V block's copy was issued with this block's K, long read)
+          if (!mbar_wait(&sm.v_full[st], (p / kVS) & 1, abort, a.status)) ok = false;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             uint4* row = reinterpret_cast<uint4*>(sm.v[st][h] + r * 128);
