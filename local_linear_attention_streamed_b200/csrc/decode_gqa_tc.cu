@@ -68,10 +68,13 @@ struct Geo {
   static constexpr int kRows = 16 * kPair;
   static constexpr int kHeads = G * kPair;
   static constexpr int NW = 4 * kHeads < 16 ? 16 : 4 * kHeads;
-  // K and V blocks travel in separate rings: a K stage is free once the
+  // K/V stages.  Where shared memory is short (the weight tiles of groups of
+  // 8 at d = 64) K and V travel in separate rings: a K stage is free once the
   // block's scores are computed, a V stage only after its value product, so
-  // V gets the deeper ring where shared memory is short.
+  // V gets the deeper ring.  Elsewhere one ring carries both (measured 3 %
+  // faster for the ungrouped decode than two rings of equal depth).
   static constexpr int kKS = (D == 64 && G == 8) ? 2 : 3, kVS = 3;
+  static constexpr bool kSepKV = kKS != kVS;
   static constexpr uint32_t kColS = 0, kColO = 2 * kRows;
   static constexpr uint32_t kTmemCols = D == 64 ? 256 : 128;
   // Key warpgroups: with 8 or more query heads a unit, two warpgroups split
@@ -126,6 +129,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
                          DecodeArgs a) {
   using Gm = Geo<D, G>;
   constexpr int NW = Gm::NW, kKS = Gm::kKS, kVS = Gm::kVS, kPair = Gm::kPair, kRows = Gm::kRows;
+  constexpr bool kSepKV = Gm::kSepKV;
   constexpr int kKW = Gm::kKW, kHW = Gm::kHW, kWCols = Gm::kWCols;
   constexpr int kThreads = Gm::kThreads;
   constexpr uint32_t kColS = Gm::kColS, kColO = Gm::kColO, kTmemCols = Gm::kTmemCols;
@@ -221,6 +225,20 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
         bool ok = true;
         for (int i = 0; i < x.nblk; ++i, ++pos) {
           const int ks = pos % kKS, vs = pos % kVS;
+          if constexpr (!kSepKV) {
+            // One ring: K and V of the block on the V stage's barriers.
+            if (!(ok = mbar_wait(&sm.v_empty[vs], ((pos / kVS) & 1) ^ 1, abort, a.status))) break;
+            if (a.inject_stall && blockIdx.x == 0) continue;
+            mbar_expect_tx(&sm.v_full[vs], 4 * kKeys * 128);
+            last_v[vs] = (int)(pos / kVS);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int row = (x.bkv + (kPair == 2 ? h : 0)) * a.L + x.kbeg + kKeys * i;
+              tma_load_2d(sm.k[ks][h], &tmK, &sm.v_full[vs], kPair == 2 ? 0 : 64 * h, row);
+              tma_load_2d(sm.v[vs][h], &tmV, &sm.v_full[vs], kPair == 2 ? 0 : 64 * h, row);
+            }
+            continue;
+          }
           if (!(ok = mbar_wait(&sm.k_empty[ks], ((pos / kKS) & 1) ^ 1, abort, a.status))) break;
           // The failure-detection test withholds CTA 0's K/V: the MMA thread's
           // bounded wait runs out and every role unwinds through the abort path.
@@ -281,7 +299,9 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
         // Scores of block bb (ring position p): S^T = K [Q; R]^T, both K-major.
         auto issue_scores = [&](uint32_t p, uint32_t bb) -> bool {
           const int st = p % kKS, sb = bb & 1;
-          if (!mbar_wait(&sm.k_full[st], (p / kKS) & 1, abort, a.status)) return false;
+          if (!(kSepKV ? mbar_wait(&sm.k_full[st], (p / kKS) & 1, abort, a.status)
+                       : mbar_wait(&sm.v_full[p % kVS], (p / kVS) & 1, abort, a.status)))
+            return false;
           if (!mbar_wait(&sm.s_free[sb], ((bb >> 1) & 1) ^ 1, abort, a.status)) return false;
           tc_fence_after();
           const uint64_t ak = sdesc(smem_u32(sm.k[st][0]), 16, 1024);
@@ -293,7 +313,7 @@ __global__ void __launch_bounds__(Geo<D, G>::kThreads, 1)
                    ks > 0 ? 1u : 0u);
           }
           mma_commit(&sm.s_full[sb]);
-          mma_commit(&sm.k_empty[st]);  // the K block is read
+          if constexpr (kSepKV) mma_commit(&sm.k_empty[st]);  // the K block is read
           return true;
         };
         if (!(ok = issue_scores(pos, blk))) break;

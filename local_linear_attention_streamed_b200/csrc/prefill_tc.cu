@@ -14,12 +14,13 @@
 //                 memory ("accumulate O1 and O2 in parallel").  Two issuing
 //                 threads keep the tensor pipe fed while either one waits on a
 //                 barrier (an MMA issue stalls until the pipe takes it).
-//   warps 2..9  two softmax warpgroups, each thread = one half (32 keys of every
-//               block, 64 output dims) of one query row (= TMEM lane): one running
-//               max and one rescale factor shared by both branches (agihunt.info
-//               summary, hardware paragraph), omega = sum w, T = sum w t in fp32,
-//               P = bf16(w) and bf16(w (t - c)) into a P buffer, and the
-//               epilogue out = ((1 + T/omega) O1 - O2) / omega.
+//   warps 2..9  two softmax warpgroups taking alternate 64-key blocks; each
+//               thread owns one query row (= TMEM lane): the whole row of its
+//               warpgroup's blocks, and half of the output dims in the epilogue.
+//               One running max and one rescale factor shared by both branches
+//               (agihunt.info summary, hardware paragraph), omega = sum w,
+//               T = sum w t in fp32, P = bf16(w) and bf16(w (t - c)) into a P
+//               buffer, and the epilogue out = ((1 + T/omega) O1 - O2) / omega.
 // TMEM (512 columns): one S stage (S1 at 0, S2 at 64: 64 fp32 columns each),
 // two P buffers at 128 and 192 (bf16 pairs: bf16(w) in columns 0..31 and
 // bf16(w (t - c)) in 32..63), O1 at 256 and O2 at 384 (128 fp32 columns each).
