@@ -671,6 +671,34 @@ def run_gpu(args, rank, world, dist):
         }
         del ht
         torch.cuda.empty_cache()
+        # Grouped cells at B=64, Hkv=8, L=4096: groups of 8 at d = 128 and the
+        # head-pair form at d = 64 (two KV heads a unit) for groups of 2, 4, 8.
+        cells = []
+        for (cd, cG) in [(128, 8), (64, 2), (64, 4), (64, 8)]:
+            cB, cHkv, cL = 64, 8, 4096
+            cH = cG * cHkv
+            cspecs = synth.decode_gqa_specs(cB, cH, cHkv, cL, cd)
+            ct = {}
+            for name, spec in cspecs.items():
+                ct[name] = torch.empty(spec.shape, dtype=torch.bfloat16, device=dev)
+                synth.device_fill(ct[name].data_ptr(), synth.BF16, seed + 9, spec)
+            csl = torch.full((cB,), cL, dtype=torch.int32, device=dev)
+            cout = torch.empty_like(ct["q"])
+
+            def cdec():
+                plx.decode_gqa(ct["q"], ct["r"], ct["K"], ct["V"], csl, out=cout)
+
+            c_total, c_per = timed(cdec, gsteps, max(3, args.warmup // 2), stream, dist)
+            if plx.get_device_status() != 0:
+                raise RuntimeError("grouped decode reported a device error")
+            c_alg = cB * cHkv * cL * cd * 2 * 2 + 3 * cB * cH * cd * 2
+            c_ach = c_alg / (float(np.mean(c_per)) * 1e-3) / 1e9
+            cells.append({"d": cd, "groups": cG, "workload": f"decode B={cB} H={cH} Hkv={cHkv} L={cL} d={cd} bf16",
+                          "kernel_gbs": round(c_ach, 1), "frac": round(c_ach / peaks["hbm_gbs"], 4),
+                          "kernel": f"decode_gqa_tc_kernel<{cd}, {cG}>", "algorithmic_bytes_per_launch": c_alg})
+            del ct
+            torch.cuda.empty_cache()
+        gqa["cells"] = cells
 
     # ---- Decode over an e4m3 KV cache: the decode workload's shape, and groups of 4.
     fp8kv = None
