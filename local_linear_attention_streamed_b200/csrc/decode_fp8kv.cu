@@ -782,23 +782,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = warp_wait(&sm.vc_free[vb], ((bb >> 1) & 1) ^ 1, abort, a.status))) break;
         const bool inside = x.kbeg + kKeys * i + r < x.n;
         const uint8_t* vr = sm.raw[st][1];
+        // All four 16-code chunks of this half row are loaded before any store:
+        // the stores into the bf16 tile could alias the raw stage as far as
+        // the compiler knows, and would otherwise serialise the loads.  Code 0
+        // converts to +0, so rows past the sequence load zeros.
+        uint4 cvv[4];
 #pragma unroll
-        for (int c = 4 * half; c < 4 * half + 4; ++c) {
+        for (int cc = 0; cc < 4; ++cc)
+          cvv[cc] = inside ? *reinterpret_cast<const uint4*>(vr + sw128_chunk(r, 4 * half + cc)) : make_uint4(0u, 0u, 0u, 0u);
+        uint8_t* dst = sm.vc[vb][half];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          // dims 64 half + 16 cc .. + 15: chunks 2 cc and 2 cc + 1 of the half's tile
           uint32_t h8[8];
-          if (inside) {
-            const uint4 cv = *reinterpret_cast<const uint4*>(vr + sw128_chunk(r, c));
-            e4m3x4_to_bf16(cv.x, h8[0], h8[1]);
-            e4m3x4_to_bf16(cv.y, h8[2], h8[3]);
-            e4m3x4_to_bf16(cv.z, h8[4], h8[5]);
-            e4m3x4_to_bf16(cv.w, h8[6], h8[7]);
-          } else {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) h8[k] = 0u;
-          }
-          // dims 16c .. 16c + 15: half c / 4, chunks 2 (c % 4) and 2 (c % 4) + 1
-          uint8_t* dst = sm.vc[vb][c >> 2];
-          *reinterpret_cast<uint4*>(dst + sw128_chunk(r, 2 * (c & 3))) = make_uint4(h8[0], h8[1], h8[2], h8[3]);
-          *reinterpret_cast<uint4*>(dst + sw128_chunk(r, 2 * (c & 3) + 1)) = make_uint4(h8[4], h8[5], h8[6], h8[7]);
+          e4m3x4_to_bf16(cvv[cc].x, h8[0], h8[1]);
+          e4m3x4_to_bf16(cvv[cc].y, h8[2], h8[3]);
+          e4m3x4_to_bf16(cvv[cc].z, h8[4], h8[5]);
+          e4m3x4_to_bf16(cvv[cc].w, h8[6], h8[7]);
+          *reinterpret_cast<uint4*>(dst + sw128_chunk(r, 2 * cc)) = make_uint4(h8[0], h8[1], h8[2], h8[3]);
+          *reinterpret_cast<uint4*>(dst + sw128_chunk(r, 2 * cc + 1)) = make_uint4(h8[4], h8[5], h8[6], h8[7]);
         }
         fence_async_smem();
         __syncwarp();
