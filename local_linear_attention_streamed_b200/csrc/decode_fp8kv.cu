@@ -31,10 +31,10 @@
 // blocks by TMA; for groups of 1 and 2 warp 1 issues the score MMAs and warp 3
 // the value MMAs (one issuing thread each: an issue waits for the tensor pipe
 // to take the MMA, and either thread's barrier waits then overlap the other's
-// issues), for larger groups warp 1 issues both; warp 2 builds the q / rho
-// operand of each unit; warps 4-7 own one key each
-// (scores, weights) and at the end of a unit one dim each (output or partial
-// record, merged by the last CTA of a (b, KV head)); warps 8-15, two per key
+// issues), for larger groups warp 1 issues both; warp 2 (with warp 3 where
+// that warp issues nothing) builds the q / rho operand of each unit; warps 4-7
+// own one key each (scores, weights) and at the end of a unit one dim each
+// (output or partial record, merged by the last CTA of a (b, KV head)); warps 8-15, two per key
 // (one per 64-dim half of its V row), convert the value rows into the bf16
 // value tile.
 //
