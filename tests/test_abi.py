@@ -101,6 +101,42 @@ def test_decode_gqa_rejects_bad_arguments(lib):
     assert lib.plx_decode_gqa_workspace_bytes(1, 16, 2, 8192, 128) > 0
 
 
+def test_fp8_cache_calls_reject_bad_arguments(lib):
+    # plx_kv_quantize_fp8(X, codes, scales, rows, d, stream)
+    assert lib.plx_kv_quantize_fp8(None, A, A, 4, 128, None) == -1
+    assert lib.plx_kv_quantize_fp8(A, A, A, 0, 128, None) == -1
+    assert lib.plx_kv_quantize_fp8(A, A, A, 4, 96, None) == -2
+    assert lib.plx_kv_quantize_fp8(A + 8, A, A, 4, 128, None) == -3
+    assert lib.plx_kv_quantize_fp8(A, A, A + 2, 4, 128, None) == -3      # scales need 4 bytes
+    # plx_decode_fp8kv(q, r, Kc, Ks, Vc, Vs, seqlens, out, B, H, Hkv, L, d, ws, ws_bytes, stream)
+    ok = [A] * 8
+    assert lib.plx_decode_fp8kv(A, A, A, None, A, A, A, A, 1, 8, 2, 64, 128, None, 0, None) == -1
+    assert lib.plx_decode_fp8kv(*ok, 1, 8, 3, 64, 128, None, 0, None) == -1   # H not a multiple of Hkv
+    assert lib.plx_decode_fp8kv(*ok, 1, 6, 2, 64, 128, None, 0, None) == -2   # group of 3
+    assert lib.plx_decode_fp8kv(*ok, 1, 32, 2, 64, 128, None, 0, None) == -2  # group of 16
+    assert lib.plx_decode_fp8kv(*ok, 1, 8, 2, 64, 64, None, 0, None) == -2    # d = 128 only
+    assert lib.plx_decode_fp8kv(A + 4, A, A, A, A, A, A, A, 1, 8, 2, 64, 128, None, 0, None) == -3
+    assert lib.plx_decode_fp8kv(A, A, A, A + 4, A, A, A, A, 1, 8, 2, 64, 128, None, 0, None) == -3  # scales 16 B
+    assert lib.plx_decode_fp8kv(A, A, A, A, A, A, A + 2, A, 1, 8, 2, 64, 128, None, 0, None) == -3  # seqlens 4 B
+    assert lib.plx_decode_fp8kv(*ok, 1 << 22, 8, 8, 64, 128, None, 0, None) == -2  # B*H above 2^24
+    assert lib.plx_decode_fp8kv_workspace_bytes(1, 8, 3, 64, 128) == 0
+    S = lib.plx_decode_num_splits(1, 2, 8192, 128)
+    assert S > 1 and lib.plx_decode_fp8kv_workspace_bytes(1, 8, 2, 8192, 128) == 8 * S * (2 * 128 + 4) * 4
+
+
+def test_dilated_prefill_rejects_bad_arguments(lib):
+    # plx_prefill_dilated(Q, K, V, R, out, B, H, Hkv, N, d, dilation, window, stream)
+    ok = [A] * 5
+    assert lib.plx_prefill_dilated(None, A, A, A, A, 1, 4, 2, 256, 128, 2, 0, None) == -1
+    assert lib.plx_prefill_dilated(*ok, 1, 4, 2, 256, 128, 0, 0, None) == -1      # dilation >= 1
+    assert lib.plx_prefill_dilated(*ok, 1, 4, 2, 256, 128, 2, -1, None) == -1     # window >= 0
+    assert lib.plx_prefill_dilated(*ok, 1, 4, 3, 256, 128, 2, 0, None) == -1      # H not a multiple of Hkv
+    assert lib.plx_prefill_dilated(*ok, 1, 4, 2, 300, 128, 7, 0, None) == -2      # ragged classes
+    assert lib.plx_prefill_dilated(*ok, 1, 4, 2, 256, 96, 2, 0, None) == -2
+    assert lib.plx_prefill_dilated(A, A, A + 8, A, A, 1, 4, 2, 256, 128, 2, 0, None) == -3
+    assert lib.plx_prefill_dilated(*ok, 1 << 20, 16, 16, 256, 128, 2, 0, None) == -2  # B*H*r above 2^24
+
+
 def test_layer_and_norm_rope_reject_bad_arguments(lib):
     assert lib.plx_qkr_norm_rope(None, A, 1, 8, 2, 128, 1e-6, 1e4, None) == -1
     assert lib.plx_qkr_norm_rope(A, A, 1, 8, 2, 96, 1e-6, 1e4, None) == -2
