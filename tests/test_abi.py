@@ -101,6 +101,20 @@ def test_decode_gqa_rejects_bad_arguments(lib):
     assert lib.plx_decode_gqa_workspace_bytes(1, 16, 2, 8192, 128) > 0
 
 
+def test_decode_kernel_choice(lib):
+    """The ungrouped bf16 decode's size rule, as plx_decode_uses_tc reports it
+    (1 = tensor-core kernel, 0 = warp-MMA kernel): at d = 128 long caches,
+    or enough (b, h) with medium ones; at d = 64 head pairs for long caches
+    over few heads only."""
+    cells = {(64, 16, 4096, 128): 1, (1, 16, 32768, 128): 1, (8, 16, 4096, 128): 0,
+             (64, 16, 1024, 128): 1, (256, 16, 16384, 128): 1, (2048, 16, 128, 128): 0,
+             (16, 16, 2048, 128): 1, (8, 16, 2048, 128): 0, (256, 16, 1024, 128): 0,
+             (1, 32, 32768, 64): 1, (64, 32, 4096, 64): 0, (1, 31, 32768, 64): 0, (4, 32, 16384, 64): 0}
+    for (B, H, L, d), want in cells.items():
+        assert lib.plx_decode_uses_tc(B, H, L, d) == want, (B, H, L, d)
+    assert lib.plx_decode_uses_tc(1, 16, 4096, 96) == -1
+
+
 def test_fp8_cache_calls_reject_bad_arguments(lib):
     # plx_kv_quantize_fp8(X, codes, scales, rows, d, stream)
     assert lib.plx_kv_quantize_fp8(None, A, A, 4, 128, None) == -1
