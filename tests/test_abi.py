@@ -176,3 +176,23 @@ def test_decode_split_plan(lib):
     # Small batches split the context; large ones do not need to.
     assert lib.plx_decode_num_splits(1, 16, 32768, 128) > 8
     assert lib.plx_decode_num_splits(2048, 16, 4096, 128) == 1
+
+
+def test_layer_workspace_slots_match_the_binding():
+    """The caller workspace of plx_layer_forward holds nine 256-byte-aligned
+    slots; the binding's views of the layer's own attention inputs and output
+    are slots 4..8, [B, H, N, d] bf16 each."""
+    import torch
+    from local_linear_attention_streamed_b200 import plx
+    for (B, N, H, d) in [(1, 1, 1, 64), (2, 100, 3, 64), (4, 8192, 16, 128), (3, 7, 5, 128)]:
+        slot = -(-(B * N * H * d * 2) // 256) * 256
+        assert plx.layer_workspace_bytes(B, N, H, d) == 9 * slot
+        if B * N * H * d > 1 << 20:
+            continue
+        ws = torch.zeros(9 * slot, dtype=torch.uint8)
+        views = plx.layer_workspace_views(ws, B, N, H, d)
+        base = ws.data_ptr()
+        for i, name in enumerate(("q", "k", "v", "rho", "attn")):
+            t = views[name]
+            assert t.dtype == torch.bfloat16 and tuple(t.shape) == (B, H, N, d)
+            assert t.data_ptr() - base == (4 + i) * slot
