@@ -147,3 +147,37 @@ def test_decode_over_quantised_cache_is_close_to_the_bf16_decode():
     want = oracle.decode_gqa_ref(q, r, K, V, sl)
     rel = np.sqrt(np.mean((got - want) ** 2) / np.mean(want * want))
     assert 1e-3 < rel < 0.15
+
+
+def test_three_e4m3_terms_hold_a_scaled_bf16_row():
+    """The e4m3-cache decode feeds q and rho to e4m3 score MMAs as three e4m3
+    terms per element (hi, then the rounding of what is left, twice), after
+    scaling the row by the power of two that puts its largest element in
+    [2^7, 2^8).  With round-to-nearest e4m3 (subnormals included) the three
+    terms give back every bf16 element to within 2^-17 of the row's largest,
+    so the three score columns add up to the score of the unrounded operand;
+    two terms do not (errors near 2^-9 of an element)."""
+    import torch
+    from oracle.layer import e4m3
+
+    rng = np.random.default_rng(5)
+    rows = rng.standard_normal((64, 128)) * 2.0 ** rng.uniform(-12, 0, (64, 128))
+    rows[0, 3] *= 2.0 ** 10                      # one element far above the rest
+    rows[1] = 0.0
+    rows[1, 7] = -3.0                            # a single non-zero element
+    x = torch.from_numpy(rows).to(torch.bfloat16).double().numpy()
+    worst3, worst2 = 0.0, 0.0
+    for row in x:
+        m = np.max(np.abs(row))
+        if m == 0:
+            continue
+        e = int(np.floor(np.log2(m))) - 7
+        y = np.ldexp(row, -e)
+        assert 2.0 ** 7 <= np.max(np.abs(y)) < 2.0 ** 8
+        t1 = e4m3(y)
+        t2 = e4m3(y - t1)
+        t3 = e4m3(y - t1 - t2)
+        worst3 = max(worst3, np.max(np.abs(y - (t1 + t2 + t3))) / np.max(np.abs(y)))
+        worst2 = max(worst2, np.max(np.abs((y - (t1 + t2)) / np.where(y == 0, 1, y))))
+    assert worst3 <= 2.0 ** -17
+    assert worst2 > 2.0 ** -10
